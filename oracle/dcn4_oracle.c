@@ -1,0 +1,315 @@
+/*
+ * dcn4_oracle.c -- plain, slow CPU restatement of DCNv4 deformable spatial
+ * aggregation, its backward pass and the FlowDCN groupwise multi-scale
+ * (MSDCN) variant.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg do.  It shares no header, helper, table or
+ * constant with the CUDA path.
+ *
+ * Sources (page title, section):
+ *  [DIGEST]  "(论文速读）DCNv4：高效可变形卷积算子" (CSDN summary of the CVPR 2024
+ *            DCNv4 paper): "移除Softmax归一化" (aggregation weights are
+ *            unbounded, no softmax), "GPU效率的理论分析" (36HWC FLOPs, the
+ *            factor 4 is the bilinear interpolation; ideal traffic
+ *            2HWC + 27HWG; worst case 64HWC), "方法1. 消除冗余工作负载" (the D = C/G
+ *            channels of a group share offsets and weights).
+ *  [FLOWDCN] "NeurIPS'24 | FlowDCN：基于可变形卷积的任意分辨率图像生成模型":
+ *            "2.2 DCN结构简介" (sample at p0 + p_k + delta p, aggregate with the
+ *            dynamic weights, concatenate the groups), "3.1 组间多尺度可变形卷积"
+ *            (delta p split into a per-group scale with prior s0_g and a
+ *            per-tap direction; the maximum scale Smax).
+ *  [CANN]    "CANN ops-nn 算子与 Stable Diffusion 的卷积实现", "2.1 标准卷积的数学
+ *            表达" (conv indexing y*s + i used for the base sampling grid).
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - offset_weight layout [N][Ho][Wo][G][kh*kw][3] holding (dx along W,
+ *    dy along H, m); tap k = i*kw + j with i along H.
+ *  - base point of tap (i, j) for output (ho, wo) is
+ *    (ho*sh - ph + i*dh, wo*sw - pw + j*dw), as in conv indexing with padding
+ *    and dilation; the sample is that point plus (dy, dx) * offset_scale.
+ *  - positions are computed in fp32: the product d*offset_scale and the sum
+ *    base + product are each rounded to nearest (this file must be built
+ *    with -ffp-contract=off so no fused multiply-add merges them).
+ *  - "zero outside the image" is per corner: a sample with x in (-1, W) and
+ *    y in (-1, H) keeps its in-image corners; any other sample (including a
+ *    NaN position) contributes nothing.
+ *  - the corner indices are floor(x), floor(y) of the fp32 position; the
+ *    fractional parts x - floor(x), y - floor(y) and the four bilinear
+ *    weights are taken in fp64, where they are exact.
+ *  - accumulation in fp64 from inputs widened exactly from their stored type.
+ *  - MSDCN: s = s0_g * softplus(raw) in fp32 with
+ *    softplus(r) = max(r, 0) + log1p(exp(-|r|)); s is clamped from above at
+ *    Smax; delta = s * dir (fp32); the sample point is then formed exactly as
+ *    in DCNv4 with delta in place of the offset.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* The oracle's own problem description (deliberately not the product's). */
+typedef struct {
+    int N, H, W, C, G;   /* input N x H x W x C, channel-last; G groups    */
+    int kh, kw;          /* kernel taps along H and W                     */
+    int sh, sw;          /* stride                                        */
+    int ph, pw;          /* padding                                       */
+    int dh, dw;          /* dilation                                      */
+    float offset_scale;  /* multiplies every offset before it is added    */
+} orc_problem;
+
+/* Output size, standard convolution arithmetic ([CANN] 2.1). Returns 0 when
+ * the problem is well formed, -1 otherwise. */
+int orc_out_hw(const orc_problem *p, int *Ho, int *Wo)
+{
+    if (!p || p->N <= 0 || p->H <= 0 || p->W <= 0 || p->C <= 0 || p->G <= 0)
+        return -1;
+    if (p->C % p->G != 0 || p->kh <= 0 || p->kw <= 0 || p->sh <= 0 ||
+        p->sw <= 0 || p->ph < 0 || p->pw < 0 || p->dh <= 0 || p->dw <= 0)
+        return -1;
+    int ho = (p->H + 2 * p->ph - p->dh * (p->kh - 1) - 1) / p->sh + 1;
+    int wo = (p->W + 2 * p->pw - p->dw * (p->kw - 1) - 1) / p->sw + 1;
+    if (ho <= 0 || wo <= 0)
+        return -1;
+    if (Ho) *Ho = ho;
+    if (Wo) *Wo = wo;
+    return 0;
+}
+
+/* The sampling position of one tap, in fp32 ([FLOWDCN] 2.2: p0 + p_k + dp). */
+static void orc_position(const orc_problem *p, int ho, int wo, int i, int j,
+                         float dx, float dy, float *x, float *y)
+{
+    float bx = (float)(wo * p->sw - p->pw + j * p->dw);
+    float by = (float)(ho * p->sh - p->ph + i * p->dh);
+    float tx = dx * p->offset_scale;
+    float ty = dy * p->offset_scale;
+    *x = bx + tx;
+    *y = by + ty;
+}
+
+/* Adds m * bilinear(img at (x, y))[c0 .. c0+D) into acc ([DIGEST]: 4 terms of
+ * the bilinear interpolation per sample; out-of-image corners are zero). */
+static void orc_splat_sample(const float *img, int H, int W, int C, int c0,
+                             int D, float x, float y, double m, double *acc)
+{
+    if (!(x > -1.0f && x < (float)W && y > -1.0f && y < (float)H))
+        return;
+    float x0f = floorf(x), y0f = floorf(y);
+    double lx = (double)x - (double)x0f, ly = (double)y - (double)y0f;
+    int x0 = (int)x0f, y0 = (int)y0f;
+    for (int a = 0; a < 2; ++a) {
+        for (int b = 0; b < 2; ++b) {
+            int yy = y0 + a, xx = x0 + b;
+            if (yy < 0 || yy >= H || xx < 0 || xx >= W)
+                continue;
+            double wy = a ? ly : 1.0 - ly;
+            double wx = b ? lx : 1.0 - lx;
+            const float *v = img + ((size_t)yy * W + xx) * C + c0;
+            for (int d = 0; d < D; ++d)
+                acc[d] += m * (wy * wx) * (double)v[d];
+        }
+    }
+}
+
+/* DCNv4 forward ([FLOWDCN] 2.2; [DIGEST] 移除Softmax归一化: m is used as given).
+ * input [N][H][W][C], offset_weight [N][Ho][Wo][G][kh*kw][3], out [N][Ho][Wo][C].
+ * Returns 0 on success, -1 on a malformed problem. */
+int orc_dcn4_forward(const orc_problem *p, const float *input,
+                     const float *offset_weight, double *out)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo) || !input || !offset_weight || !out)
+        return -1;
+    const int K = p->kh * p->kw, D = p->C / p->G;
+    const size_t img = (size_t)p->H * p->W * p->C;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int n = 0; n < p->N; ++n) {
+        for (int ho = 0; ho < Ho; ++ho) {
+            for (int wo = 0; wo < Wo; ++wo) {
+                size_t pix = ((size_t)n * Ho + ho) * Wo + wo;
+                for (int g = 0; g < p->G; ++g) {
+                    double *o = out + pix * p->C + (size_t)g * D;
+                    const float *t = offset_weight + (pix * p->G + g) * (size_t)K * 3;
+                    for (int d = 0; d < D; ++d)
+                        o[d] = 0.0;
+                    for (int i = 0; i < p->kh; ++i) {
+                        for (int j = 0; j < p->kw; ++j) {
+                            int k = i * p->kw + j;
+                            float x, y;
+                            orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);
+                            orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,
+                                             g * D, D, x, y, (double)t[3 * k + 2], o);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* DCNv4 backward: the derivative of the forward above, written out.
+ * grad_out [N][Ho][Wo][C] (values as stored), grad_input [N][H][W][C] and
+ * grad_offset_weight [N][Ho][Wo][G][kh*kw][3] are written (not accumulated).
+ *   grad m      = sum_d go_d * bilinear_d
+ *   grad dx     = offset_scale * m * sum_corners (+-wy) * <go, V_corner>
+ *   grad dy     = offset_scale * m * sum_corners (+-wx) * <go, V_corner>
+ *   grad in[c] += m * wy * wx * go        (for every in-image corner c)
+ * At an integer position the derivative taken is the one of the cell that
+ * floor() selects (the right-hand derivative). Samples outside
+ * (-1, W) x (-1, H) have zero gradient. */
+int orc_dcn4_backward(const orc_problem *p, const float *input,
+                      const float *offset_weight, const float *grad_out,
+                      double *grad_input, double *grad_offset_weight)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo) || !input || !offset_weight || !grad_out ||
+        !grad_input || !grad_offset_weight)
+        return -1;
+    const int K = p->kh * p->kw, D = p->C / p->G;
+    const size_t img = (size_t)p->H * p->W * p->C;
+    memset(grad_input, 0, sizeof(double) * img * p->N);
+    /* images are independent, so they may run in parallel */
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < p->N; ++n) {
+        const float *in_n = input + (size_t)n * img;
+        double *gin_n = grad_input + (size_t)n * img;
+        for (int ho = 0; ho < Ho; ++ho) {
+            for (int wo = 0; wo < Wo; ++wo) {
+                size_t pix = ((size_t)n * Ho + ho) * Wo + wo;
+                for (int g = 0; g < p->G; ++g) {
+                    const float *t = offset_weight + (pix * p->G + g) * (size_t)K * 3;
+                    double *gt = grad_offset_weight + (pix * p->G + g) * (size_t)K * 3;
+                    const float *go = grad_out + pix * p->C + (size_t)g * D;
+                    for (int i = 0; i < p->kh; ++i) {
+                        for (int j = 0; j < p->kw; ++j) {
+                            int k = i * p->kw + j;
+                            float x, y;
+                            orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);
+                            double m = (double)t[3 * k + 2];
+                            double gx = 0.0, gy = 0.0, gm = 0.0;
+                            if (x > -1.0f && x < (float)p->W && y > -1.0f && y < (float)p->H) {
+                                float x0f = floorf(x), y0f = floorf(y);
+                                double lx = (double)x - (double)x0f;
+                                double ly = (double)y - (double)y0f;
+                                int x0 = (int)x0f, y0 = (int)y0f;
+                                for (int a = 0; a < 2; ++a) {
+                                    for (int b = 0; b < 2; ++b) {
+                                        int yy = y0 + a, xx = x0 + b;
+                                        if (yy < 0 || yy >= p->H || xx < 0 || xx >= p->W)
+                                            continue;
+                                        double wy = a ? ly : 1.0 - ly;
+                                        double wx = b ? lx : 1.0 - lx;
+                                        size_t at = ((size_t)yy * p->W + xx) * p->C + (size_t)g * D;
+                                        double dot = 0.0;
+                                        for (int d = 0; d < D; ++d) {
+                                            dot += (double)go[d] * (double)in_n[at + d];
+                                            gin_n[at + d] += m * (wy * wx) * (double)go[d];
+                                        }
+                                        gm += wy * wx * dot;
+                                        gx += (b ? wy : -wy) * dot;
+                                        gy += (a ? wx : -wx) * dot;
+                                    }
+                                }
+                            }
+                            gt[3 * k] = (double)p->offset_scale * m * gx;
+                            gt[3 * k + 1] = (double)p->offset_scale * m * gy;
+                            gt[3 * k + 2] = gm;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* MSDCN per-group scale ([FLOWDCN] 3.1): s = min(s0 * softplus(raw), smax)
+ * in fp32. A NaN raw gives a NaN scale (and hence no contribution). */
+float orc_msdcn_scale(float raw, float s0, float smax)
+{
+    float sp = fmaxf(raw, 0.0f) + log1pf(expf(-fabsf(raw)));
+    float s = s0 * sp;
+    if (s > smax)
+        s = smax;
+    return s;
+}
+
+/* MSDCN forward ([FLOWDCN] 3.1): DCNv4 aggregation whose offset for group g
+ * and tap k is s_g(p0) * dir_{g,k}(p0).
+ * dir_weight [N][Ho][Wo][G][kh*kw][3] holds (dir_x, dir_y, m);
+ * scale_raw [N][Ho][Wo][G]; s0 [G]. */
+int orc_msdcn_forward(const orc_problem *p, const float *input,
+                      const float *dir_weight, const float *scale_raw,
+                      const float *s0, float smax, double *out)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo) || !input || !dir_weight || !scale_raw || !s0 || !out)
+        return -1;
+    const int K = p->kh * p->kw, D = p->C / p->G;
+    const size_t img = (size_t)p->H * p->W * p->C;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int n = 0; n < p->N; ++n) {
+        for (int ho = 0; ho < Ho; ++ho) {
+            for (int wo = 0; wo < Wo; ++wo) {
+                size_t pix = ((size_t)n * Ho + ho) * Wo + wo;
+                for (int g = 0; g < p->G; ++g) {
+                    double *o = out + pix * p->C + (size_t)g * D;
+                    const float *t = dir_weight + (pix * p->G + g) * (size_t)K * 3;
+                    float s = orc_msdcn_scale(scale_raw[pix * p->G + g], s0[g], smax);
+                    for (int d = 0; d < D; ++d)
+                        o[d] = 0.0;
+                    for (int i = 0; i < p->kh; ++i) {
+                        for (int j = 0; j < p->kw; ++j) {
+                            int k = i * p->kw + j;
+                            float dx = s * t[3 * k], dy = s * t[3 * k + 1];
+                            float x, y;
+                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);
+                            orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,
+                                             g * D, D, x, y, (double)t[3 * k + 2], o);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* --- cost model of [DIGEST] "GPU效率的理论分析" -------------------------- */
+
+/* FLOPs: 4 (bilinear terms) per tap per output element, i.e. 36 HWC for a
+ * 3x3 kernel with H, W the output size. */
+double orc_flops(const orc_problem *p)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo))
+        return -1.0;
+    return 4.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;
+}
+
+/* Ideal traffic in bytes: input and output once, plus 3 values per tap per
+ * group per output pixel (27 HWG for 3x3); elem_bytes per value. */
+double orc_ideal_bytes(const orc_problem *p, int elem_bytes)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo))
+        return -1.0;
+    double in = (double)p->N * p->H * p->W * p->C;
+    double out = (double)p->N * Ho * Wo * p->C;
+    double ow = 3.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->G;
+    return (in + out + ow) * elem_bytes;
+}
+
+/* Worst-case traffic with no cache: for every output element 4 reads per
+ * tap, 3 offset/weight reads per tap and one write (64 HWC for 3x3). */
+double orc_worst_bytes(const orc_problem *p, int elem_bytes)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo))
+        return -1.0;
+    double per = 4.0 * p->kh * p->kw + 3.0 * p->kh * p->kw + 1.0;
+    return per * (double)p->N * Ho * Wo * p->C * elem_bytes;
+}
