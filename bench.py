@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the DCNv4 hot path on B200.
+
+One step = DCNv4 forward + DCNv4 backward + MSDCN forward over one batch of
+the InternImage-stage workload (N64 56x56 C128 G8, bf16; MSDCN inputs of the
+same shape), inputs resident in HBM. Each op is captured once in a CUDA graph
+and replayed; L2 is flushed (256 MB write) before every timed step; CUDA
+events on the launching stream time each op. The reported value is effective
+bandwidth: the operator's ideal bytes (input and output once, 27 offset/weight
+values per pixel and group; DCNv4 digest "GPU效率的理论分析") per second of device
+time, summed over all ranks (weak scaling: every rank runs a full batch).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DCNv4 fwd/bwd GB/s and Gsample·ch/s at 1 B200; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="internimage_bf16")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- accounting
+def ideal_bytes(wl, Ho, Wo):
+    """Ideal traffic of each op in bytes (inputs read once, outputs written once)."""
+    eb = 4 if wl.dtype == "f32" else 2
+    nin = wl.N * wl.H * wl.W * wl.C
+    nout = wl.N * Ho * Wo * wl.C
+    now = wl.N * Ho * Wo * wl.G * wl.K * 3
+    return {
+        "dcn4_forward": (nin + nout + now) * eb,
+        "dcn4_backward": (nin + nout + now + nin + now) * eb,
+        "msdcn_forward": (nin + nout + now + wl.N * Ho * Wo * wl.G) * eb,
+    }
+
+
+def samples_ch(wl, Ho, Wo):
+    """Bilinear samples x channels of one forward (K per output element)."""
+    return wl.K * wl.N * Ho * Wo * wl.C
+
+
+def msdcn_variant(wl):
+    return wl.replace(kind="msdcn", offset_dist=("normal", 1.0))
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "deformable_convolution_dcn4_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = rec.get(f"{kernel}@{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value, device="cpu"):
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_step_sample(wl, n_images):
+    """The oracle's fwd + bwd + MSDCN fwd on the first n_images of the
+    workload; returns (seconds, ideal bytes processed)."""
+    import oracle
+    from deformable_convolution_dcn4_b200.workloads import make_inputs
+    orc = oracle.default()
+    sub = wl.replace(N=n_images)
+    p = orc.problem(sub.N, sub.H, sub.W, sub.C, sub.G, sub.kh, sub.kw, sub.stride, sub.pad,
+                    sub.dilation, sub.offset_scale)
+    Ho, Wo = orc.out_hw(p)
+    d = make_inputs(sub, (Ho, Wo), with_grad=True)
+    ms = make_inputs(msdcn_variant(sub), (Ho, Wo))
+    arr = {k: v.float().numpy() for k, v in d.items()}
+    marr = {k: v.float().numpy() for k, v in ms.items()}
+    t0 = time.perf_counter()
+    orc.forward(p, arr["input"], arr["offset_weight"])
+    orc.backward(p, arr["input"], arr["offset_weight"], arr["grad_out"])
+    orc.msdcn_forward(p, marr["input"], marr["dir_weight"], marr["scale_raw"], marr["s0"],
+                      sub.smax)
+    dt = time.perf_counter() - t0
+    return dt, sum(ideal_bytes(sub, Ho, Wo).values())
+
+
+def cpu_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    """Times the oracle on a bounded sample (whole images, growing until the
+    run takes about budget_s)."""
+    n, total_t, total_b, runs = 1, 0.0, 0.0, 0
+    while True:
+        dt, b = oracle_step_sample(wl, n)
+        total_t, total_b, runs = total_t + dt, total_b + b, runs + 1
+        if total_t >= budget_s or n >= wl.N:
+            break
+        n = min(wl.N, max(n + 1, int(n * budget_s / max(total_t, 1e-3) * 0.5)))
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"{runs} oracle runs of fwd+bwd+MSDCN fwd on up to {n} of {wl.N} images "
+                      f"of {wl.name}, {total_t:.1f} s total"}
+
+
+# ---------------------------------------------------------------- our arm
+def describe(wl, Ho, Wo):
+    return {"workload": f"{wl.name}: N{wl.N} {wl.H}x{wl.W} C{wl.C} G{wl.G} (D{wl.D}) "
+                        f"{wl.kh}x{wl.kw} s{wl.stride[0]} p{wl.pad[0]} d{wl.dilation[0]} "
+                        f"{wl.dtype}; offsets {wl.offset_dist[0]}({wl.offset_dist[1]}) px, "
+                        f"m ~ N(0,{wl.weight_sigma}); MSDCN inputs of the same shape "
+                        f"(dir ~ N(0,1), raw ~ N(0,1), s0 = 1,1,2,2,.., Smax {wl.smax})",
+            "ops_per_step": ["dcn4_forward", "dcn4_backward", "msdcn_forward"],
+            "N": wl.N, "H": wl.H, "W": wl.W, "C": wl.C, "G": wl.G, "Ho": Ho, "Wo": Wo,
+            "l2": "flushed before every timed step (256 MB write)",
+            "parallelism": "batch replicas, one process per GPU"}
+
+
+def run_ours(args):
+    import torch
+
+    import deformable_convolution_dcn4_b200 as dcn
+    from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    dcn.load()
+
+    wl = WORKLOADS[args.workload]
+    desc = dcn.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, 0, (wl.kh, wl.kw), wl.stride, wl.pad,
+                         wl.dilation, wl.offset_scale)
+    Ho, Wo = dcn.dcn4_out_shape(desc)
+    host = make_inputs(wl, (Ho, Wo), with_grad=True)
+    mhost = make_inputs(msdcn_variant(wl), (Ho, Wo))
+    d = {k: v.to(dev) for k, v in host.items()}
+    m = {k: (v if k == "s0" else v.to(dev)) for k, v in mhost.items()}
+    kw = dict(group=wl.G, kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad,
+              dilation=wl.dilation, offset_scale=wl.offset_scale)
+    out = torch.empty((wl.N, Ho, Wo, wl.C), dtype=d["input"].dtype, device=dev)
+    ms_out = torch.empty_like(out)
+    gin = torch.empty_like(d["input"])
+    gow = torch.empty_like(d["offset_weight"])
+    dsc = dcn.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, d["input"].dtype, (wl.kh, wl.kw),
+                        wl.stride, wl.pad, wl.dilation, wl.offset_scale)
+    ws = torch.empty(max(dcn.dcn4_backward_workspace_size(dsc), 16), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    ops = {
+        "dcn4_forward": lambda: dcn.dcn4_forward(d["input"], d["offset_weight"], out=out, **kw),
+        "dcn4_backward": lambda: dcn.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"],
+                                                   workspace=ws, grad_input=gin,
+                                                   grad_offset_weight=gow, **kw),
+        "msdcn_forward": lambda: dcn.msdcn_forward(m["input"], m["dir_weight"], m["scale_raw"],
+                                                   m["s0"], wl.smax, out=ms_out, **kw),
+    }
+    launches = {"dcn4_forward": 1, "dcn4_backward": 3, "msdcn_forward": 1}
+    for f in ops.values():  # first calls set kernel attributes outside any capture
+        f()
+    torch.cuda.synchronize()
+    graphs = {}
+    for name, f in ops.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        graphs[name] = g
+    torch.cuda.synchronize()
+    names = list(ops)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed_step():
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record(stream)
+        for i, n in enumerate(names):
+            graphs[n].replay()
+            ev[i + 1].record(stream)
+        return ev
+
+    for _ in range(args.warmup):
+        timed_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    torch.cuda.synchronize()
+    per_op = {n: 0.0 for n in names}
+    with ClockSampler(local) as clocks:
+        evs = [timed_step() for _ in range(args.steps)]
+        torch.cuda.synchronize()
+    for ev in evs:
+        for i, n in enumerate(names):
+            per_op[n] += ev[i].elapsed_time(ev[i + 1])
+    step_ms_local = sum(per_op.values()) / args.steps
+    barrier(dev)
+    torch.cuda.synchronize()
+    step_ms = max_over_ranks(step_ms_local, dev)
+    ib = ideal_bytes(wl, Ho, Wo)
+    step_bytes = sum(ib.values())
+    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    op_ms = {n: per_op[n] / args.steps for n in names}
+    peak, peak_kind = hbm_peak()
+    breakdown = {}
+    for n in names:
+        gbs = ib[n] / (op_ms[n] * 1e-3) / 1e9
+        breakdown[n] = {"ms": round(op_ms[n], 5), "ideal_bytes": ib[n], "GB/s": round(gbs, 1),
+                        f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4)}
+    breakdown["dcn4_forward"]["Gsample_ch_per_s"] = round(
+        samples_ch(wl, Ho, Wo) / (op_ms["dcn4_forward"] * 1e-3) / 1e9, 1)
+    breakdown["msdcn_forward"]["Gsample_ch_per_s"] = round(
+        samples_ch(wl, Ho, Wo) / (op_ms["msdcn_forward"] * 1e-3) / 1e9, 1)
+    dom = max(names, key=lambda n: op_ms[n])
+    dom_gbs = ib[dom] / (op_ms[dom] * 1e-3) / 1e9
+    traffic = recorded_traffic(dom, wl.name)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} copy bandwidth",
+                "bytes_per_launch": ib[dom]}
+
+    # end to end: pinned host buffers, H2D copies + the three calls + D2H reads
+    e2e = run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream,
+                  step_bytes, world)
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic (seeded; shapes and distributions of an "
+                                       "InternImage stage)",
+            "config": describe(wl, Ho, Wo), "roofline": roofline, "ops": breakdown,
+            "gpu_launches": args.steps * sum(launches.values()), "e2e": e2e,
+            "clocks": clocks.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    barrier(dev)
+    for g in graphs.values():
+        del g
+    graphs.clear()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream, step_bytes,
+            world):
+    import torch
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    mpin = {k: (v if k == "s0" else v.pin_memory()) for k, v in mhost.items()}
+    outs = [out, gin, gow, ms_out]
+    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(v.numel() * v.element_size() for v in pin.values()) + \
+        sum(v.numel() * v.element_size() for k, v in mpin.items() if k != "s0")
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def step():
+        for k, v in pin.items():
+            d[k].copy_(v, non_blocking=True)
+        for k, v in mpin.items():
+            if k != "s0":
+                m[k].copy_(v, non_blocking=True)
+        for f in ops.values():
+            f()
+        for t, h in zip(outs, hout):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    steps = max(1, min(args.steps, 10))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "path": "Python binding -> C ABI, pinned host buffers, "
+                                    "cudaMemcpyAsync both ways inside the timed region"}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    from deformable_convolution_dcn4_b200.workloads import WORKLOADS
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    n_img = min(4, wl.N)
+    for _ in range(args.warmup):
+        oracle_step_sample(wl, n_img)
+    times, nbytes = [], 0.0
+    for _ in range(args.steps):
+        dt, b = oracle_step_sample(wl, n_img)
+        times.append(dt)
+        nbytes = b
+    step_s = sum(times) / len(times)
+    value = nbytes / step_s / 1e9
+    sample = (f"fwd+bwd+MSDCN fwd of the CPU oracle on {n_img} of {wl.N} images of {wl.name} "
+              f"per step")
+    sub = wl.replace(N=n_img)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": describe(sub, wl.H, wl.W),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+"""Thin ctypes binding of libdcn4.so (the C ABI in include/dcn4.h).
+
+Argument marshalling only: tensors come from torch (device memory, the
+current stream), every step of the operator runs in the library's CUDA
+kernels. There is no CPU fallback: calls raise when the library or a CUDA
+device is missing.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libdcn4.so")
+
+STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
+          3: "DCN4_ERR_WORKSPACE", 4: "DCN4_ERR_CUDA", 5: "DCN4_ERR_TIMEOUT",
+          6: "DCN4_ERR_INTERNAL"}
+DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2}
+
+# Every symbol include/dcn4.h declares.
+EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
+           "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error")
+
+
+class Dcn4Error(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("N", "H", "W", "C", "G", "kh", "kw", "stride_h", "stride_w", "pad_h", "pad_w",
+                 "dil_h", "dil_w")] + [("offset_scale", ctypes.c_float), ("dtype", ctypes.c_int),
+                                       ("algo", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load(path=LIBRARY):
+    """Loads libdcn4.so once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libdcn4.so not built ({path}); run "
+                           "`python -m deformable_convolution_dcn4_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(Desc)
+    vp, st = ctypes.c_void_p, ctypes.c_int
+    lib.dcn4_out_shape.argtypes = [P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.dcn4_forward.argtypes = [P, vp, vp, vp, vp]
+    lib.dcn4_backward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.dcn4_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.msdcn_forward.argtypes = [P, vp, vp, vp, ctypes.POINTER(ctypes.c_float), ctypes.c_float,
+                                  vp, vp]
+    lib.dcn4_status_string.argtypes = [st]
+    lib.dcn4_status_string.restype = ctypes.c_char_p
+    lib.dcn4_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    for name in EXPORTS:
+        if name != "dcn4_status_string":
+            getattr(lib, name).restype = st
+    _lib = lib
+    return lib
+
+
+def _pair(v):
+    return (int(v), int(v)) if isinstance(v, (int, float)) else (int(v[0]), int(v[1]))
+
+
+def make_desc(N, H, W, C, G, dtype, kernel_size=3, stride=1, pad=1, dilation=1,
+              offset_scale=1.0, algo="auto"):
+    kh, kw = _pair(kernel_size)
+    sh, sw = _pair(stride)
+    ph, pw = _pair(pad)
+    dh, dw = _pair(dilation)
+    code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return Desc(N, H, W, C, G, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale), code,
+                ALGO_CODE[algo])
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise Dcn4Error(fn, rc)
+
+
+def dcn4_out_shape(desc):
+    ho, wo = ctypes.c_int(), ctypes.c_int()
+    _check("dcn4_out_shape", load().dcn4_out_shape(ctypes.byref(desc), ctypes.byref(ho),
+                                                   ctypes.byref(wo)))
+    return ho.value, wo.value
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _require(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (channel-last)")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo):
+    N, H, W, C = inp.shape
+    return make_desc(N, H, W, C, group, inp.dtype, kernel_size, stride, pad, dilation,
+                     offset_scale, algo)
+
+
+def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, dilation=1,
+                 offset_scale=1.0, algo="auto", out=None):
+    """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3]."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    ho, wo = dcn4_out_shape(desc)
+    N, _, _, C = input.shape
+    _require(input, "input", input.dtype)
+    _require(offset_weight, "offset_weight", input.dtype,
+             (N, ho, wo, group, desc.kh * desc.kw, 3))
+    if out is None:
+        out = torch.empty((N, ho, wo, C), dtype=input.dtype, device=input.device)
+    _require(out, "out", input.dtype, (N, ho, wo, C))
+    _check("dcn4_forward", load().dcn4_forward(ctypes.byref(desc), _ptr(input), _ptr(offset_weight),
+                                               _ptr(out), _stream(input)))
+    return out
+
+
+def dcn4_backward_workspace_size(desc):
+    n = ctypes.c_size_t()
+    _check("dcn4_backward_workspace_size",
+           load().dcn4_backward_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
+                  dilation=1, offset_scale=1.0, algo="auto", workspace=None,
+                  grad_input=None, grad_offset_weight=None):
+    """DCNv4 backward -> (grad_input, grad_offset_weight)."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    ho, wo = dcn4_out_shape(desc)
+    N, H, W, C = input.shape
+    _require(input, "input", input.dtype)
+    _require(offset_weight, "offset_weight", input.dtype,
+             (N, ho, wo, group, desc.kh * desc.kw, 3))
+    _require(grad_out, "grad_out", input.dtype, (N, ho, wo, C))
+    if grad_input is None:
+        grad_input = torch.empty_like(input)
+    if grad_offset_weight is None:
+        grad_offset_weight = torch.empty_like(offset_weight)
+    need = dcn4_backward_workspace_size(desc)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=input.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("dcn4_backward", load().dcn4_backward(
+        ctypes.byref(desc), _ptr(input), _ptr(offset_weight), _ptr(grad_out), _ptr(grad_input),
+        _ptr(grad_offset_weight), ws_ptr, ws_bytes, _stream(input)))
+    return grad_input, grad_offset_weight
+
+
+def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, stride=1, pad=1,
+                  dilation=1, offset_scale=1.0, algo="auto", out=None):
+    """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G]."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    ho, wo = dcn4_out_shape(desc)
+    N, _, _, C = input.shape
+    _require(input, "input", input.dtype)
+    _require(dir_weight, "dir_weight", input.dtype, (N, ho, wo, group, desc.kh * desc.kw, 3))
+    _require(scale_raw, "scale_raw", input.dtype, (N, ho, wo, group))
+    s0 = [float(v) for v in (s0.tolist() if isinstance(s0, torch.Tensor) else s0)]
+    if len(s0) != group:
+        raise ValueError("s0 must hold one prior per group")
+    s0_arr = (ctypes.c_float * group)(*s0)
+    if out is None:
+        out = torch.empty((N, ho, wo, C), dtype=input.dtype, device=input.device)
+    _require(out, "out", input.dtype, (N, ho, wo, C))
+    _check("msdcn_forward", load().msdcn_forward(
+        ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr,
+        float(smax), _ptr(out), _stream(input)))
+    return out
+
+
+def dcn4_status_string(code):
+    return load().dcn4_status_string(int(code)).decode()
+
+
+def dcn4_last_device_error():
+    """(status, raw bits) of the device error word, which it clears."""
+    bits = ctypes.c_uint()
+    rc = load().dcn4_last_device_error(ctypes.byref(bits))
+    return rc, bits.value

@@ -1,0 +1,50 @@
+"""Builds libdcn4.so (the C-ABI library) in-tree with nvcc for sm_100a.
+
+    python -m deformable_convolution_dcn4_b200.build [--force] [--verbose]
+
+No fast-math: sample positions rely on IEEE fp32 rounding of each multiply
+and add (the kernels use __fmul_rn/__fadd_rn where it matters).
+"""
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIBRARY = os.path.join(PKG, "libdcn4.so")
+SOURCES = ["dcn4_api.cu", "dcn4_kernels.cu"]
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+         "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden",
+         "-DDCN4_BUILDING_LIBRARY", "-I", INCLUDE, "-I", CSRC]
+
+
+def _inputs():
+    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
+    files.append(os.path.join(INCLUDE, "dcn4.h"))
+    return files
+
+
+def up_to_date():
+    if not os.path.exists(LIBRARY):
+        return False
+    t = os.path.getmtime(LIBRARY)
+    return all(os.path.getmtime(f) <= t for f in _inputs())
+
+
+def build(force=False, verbose=False):
+    if not force and up_to_date():
+        return LIBRARY
+    cmd = [NVCC, *FLAGS]
+    if verbose:
+        cmd += ["-Xptxas", "-v"]
+    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", LIBRARY]
+    subprocess.run(cmd, check=True)
+    return LIBRARY
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

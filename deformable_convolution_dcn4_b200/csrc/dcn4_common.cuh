@@ -1,0 +1,210 @@
+// dcn4_common.cuh -- shared device helpers and launch parameter blocks for the
+// DCNv4 / MSDCN kernels (sm_100a). Host and device code both include it.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dcn4 {
+
+// Bits of the device error word (read back by dcn4_last_device_error).
+constexpr unsigned kErrTimeout = 1u;   // a bounded mbarrier wait expired
+constexpr unsigned kErrInternal = 2u;  // a consistency check failed
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+constexpr int kMaxGroups = 1024;
+
+// Problem geometry, copied into every launch.
+struct Geometry {
+    int N, H, W, C, G, D;
+    int kh, kw, K;
+    int sh, sw, ph, pw, dh, dw;
+    int Ho, Wo;
+    float os;  // offset_scale
+};
+
+// MSDCN extras: per-group scale priors travel inside the launch parameters.
+struct MsdcnParams {
+    const void *raw;  // [N][Ho][Wo][G] in the element type
+    float smax;
+    float s0[kMaxGroups];
+};
+
+// Tiling of the shared-memory halo kernels (chosen on the host).
+struct HaloPlan {
+    int TH, TW;          // output tile
+    int Gc;              // groups per CTA (a divisor of G)
+    int R;               // offset reach covered by the halo, in pixels
+    int HR, HC;          // halo rows / columns held in shared memory
+    int full_h, full_w;  // 1: the halo is the whole image plus a 1-pixel zero border
+    int tiles_h, tiles_w, slices;
+    int slot_bytes;      // bytes per output pixel of staged offset/weight triples
+    int halo_bytes;      // HR*HC*Gc*D*elem, rounded up to 128
+    int smem_bytes;      // dynamic shared memory of one CTA
+};
+
+// ---- element types -------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static constexpr int kBytes = 4;
+    static constexpr int kPerVec = 4;  // elements per 16-byte vector
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static constexpr int kBytes = 2;
+    static constexpr int kPerVec = 8;
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+template <> struct Elem<__half> {
+    static constexpr int kBytes = 2;
+    static constexpr int kPerVec = 8;
+    static __device__ __forceinline__ float to_f(__half v) { return __half2float(v); }
+    static __device__ __forceinline__ __half from_f(float v) { return __float2half_rn(v); }
+};
+
+// ---- sample position: fp32, product and sum rounded separately -------------
+__device__ __forceinline__ float sample_coord(int base, float delta, float os) {
+    return __fadd_rn((float)base, __fmul_rn(delta, os));
+}
+
+// ---- packed fp32 pair FMA (sm_100a f32x2) -----------------------------------
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float x0, float x1, float w) {
+    unsigned long long acc, xv, wv;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(wv) : "f"(w));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(xv), "l"(wv));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+}
+
+// acc[0..kPerVec) += w * (16-byte vector v of T), fp32 arithmetic.
+template <typename T> struct VecMath;
+template <> struct VecMath<float> {
+    static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {
+        ffma2(acc[0], acc[1], __uint_as_float(v.x), __uint_as_float(v.y), w);
+        ffma2(acc[2], acc[3], __uint_as_float(v.z), __uint_as_float(v.w), w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float *a) {
+        return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]),
+                          __float_as_uint(a[2]), __float_as_uint(a[3]));
+    }
+};
+template <> struct VecMath<__nv_bfloat16> {
+    static __device__ __forceinline__ void fma2w(float *acc, unsigned w2, float w) {
+        ffma2(acc[0], acc[1], __uint_as_float(w2 << 16), __uint_as_float(w2 & 0xffff0000u), w);
+    }
+    static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {
+        fma2w(acc + 0, v.x, w);
+        fma2w(acc + 2, v.y, w);
+        fma2w(acc + 4, v.z, w);
+        fma2w(acc + 6, v.w, w);
+    }
+    static __device__ __forceinline__ unsigned pk(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<unsigned *>(&h);
+    }
+    static __device__ __forceinline__ uint4 pack(const float *a) {
+        return make_uint4(pk(a[0], a[1]), pk(a[2], a[3]), pk(a[4], a[5]), pk(a[6], a[7]));
+    }
+};
+template <> struct VecMath<__half> {
+    static __device__ __forceinline__ void fma2w(float *acc, unsigned w2, float w) {
+        __half2 h = *reinterpret_cast<__half2 *>(&w2);
+        float2 f = __half22float2(h);
+        ffma2(acc[0], acc[1], f.x, f.y, w);
+    }
+    static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {
+        fma2w(acc + 0, v.x, w);
+        fma2w(acc + 2, v.y, w);
+        fma2w(acc + 4, v.z, w);
+        fma2w(acc + 6, v.w, w);
+    }
+    static __device__ __forceinline__ unsigned pk(float lo, float hi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<unsigned *>(&h);
+    }
+    static __device__ __forceinline__ uint4 pack(const float *a) {
+        return make_uint4(pk(a[0], a[1]), pk(a[2], a[3]), pk(a[4], a[5]), pk(a[6], a[7]));
+    }
+};
+
+// ---- shared memory / async-copy primitives --------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for phase `parity` of the barrier for at most `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// 4-D tiled TMA load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
+
+// Plain (untiled) bulk copy global -> shared; 16-byte aligned addresses and size.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+}  // namespace dcn4

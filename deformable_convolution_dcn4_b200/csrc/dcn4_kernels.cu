@@ -1,0 +1,162 @@
+// dcn4_kernels.cu -- the one translation unit holding every device function of
+// libdcn4: kernel instantiations, their launchers and the device error word.
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "dcn4_common.cuh"
+
+namespace dcn4 {
+// Set by kernels whose bounded waits expire; read by dcn4_last_device_error.
+__device__ unsigned int g_error_word = 0;
+}  // namespace dcn4
+
+#include "dcn4_bwd.cuh"
+#include "dcn4_fwd.cuh"
+#include "dcn4_launch.h"
+
+namespace dcn4 {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int cached_attr(cudaDeviceAttr attr, int (&cache)[kMaxDevices]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (cache[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, attr, dev) == cudaSuccess) cache[dev] = v;
+    }
+    return cache[dev];
+}
+
+// Raises a kernel's dynamic shared memory limit once per (kernel, device).
+cudaError_t allow_smem(const void *kernel, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kernel, dev})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem_optin());
+    if (e == cudaSuccess) done.insert({kernel, dev});
+    return e;
+}
+
+int grid_for(long long work, int block) {
+    long long blocks = (work + block - 1) / block;
+    const long long cap = (long long)sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+template <typename T, int U, bool MS>
+cudaError_t launch_halo_t(const FwdLaunch &L) {
+    auto k = fwd_halo_kernel<T, U, MS>;
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.plan.smem_bytes);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
+    static const MsdcnParams kNoMs = {};
+    k<<<(unsigned)grid, 256, L.plan.smem_bytes, L.stream>>>(
+        *L.tmap, L.geo, L.plan, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+        static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
+    return cudaGetLastError();
+}
+
+template <typename T, bool MS>
+cudaError_t launch_halo_u(const FwdLaunch &L) {
+    const int U = L.geo.D * (int)sizeof(T) / 16;
+    switch (U) {
+        case 2: return launch_halo_t<T, 2, MS>(L);
+        case 4: return launch_halo_t<T, 4, MS>(L);
+        case 8: return launch_halo_t<T, 8, MS>(L);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T, bool MS>
+cudaError_t launch_generic_t(const FwdLaunch &L) {
+    const long long work = (long long)L.geo.N * L.geo.Ho * L.geo.Wo * L.geo.G * ((L.geo.D + 7) / 8);
+    static const MsdcnParams kNoMs = {};
+    fwd_generic_kernel<T, MS><<<grid_for(work, 256), 256, 0, L.stream>>>(
+        L.geo, static_cast<const T *>(L.in), static_cast<const T *>(L.ow), static_cast<T *>(L.out),
+        L.ms ? *L.ms : kNoMs);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_fwd_t(const FwdLaunch &L) {
+    if (L.halo) return L.msdcn ? launch_halo_u<T, true>(L) : launch_halo_u<T, false>(L);
+    return L.msdcn ? launch_generic_t<T, true>(L) : launch_generic_t<T, false>(L);
+}
+
+template <typename T>
+cudaError_t launch_bwd_t(const BwdLaunch &L) {
+    const Geometry &g = L.geo;
+    const long long nin = (long long)g.N * g.H * g.W * g.C;
+    zero_f32_kernel<<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(L.acc, nin);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
+    bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
+        g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+        static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (static_cast<void *>(L.acc) != L.gin) {
+        convert_f32_kernel<T><<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(
+            L.acc, static_cast<T *>(L.gin), nin);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace
+
+int sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int v = cached_attr(cudaDevAttrMultiProcessorCount, cache);
+    return v > 0 ? v : 148;
+}
+
+int max_smem_optin() {
+    static int cache[kMaxDevices] = {0};
+    int v = cached_attr(cudaDevAttrMaxSharedMemoryPerBlockOptin, cache);
+    return v > 0 ? v : 48 * 1024;
+}
+
+cudaError_t launch_forward(const FwdLaunch &L) {
+    switch (L.dtype) {
+        case Dtype::F32: return launch_fwd_t<float>(L);
+        case Dtype::BF16: return launch_fwd_t<__nv_bfloat16>(L);
+        case Dtype::F16: return launch_fwd_t<__half>(L);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_backward(const BwdLaunch &L) {
+    switch (L.dtype) {
+        case Dtype::F32: return launch_bwd_t<float>(L);
+        case Dtype::BF16: return launch_bwd_t<__nv_bfloat16>(L);
+        case Dtype::F16: return launch_bwd_t<__half>(L);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t read_clear_device_error(unsigned *bits) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v));
+    if (e != cudaSuccess) return e;
+    if (v != 0) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    }
+    *bits = v;
+    return e;
+}
+
+}  // namespace dcn4

@@ -1,0 +1,51 @@
+// dcn4_launch.h -- host-side launch interface between the C ABI (dcn4_api.cu)
+// and the kernel translation unit (dcn4_kernels.cu).
+#pragma once
+
+#include "dcn4_common.cuh"
+
+namespace dcn4 {
+
+enum class Dtype { F32 = 0, BF16 = 1, F16 = 2 };
+
+inline int elem_bytes(Dtype t) { return t == Dtype::F32 ? 4 : 2; }
+
+struct FwdLaunch {
+    Geometry geo;
+    Dtype dtype;
+    bool msdcn;
+    const void *in;
+    const void *ow;   // offset_weight (DCNv4) or dir_weight (MSDCN)
+    void *out;
+    const MsdcnParams *ms;  // MSDCN only
+    bool halo;              // use the shared-memory halo kernel
+    HaloPlan plan;
+    const CUtensorMap *tmap;
+    unsigned long long ow_bytes;
+    cudaStream_t stream;
+};
+
+struct BwdLaunch {
+    Geometry geo;
+    Dtype dtype;
+    const void *in;
+    const void *ow;
+    const void *gout;
+    void *gin;     // element type
+    void *gow;     // element type
+    float *acc;    // fp32 accumulation buffer for grad_input (== gin for fp32)
+    cudaStream_t stream;
+};
+
+cudaError_t launch_forward(const FwdLaunch &L);
+cudaError_t launch_backward(const BwdLaunch &L);
+
+// Reads and clears the device error word of the current device.
+cudaError_t read_clear_device_error(unsigned *bits);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+// Largest opt-in dynamic shared memory per block of the current device.
+int max_smem_optin();
+
+}  // namespace dcn4

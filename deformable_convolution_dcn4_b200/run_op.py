@@ -1,0 +1,49 @@
+"""Runs one operator of the library a few times on a named workload; the
+command profilers (ncu) wrap to capture single kernels.
+
+    python -m deformable_convolution_dcn4_b200.run_op --op forward \
+        --workload internimage_bf16 --iters 3 [--N 64] [--algo auto]
+"""
+import argparse
+import sys
+
+import torch
+
+from . import _binding as B
+from .workloads import WORKLOADS, make_inputs
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--op", choices=["forward", "backward", "msdcn"], default="forward")
+    p.add_argument("--workload", default="internimage_bf16")
+    p.add_argument("--iters", type=int, default=3)
+    p.add_argument("--N", type=int, default=None)
+    p.add_argument("--algo", default="auto")
+    a = p.parse_args(argv)
+    wl = WORKLOADS[a.workload]
+    if a.N:
+        wl = wl.replace(N=a.N)
+    if a.op == "msdcn" and wl.kind != "msdcn":
+        wl = wl.replace(kind="msdcn", offset_dist=("normal", 1.0))
+    desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, 0, (wl.kh, wl.kw), wl.stride, wl.pad,
+                       wl.dilation, wl.offset_scale)
+    ho, wo = B.dcn4_out_shape(desc)
+    d = make_inputs(wl, (ho, wo), with_grad=a.op == "backward", device="cuda")
+    kw = dict(group=wl.G, kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad,
+              dilation=wl.dilation, offset_scale=wl.offset_scale, algo=a.algo)
+    for _ in range(a.iters):
+        if a.op == "forward":
+            B.dcn4_forward(d["input"], d["offset_weight"], **kw)
+        elif a.op == "backward":
+            B.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"], **kw)
+        else:
+            B.msdcn_forward(d["input"], d["dir_weight"], d["scale_raw"], d["s0"], wl.smax, **kw)
+    torch.cuda.synchronize()
+    rc, bits = B.dcn4_last_device_error()
+    print(f"run_op {a.op} {wl.name} N={wl.N} iters={a.iters}: device error bits {bits}")
+    return 0 if rc == 0 else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main())

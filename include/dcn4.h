@@ -1,0 +1,152 @@
+/*
+ * dcn4.h -- C ABI of the B200 (sm_100a) DCNv4 deformable spatial aggregation
+ * library (libdcn4.so).
+ *
+ * The operation (DCNv4, CVPR 2024; as summarised in "(论文速读）DCNv4：高效可变形
+ * 卷积算子", sections "移除Softmax归一化" and "方法1. 消除冗余工作负载", and in
+ * "NeurIPS'24 | FlowDCN：基于可变形卷积的任意分辨率图像生成模型", section
+ * "2.2 DCN结构简介"): for every output pixel p0 = (ho, wo), group g and kernel
+ * tap k = (i, j), sample the channel-last input by bilinear interpolation at
+ *
+ *     x = (wo*stride_w - pad_w + j*dil_w) + dx * offset_scale
+ *     y = (ho*stride_h - pad_h + i*dil_h) + dy * offset_scale
+ *
+ * (in-image corners only; a sample outside (-1, W) x (-1, H) adds nothing),
+ * multiply the sample by the unnormalised weight m (no softmax), sum over the
+ * taps and write the D = C/G channels of group g into their slot of the
+ * C-vector (the groups are concatenated).
+ *
+ * Tensors (all dense, contiguous, channel-last, one element type per call):
+ *   input          [N][H][W][C]
+ *   offset_weight  [N][Ho][Wo][G][kh*kw][3]   triples (dx along W, dy along H, m),
+ *                                             tap k = i*kw + j, i along H
+ *   output         [N][Ho][Wo][C]
+ *   Ho = (H + 2*pad_h - dil_h*(kh-1) - 1) / stride_h + 1, likewise Wo.
+ *
+ * Arithmetic: sample positions are formed in fp32 with the product
+ * dx*offset_scale and the sum each rounded to nearest (no fused multiply-add),
+ * so corner indices match a CPU evaluation of the same formula bit for bit;
+ * interpolation weights and accumulation are fp32; results are rounded once
+ * to the element type.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are owned by the caller; the library allocates no memory
+ *     and keeps no per-call state (the one exception is a device error word,
+ *     see dcn4_last_device_error).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Calls only enqueue work; they never synchronise the device.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Argument errors are reported synchronously before anything is
+ *     launched; launch failures come back as DCN4_ERR_CUDA.
+ *   - Pointers that are not 16-byte aligned, or channel counts whose group
+ *     slice is not a multiple of 16 bytes, are legal: such calls take the
+ *     generic (slower) kernels.
+ */
+#ifndef DCN4_H
+#define DCN4_H
+
+#include <stddef.h>
+
+#if defined(DCN4_BUILDING_LIBRARY) && defined(__GNUC__)
+#define DCN4_API __attribute__((visibility("default")))
+#else
+#define DCN4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DCN4_OK = 0,
+    DCN4_ERR_INVALID_ARG = 1,  /* malformed descriptor or null pointer        */
+    DCN4_ERR_UNSUPPORTED = 2,  /* well formed but outside what is implemented */
+    DCN4_ERR_WORKSPACE = 3,    /* workspace missing or too small              */
+    DCN4_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed        */
+    DCN4_ERR_TIMEOUT = 5,      /* a device-side bounded wait expired          */
+    DCN4_ERR_INTERNAL = 6      /* a device-side consistency check failed      */
+} dcn4_status;
+
+typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
+
+/* Kernel selection. AUTO picks the staged (shared-memory halo) kernel when
+ * the call qualifies and the generic one otherwise; the other values force
+ * a variant (a forced variant the call does not qualify for returns
+ * DCN4_ERR_UNSUPPORTED). */
+typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
+
+/* The whole configuration of one call. Limits: all sizes positive, C % G == 0,
+ * G <= 1024, 1 <= kh*kw <= 64, strides and dilations >= 1, pads >= 0, every
+ * tensor below 2^31 elements, Ho and Wo positive. */
+typedef struct {
+    int N, H, W, C, G;
+    int kh, kw;
+    int stride_h, stride_w;
+    int pad_h, pad_w;
+    int dil_h, dil_w;
+    float offset_scale;
+    dcn4_dtype dtype;
+    dcn4_algo algo;
+} dcn4_desc;
+
+/* Output size for `desc` (standard convolution arithmetic, as in
+ * "CANN ops-nn 算子与 Stable Diffusion 的卷积实现", "2.1 标准卷积的数学表达").
+ * Returns DCN4_ERR_INVALID_ARG for a malformed descriptor. */
+DCN4_API dcn4_status dcn4_out_shape(const dcn4_desc *desc, int *Ho, int *Wo);
+
+/* DCNv4 forward (definition above). input, offset_weight and output are
+ * device pointers of desc->dtype with the shapes above; output must not
+ * overlap the inputs. */
+DCN4_API dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input,
+                         const void *offset_weight, void *output, void *stream);
+
+/* Bytes of device workspace dcn4_backward needs for `desc`: an fp32 copy of
+ * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. */
+DCN4_API dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes);
+
+/* DCNv4 backward: the derivative of the forward (the pages only say that
+ * DCNv4 optimised its backward operator; FlowDCN article, "2.2" and "4.1").
+ * Reads input, offset_weight and grad_out ([N][Ho][Wo][C]); writes
+ *   grad_input          [N][H][W][C]     sum over samples of m*w_corner*grad_out
+ *   grad_offset_weight  [N][Ho][Wo][G][kh*kw][3]
+ *       (d/d dx, d/d dy, d/d m) of sum(output * grad_out).
+ * At an integer sample position the derivative is that of the cell floor()
+ * selects. `workspace` (>= dcn4_backward_workspace_size bytes, 16-byte
+ * aligned, device memory owned by the caller) may be NULL when that size is 0.
+ * grad_input accumulates in fp32 with atomic adds, so its last bits may vary
+ * from run to run. */
+DCN4_API dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input,
+                          const void *offset_weight, const void *grad_out,
+                          void *grad_input, void *grad_offset_weight,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* MSDCN (groupwise multi-scale DCN) forward, "NeurIPS'24 | FlowDCN", section
+ * "3.1 组间多尺度可变形卷积": the offset of group g, tap k at pixel p0 is
+ * s_g(p0) * dir_{g,k}(p0) with
+ *     s_g = min(s0[g] * softplus(scale_raw), smax),
+ *     softplus(r) = max(r, 0) + log1p(exp(-|r|))       (fp32, expf/log1pf),
+ * after which the sample is formed exactly as in dcn4_forward (offset_scale
+ * still applies). dir_weight [N][Ho][Wo][G][kh*kw][3] holds (dir_x, dir_y, m);
+ * scale_raw [N][Ho][Wo][G] (device, desc->dtype); s0_host [G] is a HOST array
+ * of fp32 scale priors, copied into the launch. A NaN scale gives no
+ * contribution. */
+DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
+                          const void *dir_weight, const void *scale_raw,
+                          const float *s0_host, float smax, void *output,
+                          void *stream);
+
+/* Human-readable name of a status code (static storage). */
+DCN4_API const char *dcn4_status_string(dcn4_status status);
+
+/* Reads and clears the device error word that kernels set when a bounded wait
+ * expires (DCN4_ERR_TIMEOUT) or a consistency check fails
+ * (DCN4_ERR_INTERNAL). *code receives the raw bit set (0 = none). This call
+ * synchronises the current device. Returns DCN4_OK when the word was clear,
+ * otherwise the status the bits map to. */
+DCN4_API dcn4_status dcn4_last_device_error(unsigned int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN4_H */

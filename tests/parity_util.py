@@ -1,0 +1,92 @@
+"""Helpers shared by the GPU parity tests: run one case through the C ABI and
+through the CPU oracle on the same seeded inputs and compare."""
+import numpy as np
+import torch
+
+from deformable_convolution_dcn4_b200 import _binding as B
+from deformable_convolution_dcn4_b200.workloads import make_inputs
+
+# Gates (scaled error = max |gpu - ref| / max |ref|): fp32 1e-5; bf16/fp16
+# outputs are rounded to their 8/11-bit mantissas, gate 2e-2.
+TOL = {"f32": 1e-5, "bf16": 2e-2, "f16": 2e-2}
+
+
+def scaled_err(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite GPU output"
+    scale = np.abs(ref).max()
+    if scale == 0.0:
+        return float(np.abs(got).max())
+    return float(np.abs(got - ref).max() / scale)
+
+
+def f32(t):
+    return t.float().cpu().numpy()
+
+
+def desc_kw(wl):
+    return dict(kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
+                offset_scale=wl.offset_scale)
+
+
+def out_hw(wl):
+    d = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, 0, (wl.kh, wl.kw), wl.stride, wl.pad,
+                    wl.dilation, wl.offset_scale)
+    return B.dcn4_out_shape(d)
+
+
+def problem(orc, wl, N=None):
+    return orc.problem(N or wl.N, wl.H, wl.W, wl.C, wl.G, wl.kh, wl.kw, wl.stride, wl.pad,
+                       wl.dilation, wl.offset_scale)
+
+
+def gpu_forward(wl, data, algo="auto"):
+    dev = "cuda"
+    if wl.kind == "msdcn":
+        return B.msdcn_forward(data["input"].to(dev), data["dir_weight"].to(dev),
+                               data["scale_raw"].to(dev), data["s0"], wl.smax, group=wl.G,
+                               algo=algo, **desc_kw(wl))
+    return B.dcn4_forward(data["input"].to(dev), data["offset_weight"].to(dev), group=wl.G,
+                          algo=algo, **desc_kw(wl))
+
+
+def oracle_forward(orc, wl, data, images=None):
+    """Oracle output for all images, or for the listed images only."""
+    sel = slice(None) if images is None else list(images)
+    n = wl.N if images is None else len(images)
+    prob = problem(orc, wl, n)
+    x = f32(data["input"][sel])
+    if wl.kind == "msdcn":
+        return orc.msdcn_forward(prob, x, f32(data["dir_weight"][sel]),
+                                 f32(data["scale_raw"][sel]), data["s0"].numpy(), wl.smax)
+    return orc.forward(prob, x, f32(data["offset_weight"][sel]))
+
+
+def forward_case(orc, wl, algo="auto", images=None):
+    data = make_inputs(wl, out_hw(wl))
+    got = f32(gpu_forward(wl, data, algo))
+    ref = oracle_forward(orc, wl, data, images)
+    if images is not None:
+        got = got[list(images)]
+    return scaled_err(got, ref)
+
+
+def backward_case(orc, wl, algo="auto", images=None):
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    dev = "cuda"
+    gin, gow = B.dcn4_backward(data["input"].to(dev), data["offset_weight"].to(dev),
+                               data["grad_out"].to(dev), group=wl.G, algo=algo, **desc_kw(wl))
+    sel = slice(None) if images is None else list(images)
+    n = wl.N if images is None else len(images)
+    rgin, rgow = orc.backward(problem(orc, wl, n), f32(data["input"][sel]),
+                              f32(data["offset_weight"][sel]), f32(data["grad_out"][sel]))
+    gin, gow = f32(gin), f32(gow)
+    if images is not None:
+        gin, gow = gin[list(images)], gow[list(images)]
+    return scaled_err(gin, rgin), scaled_err(gow, rgow)
+
+
+def cuda_sync():
+    torch.cuda.synchronize()

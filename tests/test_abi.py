@@ -1,0 +1,113 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, and validates arguments on the host before touching CUDA."""
+import ctypes
+import re
+
+import pytest
+
+from deformable_convolution_dcn4_b200 import _binding as B
+from deformable_convolution_dcn4_b200 import build as libbuild
+
+HEADER = libbuild.INCLUDE + "/dcn4.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return B.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"DCN4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_binding_exports():
+    assert sorted(declared_symbols()) == sorted(B.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_only_the_abi_is_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    text_syms = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared_symbols()) <= text_syms
+    leaked = {s for s in text_syms if s.startswith(("dcn4", "msdcn", "_ZN4dcn4"))} - set(
+        declared_symbols())
+    assert not leaked, leaked
+
+
+def test_status_strings(lib):
+    for code, name in B.STATUS.items():
+        assert B.dcn4_status_string(code) == name
+    assert B.dcn4_status_string(99) == "DCN4_UNKNOWN_STATUS"
+
+
+def _desc(**kw):
+    base = dict(N=2, H=9, W=11, C=16, G=4, dtype=0, kernel_size=3, stride=1, pad=1, dilation=1)
+    base.update(kw)
+    return B.make_desc(base["N"], base["H"], base["W"], base["C"], base["G"], base["dtype"],
+                       base["kernel_size"], base["stride"], base["pad"], base["dilation"])
+
+
+def test_out_shape_matches_oracle(lib, orc):
+    cases = [dict(), dict(stride=2), dict(pad=0), dict(dilation=2), dict(kernel_size=5, pad=2),
+             dict(kernel_size=1, pad=0), dict(kernel_size=(3, 1), pad=(1, 0)),
+             dict(stride=(2, 3), pad=(0, 2), dilation=(2, 1)), dict(H=1, W=1, kernel_size=1, pad=0)]
+    for c in cases:
+        d = _desc(**c)
+        p = orc.problem(d.N, d.H, d.W, d.C, d.G, d.kh, d.kw, (d.stride_h, d.stride_w),
+                        (d.pad_h, d.pad_w), (d.dil_h, d.dil_w))
+        assert B.dcn4_out_shape(d) == orc.out_hw(p), c
+
+
+@pytest.mark.parametrize("bad", [dict(C=10, G=4), dict(N=0), dict(G=0), dict(stride=0),
+                                 dict(dilation=0), dict(pad=-1), dict(H=2, pad=0),
+                                 dict(dtype=7), dict(C=2048, G=2048),
+                                 dict(kernel_size=9, pad=4)])
+def test_malformed_descriptors_rejected(lib, bad):
+    d = _desc(**bad)
+    with pytest.raises(B.Dcn4Error) as e:
+        B.dcn4_out_shape(d)
+    assert e.value.code == 1
+    n = ctypes.c_size_t()
+    assert lib.dcn4_backward_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 1
+
+
+def test_null_pointers_rejected_before_any_launch(lib):
+    d = _desc()
+    z = ctypes.c_void_p(0)
+    one = ctypes.c_void_p(16)
+    assert lib.dcn4_forward(ctypes.byref(d), z, one, one, z) == 1
+    assert lib.dcn4_forward(ctypes.byref(d), one, z, one, z) == 1
+    assert lib.dcn4_forward(ctypes.byref(d), one, one, z, z) == 1
+    assert lib.dcn4_forward(None, one, one, one, z) == 1
+    s0 = (ctypes.c_float * 4)(1, 1, 2, 2)
+    assert lib.msdcn_forward(ctypes.byref(d), one, one, z, s0, 8.0, one, z) == 1
+    assert lib.msdcn_forward(ctypes.byref(d), one, one, one, None, 8.0, one, z) == 1
+    assert lib.dcn4_backward(ctypes.byref(d), one, one, one, z, one, one, 1 << 30, z) == 1
+
+
+def test_workspace_rules(lib):
+    d32 = _desc(dtype=0)
+    assert B.dcn4_backward_workspace_size(d32) == 0
+    d16 = _desc(dtype=1)
+    assert B.dcn4_backward_workspace_size(d16) == 2 * 9 * 11 * 16 * 4
+    one = ctypes.c_void_p(16)
+    z = ctypes.c_void_p(0)
+    # too small / missing workspace is reported before anything runs
+    assert lib.dcn4_backward(ctypes.byref(d16), one, one, one, one, one, z, 0, z) == 3
+    assert lib.dcn4_backward(ctypes.byref(d16), one, one, one, one, one, one, 100, z) == 3
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 8, 8, 16)
+    ow = torch.zeros(1, 8, 8, 4, 9, 3)
+    with pytest.raises(ValueError):
+        B.dcn4_forward(x, ow, group=4)

@@ -1,0 +1,235 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs, element by element (scaled max error), for every kernel
+variant, the workload shapes (reduced, then full size on sampled images) and
+the edge cases."""
+import numpy as np
+import pytest
+import torch
+
+from deformable_convolution_dcn4_b200 import _binding as B
+from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
+
+from parity_util import (TOL, backward_case, f32, forward_case, gpu_forward, oracle_forward,
+                         out_hw, problem, scaled_err)
+
+pytestmark = pytest.mark.gpu
+
+W = WORKLOADS
+ALGOS = ["auto", "generic", "halo"]
+
+# Workload shapes at sizes the oracle finishes in seconds (several tiles,
+# ragged tails where the sizes allow).
+REDUCED = {
+    "tiny_f32": W["tiny_f32"],
+    "internimage_bf16": W["internimage_bf16"].replace(N=2),
+    "internimage_f32": W["internimage_f32"].replace(N=2),
+    "ldm64_f16": W["ldm64_f16"].replace(N=1),
+    "ldm32_f16": W["ldm32_f16"].replace(N=2),
+    "flowdcn_msdcn_bf16": W["flowdcn_msdcn_bf16"].replace(N=2),
+    "highres_bf16": W["highres_bf16"].replace(N=1),
+}
+
+EDGE = {
+    "ragged_bf16": W["internimage_bf16"].replace(name="ragged", N=2, H=37, W=29, C=64, G=4),
+    "stride2_pad0_dil2_f16": W["ldm64_f16"].replace(name="s2", N=1, H=33, W=30, C=64, G=4,
+                                                    stride=(2, 2), pad=(0, 0), dilation=(2, 2)),
+    "stride_mixed_f32": W["tiny_f32"].replace(name="smix", N=2, H=21, W=18, C=32, G=2,
+                                              stride=(1, 2), pad=(2, 0), dilation=(1, 2)),
+    "offset_scale_bf16": W["internimage_bf16"].replace(name="os", N=1, H=20, W=24,
+                                                       offset_scale=0.75),
+    "far_offsets_bf16": W["internimage_bf16"].replace(name="far", N=1, H=40, W=40,
+                                                      offset_dist=("normal", 8.0)),
+    "far_offsets_f32": W["internimage_f32"].replace(name="far32", N=1, H=24, W=32,
+                                                    offset_dist=("normal", 6.0)),
+    "single_group_f16": W["ldm64_f16"].replace(name="g1", N=2, H=12, W=10, C=16, G=1),
+    "tiny_image_bf16": W["internimage_bf16"].replace(name="t", N=3, H=2, W=3, C=32, G=2),
+    "one_pixel_f32": W["tiny_f32"].replace(name="p", N=2, H=1, W=1, C=16, G=4),
+    "d64_f32": W["tiny_f32"].replace(name="d64", N=1, H=12, W=14, C=128, G=2),
+}
+
+GENERIC_ONLY = {
+    "k1x1_bf16": W["internimage_bf16"].replace(name="k1", N=1, H=10, W=12, kh=1, kw=1,
+                                                pad=(0, 0)),
+    "k5x5_f32": W["tiny_f32"].replace(name="k5", N=1, H=11, W=9, kh=5, kw=5, pad=(2, 2)),
+    "k3x1_f16": W["ldm64_f16"].replace(name="k31", N=1, H=9, W=8, C=32, G=2, kh=3, kw=1,
+                                       pad=(1, 0)),
+    "d12_bf16": W["internimage_bf16"].replace(name="d12", N=1, H=14, W=10, C=36, G=3),
+    "d6_f32": W["tiny_f32"].replace(name="d6", N=1, H=9, W=9, C=6, G=1),
+}
+
+
+def _halo_supported(wl):
+    eb = 4 if wl.dtype == "f32" else 2
+    u = wl.D * eb // 16
+    return wl.kh == 3 and wl.kw == 3 and (wl.D * eb) % 16 == 0 and u in (2, 4, 8)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("name", sorted(REDUCED))
+def test_forward_reduced(orc, name, algo):
+    wl = REDUCED[name]
+    err = forward_case(orc, wl, algo)
+    assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_forward_edge(orc, name, algo):
+    wl = EDGE[name]
+    if algo == "halo" and not _halo_supported(wl):
+        pytest.skip("halo kernel needs 3x3 taps and 32/64/128-byte group slices")
+    err = forward_case(orc, wl, algo)
+    assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", sorted(GENERIC_ONLY))
+def test_forward_generic_shapes(orc, name):
+    wl = GENERIC_ONLY[name]
+    err = forward_case(orc, wl, "auto")
+    assert err <= TOL[wl.dtype], f"{name}: {err:.3e}"
+    with pytest.raises(B.Dcn4Error) as e:
+        forward_case(orc, wl, "halo")
+    assert e.value.code == 2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("algo", ALGOS)
+def test_integer_offsets_gather_exactly(orc, dtype, algo):
+    """Integer offsets and one tap with m = 1: the output is a copy of input
+    pixels (or zero), so the GPU must equal the oracle bit for bit; this pins
+    the corner selection."""
+    wl = W["internimage_bf16"].replace(N=2, H=19, W=23, C=64, G=4, dtype=dtype)
+    Ho, Wo = out_hw(wl)
+    data = make_inputs(wl, (Ho, Wo))
+    g = torch.Generator().manual_seed(3)
+    ow = torch.zeros((wl.N, Ho, Wo, wl.G, 9, 3))
+    ow[..., :2] = torch.randint(-6, 7, (wl.N, Ho, Wo, wl.G, 9, 2), generator=g).float()
+    tap = torch.randint(0, 9, (wl.N, Ho, Wo, wl.G), generator=g)
+    ow[..., 2].scatter_(-1, tap[..., None], 1.0)
+    data["offset_weight"] = ow.to(data["input"].dtype)
+    got = f32(gpu_forward(wl, data, algo))
+    ref = oracle_forward(orc, wl, data)
+    assert np.array_equal(got, ref.astype(np.float32))
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_all_samples_out_of_bounds_give_zero(orc, algo):
+    wl = W["internimage_bf16"].replace(N=1, H=16, W=16)
+    Ho, Wo = out_hw(wl)
+    data = make_inputs(wl, (Ho, Wo))
+    ow = data["offset_weight"].float()
+    ow[..., 0] = -(wl.W + 5.0)
+    data["offset_weight"] = ow.to(torch.bfloat16)
+    assert torch.count_nonzero(gpu_forward(wl, data, algo)).item() == 0
+
+
+def test_nonfinite_offsets_contribute_nothing(orc):
+    wl = W["tiny_f32"]
+    Ho, Wo = out_hw(wl)
+    data = make_inputs(wl, (Ho, Wo))
+    ow = data["offset_weight"].clone()
+    ow[0, 3, 4, 1, 2, 0] = float("nan")
+    ow[0, 5, 6, 2, 7, 1] = float("inf")
+    data["offset_weight"] = ow
+    for algo in ALGOS:
+        got = f32(gpu_forward(wl, data, algo))
+        assert scaled_err(got, oracle_forward(orc, wl, data)) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("algo", ["auto", "halo"])
+def test_msdcn_unit_scale_is_dcn4(orc, algo):
+    """softplus(30) > Smax = 1 so every scale is exactly 1: MSDCN must equal
+    DCNv4 with offsets = directions, bit for bit."""
+    wl = REDUCED["flowdcn_msdcn_bf16"].replace(N=1, smax=1.0)
+    Ho, Wo = out_hw(wl)
+    data = make_inputs(wl, (Ho, Wo))
+    data["scale_raw"] = torch.full_like(data["scale_raw"], 30.0)
+    data["s0"] = torch.ones(wl.G)
+    ms = gpu_forward(wl, data, algo)
+    dcn = B.dcn4_forward(data["input"].cuda(), data["dir_weight"].cuda(), group=wl.G, algo=algo)
+    assert torch.equal(ms, dcn)
+
+
+def test_misaligned_pointers_take_generic_path(orc):
+    wl = W["internimage_bf16"].replace(N=1, H=12, W=12)
+    Ho, Wo = out_hw(wl)
+    data = make_inputs(wl, (Ho, Wo))
+    x = torch.empty(data["input"].numel() + 1, dtype=torch.bfloat16, device="cuda")[1:]
+    x = x.view(data["input"].shape)
+    x.copy_(data["input"])
+    assert x.data_ptr() % 16 != 0
+    out = B.dcn4_forward(x, data["offset_weight"].cuda(), group=wl.G)
+    assert scaled_err(f32(out), oracle_forward(orc, wl, data)) <= TOL["bf16"]
+    with pytest.raises(B.Dcn4Error) as e:
+        B.dcn4_forward(x, data["offset_weight"].cuda(), group=wl.G, algo="halo")
+    assert e.value.code == 2
+
+
+def test_forward_is_deterministic():
+    wl = REDUCED["internimage_bf16"]
+    data = make_inputs(wl, out_hw(wl))
+    a = gpu_forward(wl, data)
+    b = gpu_forward(wl, data)
+    assert torch.equal(a, b)
+
+
+# ---- full sizes, in the bench's launch configuration, sampled images ----
+FULL_SAMPLES = {
+    "internimage_bf16": [0, 37, 63],
+    "internimage_f32": [0, 63],
+    "ldm64_f16": [0, 7],
+    "ldm32_f16": [0, 5],
+    "flowdcn_msdcn_bf16": [0, 31],
+    "highres_bf16": [0, 3],
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL_SAMPLES))
+def test_forward_full_size_sampled(orc, name):
+    wl = W[name]
+    err = forward_case(orc, wl, "auto", images=FULL_SAMPLES[name])
+    assert err <= TOL[wl.dtype], f"{name}: {err:.3e}"
+
+
+# ---- backward ----
+BWD = {
+    "tiny_f32": W["tiny_f32"],
+    "highres_bf16_small": W["highres_bf16"].replace(N=1, H=40, W=36),
+    "internimage_bf16": W["internimage_bf16"].replace(N=1),
+    "ldm_f16": W["ldm64_f16"].replace(N=1, H=24, W=20),
+    "stride2_dil2_f32": W["tiny_f32"].replace(N=2, H=17, W=15, C=32, G=2, stride=(2, 2),
+                                              dilation=(2, 2), pad=(2, 1), offset_scale=0.5),
+    "k5_f32": W["tiny_f32"].replace(N=1, H=9, W=11, C=8, G=2, kh=5, kw=5, pad=(2, 2)),
+    "d12_bf16": W["internimage_bf16"].replace(N=1, H=10, W=9, C=36, G=3),
+    "far_bf16": W["internimage_bf16"].replace(N=1, H=24, W=24, offset_dist=("normal", 8.0)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BWD))
+def test_backward(orc, name):
+    wl = BWD[name]
+    e_in, e_ow = backward_case(orc, wl)
+    tol = TOL[wl.dtype]
+    assert e_in <= tol and e_ow <= tol, f"{name}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
+
+
+def test_backward_full_size_sampled(orc):
+    wl = W["highres_bf16"]
+    e_in, e_ow = backward_case(orc, wl, images=[0, 3])
+    assert e_in <= TOL["bf16"] and e_ow <= TOL["bf16"], (e_in, e_ow)
+
+
+def test_backward_workspace_too_small_is_rejected():
+    wl = W["tiny_f32"].replace(dtype="bf16")
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    with pytest.raises(B.Dcn4Error) as e:
+        B.dcn4_backward(data["input"].cuda(), data["offset_weight"].cuda(),
+                        data["grad_out"].cuda(), group=wl.G,
+                        workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 3
+
+
+def test_no_device_error_left_behind():
+    torch.cuda.synchronize()
+    rc, bits = B.dcn4_last_device_error()
+    assert rc == 0 and bits == 0
