@@ -18,6 +18,7 @@ STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
           6: "DCN4_ERR_INTERNAL"}
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2}
+MATH_CODE = {"f32": 0, "mixed16": 1}
 
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
@@ -34,7 +35,7 @@ class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("N", "H", "W", "C", "G", "kh", "kw", "stride_h", "stride_w", "pad_h", "pad_w",
                  "dil_h", "dil_w")] + [("offset_scale", ctypes.c_float), ("dtype", ctypes.c_int),
-                                       ("algo", ctypes.c_int)]
+                                       ("algo", ctypes.c_int), ("math", ctypes.c_int)]
 
 
 _lib = None
@@ -72,14 +73,14 @@ def _pair(v):
 
 
 def make_desc(N, H, W, C, G, dtype, kernel_size=3, stride=1, pad=1, dilation=1,
-              offset_scale=1.0, algo="auto"):
+              offset_scale=1.0, algo="auto", math="f32"):
     kh, kw = _pair(kernel_size)
     sh, sw = _pair(stride)
     ph, pw = _pair(pad)
     dh, dw = _pair(dilation)
     code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     return Desc(N, H, W, C, G, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale), code,
-                ALGO_CODE[algo])
+                ALGO_CODE[algo], MATH_CODE[math])
 
 
 def _check(fn, rc):
@@ -113,16 +114,16 @@ def _require(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo):
+def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo, math="f32"):
     N, H, W, C = inp.shape
     return make_desc(N, H, W, C, group, inp.dtype, kernel_size, stride, pad, dilation,
-                     offset_scale, algo)
+                     offset_scale, algo, math)
 
 
 def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, dilation=1,
-                 offset_scale=1.0, algo="auto", out=None):
+                 offset_scale=1.0, algo="auto", out=None, math="f32"):
     """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3]."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)
     N, _, _, C = input.shape
     _require(input, "input", input.dtype)
@@ -170,9 +171,9 @@ def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1
 
 
 def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, stride=1, pad=1,
-                  dilation=1, offset_scale=1.0, algo="auto", out=None):
+                  dilation=1, offset_scale=1.0, algo="auto", out=None, math="f32"):
     """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G]."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)
     N, _, _, C = input.shape
     _require(input, "input", input.dtype)

@@ -36,6 +36,7 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
     if (d->dtype != DCN4_F32 && d->dtype != DCN4_BF16 && d->dtype != DCN4_F16) return false;
     if (d->algo != DCN4_ALGO_AUTO && d->algo != DCN4_ALGO_GENERIC && d->algo != DCN4_ALGO_HALO)
         return false;
+    if (d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16) return false;
     int Ho = 0, Wo = 0;
     if (!out_hw(*d, &Ho, &Wo)) return false;
     const int K = d->kh * d->kw;
@@ -65,7 +66,10 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
     const int R = msdcn ? 8 : 4;
     const int smem_max = max_smem_optin();
     const int budget_two = 110 * 1024;  // two CTAs per SM
-    const int slot = ceil_to(Gc * 27 * eb, 16) + 32;
+    // record slots: room for the 16-byte superset copy plus a word of read
+    // slack, and a stride of 16 (mod 128) bytes so that the records of
+    // consecutive pixels start in different bank quads
+    const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
     auto try_tile = [&](int TH, int TW, bool force_full, int budget, HaloPlan *p) {
         TH = TH < g.Ho ? TH : g.Ho;
         TW = TW < g.Wo ? TW : g.Wo;
@@ -163,6 +167,7 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     L.ow = ow;
     L.out = output;
     L.ms = ms;
+    L.mixed = desc->math == DCN4_MATH_MIXED16;
     L.stream = static_cast<cudaStream_t>(stream);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * elem_bytes(L.dtype);
     CUtensorMap map;

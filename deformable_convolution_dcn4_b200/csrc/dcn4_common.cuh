@@ -133,6 +133,36 @@ template <> struct VecMath<__half> {
     }
 };
 
+// acc[0..8) += w * v with v eight 16-bit values and w rounded once to the
+// same 16-bit type: a mixed-precision fma (16-bit multiplicands, exact product,
+// fp32 accumulation and rounding), per element.
+template <typename T> struct VecMathMixed;
+template <> struct VecMathMixed<float> {
+    static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {
+        VecMath<float>::fma(acc, v, w);
+    }
+};
+__device__ __forceinline__ unsigned short bf16_bits(float w) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(w));
+}
+__device__ __forceinline__ unsigned short f16_bits(float w) {
+    return __half_as_ushort(__float2half_rn(w));
+}
+#define DCN4_MIXED_FMA(TY, CONV)                                                              \
+    static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {        \
+        const unsigned short cw = CONV(w);                                                    \
+        const unsigned wd[4] = {v.x, v.y, v.z, v.w};                                          \
+        _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                       \
+            const unsigned short lo = (unsigned short)(wd[e] & 0xffffu);                      \
+            const unsigned short hi = (unsigned short)(wd[e] >> 16);                          \
+            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(acc[2 * e]) : "h"(lo), "h"(cw));   \
+            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(acc[2 * e + 1]) : "h"(hi), "h"(cw)); \
+        }                                                                                     \
+    }
+template <> struct VecMathMixed<__nv_bfloat16> { DCN4_MIXED_FMA("bf16", bf16_bits) };
+template <> struct VecMathMixed<__half> { DCN4_MIXED_FMA("f16", f16_bits) };
+#undef DCN4_MIXED_FMA
+
 // ---- shared memory / async-copy primitives --------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -164,7 +164,17 @@ template <> __device__ __forceinline__ float RecordReader16<__half>::cvt_hi(unsi
 template <> struct RecordReader<__nv_bfloat16> : RecordReader16<__nv_bfloat16> {};
 template <> struct RecordReader<__half> : RecordReader16<__half> {};
 
-template <typename T, int U, bool MS>
+// Reads tap k's (dx, dy, m) of a record in shared memory (escape path).
+template <typename T>
+__device__ __forceinline__ void record_tap(const unsigned char *rec, int k, float &dx, float &dy,
+                                           float &m) {
+    const T *p = reinterpret_cast<const T *>(rec) + 3 * k;
+    dx = Elem<T>::to_f(p[0]);
+    dy = Elem<T>::to_f(p[1]);
+    m = Elem<T>::to_f(p[2]);
+}
+
+template <typename T, int U, bool MS, bool OS1, bool MIXED>
 __global__ void __launch_bounds__(256, (U >= 8 ? 1 : 2))
 fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan pl,
                 const T *__restrict__ in, const T *__restrict__ ow, T *__restrict__ out,
@@ -251,6 +261,12 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
     const int lane = threadIdx.x & 31;
     const int npairs = pl.TH * pl.TW * pl.Gc;
     const size_t img = (size_t)g.H * g.W * g.C;
+    // the staged window in image coordinates: corners x0, x0+1 are inside iff
+    // hx_lo <= x < hx_hi (NaN fails the test and goes to the escape path)
+    const float hx_lo = (float)hx0, hx_hi = (float)(hx0 + pl.HC - 1);
+    const float hy_lo = (float)hy0, hy_hi = (float)(hy0 + pl.HR - 1);
+    const float PSf = (float)PS, RSf = (float)RS;
+    const float dwf = (float)g.dw, dhf = (float)g.dh;
     for (int f = threadIdx.x; f < npairs; f += blockDim.x) {
         const int pix = f / pl.Gc;
         const int gl = f - pix * pl.Gc;
@@ -259,11 +275,13 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
         const int ho = ho0 + ty, wo = wo0 + tx;
         const unsigned long long gp = ((unsigned long long)n * g.Ho + ho) * g.Wo + wo;
         const unsigned long long start = (gp * g.G + g0) * (unsigned long long)REC;
+        const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + (start & 15ull) + gl * REC;
         float v[27];
-        RecordReader<T>::read(slots + (size_t)pix * pl.slot_bytes + (start & 15ull) + gl * REC, v);
+        RecordReader<T>::read(rec, v);
+        float s = 1.0f;
         if (MS) {
             const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + g0 + gl]);
-            const float s = msdcn_scale(raw, ms.s0[g0 + gl], ms.smax);
+            s = msdcn_scale(raw, ms.s0[g0 + gl], ms.smax);
 #pragma unroll
             for (int k = 0; k < 9; ++k) {
                 v[3 * k] = __fmul_rn(s, v[3 * k]);
@@ -278,54 +296,80 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
 
+        const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
+        const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
+        const float bys[3] = {fby, fby + dhf, fby + 2.0f * dhf};
         const unsigned char *hbase = halo + (size_t)gl * D * EB;
-        const T *gbase = in + (size_t)n * img + (size_t)(g0 + gl) * D;
+        unsigned esc = 0;
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            const int by = ho * g.sh - g.ph + i * g.dh;
-#pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                const int k = i * 3 + j;
-                const int bx = wo * g.sw - g.pw + j * g.dw;
-                const float x = sample_coord(bx, v[3 * k], g.os);
-                const float y = sample_coord(by, v[3 * k + 1], g.os);
-                const float m = v[3 * k + 2];
-                if (!(x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H)) continue;
+        for (int k = 0; k < 9; ++k) {
+            const float x = OS1 ? __fadd_rn(bxs[k % 3], v[3 * k])
+                                : __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
+            const float y = OS1 ? __fadd_rn(bys[k / 3], v[3 * k + 1])
+                                : __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            const float m = v[3 * k + 2];
+            if (x >= hx_lo && x < hx_hi && y >= hy_lo && y < hy_hi) {
                 const float x0f = floorf(x), y0f = floorf(y);
                 const float lx = x - x0f, ly = y - y0f;
-                const float mhy = m * (1.0f - ly), mly = m * ly;
-                const float w00 = mhy * (1.0f - lx), w01 = mhy * lx;
-                const float w10 = mly * (1.0f - lx), w11 = mly * lx;
-                const int x0 = (int)x0f, y0 = (int)y0f;
-                const int ix = x0 - hx0, iy = y0 - hy0;
-                if ((unsigned)ix < (unsigned)(pl.HC - 1) && (unsigned)iy < (unsigned)(pl.HR - 1)) {
-                    const unsigned char *c00 = hbase + (size_t)(iy * pl.HC + ix) * PS;
+                const float mly = m * ly, mhy = m - mly;
+                const float w01 = mhy * lx, w00 = mhy - w01;
+                const float w11 = mly * lx, w10 = mly - w11;
+                // integer-valued floats below 2^24: the byte offset is exact
+                const int off = __float2int_rz(fmaf(y0f - hy_lo, RSf, (x0f - hx_lo) * PSf));
+                const unsigned char *c00 = hbase + off;
 #pragma unroll
-                    for (int c = 0; c < U; ++c) {
-                        const int off = ((c + r) & (U - 1)) * 16;
-                        const uint4 q00 = *reinterpret_cast<const uint4 *>(c00 + off);
-                        const uint4 q01 = *reinterpret_cast<const uint4 *>(c00 + PS + off);
-                        const uint4 q10 = *reinterpret_cast<const uint4 *>(c00 + RS + off);
-                        const uint4 q11 = *reinterpret_cast<const uint4 *>(c00 + RS + PS + off);
+                for (int c = 0; c < U; ++c) {
+                    const int o = ((c + r) & (U - 1)) * 16;
+                    const uint4 q00 = *reinterpret_cast<const uint4 *>(c00 + o);
+                    const uint4 q01 = *reinterpret_cast<const uint4 *>(c00 + PS + o);
+                    const uint4 q10 = *reinterpret_cast<const uint4 *>(c00 + RS + o);
+                    const uint4 q11 = *reinterpret_cast<const uint4 *>(c00 + RS + PS + o);
+                    if (MIXED) {
+                        VecMathMixed<T>::fma(acc[c], q00, w00);
+                        VecMathMixed<T>::fma(acc[c], q01, w01);
+                        VecMathMixed<T>::fma(acc[c], q10, w10);
+                        VecMathMixed<T>::fma(acc[c], q11, w11);
+                    } else {
                         VecMath<T>::fma(acc[c], q00, w00);
                         VecMath<T>::fma(acc[c], q01, w01);
                         VecMath<T>::fma(acc[c], q10, w10);
                         VecMath<T>::fma(acc[c], q11, w11);
                     }
-                } else {
-                    // outside the staged window: 16-byte loads from global memory
-                    const float wc[4] = {w00, w01, w10, w11};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int yy = y0 + (q >> 1), xx = x0 + (q & 1);
-                        if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
-                        const uint4 *p = reinterpret_cast<const uint4 *>(
-                            gbase + ((size_t)yy * g.W + xx) * g.C);
-#pragma unroll
-                        for (int c = 0; c < U; ++c)
-                            VecMath<T>::fma(acc[c], __ldg(p + ((c + r) & (U - 1))), wc[q]);
-                    }
                 }
+            } else {
+                esc |= 1u << k;
+            }
+        }
+        // samples outside the staged window (rare): 16-byte loads from global
+        // memory, each corner tested against the image
+        const T *gbase = in + (size_t)n * img + (size_t)(g0 + gl) * D;
+        while (esc) {
+            const int k = __ffs(esc) - 1;
+            esc &= esc - 1;
+            float dx, dy, m;
+            record_tap<T>(rec, k, dx, dy, m);
+            if (MS) {
+                dx = __fmul_rn(s, dx);
+                dy = __fmul_rn(s, dy);
+            }
+            const int i = k / 3, j = k - 3 * (k / 3);
+            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            if (!(x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H)) continue;
+            const float x0f = floorf(x), y0f = floorf(y);
+            const float lx = x - x0f, ly = y - y0f;
+            const float mly = m * ly, mhy = m - mly;
+            const float w01 = mhy * lx, w11 = mly * lx;
+            const float wc[4] = {mhy - w01, w01, mly - w11, w11};
+            const int x0 = (int)x0f, y0 = (int)y0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int yy = y0 + (q >> 1), xx = x0 + (q & 1);
+                if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
+                const uint4 *p = reinterpret_cast<const uint4 *>(gbase + ((size_t)yy * g.W + xx) * g.C);
+#pragma unroll
+                for (int c = 0; c < U; ++c)
+                    VecMath<T>::fma(acc[c], __ldg(p + ((c + r) & (U - 1))), wc[q]);
             }
         }
         uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)(g0 + gl) * D);

@@ -54,9 +54,9 @@ int grid_for(long long work, int block) {
     return (int)blocks;
 }
 
-template <typename T, int U, bool MS>
+template <typename T, int U, bool MS, bool OS1, bool MIXED>
 cudaError_t launch_halo_t(const FwdLaunch &L) {
-    auto k = fwd_halo_kernel<T, U, MS>;
+    auto k = fwd_halo_kernel<T, U, MS, OS1, MIXED>;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.plan.smem_bytes);
     if (e != cudaSuccess) return e;
     const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
@@ -67,13 +67,21 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
     return cudaGetLastError();
 }
 
+template <typename T, int U, bool MS>
+cudaError_t launch_halo_m(const FwdLaunch &L) {
+    const bool os1 = L.geo.os == 1.0f;
+    if (sizeof(T) == 2 && L.mixed)
+        return os1 ? launch_halo_t<T, U, MS, true, true>(L) : launch_halo_t<T, U, MS, false, true>(L);
+    return os1 ? launch_halo_t<T, U, MS, true, false>(L) : launch_halo_t<T, U, MS, false, false>(L);
+}
+
 template <typename T, bool MS>
 cudaError_t launch_halo_u(const FwdLaunch &L) {
     const int U = L.geo.D * (int)sizeof(T) / 16;
     switch (U) {
-        case 2: return launch_halo_t<T, 2, MS>(L);
-        case 4: return launch_halo_t<T, 4, MS>(L);
-        case 8: return launch_halo_t<T, 8, MS>(L);
+        case 2: return launch_halo_m<T, 2, MS>(L);
+        case 4: return launch_halo_m<T, 4, MS>(L);
+        case 8: return launch_halo_m<T, 8, MS>(L);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -19,6 +19,7 @@ struct FwdLaunch {
     void *out;
     const MsdcnParams *ms;  // MSDCN only
     bool halo;              // use the shared-memory halo kernel
+    bool mixed;             // 16-bit weights with mixed-precision fma (bf16/fp16)
     HaloPlan plan;
     const CUtensorMap *tmap;
     unsigned long long ow_bytes;

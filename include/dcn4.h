@@ -75,6 +75,14 @@ typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
  * DCN4_ERR_UNSUPPORTED). */
 typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
 
+/* Multiply precision of the bf16/fp16 halo forward kernels (fp32 calls and the
+ * generic kernels always use fp32). F32: bilinear weights in fp32, every
+ * product and sum in fp32. MIXED16: each weight is rounded once to the
+ * input's 16-bit type and the kernel uses the mixed-precision fma
+ * (16-bit x 16-bit exact product, fp32 accumulate); the extra error is one
+ * 16-bit rounding of each weight, the size of the inputs' own quantisation. */
+typedef enum { DCN4_MATH_F32 = 0, DCN4_MATH_MIXED16 = 1 } dcn4_math;
+
 /* The whole configuration of one call. Limits: all sizes positive, C % G == 0,
  * G <= 1024, 1 <= kh*kw <= 64, strides and dilations >= 1, pads >= 0, every
  * tensor below 2^31 elements, Ho and Wo positive. */
@@ -87,6 +95,7 @@ typedef struct {
     float offset_scale;
     dcn4_dtype dtype;
     dcn4_algo algo;
+    dcn4_math math;
 } dcn4_desc;
 
 /* Output size for `desc` (standard convolution arithmetic, as in

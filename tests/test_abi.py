@@ -79,6 +79,15 @@ def test_malformed_descriptors_rejected(lib, bad):
     assert lib.dcn4_backward_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 1
 
 
+def test_bad_enum_fields_rejected(lib):
+    for field, val in (("math", 5), ("algo", 9), ("dtype", -1)):
+        d = _desc()
+        setattr(d, field, val)
+        with pytest.raises(B.Dcn4Error) as e:
+            B.dcn4_out_shape(d)
+        assert e.value.code == 1
+
+
 def test_null_pointers_rejected_before_any_launch(lib):
     d = _desc()
     z = ctypes.c_void_p(0)
