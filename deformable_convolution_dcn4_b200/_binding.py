@@ -22,7 +22,8 @@ MATH_CODE = {"f32": 0, "mixed16": 1}
 
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
-           "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error")
+           "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
+           "dcn4_backward_noalloc")
 
 
 class Dcn4Error(RuntimeError):
@@ -61,6 +62,7 @@ def load(path=LIBRARY):
     lib.dcn4_status_string.argtypes = [st]
     lib.dcn4_status_string.restype = ctypes.c_char_p
     lib.dcn4_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.dcn4_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -167,6 +169,28 @@ def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1
     _check("dcn4_backward", load().dcn4_backward(
         ctypes.byref(desc), _ptr(input), _ptr(offset_weight), _ptr(grad_out), _ptr(grad_input),
         _ptr(grad_offset_weight), ws_ptr, ws_bytes, _stream(input)))
+    return grad_input, grad_offset_weight
+
+
+def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
+                          dilation=1, offset_scale=1.0, algo="auto", grad_input=None,
+                          grad_offset_weight=None):
+    """dcn4_backward without a caller-supplied workspace: the library's own
+    fixed scratch array is used (see include/dcn4.h for its limit)."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    ho, wo = dcn4_out_shape(desc)
+    N, H, W, C = input.shape
+    _require(input, "input", input.dtype)
+    _require(offset_weight, "offset_weight", input.dtype,
+             (N, ho, wo, group, desc.kh * desc.kw, 3))
+    _require(grad_out, "grad_out", input.dtype, (N, ho, wo, C))
+    if grad_input is None:
+        grad_input = torch.empty_like(input)
+    if grad_offset_weight is None:
+        grad_offset_weight = torch.empty_like(offset_weight)
+    _check("dcn4_backward_noalloc", load().dcn4_backward_noalloc(
+        ctypes.byref(desc), _ptr(input), _ptr(offset_weight), _ptr(grad_out), _ptr(grad_input),
+        _ptr(grad_offset_weight), _stream(input)))
     return grad_input, grad_offset_weight
 
 

@@ -144,6 +144,30 @@ DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
                           const float *s0_host, float smax, void *output,
                           void *stream);
 
+/* dcn4_backward for callers that cannot allocate device memory. The paper
+ * has no counterpart; this is a deployment convenience. dcn4_backward needs
+ * an fp32 scratch buffer for bf16/fp16 that the caller must allocate; callers
+ * that may not call cudaMalloc (host callbacks and framework hooks that forbid
+ * allocation, plugins whose framework owns all device memory, real-time code
+ * that cannot accept cudaMalloc's implicit synchronisation) use this entry
+ * point instead, which takes the scratch from a fixed 32 MiB array inside the
+ * library (held on every GPU that loads the library until the process exits)
+ * and allocates nothing.
+ *   - Limit: dcn4_backward_workspace_size(desc) must be <= 32 MiB
+ *     (N*H*W*C <= 8,388,608 for bf16/fp16); larger calls return
+ *     DCN4_ERR_WORKSPACE without launching. fp32 calls need no scratch.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array; each call zeroes the part it
+ *     uses first, but calls that overlap on the GPU (different streams, or
+ *     several host threads) race on it and give wrong results.
+ * Arguments, outputs and errors are otherwise those of dcn4_backward. */
+DCN4_API dcn4_status dcn4_backward_noalloc(const dcn4_desc *desc, const void *input,
+                                           const void *offset_weight, const void *grad_out,
+                                           void *grad_input, void *grad_offset_weight,
+                                           void *stream);
+
 /* Human-readable name of a status code (static storage). */
 DCN4_API const char *dcn4_status_string(dcn4_status status);
 
