@@ -123,6 +123,12 @@ def max_over_ranks(value, device="cpu"):
     return float(t.item())
 
 
+def weak_scaling_value(step_bytes_per_rank, step_ms_max, world):
+    """Whole-job throughput in GB/s: every rank processes its own full batch
+    (step_bytes_per_rank), the job takes the slowest rank's time."""
+    return world * step_bytes_per_rank / (step_ms_max * 1e-3) / 1e9
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -333,7 +339,7 @@ def run_ours(args):
     step_ms = max_over_ranks(step_ms_local, dev)
     ib = ideal_bytes(wl, Ho, Wo)
     step_bytes = sum(ib.values())
-    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    value = weak_scaling_value(step_bytes, step_ms, world)
     op_ms = {n: per_op[n] / args.steps for n in names}
     peak, peak_kind = hbm_peak()
     breakdown = {}
@@ -413,7 +419,7 @@ def run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, strea
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
-    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(weak_scaling_value(step_bytes, ms, world), 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps, "path": "Python binding -> C ABI, pinned host buffers, "
                                     "cudaMemcpyAsync both ways inside the timed region"}

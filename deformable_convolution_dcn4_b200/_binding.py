@@ -23,7 +23,7 @@ MATH_CODE = {"f32": 0, "mixed16": 1}
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
-           "dcn4_backward_noalloc")
+           "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait")
 
 
 class Dcn4Error(RuntimeError):
@@ -63,6 +63,7 @@ def load(path=LIBRARY):
     lib.dcn4_status_string.restype = ctypes.c_char_p
     lib.dcn4_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.dcn4_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.dcn4_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -218,6 +219,12 @@ def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, 
 
 def dcn4_status_string(code):
     return load().dcn4_status_string(int(code)).decode()
+
+
+def dcn4_selftest_bounded_wait(timeout_us=2000):
+    """Launches the kernel whose bounded wait must expire (see the header)."""
+    _check("dcn4_selftest_bounded_wait", load().dcn4_selftest_bounded_wait(
+        int(timeout_us), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
 
 
 def dcn4_last_device_error():

@@ -55,24 +55,37 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 int ceil_to(int v, int m) { return (v + m - 1) / m * m; }
 
-// Chooses the halo kernel's tiling; false when no tiling fits shared memory.
+int log2_exact(int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return (1 << l) == v ? l : -1;
+}
+
+// Smallest power of two >= v.
+int pow2_ceil(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+// Chooses the halo kernel's tiling; false when the call does not fit it.
+// The staged pixel (Gc groups x D channels) must be exactly 128 bytes, the
+// stride at which random 16-byte gathers can be kept free of bank conflicts.
 bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
+    if (128 % (g.D * eb) != 0) return false;
+    const int Gc = 128 / (g.D * eb);
+    if (g.G % Gc != 0) return false;
     const int U = g.D * eb / 16;
-    int Gc = 0;
-    for (int d = 1; d <= g.G; ++d)
-        if (g.G % d == 0 && (d * U) % 8 == 0 && d * g.D <= 256) { Gc = d; break; }
-    if (Gc == 0) Gc = 1;
-    if (Gc * g.D > 256) return false;
     const int R = msdcn ? 8 : 4;
     const int smem_max = max_smem_optin();
-    const int budget_two = 110 * 1024;  // two CTAs per SM
     // record slots: room for the 16-byte superset copy plus a word of read
     // slack, and a stride of 16 (mod 128) bytes so that the records of
     // consecutive pixels start in different bank quads
     const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
-    auto try_tile = [&](int TH, int TW, bool force_full, int budget, HaloPlan *p) {
+    auto try_tile = [&](int TH, int TW, bool force_full, int stages, HaloPlan *p) {
+        if (stages == 2 && U > 4) return false;  // 16 warps need <= 128 registers
         TH = TH < g.Ho ? TH : g.Ho;
-        TW = TW < g.Wo ? TW : g.Wo;
+        TW = TW < pow2_ceil(g.Wo) ? TW : pow2_ceil(g.Wo);
         int HR = (TH - 1) * g.sh + (g.kh - 1) * g.dh + 2 * R + 2;
         int HC = (TW - 1) * g.sw + (g.kw - 1) * g.dw + 2 * R + 2;
         int full_h = force_full || HR >= g.H + 2;
@@ -80,25 +93,78 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
         if (full_h) HR = g.H + 2;
         if (full_w) HC = g.W + 2;
         if (HR > 256 || HC > 256) return false;
-        const long long halo = (long long)HR * HC * Gc * g.D * eb;
-        const long long halo_r = (halo + 127) / 128 * 128;
-        const long long total = halo_r + (long long)TH * TW * slot + 16;
-        if (total > budget || total > smem_max) return false;
-        *p = HaloPlan{TH, TW, Gc, R, HR, HC, full_h, full_w,
-                      (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc,
-                      slot, (int)halo_r, (int)total};
+        const long long halo = (long long)HR * HC * 128;
+        HaloPlan q{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
+                   (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc,
+                   slot, (int)halo, stages, 0};
+        const long long total = (long long)stages *
+                                    ((((halo + (long long)TH * TW * slot) + 127) / 128 * 128) +
+                                     8 * (2 + 16));
+        if ((long long)TH * TW * Gc > 1024) return false;
+        if (total > smem_max) return false;
+        q.smem_bytes = (int)total;
+        *p = q;
         return true;
     };
-    static const int cands[][2] = {{16, 16}, {16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
+    static const int cands[][2] = {{16, 8}, {8, 16}, {16, 16}, {8, 8}, {8, 4}, {4, 8},
                                    {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
     if (msdcn) {
         static const int big[][2] = {{32, 32}, {16, 32}, {32, 16}, {16, 16}, {8, 16}, {16, 8}, {8, 8}};
         for (auto &c : big)
-            if (try_tile(c[0], c[1], true, smem_max, out)) return true;
+            if (try_tile(c[0], c[1], true, 1, out)) return true;
     }
-    for (int budget : {budget_two, smem_max})
+    for (int stages : {2, 1})
         for (auto &c : cands)
-            if (try_tile(c[0], c[1], false, budget, out)) return true;
+            if (try_tile(c[0], c[1], false, stages, out)) return true;
+    return false;
+}
+
+// Tiling and shared-memory layout of the backward halo kernel: one
+// (pixel, group) pair per thread (512 threads), 128-byte staged pixels,
+// R = 4, and the sorted sample records (14 bytes each) must fit in the
+// window buffer they reuse.
+bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
+    if (128 % (g.D * eb) != 0) return false;
+    const int Gc = 128 / (g.D * eb);
+    if (g.G % Gc != 0) return false;
+    const int U = g.D * eb / 16;
+    if (!(U == 4 || (U == 2 && eb == 2))) return false;
+    const int R = 4;
+    const int smem_max = max_smem_optin() - 1024;  // static shared memory of the kernel
+    const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
+    static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
+                                   {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    for (auto &c : cands) {
+        const int TH = c[0] < g.Ho ? c[0] : g.Ho;
+        const int TW = c[1] < pow2_ceil(g.Wo) ? c[1] : pow2_ceil(g.Wo);
+        if (TH * TW * Gc > 512) continue;
+        int HR = (TH - 1) * g.sh + (g.kh - 1) * g.dh + 2 * R + 2;
+        int HC = (TW - 1) * g.sw + (g.kw - 1) * g.dw + 2 * R + 2;
+        const int full_h = HR >= g.H + 2, full_w = HC >= g.W + 2;
+        if (full_h) HR = g.H + 2;
+        if (full_w) HC = g.W + 2;
+        if (HR > 256 || HC > 256 || TH > 256 || TW > 256) continue;
+        const int halo = HR * HC * 128;
+        const int max_samples = TH * TW * Gc * 9;
+        const int ncells = (HR - 1) * (HC - 1) * Gc;
+        if (14 * max_samples > halo || ncells > 65535) continue;
+        BwdLayout L;
+        L.go_off = halo;
+        L.slots_off = L.go_off + TH * TW * 128;
+        L.gows_off = L.slots_off + TH * TW * slot;
+        L.counts_off = ceil_to(L.gows_off + TH * TW * Gc * 27 * eb, 16);
+        L.bar_off = ceil_to(L.counts_off + (ncells + 1) * 4, 16);
+        L.ncells = ncells;
+        L.max_samples = max_samples;
+        L.hc_magic = (unsigned)(((1ull << 32) + HC - 1) / HC);
+        L.smem_bytes = L.bar_off + 16;
+        if (L.smem_bytes > smem_max) continue;
+        *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
+                        (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
+                        L.smem_bytes};
+        *lay = L;
+        return true;
+    }
     return false;
 }
 
@@ -114,6 +180,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
+}
+
+// TMA descriptor of a channel-last [N][rows][cols][C] tensor with a box of
+// (box_c channels, box_w columns, box_h rows, 1 image); zero fill out of bounds.
+bool encode_map(Dtype dt, const void *base, int N, int rows, int cols, int C, int box_c,
+                int box_w, int box_h, CUtensorMap *map) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int eb = elem_bytes(dt);
+    const CUtensorMapDataType t = dt == Dtype::F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : dt == Dtype::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)N};
+    cuuint64_t strides[3] = {(cuuint64_t)C * eb, (cuuint64_t)cols * C * eb,
+                             (cuuint64_t)rows * cols * C * eb};
+    cuuint32_t box[4] = {(cuuint32_t)box_c, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, t, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 // TMA descriptor of the input viewed as [N][H][W][C] with a box of
@@ -145,6 +232,7 @@ bool halo_ok(const Geometry &g, Dtype dt, bool msdcn, const void *in, const void
     if ((g.D * eb) % 16 != 0) return false;
     const int U = g.D * eb / 16;
     if (U != 2 && U != 4 && U != 8) return false;
+    if (eb == 4 && U == 2) return false;
     if (!aligned16(in) || !aligned16(ow) || !aligned16(out)) return false;
     if (!plan_halo(g, eb, msdcn, plan)) return false;
     return encode_input_map(g, dt, in, *plan, map);
@@ -214,8 +302,8 @@ dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *
     size_t need = 0;
     dcn4_backward_workspace_size(desc, &need);
     if (need > 0 && (!workspace || workspace_bytes < need)) return DCN4_ERR_WORKSPACE;
-    if (desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     BwdLaunch L;
+    memset(&L, 0, sizeof(L));
     L.geo = g;
     L.dtype = static_cast<Dtype>(desc->dtype);
     L.in = input;
@@ -225,6 +313,21 @@ dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *
     L.gow = grad_offset_weight;
     L.acc = need > 0 ? static_cast<float *>(workspace) : static_cast<float *>(grad_input);
     L.stream = static_cast<cudaStream_t>(stream);
+    const int eb = elem_bytes(L.dtype);
+    L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * eb;
+    CUtensorMap map_in, map_go;
+    memset(&map_in, 0, sizeof(map_in));
+    memset(&map_go, 0, sizeof(map_go));
+    if (desc->algo != DCN4_ALGO_GENERIC) {
+        L.halo = g.kh == 3 && g.kw == 3 && aligned16(input) && aligned16(offset_weight) &&
+                 aligned16(grad_out) && aligned16(L.acc) && plan_bwd(g, eb, &L.plan, &L.layout) &&
+                 encode_input_map(g, L.dtype, input, L.plan, &map_in) &&
+                 encode_map(L.dtype, grad_out, g.N, g.Ho, g.Wo, g.C, L.plan.Gc * g.D, L.plan.TW,
+                            L.plan.TH, &map_go);
+        if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+    }
+    L.tmap_in = &map_in;
+    L.tmap_go = &map_go;
     return cuda_status(launch_backward(L));
 }
 
@@ -252,6 +355,13 @@ const char *dcn4_status_string(dcn4_status s) {
         case DCN4_ERR_INTERNAL: return "DCN4_ERR_INTERNAL";
     }
     return "DCN4_UNKNOWN_STATUS";
+}
+
+dcn4_status dcn4_selftest_bounded_wait(unsigned int timeout_us, void *stream) {
+    if (timeout_us < 1) timeout_us = 1;
+    if (timeout_us > 2000000u) timeout_us = 2000000u;
+    return cuda_status(
+        launch_selftest_wait(1000ull * timeout_us, static_cast<cudaStream_t>(stream)));
 }
 
 dcn4_status dcn4_last_device_error(unsigned int *code) {

@@ -1,0 +1,474 @@
+// dcn4_bwd_halo.cuh -- shared-memory backward kernel of DCNv4 (3x3 taps,
+// 128-byte staged pixels). Included after dcn4_fwd.cuh (shares its tile
+// geometry, record reader and staging conventions).
+//
+// The forward is out[p0, g*D+d] = sum_k m_k sum_c w_c in[corner_c, g*D+d]
+// (DCNv4 digest "方法1. 消除冗余工作负载"; FlowDCN "2.2"). Its gradients:
+//   d/dm_k  = sum_c w_c <go, V_c>,       d/ddx_k = os m_k sum_c (dw_c/dlx) <go, V_c>,
+//   d/ddy_k = os m_k sum_c (dw_c/dly) <go, V_c>,   grad_in[corner_c] += m_k w_c go.
+// The first three are gathers (like the forward). The last is a scatter;
+// scattering with per-element shared-memory atomics would cost 16 atomic
+// lane-operations per corner, so the kernel transposes instead: it sorts the
+// CTA's samples by destination cell (one integer atomic per sample), and each
+// (staged pixel, group) then gathers the contributions of the four cells it
+// is a corner of, accumulating in registers, and adds the sum to the fp32
+// workspace with 16-byte vector reductions (neighbouring tiles' windows
+// overlap, so the workspace is shared).
+//
+// One CTA per (image, output tile, group slice); NW warps; phases:
+//   stage  TMA: input window + grad_out tile; bulk copies: records
+//   A      per (pixel, group): corner gathers, the three gradients per tap,
+//          count each staged sample into its cell (rank = atomic result)
+//   B      exclusive scan of the cell counts
+//   C      per (pixel, group): write (lx, ly, m, pair) of each staged sample
+//          at offset[cell] + rank, into the window buffer (no longer needed)
+//   D      per (staged pixel, group): gather from its four cells, flush
+//   E      copy the staged grad_offset_weight out with coalesced stores
+// Samples outside the staged window take a global path with fp32 atomics.
+#pragma once
+
+#include "dcn4_fwd.cuh"
+
+namespace dcn4 {
+
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
+// <go, v> over one 16-byte chunk of T (fp32 arithmetic).
+template <typename T> struct ChunkDot;
+template <> struct ChunkDot<float> {
+    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
+        return fmaf(go[3], __uint_as_float(v.w),
+                    fmaf(go[2], __uint_as_float(v.z),
+                         fmaf(go[1], __uint_as_float(v.y), go[0] * __uint_as_float(v.x))));
+    }
+};
+template <> struct ChunkDot<__nv_bfloat16> {
+    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            a = __ffma2_rn(make_float2(go[2 * e], go[2 * e + 1]),
+                           make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u)),
+                           a);
+        return a.x + a.y;
+    }
+};
+template <> struct ChunkDot<__half> {
+    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
+            a = __ffma2_rn(make_float2(go[2 * e], go[2 * e + 1]), f, a);
+        }
+        return a.x + a.y;
+    }
+};
+
+// Unpacks a 16-byte chunk of T into fp32.
+template <typename T> struct ChunkUnpack;
+template <> struct ChunkUnpack<float> {
+    static __device__ __forceinline__ void get(const uint4 &v, float *o) {
+        o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+        o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
+    }
+};
+template <> struct ChunkUnpack<__nv_bfloat16> {
+    static __device__ __forceinline__ void get(const uint4 &v, float *o) {
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o[2 * e] = __uint_as_float(w[e] << 16);
+            o[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    }
+};
+template <> struct ChunkUnpack<__half> {
+    static __device__ __forceinline__ void get(const uint4 &v, float *o) {
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
+            o[2 * e] = f.x;
+            o[2 * e + 1] = f.y;
+        }
+    }
+};
+
+// Block-wide exclusive scan of counts[0..n) in place; counts[n] = total.
+template <int NW>
+__device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *warp_sums) {
+    const int NT = NW * 32;
+    const int per = (n + NT - 1) / NT;
+    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    int local = 0;
+    for (int i = lo; i < hi; ++i) local += counts[i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < NW ? warp_sums[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < NW) warp_sums[lane] = wi - w;  // exclusive warp prefix
+        if (lane == NW - 1) warp_sums[NW] = wi;   // total
+    }
+    __syncthreads();
+    int run = warp_sums[warp] + incl - local;
+    for (int i = lo; i < hi; ++i) {
+        const int c = counts[i];
+        counts[i] = run;
+        run += c;
+    }
+    if (threadIdx.x == 0) counts[n] = warp_sums[NW];
+    __syncthreads();
+}
+
+template <typename T, int U, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
+bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
+                const __grid_constant__ CUtensorMap tmap_go, Geometry g, HaloPlan pl,
+                BwdLayout L, const T *__restrict__ in, const T *__restrict__ ow,
+                T *__restrict__ gow, float *__restrict__ gacc, unsigned long long ow_bytes) {
+    constexpr int EB = Elem<T>::kBytes;
+    constexpr int VE = Elem<T>::kPerVec;
+    constexpr int REC = 27 * EB;
+    constexpr int PS = 128;
+    constexpr int NT = NW * 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ int warp_sums[NW + 1];
+    unsigned char *halo = smem;
+    unsigned char *gotile = smem + L.go_off;
+    unsigned char *slots = smem + L.slots_off;
+    T *gows = reinterpret_cast<T *>(smem + L.gows_off);
+    int *counts = reinterpret_cast<int *>(smem + L.counts_off);
+    const uint32_t bar = smem_u32(smem + L.bar_off);
+    // sorted sample records, written over the window after phase A
+    float *slx = reinterpret_cast<float *>(smem);
+    float *sly = slx + L.max_samples;
+    float *sm = sly + L.max_samples;
+    unsigned short *sf = reinterpret_cast<unsigned short *>(sm + L.max_samples);
+
+    const TileCoord tc = tile_coord(blockIdx.x, g, pl);
+    const int D = g.D;
+    const int RS = pl.HC * PS;
+    const int lane = threadIdx.x & 31;
+    const size_t img = (size_t)g.H * g.W * g.C;
+
+    // ---------------- stage ----------------
+    if (threadIdx.x == 0) {
+        mbar_init(bar, NT);
+        fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i <= L.ncells; i += NT) counts[i] = 0;
+    __syncthreads();
+    {
+        uint32_t tx = 0;
+        if (threadIdx.x == 0)
+            tx = (uint32_t)pl.HR * pl.HC * PS + (uint32_t)pl.TH * pl.TW * PS;
+        const int npix = pl.TH * pl.TW;
+        for (int p = threadIdx.x; p < npix; p += NT) {
+            const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
+            if (ty >= tc.th_eff || tx_ >= tc.tw_eff) continue;
+            const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx_;
+            const unsigned long long start = (gp * g.G + tc.g0) * (unsigned long long)REC;
+            const unsigned long long end = start + (unsigned long long)pl.Gc * REC;
+            const unsigned long long a = start & ~15ull;
+            const unsigned long long e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
+            if (e > a) tx += (uint32_t)(e - a);
+            unsigned char *slot = slots + (size_t)p * pl.slot_bytes;
+            for (unsigned long long q = e; q < end; q += EB) {
+                const unsigned char *sp = reinterpret_cast<const unsigned char *>(ow) + q;
+                if (EB == 4)
+                    *reinterpret_cast<unsigned *>(slot + (q - a)) = *reinterpret_cast<const unsigned *>(sp);
+                else
+                    *reinterpret_cast<unsigned short *>(slot + (q - a)) =
+                        *reinterpret_cast<const unsigned short *>(sp);
+            }
+        }
+        mbar_arrive_expect_tx(bar, tx);
+        if (threadIdx.x == 0) {
+            tma_load_4d(smem_u32(halo), &tmap_in, tc.g0 * D, tc.hx0, tc.hy0, tc.n, bar);
+            tma_load_4d(smem_u32(gotile), &tmap_go, tc.g0 * D, tc.wo0, tc.ho0, tc.n, bar);
+        }
+        for (int p = threadIdx.x; p < npix; p += NT) {
+            const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
+            if (ty >= tc.th_eff || tx_ >= tc.tw_eff) continue;
+            const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx_;
+            const unsigned long long start = (gp * g.G + tc.g0) * (unsigned long long)REC;
+            const unsigned long long end = start + (unsigned long long)pl.Gc * REC;
+            const unsigned long long a = start & ~15ull;
+            const unsigned long long e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
+            if (e > a)
+                bulk_load(smem_u32(slots + (size_t)p * pl.slot_bytes),
+                          reinterpret_cast<const unsigned char *>(ow) + a, (uint32_t)(e - a), bar);
+        }
+    }
+    const bool ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
+    if (__syncthreads_or(!ok)) {
+        if (threadIdx.x == 0) atomicOr(&g_error_word, kErrTimeout);
+        mbar_wait_bounded(bar, 0, kWaitLimitNs);
+        return;
+    }
+
+    // ---------------- A: gradients of offsets and weights; cell counts ----------------
+    const float hx_lo = (float)tc.hx0, hx_hi = (float)(tc.hx0 + pl.HC - 1);
+    const float hy_lo = (float)tc.hy0, hy_hi = (float)(tc.hy0 + pl.HR - 1);
+    const float PSf = (float)PS, RSf = (float)RS;
+    const float dwf = (float)g.dw, dhf = (float)g.dh;
+    const int npairs = pl.TH * pl.TW * pl.Gc;
+    const int cells_w = pl.HC - 1;
+    constexpr int MAXP = 1;  // pairs per thread kept in registers (host: npairs <= NT)
+    unsigned kr[9];          // (cell << 16) | rank of each staged tap; 0xffffffff otherwise
+    float v[27];
+    int f = threadIdx.x;
+    const bool has_pair = f < npairs;
+    int pix = 0, gl = 0, ho = 0, wo = 0;
+    bool valid = false;
+    unsigned long long gp = 0;
+    unsigned start = 0;  // the record's offset within its 16-byte-aligned copy
+    if (has_pair) {
+        pix = f >> pl.lgGc;
+        gl = f & (pl.Gc - 1);
+        const int ty = pix >> pl.lgTW, tx = pix & (pl.TW - 1);
+        valid = ty < tc.th_eff && tx < tc.tw_eff;
+        ho = tc.ho0 + ty;
+        wo = tc.wo0 + tx;
+        gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
+        start = ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
+    }
+#pragma unroll
+    for (int k = 0; k < 9; ++k) kr[k] = 0xffffffffu;
+    const int r = (U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1));
+    if (valid) {
+        const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
+        RecordReader<T>::read(rec, v);
+        float go[U * VE];
+        {
+            const unsigned char *gsrc = gotile + (size_t)pix * PS + gl * D * EB;
+#pragma unroll
+            for (int c = 0; c < U; ++c)
+                ChunkUnpack<T>::get(*reinterpret_cast<const uint4 *>(gsrc + c * 16), go + c * VE);
+        }
+        const unsigned char *row0[U], *row1[U];
+#pragma unroll
+        for (int c = 0; c < U; ++c) {
+            const int cc = (c + r) & (U - 1);
+            row0[c] = halo + (size_t)gl * D * EB + cc * 16;
+            row1[c] = row0[c] + RS;
+        }
+        // gor[c] = go chunk (c + r) mod U, rotated with selects so that every
+        // register index stays static
+        float gor[U][VE];
+#pragma unroll
+        for (int c = 0; c < U; ++c)
+#pragma unroll
+            for (int e = 0; e < VE; ++e) gor[c][e] = go[c * VE + e];
+#pragma unroll
+        for (int bit = 1; bit < U; bit <<= 1) {
+            const bool sw = (r & bit) != 0;
+            float tmp[U][VE];
+#pragma unroll
+            for (int c = 0; c < U; ++c)
+#pragma unroll
+                for (int e = 0; e < VE; ++e) tmp[c][e] = sw ? gor[(c + bit) & (U - 1)][e] : gor[c][e];
+#pragma unroll
+            for (int c = 0; c < U; ++c)
+#pragma unroll
+                for (int e = 0; e < VE; ++e) gor[c][e] = tmp[c][e];
+        }
+        const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
+        const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
+        const float bys[3] = {fby, fby + dhf, fby + 2.0f * dhf};
+        T *gout_rec = gows + ((size_t)pix * pl.Gc + gl) * 27;
+        unsigned esc = 0;
+#pragma unroll
+        for (int k = 0; k < 9; ++k) {
+            const float x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
+            const float y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            const float m = v[3 * k + 2];
+            float gx = 0.f, gy = 0.f, gm = 0.f;
+            // a sample outside (-1, W) x (-1, H) has no gradient and no
+            // contribution (checked explicitly: at x == -1 exactly the window
+            // would otherwise give a one-sided d/dx from the corner x0 + 1)
+            const bool inside = x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H;
+            if (!inside) {
+                // nothing to do
+            } else if (x >= hx_lo && x < hx_hi && y >= hy_lo && y < hy_hi) {
+                const float x0f = floorf(x), y0f = floorf(y);
+                const float lx = x - x0f, ly = y - y0f;
+                const float hx = 1.0f - lx, hy = 1.0f - ly;
+                const int off = __float2int_rz(fmaf(y0f - hy_lo, RSf, (x0f - hx_lo) * PSf));
+                float d00 = 0.f, d01 = 0.f, d10 = 0.f, d11 = 0.f;
+#pragma unroll
+                for (int c = 0; c < U; ++c) {
+                    const unsigned char *a0 = row0[c] + off;
+                    const unsigned char *a1 = row1[c] + off;
+                    d00 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0));
+                    d01 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0 + PS));
+                    d10 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1));
+                    d11 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1 + PS));
+                }
+                gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
+                gx = g.os * m * (hy * (d01 - d00) + ly * (d11 - d10));
+                gy = g.os * m * (hx * (d10 - d00) + lx * (d11 - d01));
+                const int cell = (((int)(y0f - hy_lo)) * cells_w + (int)(x0f - hx_lo)) * pl.Gc + gl;
+                const int rank = atomicAdd(&counts[cell], 1);
+                kr[k] = ((unsigned)cell << 16) | (unsigned)rank;
+            } else {
+                esc |= 1u << k;
+            }
+            gout_rec[3 * k] = Elem<T>::from_f(gx);
+            gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
+            gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+        }
+        // samples outside the staged window: global gathers, fp32 atomics
+        const T *gsrc = in + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D;
+        float *gdst = gacc + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D;
+        while (esc) {
+            const int k = __ffs(esc) - 1;
+            esc &= esc - 1;
+            const int i = k / 3, j = k - 3 * (k / 3);
+            float dx, dy, m;
+            record_tap<T>(rec, k, dx, dy, m);
+            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            float gx = 0.f, gy = 0.f, gm = 0.f;
+            if (x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H) {
+                const float x0f = floorf(x), y0f = floorf(y);
+                const float lx = x - x0f, ly = y - y0f;
+                const int x0 = (int)x0f, y0 = (int)y0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int a = q >> 1, b = q & 1;
+                    const int yy = y0 + a, xx = x0 + b;
+                    if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
+                    const float wy = a ? ly : 1.0f - ly, wx = b ? lx : 1.0f - lx;
+                    const size_t at = ((size_t)yy * g.W + xx) * g.C;
+                    const uint4 *p = reinterpret_cast<const uint4 *>(gsrc + at);
+                    float dot = 0.f;
+#pragma unroll
+                    for (int c = 0; c < U; ++c) dot += ChunkDot<T>::dot(go + c * VE, __ldg(p + c));
+                    gm = fmaf(wy * wx, dot, gm);
+                    gx = fmaf(b ? wy : -wy, dot, gx);
+                    gy = fmaf(a ? wx : -wx, dot, gy);
+                    const float cw = m * wy * wx;
+#pragma unroll
+                    for (int d = 0; d < U * VE; ++d) atomicAdd(gdst + at + d, cw * go[d]);
+                }
+                gx *= g.os * m;
+                gy *= g.os * m;
+            }
+            gout_rec[3 * k] = Elem<T>::from_f(gx);
+            gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
+            gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+        }
+    }
+    __syncthreads();  // window reads, counts and gows staging complete
+
+    // ---------------- B: cell offsets ----------------
+    block_exclusive_scan<NW>(counts, L.ncells, warp_sums);
+
+    // ---------------- C: sorted sample records (over the window) ----------------
+    if (valid) {
+#pragma unroll
+        for (int k = 0; k < 9; ++k) {
+            if (kr[k] == 0xffffffffu) continue;
+            const int cell = (int)(kr[k] >> 16), rank = (int)(kr[k] & 0xffffu);
+            const int i = k / 3, j = k - 3 * (k / 3);
+            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, v[3 * k], g.os);
+            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, v[3 * k + 1], g.os);
+            const int pos = counts[cell] + rank;
+            slx[pos] = x - floorf(x);
+            sly[pos] = y - floorf(y);
+            sm[pos] = v[3 * k + 2];
+            sf[pos] = (unsigned short)f;
+        }
+    }
+    __syncthreads();
+
+    // ---------------- E: grad_offset_weight out (one warp per pixel) ----------------
+    {
+        const int npix = pl.TH * pl.TW;
+        const int span = pl.Gc * 27;  // elements per pixel
+        for (int p = threadIdx.x >> 5; p < npix; p += NW) {
+            const int ty = p >> pl.lgTW, tx = p & (pl.TW - 1);
+            if (ty >= tc.th_eff || tx >= tc.tw_eff) continue;
+            const unsigned long long q = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
+            T *dst = gow + (q * g.G + tc.g0) * 27;
+            const T *src = gows + (size_t)p * span;
+            for (int e = lane; e < span; e += 32) dst[e] = src[e];
+        }
+    }
+
+    // ---------------- D: gather per (staged pixel, group) and flush ----------------
+    const int nown = pl.HR * pl.HC * pl.Gc;
+    for (int o = threadIdx.x; o < nown; o += NT) {
+        const int ogl = o & (pl.Gc - 1);
+        const int q = o >> pl.lgGc;
+        const int qy = (int)__umulhi((unsigned)q, L.hc_magic), qx = q - qy * pl.HC;
+        const int iy = tc.hy0 + qy, ix = tc.hx0 + qx;
+        if (iy < 0 || iy >= g.H || ix < 0 || ix >= g.W) continue;
+        const int rr = (U <= 8) ? (((lane & 7) * U) >> 3) : (o & (U - 1));
+        float acc[U][VE];
+#pragma unroll
+        for (int c = 0; c < U; ++c)
+#pragma unroll
+            for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
+        bool any = false;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            const int cy = qy - a;
+            if (cy < 0 || cy >= pl.HR - 1) continue;
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int cx = qx - b;
+                if (cx < 0 || cx >= pl.HC - 1) continue;
+                const int cell = (cy * cells_w + cx) * pl.Gc + ogl;
+                const int e0 = counts[cell], e1 = counts[cell + 1];
+                for (int e = e0; e < e1; ++e) {
+                    const float lx = slx[e], ly = sly[e], m = sm[e];
+                    const int sp = sf[e] >> pl.lgGc;  // source pixel of the sample
+                    const float w = (a ? ly : 1.0f - ly) * (b ? lx : 1.0f - lx) * m;
+                    const unsigned char *gsrc = gotile + (size_t)sp * PS + ogl * D * EB;
+#pragma unroll
+                    for (int c = 0; c < U; ++c) {
+                        const int cc = (c + rr) & (U - 1);
+                        VecMath<T>::fma(acc[c], *reinterpret_cast<const uint4 *>(gsrc + cc * 16), w);
+                    }
+                    any = true;
+                }
+            }
+        }
+        if (any) {
+            float *dst = gacc + (size_t)tc.n * img + ((size_t)iy * g.W + ix) * g.C +
+                         (size_t)(tc.g0 + ogl) * D;
+#pragma unroll
+            for (int c = 0; c < U; ++c) {
+                const int cc = (c + rr) & (U - 1);
+#pragma unroll
+                for (int e = 0; e < VE; e += 4)
+                    red_add_v4(dst + cc * VE + e, acc[c][e], acc[c][e + 1], acc[c][e + 2],
+                               acc[c][e + 3]);
+            }
+        }
+    }
+}
+
+}  // namespace dcn4

@@ -33,16 +33,32 @@ struct MsdcnParams {
     float s0[kMaxGroups];
 };
 
+// Shared-memory layout of the backward halo kernel (chosen on the host);
+// all offsets in bytes from the start of dynamic shared memory.
+struct BwdLayout {
+    int go_off;       // grad_out tile, TH*TW pixels x 128 bytes
+    int slots_off;    // offset/weight records, TH*TW slots
+    int gows_off;     // grad_offset_weight staging, TH*TW*Gc*27 elements
+    int counts_off;   // ncells + 1 ints: per-cell sample counts, then offsets
+    int bar_off;      // one mbarrier
+    int ncells;       // (HR-1)*(HC-1)*Gc destination cells
+    int max_samples;  // TH*TW*Gc*9; sorted sample records reuse the window
+    unsigned hc_magic;  // ceil(2^32 / HC): q / HC == __umulhi(q, hc_magic) for q < 2^16
+    int smem_bytes;
+};
+
 // Tiling of the shared-memory halo kernels (chosen on the host).
 struct HaloPlan {
-    int TH, TW;          // output tile
-    int Gc;              // groups per CTA (a divisor of G)
+    int TH, TW;          // output tile (TW a power of two)
+    int Gc;              // groups per CTA (a power of two dividing G)
+    int lgTW, lgGc;      // log2(TW), log2(Gc)
     int R;               // offset reach covered by the halo, in pixels
     int HR, HC;          // halo rows / columns held in shared memory
     int full_h, full_w;  // 1: the halo is the whole image plus a 1-pixel zero border
     int tiles_h, tiles_w, slices;
     int slot_bytes;      // bytes per output pixel of staged offset/weight triples
     int halo_bytes;      // HR*HC*Gc*D*elem, rounded up to 128
+    int stages;          // 2: double-buffered (512 threads), 1: single (256 threads)
     int smem_bytes;      // dynamic shared memory of one CTA
 };
 
@@ -72,17 +88,15 @@ __device__ __forceinline__ float sample_coord(int base, float delta, float os) {
     return __fadd_rn((float)base, __fmul_rn(delta, os));
 }
 
-// ---- packed fp32 pair FMA (sm_100a f32x2) -----------------------------------
+// ---- fp32 accumulation of 16-byte vectors -------------------------------
+// acc[0..kPerVec) += w * (16-byte vector v of T), fp32 arithmetic, using the
+// sm_100 packed fp32 pair fma (__ffma2_rn) on channel pairs.
 __device__ __forceinline__ void ffma2(float &a0, float &a1, float x0, float x1, float w) {
-    unsigned long long acc, xv, wv;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(wv) : "f"(w));
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(xv), "l"(wv));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+    const float2 r = __ffma2_rn(make_float2(x0, x1), make_float2(w, w), make_float2(a0, a1));
+    a0 = r.x;
+    a1 = r.y;
 }
 
-// acc[0..kPerVec) += w * (16-byte vector v of T), fp32 arithmetic.
 template <typename T> struct VecMath;
 template <> struct VecMath<float> {
     static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {

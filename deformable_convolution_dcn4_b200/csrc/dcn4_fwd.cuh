@@ -110,13 +110,16 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
 // Shared-memory halo kernel (3x3 taps, D*sizeof(T) = 16*U bytes)
 // ------------------------------------------------------------------------
 
-// Shared-memory byte layout of one halo CTA.
+// Shared-memory byte layout of one halo CTA: STAGES x (window, record
+// slots), each stage a multiple of 128 bytes, then the mbarriers.
 struct HaloSmem {
-    static __host__ __device__ __forceinline__ int slots_offset(const HaloPlan &p) {
-        return p.halo_bytes;
+    static __host__ __device__ __forceinline__ int stage_bytes(const HaloPlan &p) {
+        return (p.halo_bytes + p.TH * p.TW * p.slot_bytes + 127) / 128 * 128;
     }
-    static __host__ __device__ __forceinline__ int barrier_offset(const HaloPlan &p) {
-        return p.halo_bytes + p.TH * p.TW * p.slot_bytes;
+    // + the win and empty barriers of every stage and one record barrier per
+    // warp (up to 16) and stage
+    static __host__ __device__ __forceinline__ int total_bytes(const HaloPlan &p, int stages) {
+        return stages * stage_bytes(p) + 8 * stages * (2 + 16);
     }
 };
 
@@ -174,122 +177,157 @@ __device__ __forceinline__ void record_tap(const unsigned char *rec, int k, floa
     m = Elem<T>::to_f(p[2]);
 }
 
-template <typename T, int U, bool MS, bool OS1, bool MIXED>
-__global__ void __launch_bounds__(256, (U >= 8 ? 1 : 2))
-fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan pl,
-                const T *__restrict__ in, const T *__restrict__ ow, T *__restrict__ out,
-                unsigned long long ow_bytes, const __grid_constant__ MsdcnParams ms) {
+// One output tile of the halo kernel: image n, groups [g0, g0+Gc), output
+// rows [ho0, ho0+th_eff) and columns [wo0, wo0+tw_eff); the staged window
+// starts at image row hy0, column hx0.
+struct TileCoord {
+    int n, g0, ho0, wo0, hy0, hx0, th_eff, tw_eff;
+    unsigned long long gp0;  // flat output pixel index of (n, ho0, wo0)
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int t, const Geometry &g, const HaloPlan &pl) {
+    TileCoord c;
+    const int tw = t % pl.tiles_w;
+    t /= pl.tiles_w;
+    const int th = t % pl.tiles_h;
+    t /= pl.tiles_h;
+    const int sl = t % pl.slices;
+    c.n = t / pl.slices;
+    c.ho0 = th * pl.TH;
+    c.wo0 = tw * pl.TW;
+    c.g0 = sl * pl.Gc;
+    c.hy0 = pl.full_h ? -1 : c.ho0 * g.sh - g.ph - pl.R;
+    c.hx0 = pl.full_w ? -1 : c.wo0 * g.sw - g.pw - pl.R;
+    c.th_eff = min(pl.TH, g.Ho - c.ho0);
+    c.tw_eff = min(pl.TW, g.Wo - c.wo0);
+    c.gp0 = ((unsigned long long)c.n * g.Ho + c.ho0) * g.Wo + c.wo0;
+    return c;
+}
+
+// Bulk-copies into their slots the records of the tile pixels whose pairs
+// this warp computes: with NT threads, thread t handles pairs t, t + NT, ...,
+// so warp w owns pixel blocks [(32w + k*NT)/Gc, +32/Gc) for k = 0, 1, ...
+// Completes on `bar` (arrival count 1); all 32 lanes call it, lane l copies
+// pixel l of each block it has, lane 0 arrives with the warp's byte count.
+template <typename T>
+__device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometry &g,
+                                              const HaloPlan &pl, const T *__restrict__ ow,
+                                              unsigned long long ow_bytes, unsigned char *slots,
+                                              int nt, uint32_t bar) {
+    constexpr int EB = Elem<T>::kBytes;
+    constexpr unsigned long long REC = 27ull * EB;
+    const int lane = threadIdx.x & 31;
+    const int npix = pl.TH * pl.TW;
+    const bool mine = lane < (32 >> pl.lgGc);
+    auto span = [&](int p, unsigned long long &a, unsigned long long &e,
+                    unsigned long long &end) -> bool {
+        const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
+        if (p >= npix || ty >= tc.th_eff || tx_ >= tc.tw_eff) return false;
+        const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx_;
+        const unsigned long long start = (gp * g.G + tc.g0) * REC;
+        end = start + (unsigned long long)pl.Gc * REC;
+        a = start & ~15ull;
+        e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
+        return true;
+    };
+    uint32_t tx = 0;
+    for (int base = (threadIdx.x & ~31) >> pl.lgGc; base < npix; base += nt >> pl.lgGc) {
+        const int p = base + lane;
+        unsigned long long a, e, end;
+        if (!mine || !span(p, a, e, end)) continue;
+        if (e > a) tx += (uint32_t)(e - a);
+        // the tensor's last bytes when its size is not a multiple of 16
+        unsigned char *slot = slots + (size_t)p * pl.slot_bytes;
+        for (unsigned long long q = e; q < end; q += EB) {
+            const unsigned char *sp = reinterpret_cast<const unsigned char *>(ow) + q;
+            if (EB == 4)
+                *reinterpret_cast<unsigned *>(slot + (q - a)) = *reinterpret_cast<const unsigned *>(sp);
+            else
+                *reinterpret_cast<unsigned short *>(slot + (q - a)) =
+                    *reinterpret_cast<const unsigned short *>(sp);
+        }
+    }
+    uint32_t total = tx;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    // order the warp's earlier generic reads of these slots (and the tail
+    // stores above) before the async-proxy writes and the arrive
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(bar, total);
+    __syncwarp();
+    for (int base = (threadIdx.x & ~31) >> pl.lgGc; base < npix; base += nt >> pl.lgGc) {
+        const int p = base + lane;
+        unsigned long long a, e, end;
+        if (!mine || !span(p, a, e, end) || e <= a) continue;
+        bulk_load(smem_u32(slots + (size_t)p * pl.slot_bytes),
+                  reinterpret_cast<const unsigned char *>(ow) + a, (uint32_t)(e - a), bar);
+    }
+}
+
+// TMA load of a tile's input window into `halo`, completing on `bar`
+// (arrival count 1); called by one thread.
+__device__ __forceinline__ void stage_window(const TileCoord &tc, const CUtensorMap *tmap,
+                                             const Geometry &g, const HaloPlan &pl, int eb,
+                                             unsigned char *halo, uint32_t bar) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(bar, (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb);
+    tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
+}
+
+// The gathers of one staged tile: one thread per (pixel, group).
+template <typename T, int U, bool MS, bool MIXED>
+__device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry &g,
+                                             const HaloPlan &pl, const T *__restrict__ in,
+                                             T *__restrict__ out, const MsdcnParams &ms,
+                                             const unsigned char *halo,
+                                             const unsigned char *slots, int ct, int nct) {
     constexpr int EB = Elem<T>::kBytes;
     constexpr int VE = Elem<T>::kPerVec;  // elements per 16-byte chunk
     constexpr int REC = 27 * EB;          // bytes of one (pixel, group) record
-    extern __shared__ __align__(1024) unsigned char smem[];
-    unsigned char *halo = smem;
-    unsigned char *slots = smem + HaloSmem::slots_offset(pl);
-    const uint32_t bar = smem_u32(smem + HaloSmem::barrier_offset(pl));
-
-    // ---- which tile ----
-    int b = blockIdx.x;
-    const int tw = b % pl.tiles_w;
-    b /= pl.tiles_w;
-    const int th = b % pl.tiles_h;
-    b /= pl.tiles_h;
-    const int sl = b % pl.slices;
-    const int n = b / pl.slices;
-    const int ho0 = th * pl.TH, wo0 = tw * pl.TW, g0 = sl * pl.Gc;
-    const int hy0 = pl.full_h ? -1 : ho0 * g.sh - g.ph - pl.R;
-    const int hx0 = pl.full_w ? -1 : wo0 * g.sw - g.pw - pl.R;
-    const int th_eff = min(pl.TH, g.Ho - ho0), tw_eff = min(pl.TW, g.Wo - wo0);
+    constexpr int PS = 128;               // bytes per staged pixel (Gc*D*EB, host-checked)
     const int D = g.D;
-    const int PS = pl.Gc * D * EB;  // bytes per halo pixel
-    const int RS = pl.HC * PS;      // bytes per halo row
-
-    if (threadIdx.x == 0) {
-        mbar_init(bar, blockDim.x);
-        fence_barrier_init();
-    }
-    __syncthreads();
-
-    // ---- stage: halo (thread 0) + one record slot per tile pixel ----
-    {
-        uint32_t tx_bytes = 0;
-        if (threadIdx.x == 0) tx_bytes = (uint32_t)pl.HR * pl.HC * PS;
-        const int npix = pl.TH * pl.TW;
-        for (int p = threadIdx.x; p < npix; p += blockDim.x) {
-            const int ty = p / pl.TW, tx = p - ty * pl.TW;
-            if (ty >= th_eff || tx >= tw_eff) continue;
-            const unsigned long long gp = ((unsigned long long)n * g.Ho + ho0 + ty) * g.Wo + wo0 + tx;
-            const unsigned long long start = (gp * g.G + g0) * (unsigned long long)REC;
-            const unsigned long long end = start + (unsigned long long)pl.Gc * REC;
-            const unsigned long long a = start & ~15ull;
-            const unsigned long long e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
-            if (e > a) tx_bytes += (uint32_t)(e - a);
-        }
-        mbar_arrive_expect_tx(bar, tx_bytes);
-        if (threadIdx.x == 0)
-            tma_load_4d(smem_u32(halo), &tmap, g0 * D, hx0, hy0, n, bar);
-        for (int p = threadIdx.x; p < npix; p += blockDim.x) {
-            const int ty = p / pl.TW, tx = p - ty * pl.TW;
-            if (ty >= th_eff || tx >= tw_eff) continue;
-            const unsigned long long gp = ((unsigned long long)n * g.Ho + ho0 + ty) * g.Wo + wo0 + tx;
-            const unsigned long long start = (gp * g.G + g0) * (unsigned long long)REC;
-            const unsigned long long end = start + (unsigned long long)pl.Gc * REC;
-            const unsigned long long a = start & ~15ull;
-            const unsigned long long e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
-            unsigned char *slot = slots + (size_t)p * pl.slot_bytes;
-            if (e > a)
-                bulk_load(smem_u32(slot), reinterpret_cast<const unsigned char *>(ow) + a,
-                          (uint32_t)(e - a), bar);
-            // the tensor's last bytes when its size is not a multiple of 16
-            for (unsigned long long q = e; q < end; q += EB) {
-                const unsigned char *sp = reinterpret_cast<const unsigned char *>(ow) + q;
-                if (EB == 4)
-                    *reinterpret_cast<unsigned *>(slot + (q - a)) = *reinterpret_cast<const unsigned *>(sp);
-                else
-                    *reinterpret_cast<unsigned short *>(slot + (q - a)) =
-                        *reinterpret_cast<const unsigned short *>(sp);
-            }
-        }
-    }
-    const bool ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
-    if (__syncthreads_or(!ok)) {
-        if (threadIdx.x == 0) atomicOr(&g_error_word, kErrTimeout);
-        mbar_wait_bounded(bar, 0, kWaitLimitNs);  // let copies in flight land
-        return;
-    }
-
-    // ---- one thread per (pixel, group) ----
+    const int RS = pl.HC * PS;            // bytes per staged row
     const int lane = threadIdx.x & 31;
     const int npairs = pl.TH * pl.TW * pl.Gc;
     const size_t img = (size_t)g.H * g.W * g.C;
     // the staged window in image coordinates: corners x0, x0+1 are inside iff
     // hx_lo <= x < hx_hi (NaN fails the test and goes to the escape path)
-    const float hx_lo = (float)hx0, hx_hi = (float)(hx0 + pl.HC - 1);
-    const float hy_lo = (float)hy0, hy_hi = (float)(hy0 + pl.HR - 1);
+    const float hx_lo = (float)tc.hx0, hx_hi = (float)(tc.hx0 + pl.HC - 1);
+    const float hy_lo = (float)tc.hy0, hy_hi = (float)(tc.hy0 + pl.HR - 1);
     const float PSf = (float)PS, RSf = (float)RS;
     const float dwf = (float)g.dw, dhf = (float)g.dh;
-    for (int f = threadIdx.x; f < npairs; f += blockDim.x) {
-        const int pix = f / pl.Gc;
-        const int gl = f - pix * pl.Gc;
-        const int ty = pix / pl.TW, tx = pix - ty * pl.TW;
-        if (ty >= th_eff || tx >= tw_eff) continue;
-        const int ho = ho0 + ty, wo = wo0 + tx;
-        const unsigned long long gp = ((unsigned long long)n * g.Ho + ho) * g.Wo + wo;
-        const unsigned long long start = (gp * g.G + g0) * (unsigned long long)REC;
-        const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + (start & 15ull) + gl * REC;
+    for (int f = ct; f < npairs; f += nct) {
+        const int pix = f >> pl.lgGc;
+        const int gl = f & (pl.Gc - 1);
+        const int ty = pix >> pl.lgTW, tx = pix & (pl.TW - 1);
+        if (ty >= tc.th_eff || tx >= tc.tw_eff) continue;
+        const int ho = tc.ho0 + ty, wo = tc.wo0 + tx;
+        const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
+        // the record's offset within its 16-byte-aligned copy (arithmetic mod 2^32)
+        const unsigned mis = ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
+        const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + mis + gl * REC;
         float v[27];
         RecordReader<T>::read(rec, v);
         float s = 1.0f;
         if (MS) {
-            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + g0 + gl]);
-            s = msdcn_scale(raw, ms.s0[g0 + gl], ms.smax);
+            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]);
+            s = msdcn_scale(raw, ms.s0[tc.g0 + gl], ms.smax);
 #pragma unroll
             for (int k = 0; k < 9; ++k) {
                 v[3 * k] = __fmul_rn(s, v[3 * k]);
                 v[3 * k + 1] = __fmul_rn(s, v[3 * k + 1]);
             }
         }
-        // chunk rotation: lanes of one 8-lane phase start at different chunks
+        // chunk rotation: the 8 lanes of a shared-memory phase start at
+        // different 16-byte chunks, so their loads hit 8 different bank quads
         const int r = (U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1));
+        const unsigned char *row0[U], *row1[U];
+#pragma unroll
+        for (int c = 0; c < U; ++c) {
+            row0[c] = halo + (size_t)gl * D * EB + ((c + r) & (U - 1)) * 16;
+            row1[c] = row0[c] + RS;
+        }
         float acc[U][VE];
 #pragma unroll
         for (int c = 0; c < U; ++c)
@@ -299,14 +337,11 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
         const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
         const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
         const float bys[3] = {fby, fby + dhf, fby + 2.0f * dhf};
-        const unsigned char *hbase = halo + (size_t)gl * D * EB;
         unsigned esc = 0;
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
-            const float x = OS1 ? __fadd_rn(bxs[k % 3], v[3 * k])
-                                : __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
-            const float y = OS1 ? __fadd_rn(bys[k / 3], v[3 * k + 1])
-                                : __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            const float x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
+            const float y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
             const float m = v[3 * k + 2];
             if (x >= hx_lo && x < hx_hi && y >= hy_lo && y < hy_hi) {
                 const float x0f = floorf(x), y0f = floorf(y);
@@ -316,14 +351,14 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
                 const float w11 = mly * lx, w10 = mly - w11;
                 // integer-valued floats below 2^24: the byte offset is exact
                 const int off = __float2int_rz(fmaf(y0f - hy_lo, RSf, (x0f - hx_lo) * PSf));
-                const unsigned char *c00 = hbase + off;
 #pragma unroll
                 for (int c = 0; c < U; ++c) {
-                    const int o = ((c + r) & (U - 1)) * 16;
-                    const uint4 q00 = *reinterpret_cast<const uint4 *>(c00 + o);
-                    const uint4 q01 = *reinterpret_cast<const uint4 *>(c00 + PS + o);
-                    const uint4 q10 = *reinterpret_cast<const uint4 *>(c00 + RS + o);
-                    const uint4 q11 = *reinterpret_cast<const uint4 *>(c00 + RS + PS + o);
+                    const unsigned char *a0 = row0[c] + off;
+                    const unsigned char *a1 = row1[c] + off;
+                    const uint4 q00 = *reinterpret_cast<const uint4 *>(a0);
+                    const uint4 q01 = *reinterpret_cast<const uint4 *>(a0 + PS);
+                    const uint4 q10 = *reinterpret_cast<const uint4 *>(a1);
+                    const uint4 q11 = *reinterpret_cast<const uint4 *>(a1 + PS);
                     if (MIXED) {
                         VecMathMixed<T>::fma(acc[c], q00, w00);
                         VecMathMixed<T>::fma(acc[c], q01, w01);
@@ -342,7 +377,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
         }
         // samples outside the staged window (rare): 16-byte loads from global
         // memory, each corner tested against the image
-        const T *gbase = in + (size_t)n * img + (size_t)(g0 + gl) * D;
+        const T *gbase = in + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D;
         while (esc) {
             const int k = __ffs(esc) - 1;
             esc &= esc - 1;
@@ -372,9 +407,113 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
                     VecMath<T>::fma(acc[c], __ldg(p + ((c + r) & (U - 1))), wc[q]);
             }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)(g0 + gl) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)(tc.g0 + gl) * D);
 #pragma unroll
         for (int c = 0; c < U; ++c) dst[(c + r) & (U - 1)] = VecMath<T>::pack(acc[c]);
+    }
+}
+
+// Persistent halo kernel. CTA b handles tiles b, b + gridDim.x, ...; thread
+// t of the NW warps owns (pixel, group) pairs t, t + 32NW, ... of every tile,
+// so each warp consumes the records of its own tile pixels: it bulk-copies
+// those itself and waits on its own barrier (rec[w][s]). The
+// input window is shared: warp 0 loads it (win[s]) once every warp has
+// released the buffer (empty[s], NW arrivals). With STAGES == 2 the copies of
+// the next tile are in flight while the current one is computed. Every wait
+// is bounded; on expiry the warp sets the error word, lets its own copies in
+// flight land and returns.
+template <typename T, int U, bool MS, bool MIXED, int STAGES, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
+fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan pl,
+                const T *__restrict__ in, const T *__restrict__ ow, T *__restrict__ out,
+                unsigned long long ow_bytes, const __grid_constant__ MsdcnParams ms) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int stage_bytes = HaloSmem::stage_bytes(pl);
+    const uint32_t win0 = smem_u32(smem + STAGES * stage_bytes);  // win[s]   at +8s
+    const uint32_t empty0 = win0 + 8 * STAGES;                     // empty[s] at +8s
+    const uint32_t rec0 = empty0 + 8 * STAGES;                     // rec[w][s] at +8(w*STAGES+s)
+    const int ntiles = g.N * pl.slices * pl.tiles_h * pl.tiles_w;
+    const int warp = threadIdx.x >> 5;
+    const bool leader = (threadIdx.x & 31) == 0;
+    const uint32_t myrec = rec0 + 8 * (warp * STAGES);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(win0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, NW);
+        }
+        for (int b = 0; b < NW * STAGES; ++b) mbar_init(rec0 + 8 * b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // window of the CTA's k-th tile (coordinates tc), once every warp has
+    // released its stage
+    auto window = [&](const TileCoord &tc, int k) -> bool {
+        const int s = k % STAGES, use = k / STAGES;
+        if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, kWaitLimitNs)) return false;
+        if (leader)
+            stage_window(tc, &tmap, g, pl, Elem<T>::kBytes, smem + s * stage_bytes, win0 + 8 * s);
+        return true;
+    };
+    auto records = [&](const TileCoord &tc, int k) {
+        const int s = k % STAGES;
+        stage_records<T>(tc, g, pl, ow, ow_bytes, smem + s * stage_bytes + pl.halo_bytes, NW * 32,
+                         myrec + 8 * s);
+    };
+    // on an expired wait: let this warp's copies of tiles k0..k1 land
+    auto drain = [&](int k0, int k1, bool with_window) {
+        for (int k = k0 < 0 ? 0 : k0; k <= k1; ++k) {
+            mbar_wait_bounded(myrec + 8 * (k % STAGES), (k / STAGES) & 1, kWaitLimitNs);
+            if (with_window)
+                mbar_wait_bounded(win0 + 8 * (k % STAGES), (k / STAGES) & 1, kWaitLimitNs);
+        }
+    };
+
+    TileCoord cur;
+    if ((int)blockIdx.x < ntiles) {
+        cur = tile_coord(blockIdx.x, g, pl);
+        records(cur, 0);
+        if (warp == 0) window(cur, 0);
+    }
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+        const int s = i % STAGES;
+        const int tn = t + gridDim.x;
+        TileCoord nxt;
+        if (tn < ntiles) nxt = tile_coord(tn, g, pl);
+        int issued = i;
+        if (STAGES == 2 && tn < ntiles) {
+            records(nxt, i + 1);
+            if (warp == 0 && !window(nxt, i + 1)) {
+                if (leader) atomicOr(&g_error_word, kErrTimeout);
+                drain(i, i + 1, false);
+                drain(i, i, true);
+                return;
+            }
+            issued = i + 1;
+        }
+        const bool ok = mbar_wait_bounded(win0 + 8 * s, (i / STAGES) & 1, kWaitLimitNs) &&
+                        mbar_wait_bounded(myrec + 8 * s, (i / STAGES) & 1, kWaitLimitNs);
+        if (!ok) {
+            if (leader) atomicOr(&g_error_word, kErrTimeout);
+            drain(i, issued, warp == 0);
+            return;
+        }
+        const unsigned char *buf = smem + s * stage_bytes;
+        compute_tile<T, U, MS, MIXED>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
+                                      threadIdx.x, NW * 32);
+        __syncwarp();
+        if (leader) mbar_arrive(empty0 + 8 * s);
+        if (STAGES == 1 && tn < ntiles) {
+            records(nxt, i + 1);
+            if (warp == 0 && !window(nxt, i + 1)) {
+                if (leader) atomicOr(&g_error_word, kErrTimeout);
+                drain(i + 1, i + 1, false);
+                return;
+            }
+        }
+        cur = nxt;
     }
 }
 

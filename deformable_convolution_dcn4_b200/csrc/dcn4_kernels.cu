@@ -13,6 +13,7 @@ __device__ unsigned int g_error_word = 0;
 
 #include "dcn4_bwd.cuh"
 #include "dcn4_fwd.cuh"
+#include "dcn4_bwd_halo.cuh"
 #include "dcn4_launch.h"
 
 namespace dcn4 {
@@ -31,7 +32,8 @@ int cached_attr(cudaDeviceAttr attr, int (&cache)[kMaxDevices]) {
     return cache[dev];
 }
 
-// Raises a kernel's dynamic shared memory limit once per (kernel, device).
+// Raises a kernel's dynamic shared memory limit once per (kernel, device) to
+// the device's opt-in maximum minus the kernel's static shared memory.
 cudaError_t allow_smem(const void *kernel, int bytes) {
     static std::mutex mu;
     static std::set<std::pair<const void *, int>> done;
@@ -41,7 +43,12 @@ cudaError_t allow_smem(const void *kernel, int bytes) {
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     if (done.count({kernel, dev})) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem_optin());
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, kernel);
+    if (e != cudaSuccess) return e;
+    const int limit = max_smem_optin() - (int)attr.sharedSizeBytes;
+    if (bytes > limit) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
     if (e == cudaSuccess) done.insert({kernel, dev});
     return e;
 }
@@ -54,36 +61,58 @@ int grid_for(long long work, int block) {
     return (int)blocks;
 }
 
-template <typename T, int U, bool MS, bool OS1, bool MIXED>
+template <typename T, int U, bool MS, bool MIXED, int STAGES, int NW>
 cudaError_t launch_halo_t(const FwdLaunch &L) {
-    auto k = fwd_halo_kernel<T, U, MS, OS1, MIXED>;
+    auto k = fwd_halo_kernel<T, U, MS, MIXED, STAGES, NW>;
+    constexpr int NT = NW * 32;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.plan.smem_bytes);
     if (e != cudaSuccess) return e;
-    const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
+    const long long tiles = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, NT, L.plan.smem_bytes);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    long long grid = (long long)sm_count() * occ;
+    if (grid > tiles) grid = tiles;
     static const MsdcnParams kNoMs = {};
-    k<<<(unsigned)grid, 256, L.plan.smem_bytes, L.stream>>>(
+    k<<<(unsigned)grid, NT, L.plan.smem_bytes, L.stream>>>(
         *L.tmap, L.geo, L.plan, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
         static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
     return cudaGetLastError();
 }
 
+// Stage count and warps: two stages with 16 warps when a tile has 512
+// (pixel, group) pairs, 8 warps when it has fewer; the large single-stage
+// plans (MSDCN whole-image windows, 64-channel groups) use 8.
+template <typename T, int U, bool MS, bool MIXED>
+cudaError_t launch_halo_s(const FwdLaunch &L) {
+    if constexpr (U <= 4) {
+        if (L.plan.stages == 2) {
+            if (L.plan.TH * L.plan.TW * L.plan.Gc >= 512)
+                return launch_halo_t<T, U, MS, MIXED, 2, 16>(L);
+            return launch_halo_t<T, U, MS, MIXED, 2, 8>(L);
+        }
+    }
+    return launch_halo_t<T, U, MS, MIXED, 1, 8>(L);
+}
+
 template <typename T, int U, bool MS>
 cudaError_t launch_halo_m(const FwdLaunch &L) {
-    const bool os1 = L.geo.os == 1.0f;
-    if (sizeof(T) == 2 && L.mixed)
-        return os1 ? launch_halo_t<T, U, MS, true, true>(L) : launch_halo_t<T, U, MS, false, true>(L);
-    return os1 ? launch_halo_t<T, U, MS, true, false>(L) : launch_halo_t<T, U, MS, false, false>(L);
+    if constexpr (sizeof(T) == 2) {
+        if (L.mixed) return launch_halo_s<T, U, MS, true>(L);
+    }
+    return launch_halo_s<T, U, MS, false>(L);
 }
 
 template <typename T, bool MS>
 cudaError_t launch_halo_u(const FwdLaunch &L) {
     const int U = L.geo.D * (int)sizeof(T) / 16;
-    switch (U) {
-        case 2: return launch_halo_m<T, 2, MS>(L);
-        case 4: return launch_halo_m<T, 4, MS>(L);
-        case 8: return launch_halo_m<T, 8, MS>(L);
-        default: return cudaErrorInvalidValue;
+    if constexpr (sizeof(T) == 2) {
+        if (U == 2) return launch_halo_m<T, 2, MS>(L);
     }
+    if (U == 4) return launch_halo_m<T, 4, MS>(L);
+    if (U == 8) return launch_halo_m<T, 8, MS>(L);
+    return cudaErrorInvalidValue;
 }
 
 template <typename T, bool MS>
@@ -103,17 +132,40 @@ cudaError_t launch_fwd_t(const FwdLaunch &L) {
 }
 
 template <typename T>
+cudaError_t launch_bwd_halo(const BwdLaunch &L) {
+    const int U = L.geo.D * (int)sizeof(T) / 16;
+    const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
+    auto run = [&](auto kernel) {
+        cudaError_t e = allow_smem(reinterpret_cast<const void *>(kernel), L.layout.smem_bytes);
+        if (e != cudaSuccess) return e;
+        kernel<<<(unsigned)grid, 512, L.layout.smem_bytes, L.stream>>>(
+            *L.tmap_in, *L.tmap_go, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
+            static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, L.ow_bytes);
+        return cudaGetLastError();
+    };
+    if constexpr (sizeof(T) == 2) {
+        if (U == 2) return run(bwd_halo_kernel<T, 2, 16>);
+    }
+    if (U == 4) return run(bwd_halo_kernel<T, 4, 16>);
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
 cudaError_t launch_bwd_t(const BwdLaunch &L) {
     const Geometry &g = L.geo;
     const long long nin = (long long)g.N * g.H * g.W * g.C;
     zero_f32_kernel<<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(L.acc, nin);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
-    bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
-        g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
-        static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow));
-    e = cudaGetLastError();
+    if (L.halo) {
+        e = launch_bwd_halo<T>(L);
+    } else {
+        const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
+        bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
+            g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+            static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow));
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
     if (static_cast<void *>(L.acc) != L.gin) {
         convert_f32_kernel<T><<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(
@@ -123,7 +175,28 @@ cudaError_t launch_bwd_t(const BwdLaunch &L) {
     return e;
 }
 
+// One CTA whose barrier waits for 16 bytes that never come: the bounded wait
+// expires and reports a timeout through the device error word.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) unsigned long long bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(b, 16);
+    const bool ok = mbar_wait_bounded(b, 0, limit_ns);
+    if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicOr(&g_error_word, kErrTimeout);
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream) {
+    (void)cudaGetLastError();
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
+}
 
 int sm_count() {
     static int cache[kMaxDevices] = {0};
@@ -138,6 +211,7 @@ int max_smem_optin() {
 }
 
 cudaError_t launch_forward(const FwdLaunch &L) {
+    (void)cudaGetLastError();  // a pending error of an earlier call is not ours
     switch (L.dtype) {
         case Dtype::F32: return launch_fwd_t<float>(L);
         case Dtype::BF16: return launch_fwd_t<__nv_bfloat16>(L);
@@ -147,6 +221,7 @@ cudaError_t launch_forward(const FwdLaunch &L) {
 }
 
 cudaError_t launch_backward(const BwdLaunch &L) {
+    (void)cudaGetLastError();  // a pending error of an earlier call is not ours
     switch (L.dtype) {
         case Dtype::F32: return launch_bwd_t<float>(L);
         case Dtype::BF16: return launch_bwd_t<__nv_bfloat16>(L);

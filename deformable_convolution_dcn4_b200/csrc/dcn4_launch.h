@@ -35,11 +35,20 @@ struct BwdLaunch {
     void *gin;     // element type
     void *gow;     // element type
     float *acc;    // fp32 accumulation buffer for grad_input (== gin for fp32)
+    bool halo;     // use the shared-memory halo kernel
+    HaloPlan plan;
+    BwdLayout layout;
+    const CUtensorMap *tmap_in;
+    const CUtensorMap *tmap_go;
+    unsigned long long ow_bytes;
     cudaStream_t stream;
 };
 
 cudaError_t launch_forward(const FwdLaunch &L);
 cudaError_t launch_backward(const BwdLaunch &L);
+
+// Launches the bounded-wait self-test kernel (see dcn4_selftest_bounded_wait).
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 
 // Reads and clears the device error word of the current device.
 cudaError_t read_clear_device_error(unsigned *bits);

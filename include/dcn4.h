@@ -168,6 +168,15 @@ DCN4_API dcn4_status dcn4_backward_noalloc(const dcn4_desc *desc, const void *in
                                            void *grad_input, void *grad_offset_weight,
                                            void *stream);
 
+/* Diagnostic for failure detection (no counterpart on the pages): launches one
+ * CTA whose mbarrier expects 16 bytes that no copy ever delivers, so its
+ * bounded wait gives up after `timeout_us` microseconds (clamped to
+ * 1..2,000,000) and sets the DCN4_ERR_TIMEOUT bit of the device error word,
+ * exactly as a stalled copy in the real kernels would. Nothing faults or
+ * hangs; read the result with dcn4_last_device_error after the stream has
+ * drained. */
+DCN4_API dcn4_status dcn4_selftest_bounded_wait(unsigned int timeout_us, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 DCN4_API const char *dcn4_status_string(dcn4_status status);
 

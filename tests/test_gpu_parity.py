@@ -59,9 +59,13 @@ GENERIC_ONLY = {
 
 
 def _halo_supported(wl):
+    """The halo kernel stages 128-byte pixels (Gc groups of D channels) and
+    needs 3x3 taps and 32-, 64- or 128-byte group slices (16-byte chunks)."""
     eb = 4 if wl.dtype == "f32" else 2
-    u = wl.D * eb // 16
-    return wl.kh == 3 and wl.kw == 3 and (wl.D * eb) % 16 == 0 and u in (2, 4, 8)
+    slice_bytes = wl.D * eb
+    if wl.kh != 3 or wl.kw != 3 or slice_bytes not in ((32, 64, 128) if eb == 2 else (64, 128)):
+        return False
+    return wl.G % (128 // slice_bytes) == 0
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -101,7 +105,10 @@ def _kw(wl):
 def test_forward_edge(orc, name, algo):
     wl = EDGE[name]
     if algo == "halo" and not _halo_supported(wl):
-        pytest.skip("halo kernel needs 3x3 taps and 32/64/128-byte group slices")
+        with pytest.raises(B.Dcn4Error) as e:
+            forward_case(orc, wl, algo)
+        assert e.value.code == 2
+        return
     err = forward_case(orc, wl, algo)
     assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
 
@@ -266,3 +273,16 @@ def test_no_device_error_left_behind():
     rc, bits = B.dcn4_last_device_error()
     assert rc == 0 and bits == 0
 
+
+def test_bounded_wait_expiry_is_reported_and_context_survives(orc):
+    """A barrier that nothing completes: the kernel's wait gives up after 2 ms,
+    the host reads DCN4_ERR_TIMEOUT, and the context keeps working."""
+    torch.cuda.synchronize()
+    B.dcn4_last_device_error()
+    B.dcn4_selftest_bounded_wait(2000)
+    torch.cuda.synchronize()
+    rc, bits = B.dcn4_last_device_error()
+    assert rc == 5 and bits & 1, (rc, bits)
+    assert B.dcn4_last_device_error() == (0, 0)  # read clears it
+    err = forward_case(orc, W["tiny_f32"], "halo")
+    assert err <= TOL["f32"]
