@@ -18,7 +18,7 @@ STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
           6: "DCN4_ERR_INTERNAL"}
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2}
-MATH_CODE = {"f32": 0, "mixed16": 1}
+MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2}
 
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
@@ -76,7 +76,7 @@ def _pair(v):
 
 
 def make_desc(N, H, W, C, G, dtype, kernel_size=3, stride=1, pad=1, dilation=1,
-              offset_scale=1.0, algo="auto", math="f32"):
+              offset_scale=1.0, algo="auto", math="default"):
     kh, kw = _pair(kernel_size)
     sh, sw = _pair(stride)
     ph, pw = _pair(pad)
@@ -117,14 +117,14 @@ def _require(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo, math="f32"):
+def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo, math="default"):
     N, H, W, C = inp.shape
     return make_desc(N, H, W, C, group, inp.dtype, kernel_size, stride, pad, dilation,
                      offset_scale, algo, math)
 
 
 def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, dilation=1,
-                 offset_scale=1.0, algo="auto", out=None, math="f32"):
+                 offset_scale=1.0, algo="auto", out=None, math="default"):
     """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3]."""
     desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)
@@ -149,9 +149,9 @@ def dcn4_backward_workspace_size(desc):
 
 def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
                   dilation=1, offset_scale=1.0, algo="auto", workspace=None,
-                  grad_input=None, grad_offset_weight=None):
+                  grad_input=None, grad_offset_weight=None, math="default"):
     """DCNv4 backward -> (grad_input, grad_offset_weight)."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)
     N, H, W, C = input.shape
     _require(input, "input", input.dtype)
@@ -175,10 +175,10 @@ def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1
 
 def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
                           dilation=1, offset_scale=1.0, algo="auto", grad_input=None,
-                          grad_offset_weight=None):
+                          grad_offset_weight=None, math="default"):
     """dcn4_backward without a caller-supplied workspace: the library's own
     fixed scratch array is used (see include/dcn4.h for its limit)."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)
     N, H, W, C = input.shape
     _require(input, "input", input.dtype)
@@ -196,7 +196,7 @@ def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, 
 
 
 def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, stride=1, pad=1,
-                  dilation=1, offset_scale=1.0, algo="auto", out=None, math="f32"):
+                  dilation=1, offset_scale=1.0, algo="auto", out=None, math="default"):
     """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G]."""
     desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
     ho, wo = dcn4_out_shape(desc)

@@ -36,7 +36,8 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
     if (d->dtype != DCN4_F32 && d->dtype != DCN4_BF16 && d->dtype != DCN4_F16) return false;
     if (d->algo != DCN4_ALGO_AUTO && d->algo != DCN4_ALGO_GENERIC && d->algo != DCN4_ALGO_HALO)
         return false;
-    if (d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16) return false;
+    if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16)
+        return false;
     int Ho = 0, Wo = 0;
     if (!out_hw(*d, &Ho, &Wo)) return false;
     const int K = d->kh * d->kw;
@@ -147,11 +148,13 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
         const int halo = HR * HC * 128;
         const int max_samples = TH * TW * Gc * 9;
         const int ncells = (HR - 1) * (HC - 1) * Gc;
-        if (14 * max_samples > halo || ncells > 65535) continue;
+        if (16 * max_samples > halo + TH * TW * slot || ncells > 65535) continue;
         BwdLayout L;
-        L.go_off = halo;
-        L.slots_off = L.go_off + TH * TW * 128;
-        L.gows_off = L.slots_off + TH * TW * slot;
+        // window and record slots first: both are free after phase A and
+        // together hold the sorted 16-byte sample records
+        L.slots_off = halo;
+        L.go_off = ceil_to(L.slots_off + TH * TW * slot, 128);  // TMA destination
+        L.gows_off = L.go_off + TH * TW * 128;
         L.counts_off = ceil_to(L.gows_off + TH * TW * Gc * 27 * eb, 16);
         L.bar_off = ceil_to(L.counts_off + (ncells + 1) * 4, 16);
         L.ncells = ncells;
@@ -240,6 +243,12 @@ bool halo_ok(const Geometry &g, Dtype dt, bool msdcn, const void *in, const void
 
 dcn4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DCN4_OK : DCN4_ERR_CUDA; }
 
+// Whether the 16-bit kernels round the bilinear weights to the data type.
+bool use_mixed(const dcn4_desc *d) {
+    if (d->dtype == DCN4_F32) return false;
+    return d->math == DCN4_MATH_MIXED16 || d->math == DCN4_MATH_DEFAULT;
+}
+
 dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow, void *output,
                         void *stream, const MsdcnParams *ms) {
     Geometry g;
@@ -255,7 +264,7 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     L.ow = ow;
     L.out = output;
     L.ms = ms;
-    L.mixed = desc->math == DCN4_MATH_MIXED16;
+    L.mixed = use_mixed(desc);
     L.stream = static_cast<cudaStream_t>(stream);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * elem_bytes(L.dtype);
     CUtensorMap map;
@@ -312,6 +321,7 @@ dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *
     L.gin = grad_input;
     L.gow = grad_offset_weight;
     L.acc = need > 0 ? static_cast<float *>(workspace) : static_cast<float *>(grad_input);
+    L.mixed = use_mixed(desc);
     L.stream = static_cast<cudaStream_t>(stream);
     const int eb = elem_bytes(L.dtype);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * eb;

@@ -88,6 +88,16 @@ __global__ void __launch_bounds__(256) zero_f32_kernel(float *__restrict__ p, lo
         p[i] = 0.0f;
 }
 
+// Zeroes `bytes` bytes (16-byte vector body when aligned, byte tail).
+__global__ void __launch_bounds__(256) zero_bytes_kernel(unsigned char *__restrict__ p, long long bytes) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long nv = ((reinterpret_cast<uintptr_t>(p) & 15) == 0) ? bytes / 16 : 0;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride)
+        reinterpret_cast<uint4 *>(p)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (long long i = nv * 16 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < bytes; i += stride)
+        p[i] = 0;
+}
+
 // dst[i] = T(src[i]) for n elements, rounding to nearest.
 template <typename T>
 __global__ void __launch_bounds__(256)

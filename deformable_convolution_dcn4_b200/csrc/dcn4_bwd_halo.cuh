@@ -37,38 +37,24 @@ __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, 
                  : "memory");
 }
 
-// <go, v> over one 16-byte chunk of T (fp32 arithmetic).
-template <typename T> struct ChunkDot;
-template <> struct ChunkDot<float> {
-    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
-        return fmaf(go[3], __uint_as_float(v.w),
-                    fmaf(go[2], __uint_as_float(v.z),
-                         fmaf(go[1], __uint_as_float(v.y), go[0] * __uint_as_float(v.x))));
+// Adds 8 packed 16-bit values (one 16-byte vector of T) to global memory.
+template <typename T> struct Red16;
+template <> struct Red16<__nv_bfloat16> {
+    static __device__ __forceinline__ void add(void *p, const uint4 &v) {
+        asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
+                     "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
     }
 };
-template <> struct ChunkDot<__nv_bfloat16> {
-    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
-        const unsigned w[4] = {v.x, v.y, v.z, v.w};
-        float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            a = __ffma2_rn(make_float2(go[2 * e], go[2 * e + 1]),
-                           make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u)),
-                           a);
-        return a.x + a.y;
+template <> struct Red16<__half> {
+    static __device__ __forceinline__ void add(void *p, const uint4 &v) {
+        asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
+                     "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
     }
 };
-template <> struct ChunkDot<__half> {
-    static __device__ __forceinline__ float dot(const float *go, const uint4 &v) {
-        const unsigned w[4] = {v.x, v.y, v.z, v.w};
-        float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
-            a = __ffma2_rn(make_float2(go[2 * e], go[2 * e + 1]), f, a);
-        }
-        return a.x + a.y;
-    }
+template <> struct Red16<float> {
+    static __device__ __forceinline__ void add(void *, const uint4 &) {}
 };
 
 // Unpacks a 16-byte chunk of T into fp32.
@@ -100,6 +86,36 @@ template <> struct ChunkUnpack<__half> {
         }
     }
 };
+
+// <a, b> over one 16-byte chunk where both operands are stored in T. For
+// 16-bit T this is the sm_100 mixed-precision fma (the 16x16-bit products
+// are exact, the sums are fp32), so it equals the unpack-and-fma form bit
+// for bit up to the order of the additions.
+template <typename T> struct PackedDot;
+template <> struct PackedDot<float> {
+    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {
+        float s0 = __uint_as_float(a.x) * __uint_as_float(b.x);
+        float s1 = __uint_as_float(a.y) * __uint_as_float(b.y);
+        s0 = fmaf(__uint_as_float(a.z), __uint_as_float(b.z), s0);
+        s1 = fmaf(__uint_as_float(a.w), __uint_as_float(b.w), s1);
+        return s0 + s1;
+    }
+};
+#define DCN4_PACKED_DOT(TY)                                                                    \
+    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {              \
+        const unsigned wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};             \
+        float s0 = 0.f, s1 = 0.f;                                                              \
+        _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                        \
+            const unsigned short al = (unsigned short)(wa[e] & 0xffffu), ah = (unsigned short)(wa[e] >> 16); \
+            const unsigned short bl = (unsigned short)(wb[e] & 0xffffu), bh = (unsigned short)(wb[e] >> 16); \
+            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(s0) : "h"(al), "h"(bl));           \
+            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(s1) : "h"(ah), "h"(bh));           \
+        }                                                                                      \
+        return s0 + s1;                                                                        \
+    }
+template <> struct PackedDot<__nv_bfloat16> { DCN4_PACKED_DOT("bf16") };
+template <> struct PackedDot<__half> { DCN4_PACKED_DOT("f16") };
+#undef DCN4_PACKED_DOT
 
 // Block-wide exclusive scan of counts[0..n) in place; counts[n] = total.
 template <int NW>
@@ -140,12 +156,16 @@ __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *wa
     __syncthreads();
 }
 
-template <typename T, int U, int NW>
+// DIRECT: grad_input (16-bit T) accumulates in place: each CTA's fp32 sums
+// are rounded once to T and added with packed 16-bit reductions (no fp32
+// workspace). Otherwise sums go to the fp32 workspace `gacc`.
+template <typename T, int U, int NW, bool MIXED, bool DIRECT>
 __global__ void __launch_bounds__(NW * 32, 1)
 bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const __grid_constant__ CUtensorMap tmap_go, Geometry g, HaloPlan pl,
                 BwdLayout L, const T *__restrict__ in, const T *__restrict__ ow,
-                T *__restrict__ gow, float *__restrict__ gacc, unsigned long long ow_bytes) {
+                T *__restrict__ gow, float *__restrict__ gacc, T *__restrict__ gin,
+                unsigned long long ow_bytes) {
     constexpr int EB = Elem<T>::kBytes;
     constexpr int VE = Elem<T>::kPerVec;
     constexpr int REC = 27 * EB;
@@ -159,11 +179,9 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     T *gows = reinterpret_cast<T *>(smem + L.gows_off);
     int *counts = reinterpret_cast<int *>(smem + L.counts_off);
     const uint32_t bar = smem_u32(smem + L.bar_off);
-    // sorted sample records, written over the window after phase A
-    float *slx = reinterpret_cast<float *>(smem);
-    float *sly = slx + L.max_samples;
-    float *sm = sly + L.max_samples;
-    unsigned short *sf = reinterpret_cast<unsigned short *>(sm + L.max_samples);
+    // sorted sample records (lx, ly, m, byte offset of the source grad_out
+    // vector), written over the window and record slots after phase A
+    float4 *srec = reinterpret_cast<float4 *>(smem);
 
     const TileCoord tc = tile_coord(blockIdx.x, g, pl);
     const int D = g.D;
@@ -259,12 +277,11 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     if (valid) {
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
         RecordReader<T>::read(rec, v);
-        float go[U * VE];
+        uint4 gop[U];  // this pair's grad_out, packed, chunk order
         {
             const unsigned char *gsrc = gotile + (size_t)pix * PS + gl * D * EB;
 #pragma unroll
-            for (int c = 0; c < U; ++c)
-                ChunkUnpack<T>::get(*reinterpret_cast<const uint4 *>(gsrc + c * 16), go + c * VE);
+            for (int c = 0; c < U; ++c) gop[c] = *reinterpret_cast<const uint4 *>(gsrc + c * 16);
         }
         const unsigned char *row0[U], *row1[U];
 #pragma unroll
@@ -273,25 +290,19 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             row0[c] = halo + (size_t)gl * D * EB + cc * 16;
             row1[c] = row0[c] + RS;
         }
-        // gor[c] = go chunk (c + r) mod U, rotated with selects so that every
-        // register index stays static
-        float gor[U][VE];
+        // gor[c] = grad_out chunk (c + r) mod U, rotated with selects so that
+        // every register index stays static
+        uint4 gor[U];
 #pragma unroll
-        for (int c = 0; c < U; ++c)
-#pragma unroll
-            for (int e = 0; e < VE; ++e) gor[c][e] = go[c * VE + e];
+        for (int c = 0; c < U; ++c) gor[c] = gop[c];
 #pragma unroll
         for (int bit = 1; bit < U; bit <<= 1) {
             const bool sw = (r & bit) != 0;
-            float tmp[U][VE];
+            uint4 tmp[U];
 #pragma unroll
-            for (int c = 0; c < U; ++c)
+            for (int c = 0; c < U; ++c) tmp[c] = sw ? gor[(c + bit) & (U - 1)] : gor[c];
 #pragma unroll
-                for (int e = 0; e < VE; ++e) tmp[c][e] = sw ? gor[(c + bit) & (U - 1)][e] : gor[c][e];
-#pragma unroll
-            for (int c = 0; c < U; ++c)
-#pragma unroll
-                for (int e = 0; e < VE; ++e) gor[c][e] = tmp[c][e];
+            for (int c = 0; c < U; ++c) gor[c] = tmp[c];
         }
         const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
         const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
@@ -320,10 +331,10 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 for (int c = 0; c < U; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
-                    d00 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0));
-                    d01 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0 + PS));
-                    d10 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1));
-                    d11 += ChunkDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1 + PS));
+                    d00 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0));
+                    d01 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0 + PS));
+                    d10 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1));
+                    d11 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1 + PS));
                 }
                 gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
                 gx = g.os * m * (hy * (d01 - d00) + ly * (d11 - d10));
@@ -364,13 +375,26 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                     const uint4 *p = reinterpret_cast<const uint4 *>(gsrc + at);
                     float dot = 0.f;
 #pragma unroll
-                    for (int c = 0; c < U; ++c) dot += ChunkDot<T>::dot(go + c * VE, __ldg(p + c));
+                    for (int c = 0; c < U; ++c) dot += PackedDot<T>::dot(gop[c], __ldg(p + c));
                     gm = fmaf(wy * wx, dot, gm);
                     gx = fmaf(b ? wy : -wy, dot, gx);
                     gy = fmaf(a ? wx : -wx, dot, gy);
                     const float cw = m * wy * wx;
 #pragma unroll
-                    for (int d = 0; d < U * VE; ++d) atomicAdd(gdst + at + d, cw * go[d]);
+                    for (int c = 0; c < U; ++c) {
+                        float go[VE];
+                        ChunkUnpack<T>::get(gop[c], go);
+                        if (DIRECT) {
+#pragma unroll
+                            for (int d = 0; d < VE; ++d) go[d] *= cw;
+                            Red16<T>::add(gin + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D + at +
+                                              c * VE,
+                                          VecMath<T>::pack(go));
+                        } else {
+#pragma unroll
+                            for (int d = 0; d < VE; ++d) atomicAdd(gdst + at + c * VE + d, cw * go[d]);
+                        }
+                    }
                 }
                 gx *= g.os * m;
                 gy *= g.os * m;
@@ -395,10 +419,8 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, v[3 * k], g.os);
             const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, v[3 * k + 1], g.os);
             const int pos = counts[cell] + rank;
-            slx[pos] = x - floorf(x);
-            sly[pos] = y - floorf(y);
-            sm[pos] = v[3 * k + 2];
-            sf[pos] = (unsigned short)f;
+            srec[pos] = make_float4(x - floorf(x), y - floorf(y), v[3 * k + 2],
+                                    __uint_as_float((unsigned)(pix * PS + gl * D * EB)));
         }
     }
     __syncthreads();
@@ -443,29 +465,36 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const int cell = (cy * cells_w + cx) * pl.Gc + ogl;
                 const int e0 = counts[cell], e1 = counts[cell + 1];
                 for (int e = e0; e < e1; ++e) {
-                    const float lx = slx[e], ly = sly[e], m = sm[e];
-                    const int sp = sf[e] >> pl.lgGc;  // source pixel of the sample
-                    const float w = (a ? ly : 1.0f - ly) * (b ? lx : 1.0f - lx) * m;
-                    const unsigned char *gsrc = gotile + (size_t)sp * PS + ogl * D * EB;
+                    const float4 rec4 = srec[e];
+                    const float w = (a ? rec4.y : 1.0f - rec4.y) * (b ? rec4.x : 1.0f - rec4.x) * rec4.z;
+                    const unsigned char *gsrc = gotile + __float_as_uint(rec4.w);
 #pragma unroll
                     for (int c = 0; c < U; ++c) {
                         const int cc = (c + rr) & (U - 1);
-                        VecMath<T>::fma(acc[c], *reinterpret_cast<const uint4 *>(gsrc + cc * 16), w);
+                        const uint4 q = *reinterpret_cast<const uint4 *>(gsrc + cc * 16);
+                        if (MIXED)
+                            VecMathMixed<T>::fma(acc[c], q, w);
+                        else
+                            VecMath<T>::fma(acc[c], q, w);
                     }
                     any = true;
                 }
             }
         }
         if (any) {
-            float *dst = gacc + (size_t)tc.n * img + ((size_t)iy * g.W + ix) * g.C +
-                         (size_t)(tc.g0 + ogl) * D;
+            const size_t at = (size_t)tc.n * img + ((size_t)iy * g.W + ix) * g.C +
+                              (size_t)(tc.g0 + ogl) * D;
 #pragma unroll
             for (int c = 0; c < U; ++c) {
                 const int cc = (c + rr) & (U - 1);
+                if (DIRECT) {
+                    Red16<T>::add(gin + at + cc * VE, VecMath<T>::pack(acc[c]));
+                } else {
 #pragma unroll
-                for (int e = 0; e < VE; e += 4)
-                    red_add_v4(dst + cc * VE + e, acc[c][e], acc[c][e + 1], acc[c][e + 2],
-                               acc[c][e + 3]);
+                    for (int e = 0; e < VE; e += 4)
+                        red_add_v4(gacc + at + cc * VE + e, acc[c][e], acc[c][e + 1],
+                                   acc[c][e + 2], acc[c][e + 3]);
+                }
             }
         }
     }

@@ -132,7 +132,7 @@ cudaError_t launch_fwd_t(const FwdLaunch &L) {
 }
 
 template <typename T>
-cudaError_t launch_bwd_halo(const BwdLaunch &L) {
+cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
     const int U = L.geo.D * (int)sizeof(T) / 16;
     const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
     auto run = [&](auto kernel) {
@@ -140,13 +140,18 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L) {
         if (e != cudaSuccess) return e;
         kernel<<<(unsigned)grid, 512, L.layout.smem_bytes, L.stream>>>(
             *L.tmap_in, *L.tmap_go, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
-            static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, L.ow_bytes);
+            static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, static_cast<T *>(L.gin),
+            L.ow_bytes);
         return cudaGetLastError();
     };
     if constexpr (sizeof(T) == 2) {
-        if (U == 2) return run(bwd_halo_kernel<T, 2, 16>);
+        if (U == 2) {
+            if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false>)
+                           : run(bwd_halo_kernel<T, 2, 16, false, false>);
+        }
     }
-    if (U == 4) return run(bwd_halo_kernel<T, 4, 16>);
+    if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false>);
     return cudaErrorInvalidValue;
 }
 
@@ -154,11 +159,22 @@ template <typename T>
 cudaError_t launch_bwd_t(const BwdLaunch &L) {
     const Geometry &g = L.geo;
     const long long nin = (long long)g.N * g.H * g.W * g.C;
+    // 16-bit grad_input accumulates in place when the halo kernel runs in
+    // the 16-bit weight mode; otherwise through the fp32 workspace
+    const bool direct = L.halo && L.mixed && sizeof(T) == 2;
+    cudaError_t e;
+    if (direct) {
+        zero_bytes_kernel<<<grid_for(nin * (long long)sizeof(T) / 16 + 1, 256), 256, 0, L.stream>>>(
+            static_cast<unsigned char *>(L.gin), nin * (long long)sizeof(T));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_bwd_halo<T>(L, true);
+    }
     zero_f32_kernel<<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(L.acc, nin);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.halo) {
-        e = launch_bwd_halo<T>(L);
+        e = launch_bwd_halo<T>(L, false);
     } else {
         const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
         bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(

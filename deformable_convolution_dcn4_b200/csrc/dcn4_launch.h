@@ -36,6 +36,7 @@ struct BwdLaunch {
     void *gow;     // element type
     float *acc;    // fp32 accumulation buffer for grad_input (== gin for fp32)
     bool halo;     // use the shared-memory halo kernel
+    bool mixed;    // 16-bit weights with mixed-precision fma (bf16/fp16 grad_input)
     HaloPlan plan;
     BwdLayout layout;
     const CUtensorMap *tmap_in;

@@ -75,13 +75,19 @@ typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
  * DCN4_ERR_UNSUPPORTED). */
 typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
 
-/* Multiply precision of the bf16/fp16 halo forward kernels (fp32 calls and the
- * generic kernels always use fp32). F32: bilinear weights in fp32, every
- * product and sum in fp32. MIXED16: each weight is rounded once to the
- * input's 16-bit type and the kernel uses the mixed-precision fma
- * (16-bit x 16-bit exact product, fp32 accumulate); the extra error is one
- * 16-bit rounding of each weight, the size of the inputs' own quantisation. */
-typedef enum { DCN4_MATH_F32 = 0, DCN4_MATH_MIXED16 = 1 } dcn4_math;
+/* Multiply precision of the bilinear weights in the bf16/fp16 halo kernels
+ * (fp32 calls and the generic kernels always use fp32).
+ *   F32      bilinear weights in fp32; every product and sum in fp32.
+ *   MIXED16  each weight is rounded once to the input's 16-bit type and the
+ *            sm_100 mixed-precision fma multiplies it with the 16-bit data
+ *            (exact 16x16-bit product, fp32 accumulation). The extra error is
+ *            one 16-bit rounding of each weight (relative 2^-9 for bf16,
+ *            2^-12 for fp16), the size of the data's own quantisation; sums
+ *            stay fp32.
+ *   DEFAULT  MIXED16 for bf16/fp16 data, F32 for fp32 data.
+ * Dot products of two stored tensors (the backward's <grad_out, input>) use
+ * the mixed-precision fma in every mode; there it is exact. */
+typedef enum { DCN4_MATH_DEFAULT = 0, DCN4_MATH_F32 = 1, DCN4_MATH_MIXED16 = 2 } dcn4_math;
 
 /* The whole configuration of one call. Limits: all sizes positive, C % G == 0,
  * G <= 1024, 1 <= kh*kw <= 64, strides and dilations >= 1, pads >= 0, every
@@ -110,7 +116,9 @@ DCN4_API dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input,
                          const void *offset_weight, void *output, void *stream);
 
 /* Bytes of device workspace dcn4_backward needs for `desc`: an fp32 copy of
- * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. */
+ * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. (In the default
+ * math mode the staged bf16/fp16 kernel accumulates in grad_input itself and
+ * leaves the workspace unused; the generic kernel and DCN4_MATH_F32 use it.) */
 DCN4_API dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes);
 
 /* DCNv4 backward: the derivative of the forward (the pages only say that
@@ -122,8 +130,10 @@ DCN4_API dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t 
  * At an integer sample position the derivative is that of the cell floor()
  * selects. `workspace` (>= dcn4_backward_workspace_size bytes, 16-byte
  * aligned, device memory owned by the caller) may be NULL when that size is 0.
- * grad_input accumulates in fp32 with atomic adds, so its last bits may vary
- * from run to run. */
+ * grad_input sums partial results with atomic adds, so its last bits may vary
+ * from run to run: in fp32 (the workspace) for fp32 data and DCN4_MATH_F32;
+ * in the default mode the staged bf16/fp16 kernel sums each CTA's
+ * contribution in fp32 and adds it to grad_input with one 16-bit rounding. */
 DCN4_API dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input,
                           const void *offset_weight, const void *grad_out,
                           void *grad_input, void *grad_offset_weight,

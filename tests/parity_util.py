@@ -73,11 +73,12 @@ def forward_case(orc, wl, algo="auto", images=None):
     return scaled_err(got, ref)
 
 
-def backward_case(orc, wl, algo="auto", images=None):
+def backward_case(orc, wl, algo="auto", images=None, math="default"):
     data = make_inputs(wl, out_hw(wl), with_grad=True)
     dev = "cuda"
     gin, gow = B.dcn4_backward(data["input"].to(dev), data["offset_weight"].to(dev),
-                               data["grad_out"].to(dev), group=wl.G, algo=algo, **desc_kw(wl))
+                               data["grad_out"].to(dev), group=wl.G, algo=algo, math=math,
+                               **desc_kw(wl))
     sel = slice(None) if images is None else list(images)
     n = wl.N if images is None else len(images)
     rgin, rgow = orc.backward(problem(orc, wl, n), f32(data["input"][sel]),

@@ -79,18 +79,20 @@ def test_forward_reduced(orc, name, algo):
 @pytest.mark.parametrize("name", [n for n in sorted(REDUCED) if REDUCED[n].dtype != "f32"] +
                          ["ragged_bf16", "stride2_pad0_dil2_f16", "far_offsets_bf16",
                           "offset_scale_bf16"])
-def test_forward_mixed16(orc, name):
-    """16-bit weights with the mixed-precision fma: same gate as the fp32-weight path."""
+@pytest.mark.parametrize("math", ["f32", "mixed16"])
+def test_forward_math_modes(orc, name, math):
+    """fp32 weights and 16-bit weights with the mixed-precision fma (the
+    default for 16-bit data): both meet the same gate."""
     wl = REDUCED.get(name) or EDGE[name]
     data = make_inputs(wl, out_hw(wl))
     dev = "cuda"
     if wl.kind == "msdcn":
         got = B.msdcn_forward(data["input"].to(dev), data["dir_weight"].to(dev),
                               data["scale_raw"].to(dev), data["s0"], wl.smax, group=wl.G,
-                              math="mixed16", **_kw(wl))
+                              math=math, **_kw(wl))
     else:
         got = B.dcn4_forward(data["input"].to(dev), data["offset_weight"].to(dev), group=wl.G,
-                             math="mixed16", **_kw(wl))
+                             math=math, **_kw(wl))
     err = scaled_err(f32(got), oracle_forward(orc, wl, data))
     assert err <= TOL[wl.dtype], f"{name}: {err:.3e}"
 
@@ -248,6 +250,14 @@ BWD = {
 def test_backward(orc, name):
     wl = BWD[name]
     e_in, e_ow = backward_case(orc, wl)
+    tol = TOL[wl.dtype]
+    assert e_in <= tol and e_ow <= tol, f"{name}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
+
+
+@pytest.mark.parametrize("name", ["highres_bf16_small", "ldm_f16", "internimage_bf16"])
+def test_backward_f32_weights(orc, name):
+    wl = BWD[name]
+    e_in, e_ow = backward_case(orc, wl, math="f32")
     tol = TOL[wl.dtype]
     assert e_in <= tol and e_ow <= tol, f"{name}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
 

@@ -39,8 +39,11 @@ def test_noalloc_backward_matches_backward_twice_in_a_row():
     # N*H*W*C = 4,194,304 fp32 scratch values = 16 MiB, inside the 32 MiB array
     wl = WORKLOADS["highres_bf16"].replace(N=1)
     d = make_inputs(wl, (wl.H, wl.W), with_grad=True, device="cuda")
-    desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, torch.bfloat16)
-    ref_in, ref_ow = B.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"], group=wl.G)
+    # fp32-weight mode: the mode in which the backward accumulates grad_input
+    # in the fp32 scratch (the default 16-bit mode adds into grad_input)
+    desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, torch.bfloat16, math="f32")
+    ref_in, ref_ow = B.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"], group=wl.G,
+                                     math="f32")
     torch.cuda.synchronize()
     for call in range(2):
         gin = torch.full_like(d["input"], float("nan"))
