@@ -228,19 +228,21 @@ def cpu_threads():
 
 
 def cpu_baseline(wl, budget_s=10.0):
-    """Times the oracle on a bounded sample (whole images, growing until the
-    run takes about budget_s)."""
+    """Times the oracle on a bounded sample: whole images, the count growing
+    until one run takes a sizeable part of budget_s (at most the whole batch),
+    then repeated until about budget_s of oracle time has been spent."""
     n, total_t, total_b, runs = 1, 0.0, 0.0, 0
     while True:
         dt, b = oracle_step_sample(wl, n)
         total_t, total_b, runs = total_t + dt, total_b + b, runs + 1
-        if total_t >= budget_s or n >= wl.N:
+        if total_t >= budget_s or runs >= 64:
             break
-        n = min(wl.N, max(n + 1, int(n * budget_s / max(total_t, 1e-3) * 0.5)))
+        if n < wl.N:
+            n = min(wl.N, max(n + 1, int(n * budget_s / max(dt, 1e-3) * 0.25)))
     return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": cpu_threads(),
             "kind": "oracle",
-            "sample": f"{runs} oracle runs of fwd+bwd+MSDCN fwd on up to {n} of {wl.N} images "
-                      f"of {wl.name}, {total_t:.1f} s total"}
+            "sample": f"{runs} oracle runs of fwd+bwd+MSDCN fwd, the last on {n} of {wl.N} "
+                      f"images of {wl.name}, {total_t:.1f} s of oracle time"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -298,15 +300,17 @@ def run_ours(args):
         "msdcn_forward": lambda: dcn.msdcn_forward(m["input"], m["dir_weight"], m["scale_raw"],
                                                    m["s0"], wl.smax, out=ms_out, **kw),
     }
-    launches = {"dcn4_forward": 1, "dcn4_backward": 3, "msdcn_forward": 1}
     for f in ops.values():  # first calls set kernel attributes outside any capture
         f()
     torch.cuda.synchronize()
     graphs = {}
+    launches = {}  # library kernels recorded into each op's graph
     for name, f in ops.items():
         g = torch.cuda.CUDAGraph()
+        before = dcn.dcn4_kernel_launches()
         with torch.cuda.graph(g):
             f()
+        launches[name] = dcn.dcn4_kernel_launches() - before
         graphs[name] = g
     torch.cuda.synchronize()
     names = list(ops)
@@ -369,7 +373,8 @@ def run_ours(args):
             "dtype": wl.dtype, "data": "synthetic (seeded; shapes and distributions of an "
                                        "InternImage stage)",
             "config": describe(wl, Ho, Wo), "roofline": roofline, "ops": breakdown,
-            "gpu_launches": args.steps * sum(launches.values()), "e2e": e2e,
+            "gpu_launches": args.steps * sum(launches.values()),
+            "launches_per_step": launches, "e2e": e2e,
             "clocks": clocks.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -432,7 +437,7 @@ def run_reference(args):
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
-    n_img = min(4, wl.N)
+    n_img = wl.N  # the whole batch: a fraction of a second per step on 16 host cores
     for _ in range(args.warmup):
         oracle_step_sample(wl, n_img)
     times, nbytes = [], 0.0
@@ -444,12 +449,15 @@ def run_reference(args):
     value = nbytes / step_s / 1e9
     sample = (f"fwd+bwd+MSDCN fwd of the CPU oracle on {n_img} of {wl.N} images of {wl.name} "
               f"per step")
-    sub = wl.replace(N=n_img)
+    import oracle
+    orc = oracle.default()
+    Ho, Wo = orc.out_hw(orc.problem(wl.N, wl.H, wl.W, wl.C, wl.G, wl.kh, wl.kw, wl.stride,
+                                    wl.pad, wl.dilation, wl.offset_scale))
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-            "config": describe(sub, wl.H, wl.W),
+            "config": describe(wl, Ho, Wo),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

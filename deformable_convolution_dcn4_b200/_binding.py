@@ -23,7 +23,7 @@ MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2}
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
-           "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait")
+           "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches")
 
 
 class Dcn4Error(RuntimeError):
@@ -64,6 +64,7 @@ def load(path=LIBRARY):
     lib.dcn4_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.dcn4_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.dcn4_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+    lib.dcn4_kernel_launches.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -225,6 +226,14 @@ def dcn4_selftest_bounded_wait(timeout_us=2000):
     """Launches the kernel whose bounded wait must expire (see the header)."""
     _check("dcn4_selftest_bounded_wait", load().dcn4_selftest_bounded_wait(
         int(timeout_us), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+
+
+def dcn4_kernel_launches():
+    """Kernels the library has issued in this process (graph captures count
+    once, replays not at all)."""
+    n = ctypes.c_ulonglong()
+    _check("dcn4_kernel_launches", load().dcn4_kernel_launches(ctypes.byref(n)))
+    return n.value
 
 
 def dcn4_last_device_error():

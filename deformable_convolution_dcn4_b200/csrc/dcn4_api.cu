@@ -384,4 +384,10 @@ dcn4_status dcn4_last_device_error(unsigned int *code) {
     return DCN4_OK;
 }
 
+dcn4_status dcn4_kernel_launches(unsigned long long *count) {
+    if (!count) return DCN4_ERR_INVALID_ARG;
+    *count = launches_issued();
+    return DCN4_OK;
+}
+
 }  // extern "C"

@@ -117,6 +117,43 @@ template <> struct PackedDot<__nv_bfloat16> { DCN4_PACKED_DOT("bf16") };
 template <> struct PackedDot<__half> { DCN4_PACKED_DOT("f16") };
 #undef DCN4_PACKED_DOT
 
+// <a, b> where a is one 16-byte chunk of T and b the same channels already
+// unpacked to fp32 (grad_out, unpacked once per pair). For 16-bit T every
+// product is exact in fp32 (8- or 11-bit significands), so this equals
+// PackedDot bit for bit: even channels sum in .x, odd ones in .y.
+template <typename T> struct DotF;
+template <> struct DotF<float> {
+    static __device__ __forceinline__ float dot(const uint4 &a, const float *b) {
+        float s0 = __uint_as_float(a.x) * b[0];
+        float s1 = __uint_as_float(a.y) * b[1];
+        s0 = fmaf(__uint_as_float(a.z), b[2], s0);
+        s1 = fmaf(__uint_as_float(a.w), b[3], s1);
+        return s0 + s1;
+    }
+};
+template <> struct DotF<__nv_bfloat16> {
+    static __device__ __forceinline__ float dot(const uint4 &a, const float *b) {
+        const unsigned w[4] = {a.x, a.y, a.z, a.w};
+        float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            s = __ffma2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u)),
+                           make_float2(b[2 * e], b[2 * e + 1]), s);
+        return s.x + s.y;
+    }
+};
+template <> struct DotF<__half> {
+    static __device__ __forceinline__ float dot(const uint4 &a, const float *b) {
+        const unsigned w[4] = {a.x, a.y, a.z, a.w};
+        float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            s = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&w[e])),
+                           make_float2(b[2 * e], b[2 * e + 1]), s);
+        return s.x + s.y;
+    }
+};
+
 // Block-wide exclusive scan of counts[0..n) in place; counts[n] = total.
 template <int NW>
 __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *warp_sums) {
@@ -252,7 +289,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     const float dwf = (float)g.dw, dhf = (float)g.dh;
     const int npairs = pl.TH * pl.TW * pl.Gc;
     const int cells_w = pl.HC - 1;
-    constexpr int MAXP = 1;  // pairs per thread kept in registers (host: npairs <= NT)
+    const int ncpg = (pl.HR - 1) * cells_w;  // cells per group; cell = gl * ncpg + y * cells_w + x
     unsigned kr[9];          // (cell << 16) | rank of each staged tap; 0xffffffff otherwise
     float v[27];
     int f = threadIdx.x;
@@ -277,32 +314,17 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     if (valid) {
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
         RecordReader<T>::read(rec, v);
-        uint4 gop[U];  // this pair's grad_out, packed, chunk order
-        {
-            const unsigned char *gsrc = gotile + (size_t)pix * PS + gl * D * EB;
-#pragma unroll
-            for (int c = 0; c < U; ++c) gop[c] = *reinterpret_cast<const uint4 *>(gsrc + c * 16);
-        }
         const unsigned char *row0[U], *row1[U];
+        // gof[c]: this pair's grad_out chunk (c + r) mod U, unpacked to fp32
+        float gof[U][VE];
 #pragma unroll
         for (int c = 0; c < U; ++c) {
             const int cc = (c + r) & (U - 1);
             row0[c] = halo + (size_t)gl * D * EB + cc * 16;
             row1[c] = row0[c] + RS;
-        }
-        // gor[c] = grad_out chunk (c + r) mod U, rotated with selects so that
-        // every register index stays static
-        uint4 gor[U];
-#pragma unroll
-        for (int c = 0; c < U; ++c) gor[c] = gop[c];
-#pragma unroll
-        for (int bit = 1; bit < U; bit <<= 1) {
-            const bool sw = (r & bit) != 0;
-            uint4 tmp[U];
-#pragma unroll
-            for (int c = 0; c < U; ++c) tmp[c] = sw ? gor[(c + bit) & (U - 1)] : gor[c];
-#pragma unroll
-            for (int c = 0; c < U; ++c) gor[c] = tmp[c];
+            ChunkUnpack<T>::get(
+                *reinterpret_cast<const uint4 *>(gotile + (size_t)pix * PS + gl * D * EB + cc * 16),
+                gof[c]);
         }
         const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
         const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
@@ -331,15 +353,15 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 for (int c = 0; c < U; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
-                    d00 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0));
-                    d01 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a0 + PS));
-                    d10 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1));
-                    d11 += PackedDot<T>::dot(gor[c], *reinterpret_cast<const uint4 *>(a1 + PS));
+                    d00 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a0), gof[c]);
+                    d01 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a0 + PS), gof[c]);
+                    d10 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a1), gof[c]);
+                    d11 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a1 + PS), gof[c]);
                 }
                 gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
                 gx = g.os * m * (hy * (d01 - d00) + ly * (d11 - d10));
                 gy = g.os * m * (hx * (d10 - d00) + lx * (d11 - d01));
-                const int cell = (((int)(y0f - hy_lo)) * cells_w + (int)(x0f - hx_lo)) * pl.Gc + gl;
+                const int cell = gl * ncpg + ((int)(y0f - hy_lo)) * cells_w + (int)(x0f - hx_lo);
                 const int rank = atomicAdd(&counts[cell], 1);
                 kr[k] = ((unsigned)cell << 16) | (unsigned)rank;
             } else {
@@ -375,24 +397,24 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                     const uint4 *p = reinterpret_cast<const uint4 *>(gsrc + at);
                     float dot = 0.f;
 #pragma unroll
-                    for (int c = 0; c < U; ++c) dot += PackedDot<T>::dot(gop[c], __ldg(p + c));
+                    for (int c = 0; c < U; ++c) dot += DotF<T>::dot(__ldg(p + ((c + r) & (U - 1))), gof[c]);
                     gm = fmaf(wy * wx, dot, gm);
                     gx = fmaf(b ? wy : -wy, dot, gx);
                     gy = fmaf(a ? wx : -wx, dot, gy);
                     const float cw = m * wy * wx;
 #pragma unroll
                     for (int c = 0; c < U; ++c) {
+                        const int cc = (c + r) & (U - 1);
                         float go[VE];
-                        ChunkUnpack<T>::get(gop[c], go);
-                        if (DIRECT) {
 #pragma unroll
-                            for (int d = 0; d < VE; ++d) go[d] *= cw;
+                        for (int d = 0; d < VE; ++d) go[d] = cw * gof[c][d];
+                        if (DIRECT) {
                             Red16<T>::add(gin + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D + at +
-                                              c * VE,
+                                              cc * VE,
                                           VecMath<T>::pack(go));
                         } else {
 #pragma unroll
-                            for (int d = 0; d < VE; ++d) atomicAdd(gdst + at + c * VE + d, cw * go[d]);
+                            for (int d = 0; d < VE; ++d) atomicAdd(gdst + at + cc * VE + d, go[d]);
                         }
                     }
                 }
@@ -453,31 +475,33 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         for (int c = 0; c < U; ++c)
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
+        // cells are numbered group-major, so for each corner row a the two
+        // cells (cy, qx - 1) (corner b = 1) and (cy, qx) (b = 0) are adjacent
+        // and their entries form one contiguous range split at es
         bool any = false;
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
             const int cy = qy - a;
             if (cy < 0 || cy >= pl.HR - 1) continue;
+            const int row = ogl * ncpg + cy * cells_w;
+            const int e0 = counts[row + max(qx - 1, 0)];
+            const int es = counts[row + min(qx, cells_w)];
+            const int e1 = counts[row + min(qx, cells_w - 1) + 1];
+            any |= e1 > e0;
+            for (int e = e0; e < e1; ++e) {
+                const float4 rec4 = srec[e];
+                const float wy = a ? rec4.y : 1.0f - rec4.y;
+                const float wx = e < es ? rec4.x : 1.0f - rec4.x;
+                const float w = wy * wx * rec4.z;
+                const unsigned char *gsrc = gotile + __float_as_uint(rec4.w);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int cx = qx - b;
-                if (cx < 0 || cx >= pl.HC - 1) continue;
-                const int cell = (cy * cells_w + cx) * pl.Gc + ogl;
-                const int e0 = counts[cell], e1 = counts[cell + 1];
-                for (int e = e0; e < e1; ++e) {
-                    const float4 rec4 = srec[e];
-                    const float w = (a ? rec4.y : 1.0f - rec4.y) * (b ? rec4.x : 1.0f - rec4.x) * rec4.z;
-                    const unsigned char *gsrc = gotile + __float_as_uint(rec4.w);
-#pragma unroll
-                    for (int c = 0; c < U; ++c) {
-                        const int cc = (c + rr) & (U - 1);
-                        const uint4 q = *reinterpret_cast<const uint4 *>(gsrc + cc * 16);
-                        if (MIXED)
-                            VecMathMixed<T>::fma(acc[c], q, w);
-                        else
-                            VecMath<T>::fma(acc[c], q, w);
-                    }
-                    any = true;
+                for (int c = 0; c < U; ++c) {
+                    const int cc = (c + rr) & (U - 1);
+                    const uint4 q = *reinterpret_cast<const uint4 *>(gsrc + cc * 16);
+                    if (MIXED)
+                        VecMathMixed<T>::fma(acc[c], q, w);
+                    else
+                        VecMath<T>::fma(acc[c], q, w);
                 }
             }
         }

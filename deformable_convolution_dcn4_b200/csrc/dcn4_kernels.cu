@@ -1,5 +1,6 @@
 // dcn4_kernels.cu -- the one translation unit holding every device function of
 // libdcn4: kernel instantiations, their launchers and the device error word.
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -9,6 +10,7 @@
 namespace dcn4 {
 // Set by kernels whose bounded waits expire; read by dcn4_last_device_error.
 __device__ unsigned int g_error_word = 0;
+
 }  // namespace dcn4
 
 #include "dcn4_bwd.cuh"
@@ -21,6 +23,10 @@ namespace dcn4 {
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// Kernels this library has issued (launched or captured into a graph).
+std::atomic<unsigned long long> g_launches{0};
+inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int cached_attr(cudaDeviceAttr attr, int (&cache)[kMaxDevices]) {
     int dev = 0;
@@ -78,6 +84,7 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
     k<<<(unsigned)grid, NT, L.plan.smem_bytes, L.stream>>>(
         *L.tmap, L.geo, L.plan, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
         static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -122,6 +129,7 @@ cudaError_t launch_generic_t(const FwdLaunch &L) {
     fwd_generic_kernel<T, MS><<<grid_for(work, 256), 256, 0, L.stream>>>(
         L.geo, static_cast<const T *>(L.in), static_cast<const T *>(L.ow), static_cast<T *>(L.out),
         L.ms ? *L.ms : kNoMs);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -142,6 +150,7 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
             *L.tmap_in, *L.tmap_go, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
             static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, static_cast<T *>(L.gin),
             L.ow_bytes);
+        count_launch();
         return cudaGetLastError();
     };
     if constexpr (sizeof(T) == 2) {
@@ -166,11 +175,13 @@ cudaError_t launch_bwd_t(const BwdLaunch &L) {
     if (direct) {
         zero_bytes_kernel<<<grid_for(nin * (long long)sizeof(T) / 16 + 1, 256), 256, 0, L.stream>>>(
             static_cast<unsigned char *>(L.gin), nin * (long long)sizeof(T));
+        count_launch();
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         return launch_bwd_halo<T>(L, true);
     }
     zero_f32_kernel<<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(L.acc, nin);
+    count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (L.halo) {
@@ -180,12 +191,14 @@ cudaError_t launch_bwd_t(const BwdLaunch &L) {
         bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
             g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
             static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow));
+        count_launch();
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
     if (static_cast<void *>(L.acc) != L.gin) {
         convert_f32_kernel<T><<<grid_for(nin / 4 + 1, 256), 256, 0, L.stream>>>(
             L.acc, static_cast<T *>(L.gin), nin);
+        count_launch();
         e = cudaGetLastError();
     }
     return e;
@@ -211,6 +224,7 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream) {
     (void)cudaGetLastError();
     selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -257,5 +271,7 @@ cudaError_t read_clear_device_error(unsigned *bits) {
     *bits = v;
     return e;
 }
+
+unsigned long long launches_issued() { return g_launches.load(std::memory_order_relaxed); }
 
 }  // namespace dcn4

@@ -54,6 +54,9 @@ cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t strea
 // Reads and clears the device error word of the current device.
 cudaError_t read_clear_device_error(unsigned *bits);
 
+// Kernels issued by this library so far (launched, or captured into a graph).
+unsigned long long launches_issued();
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 // Largest opt-in dynamic shared memory per block of the current device.

@@ -197,6 +197,15 @@ DCN4_API const char *dcn4_status_string(dcn4_status status);
  * otherwise the status the bits map to. */
 DCN4_API dcn4_status dcn4_last_device_error(unsigned int *code);
 
+/* Number of kernels this library has issued in this process, summed over
+ * devices and threads: every kernel launch, including launches recorded into
+ * a CUDA graph under stream capture (a graph replays them without passing
+ * through the library, so a caller counts replays itself). The pages define
+ * no such call; it lets a benchmark state how many of the library's kernels
+ * ran. *count receives the value. Never fails except on a null pointer
+ * (DCN4_ERR_INVALID_ARG). */
+DCN4_API dcn4_status dcn4_kernel_launches(unsigned long long *count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -120,3 +120,10 @@ def test_binding_refuses_cpu_tensors(lib):
     ow = torch.zeros(1, 8, 8, 4, 9, 3)
     with pytest.raises(ValueError):
         B.dcn4_forward(x, ow, group=4)
+
+
+def test_launch_counter_without_gpu(lib):
+    """No kernel has run in this process: the counter reads zero, and a null
+    pointer is rejected."""
+    assert B.dcn4_kernel_launches() == 0
+    assert lib.dcn4_kernel_launches(None) == 1

@@ -296,3 +296,21 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(orc):
     assert B.dcn4_last_device_error() == (0, 0)  # read clears it
     err = forward_case(orc, W["tiny_f32"], "halo")
     assert err <= TOL["f32"]
+
+
+def test_launch_counter_counts_each_kernel():
+    """Forward on the halo path is one kernel; the 16-bit backward in the
+    default math mode is two (zero grad_input, halo kernel); with fp32
+    accumulation it is three (zero workspace, halo kernel, convert)."""
+    wl = REDUCED["internimage_bf16"]
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    x, ow, go = (data[k].cuda() for k in ("input", "offset_weight", "grad_out"))
+    n0 = B.dcn4_kernel_launches()
+    B.dcn4_forward(x, ow, group=wl.G, algo="halo")
+    n1 = B.dcn4_kernel_launches()
+    B.dcn4_backward(x, ow, go, group=wl.G, algo="halo")
+    n2 = B.dcn4_kernel_launches()
+    B.dcn4_backward(x, ow, go, group=wl.G, algo="halo", math="f32")
+    n3 = B.dcn4_kernel_launches()
+    torch.cuda.synchronize()
+    assert (n1 - n0, n2 - n1, n3 - n2) == (1, 2, 3)
