@@ -39,6 +39,9 @@ class Oracle:
         lib.orc_dcn4_backward.restype = ctypes.c_int
         lib.orc_msdcn_forward.argtypes = [P, _F32P, _F32P, _F32P, _F32P, ctypes.c_float, _F64P]
         lib.orc_msdcn_forward.restype = ctypes.c_int
+        lib.orc_msdcn_backward.argtypes = [P, _F32P, _F32P, _F32P, _F32P, ctypes.c_float, _F32P,
+                                           _F64P, _F64P, _F64P]
+        lib.orc_msdcn_backward.restype = ctypes.c_int
         lib.orc_msdcn_scale.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
         lib.orc_msdcn_scale.restype = ctypes.c_float
         for name in ("orc_flops",):
@@ -94,6 +97,18 @@ class Oracle:
         if rc:
             raise ValueError("orc_msdcn_forward failed")
         return out
+
+    def msdcn_backward(self, prob, inp, dir_weight, scale_raw, s0, smax, grad_out):
+        ho, wo = self.out_hw(prob)
+        gin = np.empty((prob.N, prob.H, prob.W, prob.C), np.float64)
+        gdw = np.empty((prob.N, ho, wo, prob.G, prob.kh * prob.kw, 3), np.float64)
+        graw = np.empty((prob.N, ho, wo, prob.G), np.float64)
+        rc = self.lib.orc_msdcn_backward(ctypes.byref(prob), self._f32(inp), self._f32(dir_weight),
+                                         self._f32(scale_raw), self._f32(s0), float(smax),
+                                         self._f32(grad_out), gin, gdw, graw)
+        if rc:
+            raise ValueError("orc_msdcn_backward failed")
+        return gin, gdw, graw
 
     def msdcn_scale(self, raw, s0, smax):
         return self.lib.orc_msdcn_scale(float(raw), float(s0), float(smax))

@@ -1,7 +1,7 @@
 /*
  * dcn4_oracle.c -- plain, slow CPU restatement of DCNv4 deformable spatial
  * aggregation, its backward pass and the FlowDCN groupwise multi-scale
- * (MSDCN) variant.
+ * (MSDCN) variant with its backward pass.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
  * calls this file; only the test suite, the package smoke check and the
@@ -43,6 +43,9 @@
  *    softplus(r) = max(r, 0) + log1p(exp(-|r|)); s is clamped from above at
  *    Smax; delta = s * dir (fp32); the sample point is then formed exactly as
  *    in DCNv4 with delta in place of the offset.
+ *  - MSDCN backward: the gradient reaches raw through
+ *    ds/draw = s0 * sigmoid(raw) while s0 * softplus(raw) <= Smax and is 0
+ *    once the clamp is active (and for a NaN raw).
  */
 #include <math.h>
 #include <stddef.h>
@@ -271,6 +274,106 @@ int orc_msdcn_forward(const orc_problem *p, const float *input,
                                              g * D, D, x, y, (double)t[3 * k + 2], o);
                         }
                     }
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* Derivative of the MSDCN scale with respect to raw: s0 * sigmoid(raw) while
+ * the clamp is inactive (s0 * softplus(raw) <= smax, the branch
+ * orc_msdcn_scale keeps), 0 once it clamps, 0 for a NaN raw. sigmoid is the
+ * derivative of softplus (read from [FLOWDCN] 3.1's softplus scale; the
+ * page prints no gradient). */
+static double orc_msdcn_scale_grad(float raw, float s0, float smax)
+{
+    float sp = fmaxf(raw, 0.0f) + log1pf(expf(-fabsf(raw)));
+    float u = s0 * sp;
+    if (!(u <= smax))
+        return 0.0;
+    return (double)s0 / (1.0 + exp(-(double)raw));
+}
+
+/* MSDCN backward: the gradients of orc_msdcn_forward's output, given
+ * grad_out, with respect to the input, to dir_weight (dir_x, dir_y, m) and to
+ * scale_raw. The sample of tap k is p0 + p_k + (s * dir_k) * offset_scale,
+ * so with g_x = m * sum_d go . dv/dx (and g_y likewise) at the sample:
+ *   d/d dir_x = s * os * g_x,   d/d dir_y = s * os * g_y,
+ *   d/d m     = sum_d go . v  (as in DCNv4),
+ *   d/d raw   = (ds/draw) * os * sum_k (g_x * dir_x + g_y * dir_y),
+ *   grad_in[corner] += m * w_corner * go.
+ * Outputs are fp64: grad_input [N][H][W][C], grad_dir_weight
+ * [N][Ho][Wo][G][kh*kw][3], grad_scale_raw [N][Ho][Wo][G]. */
+int orc_msdcn_backward(const orc_problem *p, const float *input,
+                       const float *dir_weight, const float *scale_raw,
+                       const float *s0, float smax, const float *grad_out,
+                       double *grad_input, double *grad_dir_weight,
+                       double *grad_scale_raw)
+{
+    int Ho, Wo;
+    if (orc_out_hw(p, &Ho, &Wo) || !input || !dir_weight || !scale_raw || !s0 ||
+        !grad_out || !grad_input || !grad_dir_weight || !grad_scale_raw)
+        return -1;
+    const int K = p->kh * p->kw, D = p->C / p->G;
+    const size_t img = (size_t)p->H * p->W * p->C;
+    const double os = (double)p->offset_scale;
+    memset(grad_input, 0, sizeof(double) * img * p->N);
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < p->N; ++n) {
+        const float *in_n = input + (size_t)n * img;
+        double *gin_n = grad_input + (size_t)n * img;
+        for (int ho = 0; ho < Ho; ++ho) {
+            for (int wo = 0; wo < Wo; ++wo) {
+                size_t pix = ((size_t)n * Ho + ho) * Wo + wo;
+                for (int g = 0; g < p->G; ++g) {
+                    const float *t = dir_weight + (pix * p->G + g) * (size_t)K * 3;
+                    double *gt = grad_dir_weight + (pix * p->G + g) * (size_t)K * 3;
+                    const float *go = grad_out + pix * p->C + (size_t)g * D;
+                    const float raw = scale_raw[pix * p->G + g];
+                    const float s = orc_msdcn_scale(raw, s0[g], smax);
+                    double gs = 0.0;  /* d loss / d s */
+                    for (int i = 0; i < p->kh; ++i) {
+                        for (int j = 0; j < p->kw; ++j) {
+                            int k = i * p->kw + j;
+                            float dx = s * t[3 * k], dy = s * t[3 * k + 1];
+                            float x, y;
+                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);
+                            double m = (double)t[3 * k + 2];
+                            double gx = 0.0, gy = 0.0, gm = 0.0;
+                            if (x > -1.0f && x < (float)p->W && y > -1.0f && y < (float)p->H) {
+                                float x0f = floorf(x), y0f = floorf(y);
+                                double lx = (double)x - (double)x0f;
+                                double ly = (double)y - (double)y0f;
+                                int x0 = (int)x0f, y0 = (int)y0f;
+                                for (int a = 0; a < 2; ++a) {
+                                    for (int b = 0; b < 2; ++b) {
+                                        int yy = y0 + a, xx = x0 + b;
+                                        if (yy < 0 || yy >= p->H || xx < 0 || xx >= p->W)
+                                            continue;
+                                        double wy = a ? ly : 1.0 - ly;
+                                        double wx = b ? lx : 1.0 - lx;
+                                        size_t at = ((size_t)yy * p->W + xx) * p->C + (size_t)g * D;
+                                        double dot = 0.0;
+                                        for (int d = 0; d < D; ++d) {
+                                            dot += (double)go[d] * (double)in_n[at + d];
+                                            gin_n[at + d] += m * (wy * wx) * (double)go[d];
+                                        }
+                                        gm += wy * wx * dot;
+                                        gx += (b ? wy : -wy) * dot;
+                                        gy += (a ? wx : -wx) * dot;
+                                    }
+                                }
+                            }
+                            /* gx, gy: d(sum_d go . sample) / dx, dy of the position */
+                            gt[3 * k] = (double)s * os * m * gx;
+                            gt[3 * k + 1] = (double)s * os * m * gy;
+                            gt[3 * k + 2] = gm;
+                            gs += os * m * (gx * (double)t[3 * k] + gy * (double)t[3 * k + 1]);
+                        }
+                    }
+                    grad_scale_raw[pix * p->G + g] =
+                        gs == 0.0 ? 0.0 : gs * orc_msdcn_scale_grad(raw, s0[g], smax);
                 }
             }
         }

@@ -25,6 +25,13 @@ What pins what (pages cited by title and section):
   pin_unit_columns  grad_input entries == <f(e_q), g> for unit inputs e_q
   pin_finite_diff   grad dx, dy, m == central differences (exact for a
                     piecewise-linear function away from cell edges)
+  pin_msdcn_bwd_unit  MSDCN backward at a clamped unit scale == DCNv4 backward
+                    bit for bit, and no gradient reaches raw through the clamp
+  pin_msdcn_bwd_adjoint  <f(x), g> == <x, grad_input>, <f(m), g> == <m, grad_m>
+  pin_msdcn_bwd_dir central differences for dir at a clamped scale s = 2
+                    (exact, dyadic positions): the factor s in d/d dir
+  pin_msdcn_bwd_raw central differences for raw below the clamp (smooth:
+                    softplus scale, positions kept away from cell edges)
 """
 import json
 import math
@@ -391,6 +398,107 @@ def pin_finite_diff(o):
                     f"finite difference at {idx} comp {comp}: {fd} vs {an}"
 
 
+def _msdcn_case(o, seed, N=2, H=7, W=8, C=6, G=3, os_=1.0):
+    rng = _rng(seed)
+    prob = o.problem(N, H, W, C, G, 3, 3, offset_scale=os_)
+    Ho, Wo = o.out_hw(prob)
+    x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+    dw = _ow(o, prob, rng)
+    raw = rng.standard_normal((N, Ho, Wo, G)).astype(np.float32)
+    go = rng.standard_normal((N, Ho, Wo, C)).astype(np.float32)
+    s0 = np.array([1 + g // 2 for g in range(G)], np.float32)
+    return prob, x, dw, raw, s0, go
+
+
+def pin_msdcn_bwd_unit(o):
+    """s0 = 1, raw = 30, Smax = 1: s is exactly 1 (clamped), so the MSDCN
+    gradients are DCNv4's with offsets = dir, and raw gets none."""
+    prob, x, dw, raw, s0, go = _msdcn_case(o, 81, os_=0.75)
+    raw[...] = 30.0
+    gin, gdw, graw = o.msdcn_backward(prob, x, dw, raw, np.ones(prob.G, np.float32), 1.0, go)
+    rgin, rgow = o.backward(prob, x, dw, go)
+    assert np.array_equal(gin, rgin), "grad_input at unit scale"
+    assert np.array_equal(gdw, rgow), "grad_dir_weight at unit scale"
+    assert np.all(graw == 0.0), "no gradient through an active clamp"
+
+
+def pin_msdcn_bwd_adjoint(o):
+    prob, x, dw, raw, s0, go = _msdcn_case(o, 82)
+    smax = 2.5
+    gin, gdw, _ = o.msdcn_backward(prob, x, dw, raw, s0, smax, go)
+    lhs = float(np.sum(o.msdcn_forward(prob, x, dw, raw, s0, smax) * go))
+    rhs_x = float(np.sum(x.astype(np.float64) * gin))
+    rhs_m = float(np.sum(dw[..., 2].astype(np.float64) * gdw[..., 2]))
+    assert abs(lhs - rhs_x) <= 1e-11 * max(1.0, abs(lhs)), "<f(x), g> vs <x, grad_input>"
+    assert abs(lhs - rhs_m) <= 1e-11 * max(1.0, abs(lhs)), "<f(m), g> vs <m, grad_m>"
+
+
+def pin_msdcn_bwd_dir(o):
+    """Scale clamped at exactly 2 (s0 = 4, raw >= 1, Smax = 2). dir values are
+    odd multiples of 1/1024, so s * dir is an odd multiple of 1/512 and a
+    step of 1/2048 in dir moves the sample by 1/1024 inside one bilinear
+    cell: the central difference is exact up to fp64 rounding."""
+    for seed, os_ in ((83, 1.0), (84, 0.5)):
+        prob, x, dw, raw, s0, go = _msdcn_case(o, seed, os_=os_)
+        rng = _rng(seed + 100)
+        raw = rng.uniform(1.0, 3.0, raw.shape).astype(np.float32)
+        s0 = np.full(prob.G, 4.0, np.float32)
+        dw[..., :2] = (2 * rng.integers(-900, 900, dw[..., :2].shape) + 1) / 1024.0
+        gin, gdw, graw = o.msdcn_backward(prob, x, dw, raw, s0, 2.0, go)
+        assert np.all(graw == 0.0)
+        h = 1.0 / 2048.0
+        for _ in range(20):
+            idx = tuple(int(rng.integers(0, s)) for s in dw.shape[:-1])
+            for comp in range(3):
+                hh = h / os_ if comp < 2 else h
+                dp, dm = dw.copy(), dw.copy()
+                dp[idx + (comp,)] += hh
+                dm[idx + (comp,)] -= hh
+                fd = (np.sum(o.msdcn_forward(prob, x, dp, raw, s0, 2.0) * go) -
+                      np.sum(o.msdcn_forward(prob, x, dm, raw, s0, 2.0) * go)) / (2 * hh)
+                an = gdw[idx + (comp,)]
+                assert abs(fd - an) <= 1e-8 * max(1.0, abs(an)), \
+                    f"d/d dir at {idx} comp {comp}: {fd} vs {an}"
+
+
+def pin_msdcn_bwd_raw(o):
+    """Below the clamp the loss is a smooth function of raw near the drawn
+    point as long as no sample crosses a cell edge. Samples are kept at least
+    0.05 px from every edge (directions redrawn until they are), the step is
+    1e-3 (moves a sample by < 0.02 px); the central difference then matches
+    up to O(h^2) and the fp32 rounding of positions (relative ~1e-4)."""
+    prob, x, dw, raw, s0, go = _msdcn_case(o, 85, N=1, H=6, W=6, C=4, G=2)
+    Ho, Wo = o.out_hw(prob)
+    smax = 50.0
+    rng = _rng(185)
+    s = np.array([[[[o.msdcn_scale(raw[n, i, j, g], s0[g], smax) for g in range(prob.G)]
+                    for j in range(Wo)] for i in range(Ho)] for n in range(prob.N)], np.float64)
+    for n in range(prob.N):
+        for i in range(Ho):
+            for j in range(Wo):
+                for g in range(prob.G):
+                    for k in range(9):
+                        while True:
+                            d = rng.standard_normal(2)
+                            px = j - 1 + k % 3 + s[n, i, j, g] * d[0]
+                            py = i - 1 + k // 3 + s[n, i, j, g] * d[1]
+                            fx, fy = px - math.floor(px), py - math.floor(py)
+                            if 0.05 < fx < 0.95 and 0.05 < fy < 0.95:
+                                break
+                        dw[n, i, j, g, k, :2] = d
+    _, _, graw = o.msdcn_backward(prob, x, dw, raw, s0, smax, go)
+    h = 1e-3
+    for idx in np.ndindex(raw.shape):
+        rp, rm = raw.copy(), raw.copy()
+        rp[idx] += h
+        rm[idx] -= h
+        fd = (np.sum(o.msdcn_forward(prob, x, dw, rp, s0, smax) * go) -
+              np.sum(o.msdcn_forward(prob, x, dw, rm, s0, smax) * go)) / (float(rp[idx]) - float(rm[idx]))
+        an = graw[idx]
+        assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), f"d/d raw at {idx}: {fd} vs {an}"
+
+
 ALL_PINS = [pin_conv, pin_grid_sample, pin_gather, pin_fractions, pin_out_of_bounds,
             pin_linearity, pin_equivariance, pin_msdcn, pin_cost_model, pin_adjoint,
-            pin_unit_columns, pin_finite_diff]
+            pin_unit_columns, pin_finite_diff, pin_msdcn_bwd_unit, pin_msdcn_bwd_adjoint,
+            pin_msdcn_bwd_dir, pin_msdcn_bwd_raw]

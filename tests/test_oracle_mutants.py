@@ -53,6 +53,21 @@ MUTANTS = [
     ("clamp_from_below", "if (s > smax)\n        s = smax;", "if (s < smax)\n        s = smax;", 1),
     ("msdcn_scale_per_group_ignored", "float s = orc_msdcn_scale(scale_raw[pix * p->G + g], s0[g], smax);",
      "float s = orc_msdcn_scale(scale_raw[pix * p->G + g], s0[0], smax);", 1),
+    ("msdcn_grad_dir_missing_s", "gt[3 * k] = (double)s * os * m * gx;", "gt[3 * k] = os * m * gx;", 1),
+    ("msdcn_sigmoid_sign", "return (double)s0 / (1.0 + exp(-(double)raw));",
+     "return (double)s0 / (1.0 + exp((double)raw));", 1),
+    ("msdcn_clamp_gradient_kept", "if (!(u <= smax))\n        return 0.0;",
+     "if (isnan(u))\n        return 0.0;", 1),
+    ("msdcn_grad_raw_dirs_swapped",
+     "gs += os * m * (gx * (double)t[3 * k] + gy * (double)t[3 * k + 1]);",
+     "gs += os * m * (gx * (double)t[3 * k + 1] + gy * (double)t[3 * k]);", 1),
+    ("msdcn_bwd_unscaled_offsets",
+     "float dx = s * t[3 * k], dy = s * t[3 * k + 1];\n                            float x, y;\n"
+     "                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);\n"
+     "                            double m",
+     "float dx = t[3 * k], dy = t[3 * k + 1];\n                            float x, y;\n"
+     "                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);\n"
+     "                            double m", 1),
     ("flops_factor", "return 4.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;",
      "return 2.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;", 1),
     ("ideal_offsets_per_channel", "double ow = 3.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->G;",
