@@ -16,7 +16,8 @@ from . import build as _build
 class OrcProblem(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int) for name in
                 ("N", "H", "W", "C", "G", "kh", "kw", "sh", "sw", "ph", "pw", "dh", "dw")] + \
-               [("offset_scale", ctypes.c_float)]
+               [("offset_scale", ctypes.c_float), ("softmax", ctypes.c_int),
+                ("msdcn_dilation", ctypes.c_int)]
 
 
 _F32P = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
@@ -55,9 +56,10 @@ class Oracle:
     # -- problem description -------------------------------------------------
     @staticmethod
     def problem(N, H, W, C, G, kh=3, kw=3, stride=(1, 1), pad=(1, 1), dilation=(1, 1),
-                offset_scale=1.0):
+                offset_scale=1.0, softmax=False, msdcn_dilation=False):
         return OrcProblem(N, H, W, C, G, kh, kw, stride[0], stride[1], pad[0], pad[1],
-                          dilation[0], dilation[1], offset_scale)
+                          dilation[0], dilation[1], offset_scale, int(bool(softmax)),
+                          int(bool(msdcn_dilation)))
 
     def out_hw(self, prob):
         ho, wo = ctypes.c_int(), ctypes.c_int()

@@ -60,6 +60,8 @@ typedef struct {
     int ph, pw;          /* padding                                       */
     int dh, dw;          /* dilation                                      */
     float offset_scale;  /* multiplies every offset before it is added    */
+    int softmax;         /* DCNv3 weights: softmax of m over the taps     */
+    int msdcn_dilation;  /* MSDCN reading p0 + s * (p_k + dir)            */
 } orc_problem;
 
 /* Output size, standard convolution arithmetic ([CANN] 2.1). Returns 0 when
@@ -90,6 +92,62 @@ static void orc_position(const orc_problem *p, int ho, int wo, int i, int j,
     float ty = dy * p->offset_scale;
     *x = bx + tx;
     *y = by + ty;
+}
+
+/* The aggregation weights of one (pixel, group): m as given ([DIGEST]
+ * 移除Softmax归一化), or with p->softmax the DCNv3 normalisation the same
+ * section describes, softmax over the kh*kw taps (in fp64, largest logit
+ * subtracted first). t holds the (dx, dy, m) triples; w receives K weights. */
+static void orc_tap_weights(const orc_problem *p, const float *t, double *w)
+{
+    const int K = p->kh * p->kw;
+    if (!p->softmax) {
+        for (int k = 0; k < K; ++k)
+            w[k] = (double)t[3 * k + 2];
+        return;
+    }
+    double mx = (double)t[2];
+    for (int k = 1; k < K; ++k)
+        if ((double)t[3 * k + 2] > mx)
+            mx = (double)t[3 * k + 2];
+    double sum = 0.0;
+    for (int k = 0; k < K; ++k) {
+        w[k] = exp((double)t[3 * k + 2] - mx);
+        sum += w[k];
+    }
+    for (int k = 0; k < K; ++k)
+        w[k] /= sum;
+}
+
+/* The MSDCN sample of tap (i, j) with scale s and direction (dirx, diry)
+ * ([FLOWDCN] 3.1). Default reading: the offset is s * dir, then as
+ * orc_position. With p->msdcn_dilation the scale stretches the kernel grid as
+ * well: centre + s * (p_k + dir * offset_scale), centre the middle of the
+ * kh x kw window and p_k the tap's grid offset from it; each product and sum
+ * rounded to fp32. (tx, ty) receive the factor that multiplies s, i.e. the
+ * derivative of the position with respect to s. */
+static void orc_position_ms(const orc_problem *p, int ho, int wo, int i, int j, float s,
+                            float dirx, float diry, float *x, float *y, double *tx,
+                            double *ty)
+{
+    if (!p->msdcn_dilation) {
+        float dx = s * dirx, dy = s * diry;
+        orc_position(p, ho, wo, i, j, dx, dy, x, y);
+        *tx = (double)dirx * (double)p->offset_scale;
+        *ty = (double)diry * (double)p->offset_scale;
+        return;
+    }
+    float cx = (float)(wo * p->sw - p->pw) + 0.5f * (float)((p->kw - 1) * p->dw);
+    float cy = (float)(ho * p->sh - p->ph) + 0.5f * (float)((p->kh - 1) * p->dh);
+    float kx = ((float)j - 0.5f * (float)(p->kw - 1)) * (float)p->dw;
+    float ky = ((float)i - 0.5f * (float)(p->kh - 1)) * (float)p->dh;
+    float ox = dirx * p->offset_scale, oy = diry * p->offset_scale;
+    float ux = kx + ox, uy = ky + oy;
+    float sx = s * ux, sy = s * uy;
+    *x = cx + sx;
+    *y = cy + sy;
+    *tx = (double)ux;
+    *ty = (double)uy;
 }
 
 /* Adds m * bilinear(img at (x, y))[c0 .. c0+D) into acc ([DIGEST]: 4 terms of
@@ -135,6 +193,8 @@ int orc_dcn4_forward(const orc_problem *p, const float *input,
                 for (int g = 0; g < p->G; ++g) {
                     double *o = out + pix * p->C + (size_t)g * D;
                     const float *t = offset_weight + (pix * p->G + g) * (size_t)K * 3;
+                    double wk[K];
+                    orc_tap_weights(p, t, wk);
                     for (int d = 0; d < D; ++d)
                         o[d] = 0.0;
                     for (int i = 0; i < p->kh; ++i) {
@@ -143,7 +203,7 @@ int orc_dcn4_forward(const orc_problem *p, const float *input,
                             float x, y;
                             orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);
                             orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,
-                                             g * D, D, x, y, (double)t[3 * k + 2], o);
+                                             g * D, D, x, y, wk[k], o);
                         }
                     }
                 }
@@ -162,7 +222,8 @@ int orc_dcn4_forward(const orc_problem *p, const float *input,
  *   grad in[c] += m * wy * wx * go        (for every in-image corner c)
  * At an integer position the derivative taken is the one of the cell that
  * floor() selects (the right-hand derivative). Samples outside
- * (-1, W) x (-1, H) have zero gradient. */
+ * (-1, W) x (-1, H) have zero gradient. With p->softmax, m above is the
+ * softmax weight w_k and the m-gradient is taken through the softmax. */
 int orc_dcn4_backward(const orc_problem *p, const float *input,
                       const float *offset_weight, const float *grad_out,
                       double *grad_input, double *grad_offset_weight)
@@ -186,12 +247,14 @@ int orc_dcn4_backward(const orc_problem *p, const float *input,
                     const float *t = offset_weight + (pix * p->G + g) * (size_t)K * 3;
                     double *gt = grad_offset_weight + (pix * p->G + g) * (size_t)K * 3;
                     const float *go = grad_out + pix * p->C + (size_t)g * D;
+                    double wk[K], gwk[K];  /* tap weights; d loss / d weight */
+                    orc_tap_weights(p, t, wk);
                     for (int i = 0; i < p->kh; ++i) {
                         for (int j = 0; j < p->kw; ++j) {
                             int k = i * p->kw + j;
                             float x, y;
                             orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);
-                            double m = (double)t[3 * k + 2];
+                            double m = wk[k];
                             double gx = 0.0, gy = 0.0, gm = 0.0;
                             if (x > -1.0f && x < (float)p->W && y > -1.0f && y < (float)p->H) {
                                 float x0f = floorf(x), y0f = floorf(y);
@@ -219,9 +282,16 @@ int orc_dcn4_backward(const orc_problem *p, const float *input,
                             }
                             gt[3 * k] = (double)p->offset_scale * m * gx;
                             gt[3 * k + 1] = (double)p->offset_scale * m * gy;
-                            gt[3 * k + 2] = gm;
+                            gwk[k] = gm;
                         }
                     }
+                    /* through the softmax: d/d m_k = w_k (gw_k - sum_j w_j gw_j) */
+                    double dotw = 0.0;
+                    if (p->softmax)
+                        for (int k = 0; k < K; ++k)
+                            dotw += wk[k] * gwk[k];
+                    for (int k = 0; k < K; ++k)
+                        gt[3 * k + 2] = p->softmax ? wk[k] * (gwk[k] - dotw) : gwk[k];
                 }
             }
         }
@@ -241,7 +311,9 @@ float orc_msdcn_scale(float raw, float s0, float smax)
 }
 
 /* MSDCN forward ([FLOWDCN] 3.1): DCNv4 aggregation whose offset for group g
- * and tap k is s_g(p0) * dir_{g,k}(p0).
+ * and tap k is s_g(p0) * dir_{g,k}(p0) (or, with p->msdcn_dilation, whose
+ * kernel grid is scaled too, see orc_position_ms). m is used as given
+ * (p->softmax does not apply to MSDCN).
  * dir_weight [N][Ho][Wo][G][kh*kw][3] holds (dir_x, dir_y, m);
  * scale_raw [N][Ho][Wo][G]; s0 [G]. */
 int orc_msdcn_forward(const orc_problem *p, const float *input,
@@ -267,9 +339,10 @@ int orc_msdcn_forward(const orc_problem *p, const float *input,
                     for (int i = 0; i < p->kh; ++i) {
                         for (int j = 0; j < p->kw; ++j) {
                             int k = i * p->kw + j;
-                            float dx = s * t[3 * k], dy = s * t[3 * k + 1];
                             float x, y;
-                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);
+                            double tx, ty;
+                            orc_position_ms(p, ho, wo, i, j, s, t[3 * k], t[3 * k + 1], &x, &y,
+                                            &tx, &ty);
                             orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,
                                              g * D, D, x, y, (double)t[3 * k + 2], o);
                         }
@@ -301,7 +374,8 @@ static double orc_msdcn_scale_grad(float raw, float s0, float smax)
  * so with g_x = m * sum_d go . dv/dx (and g_y likewise) at the sample:
  *   d/d dir_x = s * os * g_x,   d/d dir_y = s * os * g_y,
  *   d/d m     = sum_d go . v  (as in DCNv4),
- *   d/d raw   = (ds/draw) * os * sum_k (g_x * dir_x + g_y * dir_y),
+ *   d/d raw   = (ds/draw) * sum_k (g_x * dx/ds + g_y * dy/ds), where
+ *               dx/ds = os * dir_x (or p_kx + os * dir_x with msdcn_dilation),
  *   grad_in[corner] += m * w_corner * go.
  * Outputs are fp64: grad_input [N][H][W][C], grad_dir_weight
  * [N][Ho][Wo][G][kh*kw][3], grad_scale_raw [N][Ho][Wo][G]. */
@@ -336,9 +410,10 @@ int orc_msdcn_backward(const orc_problem *p, const float *input,
                     for (int i = 0; i < p->kh; ++i) {
                         for (int j = 0; j < p->kw; ++j) {
                             int k = i * p->kw + j;
-                            float dx = s * t[3 * k], dy = s * t[3 * k + 1];
                             float x, y;
-                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);
+                            double tx, ty;  /* d position / d s */
+                            orc_position_ms(p, ho, wo, i, j, s, t[3 * k], t[3 * k + 1], &x, &y,
+                                            &tx, &ty);
                             double m = (double)t[3 * k + 2];
                             double gx = 0.0, gy = 0.0, gm = 0.0;
                             if (x > -1.0f && x < (float)p->W && y > -1.0f && y < (float)p->H) {
@@ -369,7 +444,7 @@ int orc_msdcn_backward(const orc_problem *p, const float *input,
                             gt[3 * k] = (double)s * os * m * gx;
                             gt[3 * k + 1] = (double)s * os * m * gy;
                             gt[3 * k + 2] = gm;
-                            gs += os * m * (gx * (double)t[3 * k] + gy * (double)t[3 * k + 1]);
+                            gs += m * (gx * tx + gy * ty);
                         }
                     }
                     grad_scale_raw[pix * p->G + g] =

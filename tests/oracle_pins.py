@@ -32,6 +32,17 @@ What pins what (pages cited by title and section):
                     (exact, dyadic positions): the factor s in d/d dir
   pin_msdcn_bwd_raw central differences for raw below the clamp (smooth:
                     softplus scale, positions kept away from cell edges)
+  pin_softmax_box   DCNv3 flag, equal logits: weights 1/K, zero offsets ==
+                    box filter (torch conv2d, groups=C, float64)
+  pin_softmax_shift adding a constant to a pixel-group's logits changes
+                    nothing, even at logits of 800 (exp would overflow); one dominant
+                    logit == that tap alone (DCNv4 with a one-hot m)
+  pin_softmax_bwd   adjoint for grad_input; central differences for the
+                    logits (smooth) and the offsets (exact, dyadic)
+  pin_msdcn_dilation  scale-as-dilation reading: s = 1 with dyadic dirs ==
+                    DCNv4 bit for bit; s = 2, dir = 0 == DCNv4 at twice the
+                    dilation (pad + dilation) bit for bit; backward by central
+                    differences (dir exact at s = 2; raw smooth)
 """
 import json
 import math
@@ -498,7 +509,156 @@ def pin_msdcn_bwd_raw(o):
         assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), f"d/d raw at {idx}: {fd} vs {an}"
 
 
+def _box(x, K, stride, pad, dil, kh=3, kw=3):
+    """Depthwise conv with every weight 1/K (float64, torch)."""
+    C = x.shape[-1]
+    xt = torch.from_numpy(x.astype(np.float64)).permute(0, 3, 1, 2)
+    w = torch.full((C, 1, kh, kw), 1.0 / K, dtype=torch.float64)
+    return F.conv2d(xt, w, stride=stride, padding=pad, dilation=dil, groups=C).permute(0, 2, 3, 1).numpy()
+
+
+def pin_softmax_box(o):
+    rng = _rng(91)
+    for (N, H, W, C, G, st, pd, dl) in [(2, 7, 9, 6, 3, (1, 1), (1, 1), (1, 1)),
+                                        (1, 9, 8, 4, 2, (2, 1), (2, 1), (2, 1))]:
+        prob = o.problem(N, H, W, C, G, 3, 3, st, pd, dl, softmax=True)
+        x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+        Ho, Wo = o.out_hw(prob)
+        logit = rng.standard_normal((N, Ho, Wo, G, 1)).astype(np.float32)
+        ow = _ow(o, prob, rng, offsets=0.0, m=np.broadcast_to(logit, (N, Ho, Wo, G, 9)))
+        _close(o.forward(prob, x, ow), _box(x, 9, st, pd, dl), 1e-12, "softmax of equal logits")
+
+
+def pin_softmax_shift(o):
+    rng = _rng(92)
+    N, H, W, C, G = 2, 6, 7, 4, 2
+    prob = o.problem(N, H, W, C, G, 3, 3, softmax=True)
+    x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+    ow = _ow(o, prob, rng)
+    ow[..., :2] *= 1.5
+    ref = o.forward(prob, x, ow)
+    for c in (3.0, 800.0):
+        sh = ow.copy()
+        sh[..., 2] = (sh[..., 2].astype(np.float64) + c).astype(np.float32)
+        got = o.forward(prob, x, sh)
+        assert np.all(np.isfinite(got)), f"logits + {c}: overflow"
+        # the shifted fp32 logits differ from the originals by rounding, so
+        # compare against the softmax weights of the shifted values
+        back = sh.copy()
+        back[..., 2] = (sh[..., 2].astype(np.float64) - c).astype(np.float32)
+        _close(got, o.forward(prob, x, back), 1e-12, f"logits + {c}")
+    one = ow.copy()
+    k = 4
+    one[..., 2] = 0.0
+    one[..., k, 2] = 60.0
+    hot = ow.copy()
+    hot[..., 2] = 0.0
+    hot[..., k, 2] = 1.0
+    plain = o.problem(N, H, W, C, G, 3, 3)
+    _close(o.forward(prob, x, one), o.forward(plain, x, hot), 1e-12, "one dominant logit")
+
+
+def pin_softmax_bwd(o):
+    rng = _rng(93)
+    N, H, W, C, G = 2, 7, 8, 6, 3
+    prob = o.problem(N, H, W, C, G, 3, 3, softmax=True)
+    x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+    ow = _ow(o, prob, rng)
+    ow[..., :2] = (2 * rng.integers(-900, 900, ow[..., :2].shape) + 1) / 512.0
+    Ho, Wo = o.out_hw(prob)
+    go = rng.standard_normal((N, Ho, Wo, C)).astype(np.float32)
+    gin, gow = o.backward(prob, x, ow, go)
+    lhs = float(np.sum(o.forward(prob, x, ow) * go))
+    rhs = float(np.sum(x.astype(np.float64) * gin))
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs)), "<f(x), g> vs <x, grad_input>"
+    # the logit gradients of one pixel-group sum to zero (softmax is shift-invariant)
+    assert np.abs(gow[..., 2].sum(axis=-1)).max() <= 1e-12 * max(1.0, np.abs(gow[..., 2]).max())
+    for _ in range(20):
+        idx = tuple(int(rng.integers(0, s)) for s in ow.shape[:-1])
+        for comp, h in ((0, 1.0 / 1024.0), (1, 1.0 / 1024.0), (2, 1e-4)):
+            op, om = ow.copy(), ow.copy()
+            op[idx + (comp,)] += h
+            om[idx + (comp,)] -= h
+            step = float(op[idx + (comp,)]) - float(om[idx + (comp,)])
+            fd = (np.sum(o.forward(prob, x, op) * go) - np.sum(o.forward(prob, x, om) * go)) / step
+            an = gow[idx + (comp,)]
+            tol = 1e-8 if comp < 2 else 1e-6
+            assert abs(fd - an) <= tol * max(1.0, abs(an)), f"softmax FD at {idx} comp {comp}: {fd} vs {an}"
+
+
+def pin_msdcn_dilation(o):
+    rng = _rng(94)
+    N, H, W, C, G = 2, 9, 10, 8, 4
+    for st, pd, dl in (((1, 1), (1, 1), (1, 1)), ((2, 1), (2, 1), (1, 2))):
+        prob = o.problem(N, H, W, C, G, 3, 3, st, pd, dl, msdcn_dilation=True)
+        Ho, Wo = o.out_hw(prob)
+        x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+        dw = _ow(o, prob, rng)
+        dw[..., :2] = rng.integers(-200, 200, dw[..., :2].shape) / 64.0
+        ones = np.ones(G, np.float32)
+        raw = np.full((N, Ho, Wo, G), 30.0, np.float32)
+        got = o.msdcn_forward(prob, x, dw, raw, ones, 1.0)  # s = 1 exactly
+        plain = o.problem(N, H, W, C, G, 3, 3, st, pd, dl)
+        assert np.array_equal(got, o.forward(plain, x, dw)), "dilation reading at s = 1"
+        zero = dw.copy()
+        zero[..., :2] = 0.0
+        got = o.msdcn_forward(prob, x, zero, raw, np.full(G, 4.0, np.float32), 2.0)  # s = 2
+        wide = o.problem(N, H, W, C, G, 3, 3, st, (pd[0] + dl[0], pd[1] + dl[1]),
+                         (2 * dl[0], 2 * dl[1]))
+        assert o.out_hw(wide) == (Ho, Wo)
+        assert np.array_equal(got, o.forward(wide, x, zero)), "s = 2 is twice the dilation"
+    # backward: dir by exact central differences at s = 2, raw smoothly
+    prob = o.problem(1, 7, 8, 6, 3, 3, 3, msdcn_dilation=True, offset_scale=0.5)
+    Ho, Wo = o.out_hw(prob)
+    x = rng.standard_normal((1, 7, 8, 6)).astype(np.float32)
+    dw = _ow(o, prob, rng)
+    dw[..., :2] = (2 * rng.integers(-300, 300, dw[..., :2].shape) + 1) / 512.0
+    go = rng.standard_normal((1, Ho, Wo, 6)).astype(np.float32)
+    s0 = np.full(3, 4.0, np.float32)
+    raw = rng.uniform(1.0, 3.0, (1, Ho, Wo, 3)).astype(np.float32)
+    _, gdw, graw = o.msdcn_backward(prob, x, dw, raw, s0, 2.0, go)
+    assert np.all(graw == 0.0)
+    h = 1.0 / 2048.0
+    for _ in range(16):
+        idx = tuple(int(rng.integers(0, s)) for s in dw.shape[:-1])
+        for comp in range(3):
+            hh = h / 0.5 if comp < 2 else h
+            dp, dm = dw.copy(), dw.copy()
+            dp[idx + (comp,)] += hh
+            dm[idx + (comp,)] -= hh
+            fd = (np.sum(o.msdcn_forward(prob, x, dp, raw, s0, 2.0) * go) -
+                  np.sum(o.msdcn_forward(prob, x, dm, raw, s0, 2.0) * go)) / (2 * hh)
+            an = gdw[idx + (comp,)]
+            assert abs(fd - an) <= 1e-8 * max(1.0, abs(an)), f"dilation d/d dir {idx} {comp}"
+    # raw below the clamp: keep every sample 0.05 px from cell edges
+    s0 = np.array([1.0, 1.0, 2.0], np.float32)
+    raw = rng.standard_normal((1, Ho, Wo, 3)).astype(np.float32)
+    smax = 50.0
+    for i in range(Ho):
+        for j in range(Wo):
+            for g in range(3):
+                s = o.msdcn_scale(raw[0, i, j, g], s0[g], smax)
+                for k in range(9):
+                    while True:
+                        d = rng.standard_normal(2)
+                        px = j + s * ((k % 3 - 1) + 0.5 * d[0])
+                        py = i + s * ((k // 3 - 1) + 0.5 * d[1])
+                        fx, fy = px - math.floor(px), py - math.floor(py)
+                        if 0.05 < fx < 0.95 and 0.05 < fy < 0.95:
+                            break
+                    dw[0, i, j, g, k, :2] = d
+    _, _, graw = o.msdcn_backward(prob, x, dw, raw, s0, smax, go)
+    for idx in np.ndindex(raw.shape):
+        rp, rm = raw.copy(), raw.copy()
+        rp[idx] += 1e-3
+        rm[idx] -= 1e-3
+        fd = (np.sum(o.msdcn_forward(prob, x, dw, rp, s0, smax) * go) -
+              np.sum(o.msdcn_forward(prob, x, dw, rm, s0, smax) * go)) / (float(rp[idx]) - float(rm[idx]))
+        assert abs(fd - graw[idx]) <= 2e-3 * max(1.0, abs(graw[idx])), f"dilation d/d raw {idx}"
+
+
 ALL_PINS = [pin_conv, pin_grid_sample, pin_gather, pin_fractions, pin_out_of_bounds,
             pin_linearity, pin_equivariance, pin_msdcn, pin_cost_model, pin_adjoint,
             pin_unit_columns, pin_finite_diff, pin_msdcn_bwd_unit, pin_msdcn_bwd_adjoint,
-            pin_msdcn_bwd_dir, pin_msdcn_bwd_raw]
+            pin_msdcn_bwd_dir, pin_msdcn_bwd_raw, pin_softmax_box, pin_softmax_shift,
+            pin_softmax_bwd, pin_msdcn_dilation]

@@ -28,11 +28,11 @@ MUTANTS = [
     ("transpose_taps", "int k = i * p->kw + j;\n                            float x, y;\n"
                        "                            orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);\n"
                        "                            orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,\n"
-                       "                                             g * D, D, x, y, (double)t[3 * k + 2], o);",
+                       "                                             g * D, D, x, y, wk[k], o);",
      "int k = j * p->kh + i;\n                            float x, y;\n"
      "                            orc_position(p, ho, wo, i, j, t[3 * k], t[3 * k + 1], &x, &y);\n"
      "                            orc_splat_sample(input + (size_t)n * img, p->H, p->W, p->C,\n"
-     "                                             g * D, D, x, y, (double)t[3 * k + 2], o);", 1),
+     "                                             g * D, D, x, y, wk[k], o);", 1),
     ("ignore_offset_scale", "float tx = dx * p->offset_scale;", "float tx = dx;", 1),
     ("stride_ignored", "float bx = (float)(wo * p->sw - p->pw + j * p->dw);",
      "float bx = (float)(wo - p->pw + j * p->dw);", 1),
@@ -59,15 +59,21 @@ MUTANTS = [
     ("msdcn_clamp_gradient_kept", "if (!(u <= smax))\n        return 0.0;",
      "if (isnan(u))\n        return 0.0;", 1),
     ("msdcn_grad_raw_dirs_swapped",
-     "gs += os * m * (gx * (double)t[3 * k] + gy * (double)t[3 * k + 1]);",
-     "gs += os * m * (gx * (double)t[3 * k + 1] + gy * (double)t[3 * k]);", 1),
+     "*tx = (double)dirx * (double)p->offset_scale;\n        *ty = (double)diry * (double)p->offset_scale;",
+     "*tx = (double)diry * (double)p->offset_scale;\n        *ty = (double)dirx * (double)p->offset_scale;", 1),
     ("msdcn_bwd_unscaled_offsets",
-     "float dx = s * t[3 * k], dy = s * t[3 * k + 1];\n                            float x, y;\n"
-     "                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);\n"
-     "                            double m",
-     "float dx = t[3 * k], dy = t[3 * k + 1];\n                            float x, y;\n"
-     "                            orc_position(p, ho, wo, i, j, dx, dy, &x, &y);\n"
-     "                            double m", 1),
+     "orc_position_ms(p, ho, wo, i, j, s, t[3 * k], t[3 * k + 1], &x, &y,\n"
+     "                                            &tx, &ty);\n                            double m",
+     "orc_position_ms(p, ho, wo, i, j, 1.0f, t[3 * k], t[3 * k + 1], &x, &y,\n"
+     "                                            &tx, &ty);\n                            double m", 1),
+    ("softmax_no_max_shift", "w[k] = exp((double)t[3 * k + 2] - mx);", "w[k] = exp((double)t[3 * k + 2]);", 1),
+    ("softmax_unnormalised", "        w[k] /= sum;", "        w[k] /= 9.0;", 1),
+    ("softmax_grad_missing_sum", "dotw += wk[k] * gwk[k];", "dotw += 0.0 * gwk[k];", 1),
+    ("softmax_grad_input_raw_logit", "double m = wk[k];", "double m = (double)t[3 * k + 2];", 1),
+    ("dilation_centre_off", "float cx = (float)(wo * p->sw - p->pw) + 0.5f * (float)((p->kw - 1) * p->dw);",
+     "float cx = (float)(wo * p->sw - p->pw);", 1),
+    ("dilation_grid_unscaled", "*x = cx + sx;", "*x = cx + kx + s * ox;", 1),
+    ("dilation_ds_missing_grid", "*tx = (double)ux;", "*tx = (double)ox;", 1),
     ("flops_factor", "return 4.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;",
      "return 2.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;", 1),
     ("ideal_offsets_per_channel", "double ow = 3.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->G;",
