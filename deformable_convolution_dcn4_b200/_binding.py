@@ -19,11 +19,13 @@ STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2}
 MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2}
+MSDCN_MODE_CODE = {"offset": 0, "dilation": 1}
 
 # Every symbol include/dcn4.h declares.
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
-           "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches")
+           "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches",
+           "msdcn_backward")
 
 
 class Dcn4Error(RuntimeError):
@@ -36,7 +38,8 @@ class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("N", "H", "W", "C", "G", "kh", "kw", "stride_h", "stride_w", "pad_h", "pad_w",
                  "dil_h", "dil_w")] + [("offset_scale", ctypes.c_float), ("dtype", ctypes.c_int),
-                                       ("algo", ctypes.c_int), ("math", ctypes.c_int)]
+                                       ("algo", ctypes.c_int), ("math", ctypes.c_int),
+                                       ("weights", ctypes.c_int), ("msdcn_mode", ctypes.c_int)]
 
 
 _lib = None
@@ -57,6 +60,8 @@ def load(path=LIBRARY):
     lib.dcn4_forward.argtypes = [P, vp, vp, vp, vp]
     lib.dcn4_backward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.dcn4_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.msdcn_backward.argtypes = [P, vp, vp, vp, ctypes.POINTER(ctypes.c_float), ctypes.c_float,
+                                   vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.msdcn_forward.argtypes = [P, vp, vp, vp, ctypes.POINTER(ctypes.c_float), ctypes.c_float,
                                   vp, vp]
     lib.dcn4_status_string.argtypes = [st]
@@ -77,14 +82,15 @@ def _pair(v):
 
 
 def make_desc(N, H, W, C, G, dtype, kernel_size=3, stride=1, pad=1, dilation=1,
-              offset_scale=1.0, algo="auto", math="default"):
+              offset_scale=1.0, algo="auto", math="default", softmax=False, msdcn_mode="offset"):
     kh, kw = _pair(kernel_size)
     sh, sw = _pair(stride)
     ph, pw = _pair(pad)
     dh, dw = _pair(dilation)
     code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     return Desc(N, H, W, C, G, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale), code,
-                ALGO_CODE[algo], MATH_CODE[math])
+                ALGO_CODE[algo], MATH_CODE[math], 1 if softmax else 0,
+                MSDCN_MODE_CODE[msdcn_mode])
 
 
 def _check(fn, rc):
@@ -118,16 +124,19 @@ def _require(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo, math="default"):
+def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo, math="default",
+              softmax=False, msdcn_mode="offset"):
     N, H, W, C = inp.shape
     return make_desc(N, H, W, C, group, inp.dtype, kernel_size, stride, pad, dilation,
-                     offset_scale, algo, math)
+                     offset_scale, algo, math, softmax, msdcn_mode)
 
 
 def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, dilation=1,
-                 offset_scale=1.0, algo="auto", out=None, math="default"):
-    """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3]."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
+                 offset_scale=1.0, algo="auto", out=None, math="default", softmax=False):
+    """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3].
+    softmax=True normalises m over the taps (DCNv3 weights)."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     softmax)
     ho, wo = dcn4_out_shape(desc)
     N, _, _, C = input.shape
     _require(input, "input", input.dtype)
@@ -150,9 +159,10 @@ def dcn4_backward_workspace_size(desc):
 
 def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
                   dilation=1, offset_scale=1.0, algo="auto", workspace=None,
-                  grad_input=None, grad_offset_weight=None, math="default"):
+                  grad_input=None, grad_offset_weight=None, math="default", softmax=False):
     """DCNv4 backward -> (grad_input, grad_offset_weight)."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     softmax)
     ho, wo = dcn4_out_shape(desc)
     N, H, W, C = input.shape
     _require(input, "input", input.dtype)
@@ -176,10 +186,11 @@ def dcn4_backward(input, offset_weight, grad_out, group, kernel_size=3, stride=1
 
 def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, stride=1, pad=1,
                           dilation=1, offset_scale=1.0, algo="auto", grad_input=None,
-                          grad_offset_weight=None, math="default"):
+                          grad_offset_weight=None, math="default", softmax=False):
     """dcn4_backward without a caller-supplied workspace: the library's own
     fixed scratch array is used (see include/dcn4.h for its limit)."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     softmax)
     ho, wo = dcn4_out_shape(desc)
     N, H, W, C = input.shape
     _require(input, "input", input.dtype)
@@ -197,9 +208,12 @@ def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, 
 
 
 def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, stride=1, pad=1,
-                  dilation=1, offset_scale=1.0, algo="auto", out=None, math="default"):
-    """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G]."""
-    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math)
+                  dilation=1, offset_scale=1.0, algo="auto", out=None, math="default",
+                  msdcn_mode="offset"):
+    """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G].
+    msdcn_mode "offset" (s * dir) or "dilation" (s * (p_k + dir))."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     False, msdcn_mode)
     ho, wo = dcn4_out_shape(desc)
     N, _, _, C = input.shape
     _require(input, "input", input.dtype)
@@ -216,6 +230,41 @@ def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, 
         ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr,
         float(smax), _ptr(out), _stream(input)))
     return out
+
+
+def msdcn_backward(input, dir_weight, scale_raw, s0, smax, grad_out, group, kernel_size=3,
+                   stride=1, pad=1, dilation=1, offset_scale=1.0, algo="auto", workspace=None,
+                   grad_input=None, grad_dir_weight=None, grad_scale_raw=None, math="default",
+                   msdcn_mode="offset"):
+    """MSDCN backward -> (grad_input, grad_dir_weight, grad_scale_raw)."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     False, msdcn_mode)
+    ho, wo = dcn4_out_shape(desc)
+    N, H, W, C = input.shape
+    _require(input, "input", input.dtype)
+    _require(dir_weight, "dir_weight", input.dtype, (N, ho, wo, group, desc.kh * desc.kw, 3))
+    _require(scale_raw, "scale_raw", input.dtype, (N, ho, wo, group))
+    _require(grad_out, "grad_out", input.dtype, (N, ho, wo, C))
+    s0 = [float(v) for v in (s0.tolist() if isinstance(s0, torch.Tensor) else s0)]
+    if len(s0) != group:
+        raise ValueError("s0 must hold one prior per group")
+    s0_arr = (ctypes.c_float * group)(*s0)
+    if grad_input is None:
+        grad_input = torch.empty_like(input)
+    if grad_dir_weight is None:
+        grad_dir_weight = torch.empty_like(dir_weight)
+    if grad_scale_raw is None:
+        grad_scale_raw = torch.empty_like(scale_raw)
+    need = dcn4_backward_workspace_size(desc)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=input.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("msdcn_backward", load().msdcn_backward(
+        ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr, float(smax),
+        _ptr(grad_out), _ptr(grad_input), _ptr(grad_dir_weight), _ptr(grad_scale_raw), ws_ptr,
+        ws_bytes, _stream(input)))
+    return grad_input, grad_dir_weight, grad_scale_raw
 
 
 def dcn4_status_string(code):

@@ -38,6 +38,9 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
         return false;
     if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16)
         return false;
+    if (d->weights != DCN4_WEIGHTS_PLAIN && d->weights != DCN4_WEIGHTS_SOFTMAX) return false;
+    if (d->msdcn_mode != DCN4_MSDCN_SCALE_OFFSET && d->msdcn_mode != DCN4_MSDCN_SCALE_DILATION)
+        return false;
     int Ho = 0, Wo = 0;
     if (!out_hw(*d, &Ho, &Wo)) return false;
     const int K = d->kh * d->kw;
@@ -48,7 +51,8 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
     if (!(d->offset_scale == d->offset_scale)) return false;  // NaN
     *g = Geometry{d->N, d->H, d->W, d->C, d->G, d->C / d->G, d->kh, d->kw, K,
                   d->stride_h, d->stride_w, d->pad_h, d->pad_w, d->dil_h, d->dil_w,
-                  Ho, Wo, d->offset_scale};
+                  Ho, Wo, d->offset_scale, d->weights == DCN4_WEIGHTS_SOFTMAX ? 1 : 0,
+                  d->msdcn_mode == DCN4_MSDCN_SCALE_DILATION ? 1 : 0};
     return true;
 }
 
@@ -133,9 +137,13 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
     const int R = 4;
     const int smem_max = max_smem_optin() - 1024;  // static shared memory of the kernel
     const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
-    static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
+    // first choice: a 256-pair tile small enough for two CTAs per SM (the
+    // phases of one CTA then overlap the other's); else the largest tile
+    static const int cands[][2] = {{8, 8}, {16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
                                    {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
-    for (auto &c : cands) {
+    const int per_sm = max_smem_per_sm();
+    for (int ci = 0; ci < (int)(sizeof(cands) / sizeof(cands[0])); ++ci) {
+        const int *c = cands[ci];
         const int TH = c[0] < g.Ho ? c[0] : g.Ho;
         const int TW = c[1] < pow2_ceil(g.Wo) ? c[1] : pow2_ceil(g.Wo);
         if (TH * TW * Gc > 512) continue;
@@ -162,6 +170,9 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
         L.hc_magic = (unsigned)(((1ull << 32) + HC - 1) / HC);
         L.smem_bytes = L.bar_off + 16;
         if (L.smem_bytes > smem_max) continue;
+        const bool two = TH * TW * Gc <= 256 && 2 * (L.smem_bytes + 1024 + 1024) <= per_sm;
+        if (ci == 0 && !(two && TH * TW * Gc == 256)) continue;
+        L.threads = two ? 256 : 512;
         *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                         (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
                         L.smem_bytes};
@@ -301,13 +312,21 @@ dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes) {
     return DCN4_OK;
 }
 
-dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *offset_weight,
-                          const void *grad_out, void *grad_input, void *grad_offset_weight,
-                          void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by dcn4_backward and msdcn_backward (ms != nullptr: the FlowDCN
+// multi-scale variant, graw receives the gradient of scale_raw).
+dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *offset_weight,
+                         const void *grad_out, void *grad_input, void *grad_offset_weight,
+                         void *workspace, size_t workspace_bytes, void *stream,
+                         const MsdcnParams *ms, void *graw) {
     Geometry g;
     if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
     if (!input || !offset_weight || !grad_out || !grad_input || !grad_offset_weight)
         return DCN4_ERR_INVALID_ARG;
+    if (ms && !graw) return DCN4_ERR_INVALID_ARG;
     size_t need = 0;
     dcn4_backward_workspace_size(desc, &need);
     if (need > 0 && (!workspace || workspace_bytes < need)) return DCN4_ERR_WORKSPACE;
@@ -323,14 +342,18 @@ dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *
     L.acc = need > 0 ? static_cast<float *>(workspace) : static_cast<float *>(grad_input);
     L.mixed = use_mixed(desc);
     L.stream = static_cast<cudaStream_t>(stream);
+    L.msdcn = ms != nullptr;
+    L.ms = ms;
+    L.graw = graw;
     const int eb = elem_bytes(L.dtype);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * eb;
     CUtensorMap map_in, map_go;
     memset(&map_in, 0, sizeof(map_in));
     memset(&map_go, 0, sizeof(map_go));
     if (desc->algo != DCN4_ALGO_GENERIC) {
-        L.halo = g.kh == 3 && g.kw == 3 && aligned16(input) && aligned16(offset_weight) &&
-                 aligned16(grad_out) && aligned16(L.acc) && plan_bwd(g, eb, &L.plan, &L.layout) &&
+        L.halo = !L.msdcn && g.kh == 3 && g.kw == 3 && aligned16(input) &&
+                 aligned16(offset_weight) && aligned16(grad_out) && aligned16(L.acc) &&
+                 plan_bwd(g, eb, &L.plan, &L.layout) &&
                  encode_input_map(g, L.dtype, input, L.plan, &map_in) &&
                  encode_map(L.dtype, grad_out, g.N, g.Ho, g.Wo, g.C, L.plan.Gc * g.D, L.plan.TW,
                             L.plan.TH, &map_go);
@@ -341,12 +364,41 @@ dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *
     return cuda_status(launch_backward(L));
 }
 
+}  // namespace
+
+extern "C" {
+
+dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input, const void *offset_weight,
+                          const void *grad_out, void *grad_input, void *grad_offset_weight,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    return run_backward(desc, input, offset_weight, grad_out, grad_input, grad_offset_weight,
+                        workspace, workspace_bytes, stream, nullptr, nullptr);
+}
+
+dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input, const void *dir_weight,
+                           const void *scale_raw, const float *s0_host, float smax,
+                           const void *grad_out, void *grad_input, void *grad_dir_weight,
+                           void *grad_scale_raw, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    Geometry g;
+    if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
+    if (!s0_host || !scale_raw || !grad_scale_raw) return DCN4_ERR_INVALID_ARG;
+    if (g.softmax) return DCN4_ERR_UNSUPPORTED;
+    static thread_local MsdcnParams ms;
+    ms.raw = scale_raw;
+    ms.smax = smax;
+    for (int i = 0; i < g.G; ++i) ms.s0[i] = s0_host[i];
+    return run_backward(desc, input, dir_weight, grad_out, grad_input, grad_dir_weight,
+                        workspace, workspace_bytes, stream, &ms, grad_scale_raw);
+}
+
 dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input, const void *dir_weight,
                           const void *scale_raw, const float *s0_host, float smax, void *output,
                           void *stream) {
     Geometry g;
     if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
     if (!s0_host || !scale_raw) return DCN4_ERR_INVALID_ARG;
+    if (g.softmax) return DCN4_ERR_UNSUPPORTED;
     static thread_local MsdcnParams ms;
     ms.raw = scale_raw;
     ms.smax = smax;

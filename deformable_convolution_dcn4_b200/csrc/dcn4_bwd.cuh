@@ -16,10 +16,15 @@
 namespace dcn4 {
 
 // One thread per (pixel, group); scalar loads; any shape and alignment.
-template <typename T>
+// MS: the FlowDCN multi-scale variant ("3.1"): ow holds (dir_x, dir_y, m),
+// the offset is s * dir with s = msdcn_scale(raw); by the chain rule
+// d/d dir = s * d/d offset and d/d raw = (ds/draw) * sum_k <d/d offset_k, dir_k>,
+// written to graw [N][Ho][Wo][G].
+template <typename T, bool MS>
 __global__ void __launch_bounds__(256)
 bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
-                   const T *__restrict__ gout, float *__restrict__ gin, T *__restrict__ gow) {
+                   const T *__restrict__ gout, float *__restrict__ gin, T *__restrict__ gow,
+                   const __grid_constant__ MsdcnParams ms, T *__restrict__ graw) {
     const long long total = (long long)g.N * g.Ho * g.Wo * g.G;
     const size_t img = (size_t)g.H * g.W * g.C;
     for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < total;
@@ -35,14 +40,35 @@ bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
         const T *go = gout + (size_t)pix * g.C + (size_t)grp * g.D;
         const T *src = in + (size_t)n * img + (size_t)grp * g.D;
         float *dst = gin + (size_t)n * img + (size_t)grp * g.D;
+        float s = 1.0f, gs = 0.0f;
+        if (MS) s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[t]), ms.s0[grp], ms.smax);
+        // DCNv3 weights: softmax over the taps; the gradients with respect to
+        // the weights are kept (fp32, up to kMaxTaps) to form the logit
+        // gradient w_k (gw_k - sum_j w_j gw_j) after the loop
+        SoftmaxNorm sn{0.0f, 1.0f};
+        float gwk[kMaxTaps];
+        float dotw = 0.0f;
+        if (!MS && g.softmax) {
+            float mx = -INFINITY, sum = 0.0f;
+            for (int k = 0; k < g.K; ++k) mx = fmaxf(mx, Elem<T>::to_f(rec[3 * k + 2]));
+            for (int k = 0; k < g.K; ++k) sum += expf(Elem<T>::to_f(rec[3 * k + 2]) - mx);
+            sn = SoftmaxNorm{mx, 1.0f / sum};
+        }
         for (int i = 0; i < g.kh; ++i) {
             for (int j = 0; j < g.kw; ++j) {
                 const int k = i * g.kw + j;
                 const float dx = Elem<T>::to_f(rec[3 * k]);
                 const float dy = Elem<T>::to_f(rec[3 * k + 1]);
-                const float m = Elem<T>::to_f(rec[3 * k + 2]);
-                const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
-                const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+                float m = Elem<T>::to_f(rec[3 * k + 2]);
+                if (!MS && g.softmax) m = sn.weight(m);
+                float x, y, dsx = 0.0f, dsy = 0.0f;  // ds*: d position / d s (MSDCN)
+                if (MS) {
+                    x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, j, g.kw, g.dw, s, dx, g.os, &dsx);
+                    y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, i, g.kh, g.dh, s, dy, g.os, &dsy);
+                } else {
+                    x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+                    y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+                }
                 float gx = 0.0f, gy = 0.0f, gm = 0.0f;
                 if (x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H) {
                     const float x0f = floorf(x), y0f = floorf(y);
@@ -70,10 +96,25 @@ bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
                         }
                     }
                 }
-                grec[3 * k] = Elem<T>::from_f(g.os * m * gx);
-                grec[3 * k + 1] = Elem<T>::from_f(g.os * m * gy);
-                grec[3 * k + 2] = Elem<T>::from_f(gm);
+                const float tx = g.os * m * gx, ty = g.os * m * gy;  // d/d offset
+                grec[3 * k] = Elem<T>::from_f(MS ? s * tx : tx);
+                grec[3 * k + 1] = Elem<T>::from_f(MS ? s * ty : ty);
+                if (!MS && g.softmax) {
+                    gwk[k] = gm;
+                    dotw = fmaf(m, gm, dotw);
+                } else {
+                    grec[3 * k + 2] = Elem<T>::from_f(gm);
+                }
+                if (MS) gs = fmaf(m * gx, dsx, fmaf(m * gy, dsy, gs));
             }
+        }
+        if (!MS && g.softmax)
+            for (int k = 0; k < g.K; ++k)
+                grec[3 * k + 2] = Elem<T>::from_f(
+                    sn.weight(Elem<T>::to_f(rec[3 * k + 2])) * (gwk[k] - dotw));
+        if (MS) {
+            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[t]);
+            graw[t] = Elem<T>::from_f(gs == 0.0f ? 0.0f : gs * msdcn_scale_grad(raw, ms.s0[grp], ms.smax));
         }
     }
 }

@@ -197,7 +197,7 @@ __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *wa
 // are rounded once to T and added with packed 16-bit reductions (no fp32
 // workspace). Otherwise sums go to the fp32 workspace `gacc`.
 template <typename T, int U, int NW, bool MIXED, bool DIRECT>
-__global__ void __launch_bounds__(NW * 32, 1)
+__global__ void __launch_bounds__(NW * 32, 512 / (NW * 32))
 bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const __grid_constant__ CUtensorMap tmap_go, Geometry g, HaloPlan pl,
                 BwdLayout L, const T *__restrict__ in, const T *__restrict__ ow,
@@ -314,6 +314,26 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     if (valid) {
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
         RecordReader<T>::read(rec, v);
+        // DCNv3 weights: softmax of the logits over the taps; the logit
+        // gradient w_k (gw_k - sum_j w_j gw_j) is formed after the taps from
+        // the staged gw_k
+        SoftmaxNorm sn{0.0f, 1.0f};
+        if (g.softmax) {
+            float mx = v[2];
+#pragma unroll
+            for (int k = 1; k < 9; ++k) mx = fmaxf(mx, v[3 * k + 2]);
+            float sum = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 9; ++k) {
+                v[3 * k + 2] = expf(v[3 * k + 2] - mx);
+                sum += v[3 * k + 2];
+            }
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int k = 0; k < 9; ++k) v[3 * k + 2] *= inv;
+            sn = SoftmaxNorm{mx, inv};
+        }
+        float dotw = 0.0f;
         const unsigned char *row0[U], *row1[U];
         // gof[c]: this pair's grad_out chunk (c + r) mod U, unpacked to fp32
         float gof[U][VE];
@@ -370,6 +390,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             gout_rec[3 * k] = Elem<T>::from_f(gx);
             gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
             gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            dotw = fmaf(m, gm, dotw);
         }
         // samples outside the staged window: global gathers, fp32 atomics
         const T *gsrc = in + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D;
@@ -380,6 +401,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const int i = k / 3, j = k - 3 * (k / 3);
             float dx, dy, m;
             record_tap<T>(rec, k, dx, dy, m);
+            if (g.softmax) m = sn.weight(m);
             const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
             const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
             float gx = 0.f, gy = 0.f, gm = 0.f;
@@ -424,6 +446,13 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             gout_rec[3 * k] = Elem<T>::from_f(gx);
             gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
             gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            dotw = fmaf(m, gm, dotw);
+        }
+        if (g.softmax) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k)
+                gout_rec[3 * k + 2] =
+                    Elem<T>::from_f(v[3 * k + 2] * (Elem<T>::to_f(gout_rec[3 * k + 2]) - dotw));
         }
     }
     __syncthreads();  // window reads, counts and gows staging complete
@@ -450,14 +479,26 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     // ---------------- E: grad_offset_weight out (one warp per pixel) ----------------
     {
         const int npix = pl.TH * pl.TW;
-        const int span = pl.Gc * 27;  // elements per pixel
+        const int span = pl.Gc * 27 * EB;  // bytes per pixel, contiguous in gow
         for (int p = threadIdx.x >> 5; p < npix; p += NW) {
             const int ty = p >> pl.lgTW, tx = p & (pl.TW - 1);
             if (ty >= tc.th_eff || tx >= tc.tw_eff) continue;
             const unsigned long long q = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
-            T *dst = gow + (q * g.G + tc.g0) * 27;
-            const T *src = gows + (size_t)p * span;
-            for (int e = lane; e < span; e += 32) dst[e] = src[e];
+            unsigned char *dst = reinterpret_cast<unsigned char *>(gow + (q * g.G + tc.g0) * 27);
+            const unsigned char *src = reinterpret_cast<const unsigned char *>(gows) + (size_t)p * span;
+            // widest word that divides both addresses and the span
+            const unsigned al = (unsigned)(reinterpret_cast<uintptr_t>(dst) |
+                                           reinterpret_cast<uintptr_t>(src) | (uintptr_t)span);
+            if ((al & 7) == 0) {
+                for (int e = lane * 8; e < span; e += 256)
+                    *reinterpret_cast<uint2 *>(dst + e) = *reinterpret_cast<const uint2 *>(src + e);
+            } else if ((al & 3) == 0) {
+                for (int e = lane * 4; e < span; e += 128)
+                    *reinterpret_cast<unsigned *>(dst + e) = *reinterpret_cast<const unsigned *>(src + e);
+            } else {
+                for (int e = lane * EB; e < span; e += 32 * EB)
+                    *reinterpret_cast<T *>(dst + e) = *reinterpret_cast<const T *>(src + e);
+            }
         }
     }
 

@@ -16,6 +16,7 @@ constexpr unsigned kErrInternal = 2u;  // a consistency check failed
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
 constexpr int kMaxGroups = 1024;
+constexpr int kMaxTaps = 64;  // kh * kw
 
 // Problem geometry, copied into every launch.
 struct Geometry {
@@ -23,10 +24,29 @@ struct Geometry {
     int kh, kw, K;
     int sh, sw, ph, pw, dh, dw;
     int Ho, Wo;
-    float os;  // offset_scale
+    float os;     // offset_scale
+    int softmax;  // DCNv3 weights: softmax of m over the K taps
+    int msd_dil;  // MSDCN scale-as-dilation reading
 };
 
 // MSDCN extras: per-group scale priors travel inside the launch parameters.
+// s = min(s0 * softplus(raw), smax), softplus(r) = max(r, 0) + log1p(exp(-|r|)).
+__device__ __forceinline__ float msdcn_scale(float raw, float s0, float smax) {
+    float sp = __fadd_rn(fmaxf(raw, 0.0f), log1pf(expf(-fabsf(raw))));
+    float s = __fmul_rn(s0, sp);
+    return (s > smax) ? smax : s;
+}
+
+// d s / d raw for the scale above: s0 * sigmoid(raw) (sigmoid is the
+// derivative of softplus) while s0 * softplus(raw) <= smax, the branch
+// msdcn_scale keeps; 0 once the clamp is active or raw is NaN.
+__device__ __forceinline__ float msdcn_scale_grad(float raw, float s0, float smax) {
+    const float sp = __fadd_rn(fmaxf(raw, 0.0f), log1pf(expf(-fabsf(raw))));
+    const float u = __fmul_rn(s0, sp);
+    if (!(u <= smax)) return 0.0f;
+    return s0 / (1.0f + expf(-raw));
+}
+
 struct MsdcnParams {
     const void *raw;  // [N][Ho][Wo][G] in the element type
     float smax;
@@ -45,6 +65,7 @@ struct BwdLayout {
     int max_samples;  // TH*TW*Gc*9; sorted sample records reuse the window
     unsigned hc_magic;  // ceil(2^32 / HC): q / HC == __umulhi(q, hc_magic) for q < 2^16
     int smem_bytes;
+    int threads;      // 256 (two CTAs per SM) or 512
 };
 
 // Tiling of the shared-memory halo kernels (chosen on the host).
@@ -87,6 +108,33 @@ template <> struct Elem<__half> {
 __device__ __forceinline__ float sample_coord(int base, float delta, float os) {
     return __fadd_rn((float)base, __fmul_rn(delta, os));
 }
+
+// MSDCN sample coordinate along one axis for tap index t (j along W, i along
+// H) of a window of `kt` taps with dilation `dil`, output base
+// `base` = o*stride - pad, scale s and direction d:
+//   scale-as-offset  base + t*dil + (s*d)*os
+//   scale-as-dilation  c + s*(p_t + d*os), c = base + (kt-1)/2 * dil the
+//                      window centre, p_t = (t - (kt-1)/2) * dil
+// (each product and sum rounded to fp32). *ds receives d coord / d s.
+__device__ __forceinline__ float msdcn_coord(bool dilation, int base, int t, int kt, int dil,
+                                             float s, float d, float os, float *ds) {
+    if (!dilation) {
+        *ds = __fmul_rn(d, os);
+        return sample_coord(base + t * dil, __fmul_rn(s, d), os);
+    }
+    const float c = (float)base + 0.5f * (float)((kt - 1) * dil);
+    const float p = ((float)t - 0.5f * (float)(kt - 1)) * (float)dil;
+    const float u = __fadd_rn(p, __fmul_rn(d, os));
+    *ds = u;
+    return __fadd_rn(c, __fmul_rn(s, u));
+}
+
+// DCNv3 weights: softmax over the K logits m of one (pixel, group); the
+// weight of logit m is expf(m - mx) * inv.
+struct SoftmaxNorm {
+    float mx, inv;
+    __device__ __forceinline__ float weight(float m) const { return expf(m - mx) * inv; }
+};
 
 // ---- fp32 accumulation of 16-byte vectors -------------------------------
 // acc[0..kPerVec) += w * (16-byte vector v of T), fp32 arithmetic, using the

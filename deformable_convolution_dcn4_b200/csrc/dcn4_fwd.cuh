@@ -28,12 +28,6 @@ namespace dcn4 {
 
 // The device error word (defined once, in dcn4_kernels.cu, before this file).
 
-// s = min(s0 * softplus(raw), smax), softplus(r) = max(r, 0) + log1p(exp(-|r|)).
-__device__ __forceinline__ float msdcn_scale(float raw, float s0, float smax) {
-    float sp = __fadd_rn(fmaxf(raw, 0.0f), log1pf(expf(-fabsf(raw))));
-    float s = __fmul_rn(s0, sp);
-    return (s > smax) ? smax : s;
-}
 
 // ------------------------------------------------------------------------
 // Generic kernel
@@ -64,6 +58,13 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
             const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[pix * g.G + grp]);
             s = msdcn_scale(raw, ms.s0[grp], ms.smax);
         }
+        SoftmaxNorm sn{0.0f, 1.0f};
+        if (!MS && g.softmax) {
+            float mx = -INFINITY, sum = 0.0f;
+            for (int k = 0; k < g.K; ++k) mx = fmaxf(mx, Elem<T>::to_f(rec[3 * k + 2]));
+            for (int k = 0; k < g.K; ++k) sum += expf(Elem<T>::to_f(rec[3 * k + 2]) - mx);
+            sn = SoftmaxNorm{mx, 1.0f / sum};
+        }
         float acc[CH];
 #pragma unroll
         for (int d = 0; d < CH; ++d) acc[d] = 0.0f;
@@ -71,15 +72,18 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
         for (int i = 0; i < g.kh; ++i) {
             for (int j = 0; j < g.kw; ++j) {
                 const int k = i * g.kw + j;
-                float dx = Elem<T>::to_f(rec[3 * k]);
-                float dy = Elem<T>::to_f(rec[3 * k + 1]);
-                const float m = Elem<T>::to_f(rec[3 * k + 2]);
+                const float dx = Elem<T>::to_f(rec[3 * k]);
+                const float dy = Elem<T>::to_f(rec[3 * k + 1]);
+                float m = Elem<T>::to_f(rec[3 * k + 2]);
+                if (!MS && g.softmax) m = sn.weight(m);
+                float x, y, dsx, dsy;
                 if (MS) {
-                    dx = __fmul_rn(s, dx);
-                    dy = __fmul_rn(s, dy);
+                    x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, j, g.kw, g.dw, s, dx, g.os, &dsx);
+                    y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, i, g.kh, g.dh, s, dy, g.os, &dsy);
+                } else {
+                    x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+                    y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
                 }
-                const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
-                const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
                 if (!(x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H)) continue;
                 const float x0f = floorf(x), y0f = floorf(y);
                 const float lx = x - x0f, ly = y - y0f;
@@ -310,14 +314,33 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
         float v[27];
         RecordReader<T>::read(rec, v);
         float s = 1.0f;
+        const bool dil = MS && g.msd_dil;
         if (MS) {
             const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]);
             s = msdcn_scale(raw, ms.s0[tc.g0 + gl], ms.smax);
+            if (!dil) {
+#pragma unroll
+                for (int k = 0; k < 9; ++k) {
+                    v[3 * k] = __fmul_rn(s, v[3 * k]);
+                    v[3 * k + 1] = __fmul_rn(s, v[3 * k + 1]);
+                }
+            }
+        }
+        SoftmaxNorm sn{0.0f, 1.0f};
+        if (!MS && g.softmax) {
+            float mx = v[2];
+#pragma unroll
+            for (int k = 1; k < 9; ++k) mx = fmaxf(mx, v[3 * k + 2]);
+            float sum = 0.0f;
 #pragma unroll
             for (int k = 0; k < 9; ++k) {
-                v[3 * k] = __fmul_rn(s, v[3 * k]);
-                v[3 * k + 1] = __fmul_rn(s, v[3 * k + 1]);
+                v[3 * k + 2] = expf(v[3 * k + 2] - mx);
+                sum += v[3 * k + 2];
             }
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int k = 0; k < 9; ++k) v[3 * k + 2] *= inv;
+            sn = SoftmaxNorm{mx, inv};
         }
         // chunk rotation: the 8 lanes of a shared-memory phase start at
         // different 16-byte chunks, so their loads hit 8 different bank quads
@@ -340,8 +363,16 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
         unsigned esc = 0;
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
-            const float x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
-            const float y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            float x, y;
+            if (dil) {  // centre + s * (grid offset + dir * os)
+                x = __fadd_rn(bxs[1], __fmul_rn(s, __fadd_rn((float)(k % 3 - 1) * dwf,
+                                                              __fmul_rn(v[3 * k], g.os))));
+                y = __fadd_rn(bys[1], __fmul_rn(s, __fadd_rn((float)(k / 3 - 1) * dhf,
+                                                              __fmul_rn(v[3 * k + 1], g.os))));
+            } else {
+                x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
+                y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            }
             const float m = v[3 * k + 2];
             if (x >= hx_lo && x < hx_hi && y >= hy_lo && y < hy_hi) {
                 const float x0f = floorf(x), y0f = floorf(y);
@@ -383,13 +414,16 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
             esc &= esc - 1;
             float dx, dy, m;
             record_tap<T>(rec, k, dx, dy, m);
-            if (MS) {
-                dx = __fmul_rn(s, dx);
-                dy = __fmul_rn(s, dy);
-            }
+            if (!MS && g.softmax) m = sn.weight(m);
             const int i = k / 3, j = k - 3 * (k / 3);
-            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
-            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            float x, y, dsx, dsy;
+            if (MS) {
+                x = msdcn_coord(dil, wo * g.sw - g.pw, j, 3, g.dw, s, dx, g.os, &dsx);
+                y = msdcn_coord(dil, ho * g.sh - g.ph, i, 3, g.dh, s, dy, g.os, &dsy);
+            } else {
+                x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+                y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            }
             if (!(x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H)) continue;
             const float x0f = floorf(x), y0f = floorf(y);
             const float lx = x - x0f, ly = y - y0f;

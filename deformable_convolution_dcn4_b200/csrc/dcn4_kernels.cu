@@ -24,6 +24,9 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Kernel argument for launches without the multi-scale variant.
+const MsdcnParams kNoMs = {};
+
 // Kernels this library has issued (launched or captured into a graph).
 std::atomic<unsigned long long> g_launches{0};
 inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -80,7 +83,6 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
     if (occ < 1) return cudaErrorInvalidConfiguration;
     long long grid = (long long)sm_count() * occ;
     if (grid > tiles) grid = tiles;
-    static const MsdcnParams kNoMs = {};
     k<<<(unsigned)grid, NT, L.plan.smem_bytes, L.stream>>>(
         *L.tmap, L.geo, L.plan, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
         static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
@@ -125,7 +127,6 @@ cudaError_t launch_halo_u(const FwdLaunch &L) {
 template <typename T, bool MS>
 cudaError_t launch_generic_t(const FwdLaunch &L) {
     const long long work = (long long)L.geo.N * L.geo.Ho * L.geo.Wo * L.geo.G * ((L.geo.D + 7) / 8);
-    static const MsdcnParams kNoMs = {};
     fwd_generic_kernel<T, MS><<<grid_for(work, 256), 256, 0, L.stream>>>(
         L.geo, static_cast<const T *>(L.in), static_cast<const T *>(L.ow), static_cast<T *>(L.out),
         L.ms ? *L.ms : kNoMs);
@@ -143,10 +144,11 @@ template <typename T>
 cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
     const int U = L.geo.D * (int)sizeof(T) / 16;
     const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
+    const int nt = L.layout.threads;
     auto run = [&](auto kernel) {
         cudaError_t e = allow_smem(reinterpret_cast<const void *>(kernel), L.layout.smem_bytes);
         if (e != cudaSuccess) return e;
-        kernel<<<(unsigned)grid, 512, L.layout.smem_bytes, L.stream>>>(
+        kernel<<<(unsigned)grid, nt, L.layout.smem_bytes, L.stream>>>(
             *L.tmap_in, *L.tmap_go, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
             static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, static_cast<T *>(L.gin),
             L.ow_bytes);
@@ -154,12 +156,18 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
         return cudaGetLastError();
     };
     if constexpr (sizeof(T) == 2) {
+        if (U == 2 && nt == 256) {
+            if (direct) return run(bwd_halo_kernel<T, 2, 8, true, true>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 8, true, false>)
+                           : run(bwd_halo_kernel<T, 2, 8, false, false>);
+        }
         if (U == 2) {
             if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true>);
             return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false>)
                            : run(bwd_halo_kernel<T, 2, 16, false, false>);
         }
     }
+    if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false>);
     if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false>);
     return cudaErrorInvalidValue;
 }
@@ -188,9 +196,15 @@ cudaError_t launch_bwd_t(const BwdLaunch &L) {
         e = launch_bwd_halo<T>(L, false);
     } else {
         const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
-        bwd_generic_kernel<T><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
-            g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
-            static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow));
+        if (L.msdcn)
+            bwd_generic_kernel<T, true><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
+                g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+                static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow), *L.ms,
+                static_cast<T *>(L.graw));
+        else
+            bwd_generic_kernel<T, false><<<grid_for(pairs, 256), 256, 0, L.stream>>>(
+                g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+                static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow), kNoMs, nullptr);
         count_launch();
         e = cudaGetLastError();
     }
@@ -232,6 +246,12 @@ int sm_count() {
     static int cache[kMaxDevices] = {0};
     int v = cached_attr(cudaDevAttrMultiProcessorCount, cache);
     return v > 0 ? v : 148;
+}
+
+int max_smem_per_sm() {
+    static int cache[kMaxDevices] = {0};
+    int v = cached_attr(cudaDevAttrMaxSharedMemoryPerMultiprocessor, cache);
+    return v > 0 ? v : 64 * 1024;
 }
 
 int max_smem_optin() {

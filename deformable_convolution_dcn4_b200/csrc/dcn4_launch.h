@@ -43,6 +43,9 @@ struct BwdLaunch {
     const CUtensorMap *tmap_go;
     unsigned long long ow_bytes;
     cudaStream_t stream;
+    bool msdcn;             // FlowDCN multi-scale variant: ow holds (dir_x, dir_y, m)
+    const MsdcnParams *ms;  // MSDCN only
+    void *graw;             // MSDCN only: grad of scale_raw [N][Ho][Wo][G], element type
 };
 
 cudaError_t launch_forward(const FwdLaunch &L);
@@ -61,5 +64,7 @@ unsigned long long launches_issued();
 int sm_count();
 // Largest opt-in dynamic shared memory per block of the current device.
 int max_smem_optin();
+// Shared memory per SM of the current device.
+int max_smem_per_sm();
 
 }  // namespace dcn4

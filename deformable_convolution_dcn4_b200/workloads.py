@@ -47,6 +47,8 @@ class Workload:
     kind: str = "dcn4"                                   # "dcn4" | "msdcn"
     smax: float = 8.0
     seed: int = 0
+    softmax: bool = False                                # DCNv3 weights (DCNv4 kind only)
+    msdcn_mode: str = "offset"                           # "offset" | "dilation" (MSDCN only)
 
     @property
     def D(self):

@@ -89,6 +89,25 @@ typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } d
  * the mixed-precision fma in every mode; there it is exact. */
 typedef enum { DCN4_MATH_DEFAULT = 0, DCN4_MATH_F32 = 1, DCN4_MATH_MIXED16 = 2 } dcn4_math;
 
+/* Aggregation weights ("(论文速读）DCNv4：高效可变形卷积算子", "移除Softmax归一化"):
+ *   PLAIN    DCNv4: m is used as given (unbounded, no normalisation).
+ *   SOFTMAX  DCNv3 compatibility: the K values m of one (pixel, group) are
+ *            replaced by softmax(m) over the taps (largest subtracted first,
+ *            fp32 expf); the backward returns the gradient with respect to
+ *            the logits m. DCNv4 calls only (MSDCN returns UNSUPPORTED). */
+typedef enum { DCN4_WEIGHTS_PLAIN = 0, DCN4_WEIGHTS_SOFTMAX = 1 } dcn4_weights;
+
+/* Where the MSDCN scale acts ("NeurIPS'24 | FlowDCN", "3.1"; the page's
+ * formula is missing and both readings fit its text):
+ *   SCALE_OFFSET    the offset is s * dir: sample = p0 + p_k + s*dir*os.
+ *   SCALE_DILATION  the scale stretches the kernel grid too:
+ *                   sample = c + s * (p_k + dir*os), c the centre of the
+ *                   kh x kw window, p_k the tap's grid offset from it
+ *                   ((j - (kw-1)/2) * dil_w, (i - (kh-1)/2) * dil_h);
+ *                   every product and sum rounded to fp32 in that order.
+ * DCNv4 calls ignore this field. */
+typedef enum { DCN4_MSDCN_SCALE_OFFSET = 0, DCN4_MSDCN_SCALE_DILATION = 1 } dcn4_msdcn_mode;
+
 /* The whole configuration of one call. Limits: all sizes positive, C % G == 0,
  * G <= 1024, 1 <= kh*kw <= 64, strides and dilations >= 1, pads >= 0, every
  * tensor below 2^31 elements, Ho and Wo positive. */
@@ -102,6 +121,8 @@ typedef struct {
     dcn4_dtype dtype;
     dcn4_algo algo;
     dcn4_math math;
+    dcn4_weights weights;
+    dcn4_msdcn_mode msdcn_mode;
 } dcn4_desc;
 
 /* Output size for `desc` (standard convolution arithmetic, as in
@@ -153,6 +174,29 @@ DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
                           const void *dir_weight, const void *scale_raw,
                           const float *s0_host, float smax, void *output,
                           void *stream);
+
+/* MSDCN backward: the derivative of msdcn_forward (FlowDCN article, "3.1";
+ * the page prints no gradient, these follow by the chain rule). With
+ * g_x, g_y the derivatives of sum(output * grad_out) with respect to the
+ * sample position of tap k (computed as in dcn4_backward):
+ *   grad_input        [N][H][W][C]           as in dcn4_backward
+ *   grad_dir_weight   [N][Ho][Wo][G][kh*kw][3]
+ *       d/d dir_x = s * offset_scale * g_x, d/d dir_y = s * offset_scale * g_y,
+ *       d/d m as in dcn4_backward
+ *   grad_scale_raw    [N][Ho][Wo][G]
+ *       (ds/draw) * offset_scale * sum_k (g_x dir_x + g_y dir_y), where
+ *       ds/draw = s0 * sigmoid(raw) while s0 * softplus(raw) <= smax and 0
+ *       once the clamp is active (or raw is NaN).
+ * Arguments as in msdcn_forward and dcn4_backward (grad outputs in
+ * desc->dtype, device; the same workspace size, dcn4_backward_workspace_size).
+ * This version runs one thread per (pixel, group) with fp32 atomics into the
+ * workspace (fp32 data: into grad_input); DCN4_ALGO_HALO returns
+ * DCN4_ERR_UNSUPPORTED. */
+DCN4_API dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input,
+                          const void *dir_weight, const void *scale_raw,
+                          const float *s0_host, float smax, const void *grad_out,
+                          void *grad_input, void *grad_dir_weight, void *grad_scale_raw,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /* dcn4_backward for callers that cannot allocate device memory. The paper
  * has no counterpart; this is a deployment convenience. dcn4_backward needs

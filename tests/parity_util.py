@@ -27,8 +27,13 @@ def f32(t):
 
 
 def desc_kw(wl):
-    return dict(kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
-                offset_scale=wl.offset_scale)
+    kw = dict(kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
+              offset_scale=wl.offset_scale)
+    if wl.kind == "msdcn":
+        kw["msdcn_mode"] = wl.msdcn_mode
+    else:
+        kw["softmax"] = wl.softmax
+    return kw
 
 
 def out_hw(wl):
@@ -39,7 +44,8 @@ def out_hw(wl):
 
 def problem(orc, wl, N=None):
     return orc.problem(N or wl.N, wl.H, wl.W, wl.C, wl.G, wl.kh, wl.kw, wl.stride, wl.pad,
-                       wl.dilation, wl.offset_scale)
+                       wl.dilation, wl.offset_scale, softmax=wl.softmax,
+                       msdcn_dilation=wl.msdcn_mode == "dilation")
 
 
 def gpu_forward(wl, data, algo="auto"):
@@ -87,6 +93,25 @@ def backward_case(orc, wl, algo="auto", images=None, math="default"):
     if images is not None:
         gin, gow = gin[list(images)], gow[list(images)]
     return scaled_err(gin, rgin), scaled_err(gow, rgow)
+
+
+def msdcn_backward_case(orc, wl, algo="auto", images=None, math="default"):
+    """Scaled errors of (grad_input, grad_dir_weight, grad_scale_raw)."""
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    dev = "cuda"
+    gin, gdw, graw = B.msdcn_backward(data["input"].to(dev), data["dir_weight"].to(dev),
+                                      data["scale_raw"].to(dev), data["s0"], wl.smax,
+                                      data["grad_out"].to(dev), group=wl.G, algo=algo, math=math,
+                                      **desc_kw(wl))
+    sel = slice(None) if images is None else list(images)
+    n = wl.N if images is None else len(images)
+    r = orc.msdcn_backward(problem(orc, wl, n), f32(data["input"][sel]),
+                           f32(data["dir_weight"][sel]), f32(data["scale_raw"][sel]),
+                           data["s0"].numpy(), wl.smax, f32(data["grad_out"][sel]))
+    got = [f32(gin), f32(gdw), f32(graw)]
+    if images is not None:
+        got = [t[list(images)] for t in got]
+    return tuple(scaled_err(a, b) for a, b in zip(got, r))
 
 
 def cuda_sync():

@@ -9,7 +9,7 @@ import torch
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
 
-from parity_util import (TOL, backward_case, f32, forward_case, gpu_forward, oracle_forward,
+from parity_util import (TOL, backward_case, msdcn_backward_case, f32, forward_case, gpu_forward, oracle_forward,
                          out_hw, problem, scaled_err)
 
 pytestmark = pytest.mark.gpu
@@ -314,3 +314,104 @@ def test_launch_counter_counts_each_kernel():
     n3 = B.dcn4_kernel_launches()
     torch.cuda.synchronize()
     assert (n1 - n0, n2 - n1, n3 - n2) == (1, 2, 3)
+
+
+MSDCN_BWD = {
+    "flowdcn_msdcn_bf16": REDUCED["flowdcn_msdcn_bf16"].replace(N=1),
+    "msdcn_d16_bf16": W["internimage_bf16"].replace(name="msd16", N=1, H=20, W=24, kind="msdcn",
+                                                    offset_dist=("normal", 1.0), smax=8.0),
+    "msdcn_d16_f32": W["internimage_f32"].replace(name="msd16f", N=1, H=13, W=17, kind="msdcn",
+                                                  offset_dist=("normal", 1.0), smax=3.0),
+    "msdcn_stride_f16": W["ldm64_f16"].replace(name="msds", N=2, H=15, W=11, C=32, G=4,
+                                               kind="msdcn", offset_dist=("normal", 1.0),
+                                               stride=(2, 1), pad=(0, 1), dilation=(1, 2),
+                                               offset_scale=0.5, smax=2.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MSDCN_BWD))
+@pytest.mark.parametrize("math", ["default", "f32"])
+def test_msdcn_backward(orc, name, math):
+    wl = MSDCN_BWD[name]
+    errs = msdcn_backward_case(orc, wl, math=math)
+    tol = TOL[wl.dtype]
+    assert all(e <= tol for e in errs), f"{name}: grad_input/dir/raw errors {errs}"
+
+
+def test_msdcn_backward_full_size_sampled(orc):
+    wl = W["flowdcn_msdcn_bf16"]
+    errs = msdcn_backward_case(orc, wl, images=[0, 31])
+    assert all(e <= TOL["bf16"] for e in errs), errs
+
+
+def test_msdcn_backward_halo_request_is_unsupported():
+    wl = MSDCN_BWD["msdcn_d16_bf16"]
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    with pytest.raises(B.Dcn4Error) as e:
+        B.msdcn_backward(data["input"].cuda(), data["dir_weight"].cuda(), data["scale_raw"].cuda(),
+                         data["s0"], wl.smax, data["grad_out"].cuda(), group=wl.G, algo="halo")
+    assert e.value.code == 2
+
+
+# DCNv3 compatibility (softmax over the taps) and the MSDCN scale-as-dilation
+# reading, against the oracle's own definitions of both
+SOFTMAX = {
+    "softmax_bf16": W["internimage_bf16"].replace(name="sm", N=2, H=20, W=24, softmax=True,
+                                                  weight_sigma=1.0),
+    "softmax_f32": W["internimage_f32"].replace(name="smf", N=1, H=13, W=17, softmax=True,
+                                                weight_sigma=1.0),
+    "softmax_f16_stride": W["ldm64_f16"].replace(name="sms", N=1, H=15, W=11, C=64, G=4,
+                                                 stride=(2, 1), pad=(1, 2), dilation=(1, 2),
+                                                 softmax=True, weight_sigma=2.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SOFTMAX))
+@pytest.mark.parametrize("algo", ["auto", "generic"])
+def test_softmax_forward(orc, name, algo):
+    wl = SOFTMAX[name]
+    err = forward_case(orc, wl, algo)
+    assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", sorted(SOFTMAX))
+@pytest.mark.parametrize("algo", ["auto", "generic"])
+def test_softmax_backward(orc, name, algo):
+    wl = SOFTMAX[name]
+    e_in, e_ow = backward_case(orc, wl, algo)
+    tol = TOL[wl.dtype]
+    assert e_in <= tol and e_ow <= tol, f"{name}/{algo}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
+
+
+DILATION = {
+    "dil_bf16": MSDCN_BWD["msdcn_d16_bf16"].replace(name="dil16", msdcn_mode="dilation", smax=3.0),
+    "dil_f32": MSDCN_BWD["msdcn_d16_f32"].replace(name="dil32", msdcn_mode="dilation", smax=2.5),
+    "dil_flowdcn_bf16": REDUCED["flowdcn_msdcn_bf16"].replace(N=1, msdcn_mode="dilation"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DILATION))
+@pytest.mark.parametrize("algo", ["auto", "generic"])
+def test_msdcn_dilation_forward(orc, name, algo):
+    wl = DILATION[name]
+    err = forward_case(orc, wl, algo)
+    assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", sorted(DILATION))
+def test_msdcn_dilation_backward(orc, name):
+    wl = DILATION[name]
+    errs = msdcn_backward_case(orc, wl)
+    assert all(e <= TOL[wl.dtype] for e in errs), f"{name}: {errs}"
+
+
+def test_msdcn_rejects_softmax():
+    wl = MSDCN_BWD["msdcn_d16_bf16"]
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, torch.bfloat16, softmax=True)
+    out = torch.empty_like(data["input"]).cuda()
+    s0 = (B.ctypes.c_float * wl.G)(*data["s0"].tolist())
+    rc = B.load().msdcn_forward(B.ctypes.byref(desc), B._ptr(data["input"].cuda()),
+                                B._ptr(data["dir_weight"].cuda()), B._ptr(data["scale_raw"].cuda()),
+                                s0, 8.0, B._ptr(out), None)
+    assert rc == 2
