@@ -36,7 +36,8 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
     if (d->dtype != DCN4_F32 && d->dtype != DCN4_BF16 && d->dtype != DCN4_F16) return false;
     if (d->algo != DCN4_ALGO_AUTO && d->algo != DCN4_ALGO_GENERIC && d->algo != DCN4_ALGO_HALO)
         return false;
-    if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16)
+    if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16 &&
+        d->math != DCN4_MATH_PACKED16)
         return false;
     if (d->weights != DCN4_WEIGHTS_PLAIN && d->weights != DCN4_WEIGHTS_SOFTMAX) return false;
     if (d->msdcn_mode != DCN4_MSDCN_SCALE_OFFSET && d->msdcn_mode != DCN4_MSDCN_SCALE_DILATION)
@@ -255,9 +256,17 @@ bool halo_ok(const Geometry &g, Dtype dt, bool msdcn, const void *in, const void
 dcn4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DCN4_OK : DCN4_ERR_CUDA; }
 
 // Whether the 16-bit kernels round the bilinear weights to the data type.
+// 16-bit weights (mixed-precision fma) in the backward's gather of grad_input
 bool use_mixed(const dcn4_desc *d) {
     if (d->dtype == DCN4_F32) return false;
-    return d->math == DCN4_MATH_MIXED16 || d->math == DCN4_MATH_DEFAULT;
+    return d->math == DCN4_MATH_MIXED16 || d->math == DCN4_MATH_DEFAULT ||
+           d->math == DCN4_MATH_PACKED16;
+}
+
+// forward multiply variant: 0 fp32 weights, 1 mixed-precision fma, 2 packed
+int forward_math(const dcn4_desc *d) {
+    if (d->dtype == DCN4_F32 || d->math == DCN4_MATH_F32) return 0;
+    return d->math == DCN4_MATH_PACKED16 ? 2 : 1;
 }
 
 dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow, void *output,
@@ -275,7 +284,7 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     L.ow = ow;
     L.out = output;
     L.ms = ms;
-    L.mixed = use_mixed(desc);
+    L.mathv = forward_math(desc);
     L.stream = static_cast<cudaStream_t>(stream);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * elem_bytes(L.dtype);
     CUtensorMap map;
@@ -359,6 +368,12 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
                             L.plan.TH, &map_go);
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     }
+    // vectorised global-memory kernel: whole 16-byte vectors per group, a
+    // power-of-two count of them (<= 16), 16-byte aligned tensors
+    const int vb = g.D * eb;
+    L.vec = !L.halo && desc->algo != DCN4_ALGO_GENERIC && vb % 16 == 0 && vb <= 256 &&
+            ((vb / 16) & (vb / 16 - 1)) == 0 && aligned16(input) && aligned16(grad_out) &&
+            aligned16(L.acc);
     L.tmap_in = &map_in;
     L.tmap_go = &map_go;
     return cuda_status(launch_backward(L));

@@ -225,6 +225,45 @@ template <> struct VecMathMixed<__nv_bfloat16> { DCN4_MIXED_FMA("bf16", bf16_bit
 template <> struct VecMathMixed<__half> { DCN4_MIXED_FMA("f16", f16_bits) };
 #undef DCN4_MIXED_FMA
 
+// acc[0..8) += w00*q00 + w01*q01 + w10*q10 + w11*q11 over eight 16-bit
+// channels, the four-corner blend formed in packed 16-bit arithmetic (each
+// weight rounded to T, each fused multiply-add rounded to T: the pages'
+// half-precision kernel arithmetic) and added to the fp32 accumulators.
+template <typename T> struct VecMathPacked;
+template <> struct VecMathPacked<float> {
+    static __device__ __forceinline__ void blend4(float *acc, const uint4 &q00, const uint4 &q01,
+                                                  const uint4 &q10, const uint4 &q11, float w00,
+                                                  float w01, float w10, float w11) {
+        VecMath<float>::fma(acc, q00, w00);
+        VecMath<float>::fma(acc, q01, w01);
+        VecMath<float>::fma(acc, q10, w10);
+        VecMath<float>::fma(acc, q11, w11);
+    }
+};
+#define DCN4_PACKED_BLEND(T2, CVTW, TOF2)                                                        \
+    static __device__ __forceinline__ void blend4(float *acc, const uint4 &q00, const uint4 &q01, \
+                                                  const uint4 &q10, const uint4 &q11, float w00,  \
+                                                  float w01, float w10, float w11) {              \
+        const T2 a = CVTW(w00), b = CVTW(w01), c = CVTW(w10), d = CVTW(w11);                   \
+        const unsigned x0[4] = {q00.x, q00.y, q00.z, q00.w}, x1[4] = {q01.x, q01.y, q01.z, q01.w}; \
+        const unsigned x2[4] = {q10.x, q10.y, q10.z, q10.w}, x3[4] = {q11.x, q11.y, q11.z, q11.w}; \
+        _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                          \
+            T2 r = __hmul2(*reinterpret_cast<const T2 *>(&x0[e]), a);                             \
+            r = __hfma2(*reinterpret_cast<const T2 *>(&x1[e]), b, r);                             \
+            r = __hfma2(*reinterpret_cast<const T2 *>(&x2[e]), c, r);                             \
+            r = __hfma2(*reinterpret_cast<const T2 *>(&x3[e]), d, r);                             \
+            const float2 f = TOF2(r);                                                            \
+            const float2 s = __fadd2_rn(make_float2(acc[2 * e], acc[2 * e + 1]), f);              \
+            acc[2 * e] = s.x;                                                                    \
+            acc[2 * e + 1] = s.y;                                                                \
+        }                                                                                        \
+    }
+template <> struct VecMathPacked<__nv_bfloat16> {
+    DCN4_PACKED_BLEND(__nv_bfloat162, __float2bfloat162_rn, __bfloat1622float2)
+};
+template <> struct VecMathPacked<__half> { DCN4_PACKED_BLEND(__half2, __float2half2_rn, __half22float2) };
+#undef DCN4_PACKED_BLEND
+
 // ---- shared memory / async-copy primitives --------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -280,7 +280,7 @@ __device__ __forceinline__ void stage_window(const TileCoord &tc, const CUtensor
 }
 
 // The gathers of one staged tile: one thread per (pixel, group).
-template <typename T, int U, bool MS, bool MIXED>
+template <typename T, int U, bool MS, int MV>
 __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry &g,
                                              const HaloPlan &pl, const T *__restrict__ in,
                                              T *__restrict__ out, const MsdcnParams &ms,
@@ -390,7 +390,9 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                     const uint4 q01 = *reinterpret_cast<const uint4 *>(a0 + PS);
                     const uint4 q10 = *reinterpret_cast<const uint4 *>(a1);
                     const uint4 q11 = *reinterpret_cast<const uint4 *>(a1 + PS);
-                    if (MIXED) {
+                    if (MV == 2) {
+                        VecMathPacked<T>::blend4(acc[c], q00, q01, q10, q11, w00, w01, w10, w11);
+                    } else if (MV == 1) {
                         VecMathMixed<T>::fma(acc[c], q00, w00);
                         VecMathMixed<T>::fma(acc[c], q01, w01);
                         VecMathMixed<T>::fma(acc[c], q10, w10);
@@ -456,7 +458,7 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
 // the next tile are in flight while the current one is computed. Every wait
 // is bounded; on expiry the warp sets the error word, lets its own copies in
 // flight land and returns.
-template <typename T, int U, bool MS, bool MIXED, int STAGES, int NW>
+template <typename T, int U, bool MS, int MV, int STAGES, int NW>
 __global__ void __launch_bounds__(NW * 32, 1)
 fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan pl,
                 const T *__restrict__ in, const T *__restrict__ ow, T *__restrict__ out,
@@ -535,7 +537,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
             return;
         }
         const unsigned char *buf = smem + s * stage_bytes;
-        compute_tile<T, U, MS, MIXED>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
+        compute_tile<T, U, MS, MV>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
                                       threadIdx.x, NW * 32);
         __syncwarp();
         if (leader) mbar_arrive(empty0 + 8 * s);

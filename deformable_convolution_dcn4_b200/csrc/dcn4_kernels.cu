@@ -16,6 +16,7 @@ __device__ unsigned int g_error_word = 0;
 #include "dcn4_bwd.cuh"
 #include "dcn4_fwd.cuh"
 #include "dcn4_bwd_halo.cuh"
+#include "dcn4_bwd_vec.cuh"
 #include "dcn4_launch.h"
 
 namespace dcn4 {
@@ -70,9 +71,9 @@ int grid_for(long long work, int block) {
     return (int)blocks;
 }
 
-template <typename T, int U, bool MS, bool MIXED, int STAGES, int NW>
+template <typename T, int U, bool MS, int MV, int STAGES, int NW>
 cudaError_t launch_halo_t(const FwdLaunch &L) {
-    auto k = fwd_halo_kernel<T, U, MS, MIXED, STAGES, NW>;
+    auto k = fwd_halo_kernel<T, U, MS, MV, STAGES, NW>;
     constexpr int NT = NW * 32;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.plan.smem_bytes);
     if (e != cudaSuccess) return e;
@@ -93,24 +94,25 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
 // Stage count and warps: two stages with 16 warps when a tile has 512
 // (pixel, group) pairs, 8 warps when it has fewer; the large single-stage
 // plans (MSDCN whole-image windows, 64-channel groups) use 8.
-template <typename T, int U, bool MS, bool MIXED>
+template <typename T, int U, bool MS, int MV>
 cudaError_t launch_halo_s(const FwdLaunch &L) {
     if constexpr (U <= 4) {
         if (L.plan.stages == 2) {
             if (L.plan.TH * L.plan.TW * L.plan.Gc >= 512)
-                return launch_halo_t<T, U, MS, MIXED, 2, 16>(L);
-            return launch_halo_t<T, U, MS, MIXED, 2, 8>(L);
+                return launch_halo_t<T, U, MS, MV, 2, 16>(L);
+            return launch_halo_t<T, U, MS, MV, 2, 8>(L);
         }
     }
-    return launch_halo_t<T, U, MS, MIXED, 1, 8>(L);
+    return launch_halo_t<T, U, MS, MV, 1, 8>(L);
 }
 
 template <typename T, int U, bool MS>
 cudaError_t launch_halo_m(const FwdLaunch &L) {
     if constexpr (sizeof(T) == 2) {
-        if (L.mixed) return launch_halo_s<T, U, MS, true>(L);
+        if (L.mathv == 2) return launch_halo_s<T, U, MS, 2>(L);
+        if (L.mathv == 1) return launch_halo_s<T, U, MS, 1>(L);
     }
-    return launch_halo_s<T, U, MS, false>(L);
+    return launch_halo_s<T, U, MS, 0>(L);
 }
 
 template <typename T, bool MS>
@@ -172,6 +174,35 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
     return cudaErrorInvalidValue;
 }
 
+template <typename T, bool MS, int LPP>
+cudaError_t launch_bwd_vec_l(const BwdLaunch &L) {
+    const Geometry &g = L.geo;
+    const long long total = (long long)g.N * g.Ho * g.Wo * g.G * LPP;
+    bwd_vec_kernel<T, MS, LPP><<<grid_for(total, 256), 256, 0, L.stream>>>(
+        g, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
+        static_cast<const T *>(L.gout), L.acc, static_cast<T *>(L.gow), L.ms ? *L.ms : kNoMs,
+        static_cast<T *>(L.graw));
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <typename T, bool MS>
+cudaError_t launch_bwd_vec_m(const BwdLaunch &L) {
+    switch (L.geo.D * (int)sizeof(T) / 16) {
+        case 1: return launch_bwd_vec_l<T, MS, 1>(L);
+        case 2: return launch_bwd_vec_l<T, MS, 2>(L);
+        case 4: return launch_bwd_vec_l<T, MS, 4>(L);
+        case 8: return launch_bwd_vec_l<T, MS, 8>(L);
+        case 16: return launch_bwd_vec_l<T, MS, 16>(L);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_bwd_vec(const BwdLaunch &L) {
+    return L.msdcn ? launch_bwd_vec_m<T, true>(L) : launch_bwd_vec_m<T, false>(L);
+}
+
 template <typename T>
 cudaError_t launch_bwd_t(const BwdLaunch &L) {
     const Geometry &g = L.geo;
@@ -194,6 +225,8 @@ cudaError_t launch_bwd_t(const BwdLaunch &L) {
     if (e != cudaSuccess) return e;
     if (L.halo) {
         e = launch_bwd_halo<T>(L, false);
+    } else if (L.vec) {
+        e = launch_bwd_vec<T>(L);
     } else {
         const long long pairs = (long long)g.N * g.Ho * g.Wo * g.G;
         if (L.msdcn)

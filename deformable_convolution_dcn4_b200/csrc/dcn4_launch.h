@@ -19,7 +19,7 @@ struct FwdLaunch {
     void *out;
     const MsdcnParams *ms;  // MSDCN only
     bool halo;              // use the shared-memory halo kernel
-    bool mixed;             // 16-bit weights with mixed-precision fma (bf16/fp16)
+    int mathv;              // 0 fp32 weights, 1 mixed-precision fma, 2 packed 16-bit blend
     HaloPlan plan;
     const CUtensorMap *tmap;
     unsigned long long ow_bytes;
@@ -36,6 +36,7 @@ struct BwdLaunch {
     void *gow;     // element type
     float *acc;    // fp32 accumulation buffer for grad_input (== gin for fp32)
     bool halo;     // use the shared-memory halo kernel
+    bool vec;      // otherwise the vectorised global-memory kernel (else scalar)
     bool mixed;    // 16-bit weights with mixed-precision fma (bf16/fp16 grad_input)
     HaloPlan plan;
     BwdLayout layout;

@@ -79,10 +79,10 @@ def test_forward_reduced(orc, name, algo):
 @pytest.mark.parametrize("name", [n for n in sorted(REDUCED) if REDUCED[n].dtype != "f32"] +
                          ["ragged_bf16", "stride2_pad0_dil2_f16", "far_offsets_bf16",
                           "offset_scale_bf16"])
-@pytest.mark.parametrize("math", ["f32", "mixed16"])
+@pytest.mark.parametrize("math", ["f32", "mixed16", "packed16"])
 def test_forward_math_modes(orc, name, math):
-    """fp32 weights and 16-bit weights with the mixed-precision fma (the
-    default for 16-bit data): both meet the same gate."""
+    """fp32 weights, 16-bit weights with the mixed-precision fma (the default
+    for 16-bit data) and the packed 16-bit corner blend: all meet the gate."""
     wl = REDUCED.get(name) or EDGE[name]
     data = make_inputs(wl, out_hw(wl))
     dev = "cuda"
@@ -415,3 +415,37 @@ def test_msdcn_rejects_softmax():
                                 B._ptr(data["dir_weight"].cuda()), B._ptr(data["scale_raw"].cuda()),
                                 s0, 8.0, B._ptr(out), None)
     assert rc == 2
+
+
+# Shapes the shared-memory backward does not take: AUTO runs the vectorised
+# global-memory kernel (whole 16-byte vectors per group) or, for group widths
+# that are not, the scalar one; "generic" forces the scalar kernel.
+BWD_VEC = {
+    "d64_bf16": W["flowdcn_msdcn_bf16"].replace(name="d64", kind="dcn4", N=1, H=12, W=14,
+                                                C=256, G=4, offset_dist=("normal", 2.0)),
+    "d64_f32": W["tiny_f32"].replace(name="d64f", N=1, H=9, W=10, C=128, G=2),
+    "k5_bf16": W["internimage_bf16"].replace(name="k5b", N=1, H=11, W=9, C=64, G=4, kh=5, kw=5,
+                                             pad=(2, 2)),
+    "k3x1_f16_d8": W["ldm64_f16"].replace(name="k31", N=2, H=9, W=8, C=32, G=4, kh=3, kw=1,
+                                          pad=(1, 0)),
+    "d12_bf16": BWD["d12_bf16"],
+    "softmax_d64_bf16": W["flowdcn_msdcn_bf16"].replace(name="smd64", kind="dcn4", N=1, H=10,
+                                                        W=10, C=128, G=2, softmax=True,
+                                                        weight_sigma=1.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BWD_VEC))
+@pytest.mark.parametrize("algo", ["auto", "generic"])
+def test_backward_global_kernels(orc, name, algo):
+    wl = BWD_VEC[name]
+    e_in, e_ow = backward_case(orc, wl, algo)
+    tol = TOL[wl.dtype]
+    assert e_in <= tol and e_ow <= tol, f"{name}/{algo}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
+
+
+@pytest.mark.parametrize("name", ["msdcn_d16_bf16", "msdcn_stride_f16"])
+def test_msdcn_backward_scalar_kernel(orc, name):
+    wl = MSDCN_BWD[name]
+    errs = msdcn_backward_case(orc, wl, algo="generic")
+    assert all(e <= TOL[wl.dtype] for e in errs), f"{name}: {errs}"
