@@ -82,13 +82,12 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
     const int Gc = 128 / (g.D * eb);
     if (g.G % Gc != 0) return false;
     const int U = g.D * eb / 16;
-    const int R = msdcn ? 8 : 4;
     const int smem_max = max_smem_optin();
     // record slots: room for the 16-byte superset copy plus a word of read
     // slack, and a stride of 16 (mod 128) bytes so that the records of
     // consecutive pixels start in different bank quads
     const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
-    auto try_tile = [&](int TH, int TW, bool force_full, int stages, HaloPlan *p) {
+    auto try_tile = [&](int TH, int TW, bool force_full, int stages, HaloPlan *p, int R) {
         if (stages == 2 && U > 4) return false;  // 16 warps need <= 128 registers
         TH = TH < g.Ho ? TH : g.Ho;
         TW = TW < pow2_ceil(g.Wo) ? TW : pow2_ceil(g.Wo);
@@ -114,14 +113,21 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
     };
     static const int cands[][2] = {{16, 8}, {8, 16}, {16, 16}, {8, 8}, {8, 4}, {4, 8},
                                    {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    // MSDCN offsets scale with s up to Smax: the whole image when it fits,
+    // else the widest window (R <= 8) a two-stage 16 x 8 tile allows
+    // (measured on the InternImage shape: R = 5 two-stage beats R = 8
+    // one-stage and 8 x 8 tiles), else R = 8 on smaller tiles
     if (msdcn) {
         static const int big[][2] = {{32, 32}, {16, 32}, {32, 16}, {16, 16}, {8, 16}, {16, 8}, {8, 8}};
         for (auto &c : big)
-            if (try_tile(c[0], c[1], true, 1, out)) return true;
+            if (try_tile(c[0], c[1], true, 1, out, 8)) return true;
+        for (int R = 8; R >= 5; --R)
+            if (try_tile(16, 8, false, 2, out, R)) return true;
     }
+    const int R = msdcn ? 8 : 4;
     for (int stages : {2, 1})
         for (auto &c : cands)
-            if (try_tile(c[0], c[1], false, stages, out)) return true;
+            if (try_tile(c[0], c[1], false, stages, out, R)) return true;
     return false;
 }
 

@@ -70,9 +70,11 @@ typedef enum {
 typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
 
 /* Kernel selection. AUTO picks the staged (shared-memory halo) kernel when
- * the call qualifies and the generic one otherwise; the other values force
- * a variant (a forced variant the call does not qualify for returns
- * DCN4_ERR_UNSUPPORTED). */
+ * the call qualifies and a global-memory kernel otherwise (for the backward:
+ * the vectorised one when the group width is a power-of-two count of 16-byte
+ * vectors and the tensors are 16-byte aligned, else the scalar one). GENERIC
+ * forces the scalar global-memory kernel and HALO the staged one (a forced
+ * variant the call does not qualify for returns DCN4_ERR_UNSUPPORTED). */
 typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
 
 /* Multiply precision of the bilinear weights in the bf16/fp16 halo kernels
@@ -202,9 +204,13 @@ DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
  *       once the clamp is active (or raw is NaN).
  * Arguments as in msdcn_forward and dcn4_backward (grad outputs in
  * desc->dtype, device; the same workspace size, dcn4_backward_workspace_size).
- * This version runs one thread per (pixel, group) with fp32 atomics into the
- * workspace (fp32 data: into grad_input); DCN4_ALGO_HALO returns
- * DCN4_ERR_UNSUPPORTED. */
+ * grad_input accumulates with fp32 atomics in the workspace (fp32 data: in
+ * grad_input): AUTO runs D*sizeof(T)/16 lanes per (pixel, group) with 16-byte
+ * vector loads and atomics when the group is a power-of-two count of 16-byte
+ * vectors (up to 16) and the tensors are 16-byte aligned, else (and under
+ * DCN4_ALGO_GENERIC) one thread per (pixel, group) with scalar atomics;
+ * DCN4_ALGO_HALO returns DCN4_ERR_UNSUPPORTED. desc->weights must be
+ * DCN4_WEIGHTS_PLAIN. */
 DCN4_API dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input,
                           const void *dir_weight, const void *scale_raw,
                           const float *s0_host, float smax, const void *grad_out,
