@@ -77,16 +77,19 @@ int pow2_ceil(int v) {
 // Chooses the halo kernel's tiling; false when the call does not fit it.
 // The staged pixel (Gc groups x D channels) must be exactly 128 bytes, the
 // stride at which random 16-byte gathers can be kept free of bank conflicts.
-bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
+bool plan_halo(const Geometry &g, int eb, bool msdcn, bool rec_tma, HaloPlan *out) {
     if (128 % (g.D * eb) != 0) return false;
     const int Gc = 128 / (g.D * eb);
     if (g.G % Gc != 0) return false;
     const int U = g.D * eb / 16;
     const int smem_max = max_smem_optin();
-    // record slots: room for the 16-byte superset copy plus a word of read
-    // slack, and a stride of 16 (mod 128) bytes so that the records of
-    // consecutive pixels start in different bank quads
-    const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
+    // record slots. Per-pixel bulk copies: room for the 16-byte superset copy
+    // plus a word of read slack, stride 16 (mod 128) bytes. One TMA tile copy
+    // per tile (rec_tma): the group slice starting at the 16-byte boundary
+    // at or below it, rec_box elements per pixel.
+    const int al = 16 / eb;
+    const int rec_box = ceil_to(Gc * 27 + al - 1, al);
+    const int slot = rec_tma ? rec_box * eb : ceil_to(Gc * 27 * eb + 16, 128) + 16;
     auto try_tile = [&](int TH, int TW, bool force_full, int stages, HaloPlan *p, int R) {
         if (stages == 2 && U > 4) return false;  // 16 warps need <= 128 registers
         TH = TH < g.Ho ? TH : g.Ho;
@@ -101,7 +104,7 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, HaloPlan *out) {
         const long long halo = (long long)HR * HC * 128;
         HaloPlan q{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                    (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc,
-                   slot, (int)halo, stages, 0};
+                   slot, (int)halo, stages, 0, rec_tma ? 1 : 0, rec_box};
         const long long total = (long long)stages *
                                     ((((halo + (long long)TH * TW * slot) + 127) / 128 * 128) +
                                      8 * (2 + 16));
@@ -182,7 +185,7 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
         L.threads = two ? 256 : 512;
         *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                         (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
-                        L.smem_bytes};
+                        L.smem_bytes, 0, 0};
         *lay = L;
         return true;
     }
@@ -245,9 +248,11 @@ bool encode_input_map(const Geometry &g, Dtype dt, const void *in, const HaloPla
     return r == CUDA_SUCCESS;
 }
 
-// Whether the halo kernel can run this call; fills plan and tensor map.
+// Whether the halo kernel can run this call; fills plan and tensor maps.
+// The records arrive by TMA (map_ow) when a pixel's G*27 values span a
+// multiple of 16 bytes (the TMA stride rule), else by per-pixel bulk copies.
 bool halo_ok(const Geometry &g, Dtype dt, bool msdcn, const void *in, const void *ow,
-             const void *out, HaloPlan *plan, CUtensorMap *map) {
+             const void *out, HaloPlan *plan, CUtensorMap *map, CUtensorMap *map_ow) {
     const int eb = elem_bytes(dt);
     if (g.kh != 3 || g.kw != 3) return false;
     if ((g.D * eb) % 16 != 0) return false;
@@ -255,7 +260,12 @@ bool halo_ok(const Geometry &g, Dtype dt, bool msdcn, const void *in, const void
     if (U != 2 && U != 4 && U != 8) return false;
     if (eb == 4 && U == 2) return false;
     if (!aligned16(in) || !aligned16(ow) || !aligned16(out)) return false;
-    if (!plan_halo(g, eb, msdcn, plan)) return false;
+    const bool rec_tma = (g.G * 27 * eb) % 16 == 0;
+    if (rec_tma && plan_halo(g, eb, msdcn, true, plan) &&
+        encode_map(dt, ow, g.N, g.Ho, g.Wo, g.G * 27, plan->rec_box, plan->TW, plan->TH, map_ow) &&
+        encode_input_map(g, dt, in, *plan, map))
+        return true;
+    if (!plan_halo(g, eb, msdcn, false, plan)) return false;
     return encode_input_map(g, dt, in, *plan, map);
 }
 
@@ -293,13 +303,15 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     L.mathv = forward_math(desc);
     L.stream = static_cast<cudaStream_t>(stream);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * elem_bytes(L.dtype);
-    CUtensorMap map;
+    CUtensorMap map, map_ow;
     memset(&map, 0, sizeof(map));
+    memset(&map_ow, 0, sizeof(map_ow));
     if (desc->algo != DCN4_ALGO_GENERIC) {
-        L.halo = halo_ok(g, L.dtype, L.msdcn, input, ow, output, &L.plan, &map);
+        L.halo = halo_ok(g, L.dtype, L.msdcn, input, ow, output, &L.plan, &map, &map_ow);
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     }
     L.tmap = &map;
+    L.tmap_ow = &map_ow;
     return cuda_status(launch_forward(L));
 }
 

@@ -81,6 +81,8 @@ struct HaloPlan {
     int halo_bytes;      // HR*HC*Gc*D*elem, rounded up to 128
     int stages;          // 2: double-buffered (512 threads), 1: single (256 threads)
     int smem_bytes;      // dynamic shared memory of one CTA
+    int rec_tma;         // 1: records arrive by one TMA tile copy per tile (forward)
+    int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)
 };
 
 // ---- element types -------------------------------------------------------

@@ -279,6 +279,22 @@ __device__ __forceinline__ void stage_window(const TileCoord &tc, const CUtensor
     tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
 }
 
+// With pl.rec_tma: the tile's input window and its records ([TH][TW]
+// x rec_box elements from the 16-byte boundary at or below the slice's first
+// value; zero fill past the image) on one barrier; called by one thread.
+__device__ __forceinline__ void stage_window_records(const TileCoord &tc, const CUtensorMap *tmap,
+                                                     const CUtensorMap *tmap_ow, const Geometry &g,
+                                                     const HaloPlan &pl, int eb,
+                                                     unsigned char *halo, unsigned char *slots,
+                                                     uint32_t bar) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(bar, (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb +
+                                   (uint32_t)pl.TH * pl.TW * pl.rec_box * eb);
+    tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
+    const int x0 = (tc.g0 * 27) & ~(16 / eb - 1);
+    tma_load_4d(smem_u32(slots), tmap_ow, x0, tc.wo0, tc.ho0, tc.n, bar);
+}
+
 // The gathers of one staged tile: one thread per (pixel, group).
 template <typename T, int U, bool MS, int MV>
 __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry &g,
@@ -309,7 +325,9 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
         const int ho = tc.ho0 + ty, wo = tc.wo0 + tx;
         const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
         // the record's offset within its 16-byte-aligned copy (arithmetic mod 2^32)
-        const unsigned mis = ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
+        const unsigned mis = pl.rec_tma
+                                 ? ((unsigned)(tc.g0 * 27) & (unsigned)(16 / EB - 1)) * (unsigned)EB
+                                 : ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + mis + gl * REC;
         float v[27];
         RecordReader<T>::read(rec, v);
@@ -460,9 +478,10 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
 // flight land and returns.
 template <typename T, int U, bool MS, int MV, int STAGES, int NW>
 __global__ void __launch_bounds__(NW * 32, 1)
-fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan pl,
-                const T *__restrict__ in, const T *__restrict__ ow, T *__restrict__ out,
-                unsigned long long ow_bytes, const __grid_constant__ MsdcnParams ms) {
+fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_ow,
+                Geometry g, HaloPlan pl, const T *__restrict__ in, const T *__restrict__ ow,
+                T *__restrict__ out, unsigned long long ow_bytes,
+                const __grid_constant__ MsdcnParams ms) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int stage_bytes = HaloSmem::stage_bytes(pl);
     const uint32_t win0 = smem_u32(smem + STAGES * stage_bytes);  // win[s]   at +8s
@@ -488,19 +507,32 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
     auto window = [&](const TileCoord &tc, int k) -> bool {
         const int s = k % STAGES, use = k / STAGES;
         if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, kWaitLimitNs)) return false;
-        if (leader)
-            stage_window(tc, &tmap, g, pl, Elem<T>::kBytes, smem + s * stage_bytes, win0 + 8 * s);
+        if (leader) {
+            unsigned char *buf = smem + s * stage_bytes;
+            if (pl.rec_tma)
+                stage_window_records(tc, &tmap, &tmap_ow, g, pl, Elem<T>::kBytes, buf,
+                                     buf + pl.halo_bytes, win0 + 8 * s);
+            else
+                stage_window(tc, &tmap, g, pl, Elem<T>::kBytes, buf, win0 + 8 * s);
+        }
         return true;
     };
+    // per-warp record copies (the records of the warp's own pairs), unless
+    // they come with the window
     auto records = [&](const TileCoord &tc, int k) {
+        if (pl.rec_tma) return;
         const int s = k % STAGES;
         stage_records<T>(tc, g, pl, ow, ow_bytes, smem + s * stage_bytes + pl.halo_bytes, NW * 32,
                          myrec + 8 * s);
     };
+    auto records_ready = [&](int k) -> bool {
+        return pl.rec_tma ||
+               mbar_wait_bounded(myrec + 8 * (k % STAGES), (k / STAGES) & 1, kWaitLimitNs);
+    };
     // on an expired wait: let this warp's copies of tiles k0..k1 land
     auto drain = [&](int k0, int k1, bool with_window) {
         for (int k = k0 < 0 ? 0 : k0; k <= k1; ++k) {
-            mbar_wait_bounded(myrec + 8 * (k % STAGES), (k / STAGES) & 1, kWaitLimitNs);
+            records_ready(k);
             if (with_window)
                 mbar_wait_bounded(win0 + 8 * (k % STAGES), (k / STAGES) & 1, kWaitLimitNs);
         }
@@ -530,7 +562,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, Geometry g, HaloPlan p
             issued = i + 1;
         }
         const bool ok = mbar_wait_bounded(win0 + 8 * s, (i / STAGES) & 1, kWaitLimitNs) &&
-                        mbar_wait_bounded(myrec + 8 * s, (i / STAGES) & 1, kWaitLimitNs);
+                        records_ready(i);
         if (!ok) {
             if (leader) atomicOr(&g_error_word, kErrTimeout);
             drain(i, issued, warp == 0);

@@ -85,8 +85,8 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
     long long grid = (long long)sm_count() * occ;
     if (grid > tiles) grid = tiles;
     k<<<(unsigned)grid, NT, L.plan.smem_bytes, L.stream>>>(
-        *L.tmap, L.geo, L.plan, static_cast<const T *>(L.in), static_cast<const T *>(L.ow),
-        static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
+        *L.tmap, *L.tmap_ow, L.geo, L.plan, static_cast<const T *>(L.in),
+        static_cast<const T *>(L.ow), static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
     count_launch();
     return cudaGetLastError();
 }

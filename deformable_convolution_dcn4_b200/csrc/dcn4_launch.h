@@ -22,6 +22,7 @@ struct FwdLaunch {
     int mathv;              // 0 fp32 weights, 1 mixed-precision fma, 2 packed 16-bit blend
     HaloPlan plan;
     const CUtensorMap *tmap;
+    const CUtensorMap *tmap_ow;  // records, when plan.rec_tma
     unsigned long long ow_bytes;
     cudaStream_t stream;
 };

@@ -80,7 +80,8 @@ def test_malformed_descriptors_rejected(lib, bad):
 
 
 def test_bad_enum_fields_rejected(lib):
-    for field, val in (("math", 5), ("algo", 9), ("dtype", -1)):
+    for field, val in (("math", 5), ("algo", 9), ("dtype", -1), ("weights", 2),
+                       ("msdcn_mode", -1), ("msdcn_mode", 2)):
         d = _desc()
         setattr(d, field, val)
         with pytest.raises(B.Dcn4Error) as e:
@@ -100,6 +101,24 @@ def test_null_pointers_rejected_before_any_launch(lib):
     assert lib.msdcn_forward(ctypes.byref(d), one, one, z, s0, 8.0, one, z) == 1
     assert lib.msdcn_forward(ctypes.byref(d), one, one, one, None, 8.0, one, z) == 1
     assert lib.dcn4_backward(ctypes.byref(d), one, one, one, z, one, one, 1 << 30, z) == 1
+    # msdcn_backward: every pointer, including the scale gradient and s0
+    args = [one, one, one, s0, 8.0, one, one, one, one, one, 1 << 30, z]
+    for i in (0, 1, 2, 3, 5, 6, 7, 8):
+        bad = list(args)
+        bad[i] = None if i == 3 else z
+        assert lib.msdcn_backward(ctypes.byref(d), *bad) == 1, i
+    assert lib.msdcn_backward(None, *args) == 1
+
+
+def test_msdcn_rejects_softmax_weights_before_any_launch(lib):
+    d = _desc(dtype=1)
+    d.weights = 1
+    one = ctypes.c_void_p(16)
+    z = ctypes.c_void_p(0)
+    s0 = (ctypes.c_float * 4)(1, 1, 2, 2)
+    assert lib.msdcn_forward(ctypes.byref(d), one, one, one, s0, 8.0, one, z) == 2
+    assert lib.msdcn_backward(ctypes.byref(d), one, one, one, s0, 8.0, one, one, one, one, one,
+                              1 << 30, z) == 2
 
 
 def test_workspace_rules(lib):
