@@ -138,7 +138,7 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, bool rec_tma, HaloPlan *ou
 // (pixel, group) pair per thread (512 threads), 128-byte staged pixels,
 // R = 4, and the sorted sample records (14 bytes each) must fit in the
 // window buffer they reuse.
-bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
+bool plan_bwd(const Geometry &g, int eb, bool rec_tma, HaloPlan *out, BwdLayout *lay) {
     if (128 % (g.D * eb) != 0) return false;
     const int Gc = 128 / (g.D * eb);
     if (g.G % Gc != 0) return false;
@@ -146,7 +146,10 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
     if (!(U == 4 || (U == 2 && eb == 2))) return false;
     const int R = 4;
     const int smem_max = max_smem_optin() - 1024;  // static shared memory of the kernel
-    const int slot = ceil_to(Gc * 27 * eb + 16, 128) + 16;
+    // record slots as in plan_halo: per-pixel bulk copies, or one TMA tile copy
+    const int al = 16 / eb;
+    const int rec_box = ceil_to(Gc * 27 + al - 1, al);
+    const int slot = rec_tma ? rec_box * eb : ceil_to(Gc * 27 * eb + 16, 128) + 16;
     // first choice: a 256-pair tile small enough for two CTAs per SM (the
     // phases of one CTA then overlap the other's); else the largest tile
     static const int cands[][2] = {{8, 8}, {16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
@@ -185,7 +188,7 @@ bool plan_bwd(const Geometry &g, int eb, HaloPlan *out, BwdLayout *lay) {
         L.threads = two ? 256 : 512;
         *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                         (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
-                        L.smem_bytes, 0, 0};
+                        L.smem_bytes, rec_tma ? 1 : 0, rec_box};
         *lay = L;
         return true;
     }
@@ -374,16 +377,26 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
     L.graw = graw;
     const int eb = elem_bytes(L.dtype);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * eb;
-    CUtensorMap map_in, map_go;
+    CUtensorMap map_in, map_go, map_ow;
     memset(&map_in, 0, sizeof(map_in));
     memset(&map_go, 0, sizeof(map_go));
+    memset(&map_ow, 0, sizeof(map_ow));
     if (desc->algo != DCN4_ALGO_GENERIC) {
-        L.halo = !L.msdcn && g.kh == 3 && g.kw == 3 && aligned16(input) &&
-                 aligned16(offset_weight) && aligned16(grad_out) && aligned16(L.acc) &&
-                 plan_bwd(g, eb, &L.plan, &L.layout) &&
-                 encode_input_map(g, L.dtype, input, L.plan, &map_in) &&
-                 encode_map(L.dtype, grad_out, g.N, g.Ho, g.Wo, g.C, L.plan.Gc * g.D, L.plan.TW,
-                            L.plan.TH, &map_go);
+        const bool base = !L.msdcn && g.kh == 3 && g.kw == 3 && aligned16(input) &&
+                          aligned16(offset_weight) && aligned16(grad_out) && aligned16(L.acc);
+        auto maps = [&]() {
+            return encode_input_map(g, L.dtype, input, L.plan, &map_in) &&
+                   encode_map(L.dtype, grad_out, g.N, g.Ho, g.Wo, g.C, L.plan.Gc * g.D,
+                              L.plan.TW, L.plan.TH, &map_go);
+        };
+        // records by one TMA tile copy when a pixel's G*27 values span a
+        // multiple of 16 bytes, else by per-pixel bulk copies
+        L.halo = base && (g.G * 27 * eb) % 16 == 0 && plan_bwd(g, eb, true, &L.plan, &L.layout) &&
+                 maps() &&
+                 encode_map(L.dtype, offset_weight, g.N, g.Ho, g.Wo, g.G * 27, L.plan.rec_box,
+                            L.plan.TW, L.plan.TH, &map_ow);
+        if (!L.halo)
+            L.halo = base && plan_bwd(g, eb, false, &L.plan, &L.layout) && maps();
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     }
     // vectorised global-memory kernel: whole 16-byte vectors per group, a
@@ -394,6 +407,7 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
             aligned16(L.acc);
     L.tmap_in = &map_in;
     L.tmap_go = &map_go;
+    L.tmap_ow = &map_ow;
     return cuda_status(launch_backward(L));
 }
 

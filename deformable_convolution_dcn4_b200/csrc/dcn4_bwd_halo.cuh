@@ -199,7 +199,8 @@ __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *wa
 template <typename T, int U, int NW, bool MIXED, bool DIRECT>
 __global__ void __launch_bounds__(NW * 32, 512 / (NW * 32))
 bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
-                const __grid_constant__ CUtensorMap tmap_go, Geometry g, HaloPlan pl,
+                const __grid_constant__ CUtensorMap tmap_go,
+                const __grid_constant__ CUtensorMap tmap_ow, Geometry g, HaloPlan pl,
                 BwdLayout L, const T *__restrict__ in, const T *__restrict__ ow,
                 T *__restrict__ gow, float *__restrict__ gacc, T *__restrict__ gin,
                 unsigned long long ow_bytes) {
@@ -236,8 +237,9 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     {
         uint32_t tx = 0;
         if (threadIdx.x == 0)
-            tx = (uint32_t)pl.HR * pl.HC * PS + (uint32_t)pl.TH * pl.TW * PS;
-        const int npix = pl.TH * pl.TW;
+            tx = (uint32_t)pl.HR * pl.HC * PS + (uint32_t)pl.TH * pl.TW * PS +
+                 (pl.rec_tma ? (uint32_t)pl.TH * pl.TW * pl.rec_box * EB : 0u);
+        const int npix = pl.rec_tma ? 0 : pl.TH * pl.TW;  // per-pixel copies
         for (int p = threadIdx.x; p < npix; p += NT) {
             const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
             if (ty >= tc.th_eff || tx_ >= tc.tw_eff) continue;
@@ -261,6 +263,9 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         if (threadIdx.x == 0) {
             tma_load_4d(smem_u32(halo), &tmap_in, tc.g0 * D, tc.hx0, tc.hy0, tc.n, bar);
             tma_load_4d(smem_u32(gotile), &tmap_go, tc.g0 * D, tc.wo0, tc.ho0, tc.n, bar);
+            if (pl.rec_tma)
+                tma_load_4d(smem_u32(slots), &tmap_ow, (tc.g0 * 27) & ~(16 / EB - 1), tc.wo0, tc.ho0,
+                            tc.n, bar);
         }
         for (int p = threadIdx.x; p < npix; p += NT) {
             const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
@@ -306,7 +311,8 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         ho = tc.ho0 + ty;
         wo = tc.wo0 + tx;
         gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
-        start = ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
+        start = pl.rec_tma ? ((unsigned)(tc.g0 * 27) & (unsigned)(16 / EB - 1)) * (unsigned)EB
+                           : ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
     }
 #pragma unroll
     for (int k = 0; k < 9; ++k) kr[k] = 0xffffffffu;

@@ -151,7 +151,7 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
         cudaError_t e = allow_smem(reinterpret_cast<const void *>(kernel), L.layout.smem_bytes);
         if (e != cudaSuccess) return e;
         kernel<<<(unsigned)grid, nt, L.layout.smem_bytes, L.stream>>>(
-            *L.tmap_in, *L.tmap_go, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
+            *L.tmap_in, *L.tmap_go, *L.tmap_ow, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
             static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, static_cast<T *>(L.gin),
             L.ow_bytes);
         count_launch();

@@ -43,6 +43,7 @@ struct BwdLaunch {
     BwdLayout layout;
     const CUtensorMap *tmap_in;
     const CUtensorMap *tmap_go;
+    const CUtensorMap *tmap_ow;  // records, when plan.rec_tma
     unsigned long long ow_bytes;
     cudaStream_t stream;
     bool msdcn;             // FlowDCN multi-scale variant: ow holds (dir_x, dir_y, m)
