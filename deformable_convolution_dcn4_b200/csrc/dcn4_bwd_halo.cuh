@@ -87,40 +87,10 @@ template <> struct ChunkUnpack<__half> {
     }
 };
 
-// <a, b> over one 16-byte chunk where both operands are stored in T. For
-// 16-bit T this is the sm_100 mixed-precision fma (the 16x16-bit products
-// are exact, the sums are fp32), so it equals the unpack-and-fma form bit
-// for bit up to the order of the additions.
-template <typename T> struct PackedDot;
-template <> struct PackedDot<float> {
-    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {
-        float s0 = __uint_as_float(a.x) * __uint_as_float(b.x);
-        float s1 = __uint_as_float(a.y) * __uint_as_float(b.y);
-        s0 = fmaf(__uint_as_float(a.z), __uint_as_float(b.z), s0);
-        s1 = fmaf(__uint_as_float(a.w), __uint_as_float(b.w), s1);
-        return s0 + s1;
-    }
-};
-#define DCN4_PACKED_DOT(TY)                                                                    \
-    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {              \
-        const unsigned wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};             \
-        float s0 = 0.f, s1 = 0.f;                                                              \
-        _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                        \
-            const unsigned short al = (unsigned short)(wa[e] & 0xffffu), ah = (unsigned short)(wa[e] >> 16); \
-            const unsigned short bl = (unsigned short)(wb[e] & 0xffffu), bh = (unsigned short)(wb[e] >> 16); \
-            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(s0) : "h"(al), "h"(bl));           \
-            asm("fma.rn.f32." TY " %0, %1, %2, %0;" : "+f"(s1) : "h"(ah), "h"(bh));           \
-        }                                                                                      \
-        return s0 + s1;                                                                        \
-    }
-template <> struct PackedDot<__nv_bfloat16> { DCN4_PACKED_DOT("bf16") };
-template <> struct PackedDot<__half> { DCN4_PACKED_DOT("f16") };
-#undef DCN4_PACKED_DOT
-
 // <a, b> where a is one 16-byte chunk of T and b the same channels already
 // unpacked to fp32 (grad_out, unpacked once per pair). For 16-bit T every
-// product is exact in fp32 (8- or 11-bit significands), so this equals
-// PackedDot bit for bit: even channels sum in .x, odd ones in .y.
+// product of two stored values is exact in fp32 (8- or 11-bit significands);
+// the sums are fp32, even channels in .x, odd ones in .y.
 template <typename T> struct DotF;
 template <> struct DotF<float> {
     static __device__ __forceinline__ float dot(const uint4 &a, const float *b) {
@@ -220,6 +190,11 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     // sorted sample records (lx, ly, m, byte offset of the source grad_out
     // vector), written over the window and record slots after phase A
     float4 *srec = reinterpret_cast<float4 *>(smem);
+    // DIRECT (16-bit weights, 16-bit grad_input): 8-byte records instead,
+    // {bf16 (1-ly)*m | bf16 ly*m, fp16 lx | grad_out offset / 16}: the owner
+    // gather reads them at random addresses, where bytes are the cost
+    constexpr bool CR = DIRECT && sizeof(T) == 2;
+    uint2 *srec8 = reinterpret_cast<uint2 *>(smem);
 
     const TileCoord tc = tile_coord(blockIdx.x, g, pl);
     const int D = g.D;
@@ -476,8 +451,16 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, v[3 * k], g.os);
             const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, v[3 * k + 1], g.os);
             const int pos = counts[cell] + rank;
-            srec[pos] = make_float4(x - floorf(x), y - floorf(y), v[3 * k + 2],
-                                    __uint_as_float((unsigned)(pix * PS + gl * D * EB)));
+            const float lx = x - floorf(x), ly = y - floorf(y), m = v[3 * k + 2];
+            const unsigned goff = (unsigned)(pix * PS + gl * D * EB);
+            if (CR) {
+                const __nv_bfloat162 wy2 = __floats2bfloat162_rn(m - ly * m, ly * m);
+                srec8[pos] = make_uint2(*reinterpret_cast<const unsigned *>(&wy2),
+                                        (unsigned)__half_as_ushort(__float2half_rn(lx)) |
+                                            ((goff >> 4) << 16));
+            } else {
+                srec[pos] = make_float4(lx, ly, m, __uint_as_float(goff));
+            }
         }
     }
     __syncthreads();
@@ -536,11 +519,21 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const int e1 = counts[row + min(qx, cells_w - 1) + 1];
             any |= e1 > e0;
             for (int e = e0; e < e1; ++e) {
-                const float4 rec4 = srec[e];
-                const float wy = a ? rec4.y : 1.0f - rec4.y;
-                const float wx = e < es ? rec4.x : 1.0f - rec4.x;
-                const float w = wy * wx * rec4.z;
-                const unsigned char *gsrc = gotile + __float_as_uint(rec4.w);
+                float w;
+                const unsigned char *gsrc;
+                if (CR) {
+                    const uint2 r = srec8[e];
+                    const float wy = __uint_as_float(a ? (r.x & 0xffff0000u) : (r.x << 16));
+                    const float lx = __half2float(__ushort_as_half((unsigned short)(r.y & 0xffffu)));
+                    w = wy * (e < es ? lx : 1.0f - lx);
+                    gsrc = gotile + ((r.y >> 16) << 4);
+                } else {
+                    const float4 rec4 = srec[e];
+                    const float wy = a ? rec4.y : 1.0f - rec4.y;
+                    const float wx = e < es ? rec4.x : 1.0f - rec4.x;
+                    w = wy * wx * rec4.z;
+                    gsrc = gotile + __float_as_uint(rec4.w);
+                }
 #pragma unroll
                 for (int c = 0; c < U; ++c) {
                     const int cc = (c + rr) & (U - 1);

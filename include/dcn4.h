@@ -95,8 +95,8 @@ typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } d
  *            ~4e-4 for fp16, against ~1.7e-3 / ~2e-4 for the rounding of
  *            the output itself), for fewer instructions per tap.
  *   DEFAULT  MIXED16 for bf16/fp16 data, F32 for fp32 data.
- * Dot products of two stored tensors (the backward's <grad_out, input>) use
- * the mixed-precision fma in every mode; there it is exact. */
+ * Dot products of two stored tensors (the backward's <grad_out, input>) are
+ * exact products of the stored values summed in fp32 in every mode. */
 typedef enum {
     DCN4_MATH_DEFAULT = 0,
     DCN4_MATH_F32 = 1,
