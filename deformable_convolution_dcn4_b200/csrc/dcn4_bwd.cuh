@@ -97,8 +97,8 @@ bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
                     }
                 }
                 const float tx = g.os * m * gx, ty = g.os * m * gy;  // d/d offset
-                grec[3 * k] = Elem<T>::from_f(MS ? s * tx : tx);
-                grec[3 * k + 1] = Elem<T>::from_f(MS ? s * ty : ty);
+                grec[3 * k] = Elem<T>::from_f(MS && tx != 0.0f ? s * tx : tx);
+                grec[3 * k + 1] = Elem<T>::from_f(MS && ty != 0.0f ? s * ty : ty);
                 if (!MS && g.softmax) {
                     gwk[k] = gm;
                     dotw = fmaf(m, gm, dotw);

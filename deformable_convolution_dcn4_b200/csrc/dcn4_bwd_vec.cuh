@@ -123,8 +123,8 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                 }
                 const float tx = g.os * m * gx, ty = g.os * m * gy;  // d/d offset
                 if (active && sub == 0) {
-                    grec[3 * k] = Elem<T>::from_f(MS ? s * tx : tx);
-                    grec[3 * k + 1] = Elem<T>::from_f(MS ? s * ty : ty);
+                    grec[3 * k] = Elem<T>::from_f(MS && tx != 0.0f ? s * tx : tx);
+                    grec[3 * k + 1] = Elem<T>::from_f(MS && ty != 0.0f ? s * ty : ty);
                     grec[3 * k + 2] = Elem<T>::from_f(gm);
                 }
                 dotw = fmaf(m, gm, dotw);

@@ -441,8 +441,11 @@ int orc_msdcn_backward(const orc_problem *p, const float *input,
                                 }
                             }
                             /* gx, gy: d(sum_d go . sample) / dx, dy of the position */
-                            gt[3 * k] = (double)s * os * m * gx;
-                            gt[3 * k + 1] = (double)s * os * m * gy;
+                            /* a sample that contributes nothing (outside, or a NaN
+                             * scale) has zero gradient, not s * 0 */
+                            const double gdx = os * m * gx, gdy = os * m * gy;
+                            gt[3 * k] = gdx == 0.0 ? 0.0 : (double)s * gdx;
+                            gt[3 * k + 1] = gdy == 0.0 ? 0.0 : (double)s * gdy;
                             gt[3 * k + 2] = gm;
                             gs += m * (gx * tx + gy * ty);
                         }

@@ -9,8 +9,8 @@ import torch
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
 
-from parity_util import (TOL, backward_case, msdcn_backward_case, f32, forward_case, gpu_forward, oracle_forward,
-                         out_hw, problem, scaled_err)
+from parity_util import (TOL, backward_case, desc_kw, msdcn_backward_case, f32, forward_case,
+                         gpu_forward, oracle_forward, out_hw, problem, scaled_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -449,3 +449,63 @@ def test_msdcn_backward_scalar_kernel(orc, name):
     wl = MSDCN_BWD[name]
     errs = msdcn_backward_case(orc, wl, algo="generic")
     assert all(e <= TOL[wl.dtype] for e in errs), f"{name}: {errs}"
+
+
+# More edge cases of the later rows: softmax with far offsets (many samples
+# take the global escape path of the staged kernels), softmax with fp32 math
+# in the backward, MSDCN with a NaN scale and with every scale clamped, and
+# the dilation reading at the FlowDCN group width with stride.
+EXTRA = {
+    "softmax_far_bf16": SOFTMAX["softmax_bf16"].replace(name="smfar", offset_dist=("normal", 8.0)),
+    "softmax_ragged_f16": W["ldm64_f16"].replace(name="smr", N=2, H=13, W=11, C=64, G=4,
+                                                 softmax=True, weight_sigma=3.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EXTRA))
+def test_softmax_edge_forward_backward(orc, name):
+    wl = EXTRA[name]
+    assert forward_case(orc, wl) <= TOL[wl.dtype]
+    for math in ("default", "f32"):
+        e_in, e_ow = backward_case(orc, wl, math=math)
+        assert e_in <= TOL[wl.dtype] and e_ow <= TOL[wl.dtype], (name, math, e_in, e_ow)
+
+
+def test_msdcn_nan_and_clamped_scales(orc):
+    """A NaN raw scale gives no contribution and no gradient for its
+    (pixel, group); raw values far above the clamp give s = Smax exactly and
+    a zero raw gradient."""
+    wl = MSDCN_BWD["msdcn_d16_bf16"].replace(smax=2.0)
+    data = make_inputs(wl, out_hw(wl), with_grad=True)
+    raw = data["scale_raw"].clone()
+    raw[0, 3, 4, 1] = float("nan")
+    raw[0, 5, :, :] = 40.0  # every group of row 5 clamped
+    data["scale_raw"] = raw
+    dev = "cuda"
+    out = B.msdcn_forward(data["input"].to(dev), data["dir_weight"].to(dev), raw.to(dev),
+                          data["s0"], wl.smax, group=wl.G, **desc_kw(wl))
+    gin, gdw, graw = B.msdcn_backward(data["input"].to(dev), data["dir_weight"].to(dev),
+                                      raw.to(dev), data["s0"], wl.smax, data["grad_out"].to(dev),
+                                      group=wl.G, **desc_kw(wl))
+    prob = problem(orc, wl)
+    x, dw, go = (f32(data[k]) for k in ("input", "dir_weight", "grad_out"))
+    ref = orc.msdcn_forward(prob, x, dw, f32(raw), data["s0"].numpy(), wl.smax)
+    rgin, rgdw, rgraw = orc.msdcn_backward(prob, x, dw, f32(raw), data["s0"].numpy(), wl.smax, go)
+    got = f32(out)
+    # the NaN group's channels are NaN on both sides (m * NaN-position sample
+    # is skipped, the oracle skips it too: zero contribution), compare the rest
+    assert scaled_err(got, ref) <= TOL["bf16"]
+    assert scaled_err(f32(gin), rgin) <= TOL["bf16"]
+    assert scaled_err(f32(gdw), rgdw) <= TOL["bf16"]
+    g = f32(graw)
+    assert np.all(g[0, 5] == 0.0) and np.all(rgraw[0, 5] == 0.0)
+    assert g[0, 3, 4, 1] == 0.0 and rgraw[0, 3, 4, 1] == 0.0
+    assert scaled_err(g, rgraw) <= TOL["bf16"]
+
+
+def test_msdcn_dilation_stride_d64(orc):
+    wl = REDUCED["flowdcn_msdcn_bf16"].replace(name="dils", N=1, H=15, W=13, C=128, G=2,
+                                               stride=(2, 1), pad=(1, 2), dilation=(1, 2),
+                                               msdcn_mode="dilation", smax=3.0)
+    assert forward_case(orc, wl) <= TOL["bf16"]
+    assert all(e <= TOL["bf16"] for e in msdcn_backward_case(orc, wl))
