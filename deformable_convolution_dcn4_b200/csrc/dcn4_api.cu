@@ -316,6 +316,10 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     if (desc->algo != DCN4_ALGO_GENERIC) {
         L.halo = halo_ok(g, L.dtype, L.msdcn, input, ow, output, &L.plan, &map, &map_ow);
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+        // vectorised global-memory kernel: whole 16-byte vectors per group,
+        // 16-byte aligned input and output
+        const int eb = elem_bytes(L.dtype);
+        L.vec = !L.halo && (g.D * eb) % 16 == 0 && aligned16(input) && aligned16(output);
     }
     L.tmap = &map;
     L.tmap_ow = &map_ow;

@@ -1,6 +1,7 @@
-// dcn4_bwd_vec.cuh -- vectorised global-memory backward of DCNv4 and of the
-// FlowDCN multi-scale variant, for the calls the shared-memory kernel does
-// not take (MSDCN, group widths other than 16/32 bytes, other kernel sizes).
+// dcn4_bwd_vec.cuh -- vectorised global-memory forward and backward of DCNv4
+// and of the FlowDCN multi-scale variant, for the calls the shared-memory
+// kernels do not take (MSDCN backward, group widths other than 32-128 bytes,
+// kernel sizes other than 3x3).
 // Included after dcn4_bwd_halo.cuh (uses its DotF, ChunkUnpack, red_add_v4).
 //
 // LPP = D * sizeof(T) / 16 lanes share one (pixel, group): lane `sub` owns
@@ -16,6 +17,82 @@
 #include "dcn4_bwd_halo.cuh"
 
 namespace dcn4 {
+
+// Forward: thread t of a (pixel, group)'s VPP = D*sizeof(T)/16 threads owns
+// one 16-byte vector of the group's channels; per tap it loads that vector
+// of each in-image corner (L1/L2) and accumulates in fp32. Positions,
+// weights and the MSDCN scale / DCNv3 softmax are formed as in
+// fwd_generic_kernel (dcn4_fwd.cuh); no lane exchanges anything.
+template <typename T, bool MS>
+__global__ void __launch_bounds__(256)
+fwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
+               T *__restrict__ out, const __grid_constant__ MsdcnParams ms) {
+    constexpr int VE = Elem<T>::kPerVec;
+    const int vpp = g.D / VE;
+    const long long total = (long long)g.N * g.Ho * g.Wo * g.G * vpp;
+    const size_t img = (size_t)g.H * g.W * g.C;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+         t += (long long)gridDim.x * blockDim.x) {
+        const int sub = (int)(t % vpp);
+        const long long pr = t / vpp;
+        const int grp = (int)(pr % g.G);
+        const long long pix = pr / g.G;
+        const int wo = (int)(pix % g.Wo);
+        const long long r2 = pix / g.Wo;
+        const int ho = (int)(r2 % g.Ho);
+        const int n = (int)(r2 / g.Ho);
+        const T *rec = ow + (size_t)pr * g.K * 3;
+        const int c0 = grp * g.D + sub * VE;
+        const T *src = in + (size_t)n * img + c0;
+        float s = 1.0f;
+        if (MS) s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[pr]), ms.s0[grp], ms.smax);
+        SoftmaxNorm sn{0.0f, 1.0f};
+        if (!MS && g.softmax) {
+            float mx = -INFINITY, sum = 0.0f;
+            for (int k = 0; k < g.K; ++k) mx = fmaxf(mx, Elem<T>::to_f(rec[3 * k + 2]));
+            for (int k = 0; k < g.K; ++k) sum += expf(Elem<T>::to_f(rec[3 * k + 2]) - mx);
+            sn = SoftmaxNorm{mx, 1.0f / sum};
+        }
+        float acc[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
+        for (int i = 0; i < g.kh; ++i) {
+            for (int j = 0; j < g.kw; ++j) {
+                const int k = i * g.kw + j;
+                const float dx = Elem<T>::to_f(rec[3 * k]);
+                const float dy = Elem<T>::to_f(rec[3 * k + 1]);
+                float m = Elem<T>::to_f(rec[3 * k + 2]);
+                if (!MS && g.softmax) m = sn.weight(m);
+                float x, y, dsx, dsy;
+                if (MS) {
+                    x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, j, g.kw, g.dw, s, dx, g.os, &dsx);
+                    y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, i, g.kh, g.dh, s, dy, g.os, &dsy);
+                } else {
+                    x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+                    y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+                }
+                if (!(x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H)) continue;
+                const float x0f = floorf(x), y0f = floorf(y);
+                const float lx = x - x0f, ly = y - y0f;
+                const int x0 = (int)x0f, y0 = (int)y0f;
+                uint4 q[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int yy = y0 + (c >> 1), xx = x0 + (c & 1);
+                    q[c] = (yy >= 0 && yy < g.H && xx >= 0 && xx < g.W)
+                               ? __ldg(reinterpret_cast<const uint4 *>(src + ((size_t)yy * g.W + xx) * g.C))
+                               : make_uint4(0u, 0u, 0u, 0u);
+                }
+                const float mly = m * ly, mhy = m - mly;
+                VecMath<T>::fma(acc, q[0], mhy - mhy * lx);
+                VecMath<T>::fma(acc, q[1], mhy * lx);
+                VecMath<T>::fma(acc, q[2], mly - mly * lx);
+                VecMath<T>::fma(acc, q[3], mly * lx);
+            }
+        }
+        *reinterpret_cast<uint4 *>(out + (size_t)pix * g.C + c0) = VecMath<T>::pack(acc);
+    }
+}
 
 template <typename T, bool MS, int LPP>
 __global__ void __launch_bounds__(256)

@@ -136,9 +136,21 @@ cudaError_t launch_generic_t(const FwdLaunch &L) {
     return cudaGetLastError();
 }
 
+template <typename T, bool MS>
+cudaError_t launch_fwd_vec_t(const FwdLaunch &L) {
+    const long long work = (long long)L.geo.N * L.geo.Ho * L.geo.Wo * L.geo.G *
+                           (L.geo.D / Elem<T>::kPerVec);
+    fwd_vec_kernel<T, MS><<<grid_for(work, 256), 256, 0, L.stream>>>(
+        L.geo, static_cast<const T *>(L.in), static_cast<const T *>(L.ow), static_cast<T *>(L.out),
+        L.ms ? *L.ms : kNoMs);
+    count_launch();
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_fwd_t(const FwdLaunch &L) {
     if (L.halo) return L.msdcn ? launch_halo_u<T, true>(L) : launch_halo_u<T, false>(L);
+    if (L.vec) return L.msdcn ? launch_fwd_vec_t<T, true>(L) : launch_fwd_vec_t<T, false>(L);
     return L.msdcn ? launch_generic_t<T, true>(L) : launch_generic_t<T, false>(L);
 }
 

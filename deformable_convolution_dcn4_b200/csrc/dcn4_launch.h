@@ -19,6 +19,7 @@ struct FwdLaunch {
     void *out;
     const MsdcnParams *ms;  // MSDCN only
     bool halo;              // use the shared-memory halo kernel
+    bool vec;               // otherwise the vectorised global-memory kernel (else scalar)
     int mathv;              // 0 fp32 weights, 1 mixed-precision fma, 2 packed 16-bit blend
     HaloPlan plan;
     const CUtensorMap *tmap;

@@ -70,11 +70,12 @@ typedef enum {
 typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
 
 /* Kernel selection. AUTO picks the staged (shared-memory halo) kernel when
- * the call qualifies and a global-memory kernel otherwise (for the backward:
- * the vectorised one when the group width is a power-of-two count of 16-byte
- * vectors and the tensors are 16-byte aligned, else the scalar one). GENERIC
- * forces the scalar global-memory kernel and HALO the staged one (a forced
- * variant the call does not qualify for returns DCN4_ERR_UNSUPPORTED). */
+ * the call qualifies and a global-memory kernel otherwise: the vectorised one
+ * (16-byte vector loads, several threads per (pixel, group)) when a group's
+ * channels are whole 16-byte vectors (backward: a power-of-two count of them,
+ * at most 16) and the tensors are 16-byte aligned, else the scalar one.
+ * GENERIC forces the scalar global-memory kernel and HALO the staged one (a
+ * forced variant the call does not qualify for returns DCN4_ERR_UNSUPPORTED). */
 typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
 
 /* Multiply precision of the bilinear weights in the bf16/fp16 halo kernels

@@ -509,3 +509,28 @@ def test_msdcn_dilation_stride_d64(orc):
                                                msdcn_mode="dilation", smax=3.0)
     assert forward_case(orc, wl) <= TOL["bf16"]
     assert all(e <= TOL["bf16"] for e in msdcn_backward_case(orc, wl))
+
+
+# Forward shapes the staged kernel does not take, on both global-memory
+# kernels: AUTO runs the vectorised one (whole 16-byte vectors per group,
+# aligned tensors), "generic" the scalar one.
+FWD_VEC = {
+    "k5_bf16": BWD_VEC["k5_bf16"],
+    "k3x1_f16": BWD_VEC["k3x1_f16_d8"],
+    "d64_f32": BWD_VEC["d64_f32"],
+    "d256_bf16": W["internimage_bf16"].replace(name="d256", N=1, H=9, W=7, C=512, G=2),
+    "softmax_k5_f32": W["tiny_f32"].replace(name="smk5", N=1, H=10, W=9, C=32, G=2, kh=5, kw=5,
+                                            pad=(2, 2), softmax=True, weight_sigma=1.0),
+    "msdcn_k5_bf16": MSDCN_BWD["msdcn_d16_bf16"].replace(name="msk5", H=12, W=11, kh=5, kw=5,
+                                                        pad=(2, 2)),
+    "msdcn_dil_k5_f32": MSDCN_BWD["msdcn_d16_f32"].replace(name="msdk5", kh=5, kw=5, pad=(2, 2),
+                                                          msdcn_mode="dilation", smax=2.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FWD_VEC))
+@pytest.mark.parametrize("algo", ["auto", "generic"])
+def test_forward_global_kernels(orc, name, algo):
+    wl = FWD_VEC[name]
+    err = forward_case(orc, wl, algo)
+    assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
