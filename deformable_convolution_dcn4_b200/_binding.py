@@ -17,7 +17,7 @@ STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
           3: "DCN4_ERR_WORKSPACE", 4: "DCN4_ERR_CUDA", 5: "DCN4_ERR_TIMEOUT",
           6: "DCN4_ERR_INTERNAL"}
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
-ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2}
+ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2, "vector": 3}
 MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2, "packed16": 3}
 MSDCN_MODE_CODE = {"offset": 0, "dilation": 1}
 

@@ -34,7 +34,8 @@ bool out_hw(const dcn4_desc &d, int *Ho, int *Wo) {
 bool make_geometry(const dcn4_desc *d, Geometry *g) {
     if (!d) return false;
     if (d->dtype != DCN4_F32 && d->dtype != DCN4_BF16 && d->dtype != DCN4_F16) return false;
-    if (d->algo != DCN4_ALGO_AUTO && d->algo != DCN4_ALGO_GENERIC && d->algo != DCN4_ALGO_HALO)
+    if (d->algo != DCN4_ALGO_AUTO && d->algo != DCN4_ALGO_GENERIC && d->algo != DCN4_ALGO_HALO &&
+        d->algo != DCN4_ALGO_VECTOR)
         return false;
     if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16 &&
         d->math != DCN4_MATH_PACKED16)
@@ -313,13 +314,16 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     CUtensorMap map, map_ow;
     memset(&map, 0, sizeof(map));
     memset(&map_ow, 0, sizeof(map_ow));
-    if (desc->algo != DCN4_ALGO_GENERIC) {
+    if (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) {
         L.halo = halo_ok(g, L.dtype, L.msdcn, input, ow, output, &L.plan, &map, &map_ow);
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+    }
+    if (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_VECTOR) {
         // vectorised global-memory kernel: whole 16-byte vectors per group,
         // 16-byte aligned input and output
         const int eb = elem_bytes(L.dtype);
         L.vec = !L.halo && (g.D * eb) % 16 == 0 && aligned16(input) && aligned16(output);
+        if (!L.vec && desc->algo == DCN4_ALGO_VECTOR) return DCN4_ERR_UNSUPPORTED;
     }
     L.tmap = &map;
     L.tmap_ow = &map_ow;
@@ -389,7 +393,7 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
     memset(&map_in, 0, sizeof(map_in));
     memset(&map_go, 0, sizeof(map_go));
     memset(&map_ow, 0, sizeof(map_ow));
-    if (desc->algo != DCN4_ALGO_GENERIC) {
+    if (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) {
         const bool base = !L.msdcn && g.kh == 3 && g.kw == 3 && aligned16(input) &&
                           aligned16(offset_weight) && aligned16(grad_out) && aligned16(L.acc);
         auto maps = [&]() {
@@ -410,9 +414,10 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
     // vectorised global-memory kernel: whole 16-byte vectors per group, a
     // power-of-two count of them (<= 16), 16-byte aligned tensors
     const int vb = g.D * eb;
-    L.vec = !L.halo && desc->algo != DCN4_ALGO_GENERIC && vb % 16 == 0 && vb <= 256 &&
-            ((vb / 16) & (vb / 16 - 1)) == 0 && aligned16(input) && aligned16(grad_out) &&
-            aligned16(L.acc);
+    L.vec = !L.halo && (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_VECTOR) &&
+            vb % 16 == 0 && vb <= 256 && ((vb / 16) & (vb / 16 - 1)) == 0 && aligned16(input) &&
+            aligned16(grad_out) && aligned16(L.acc);
+    if (!L.vec && desc->algo == DCN4_ALGO_VECTOR) return DCN4_ERR_UNSUPPORTED;
     L.tmap_in = &map_in;
     L.tmap_go = &map_go;
     L.tmap_ow = &map_ow;

@@ -74,9 +74,15 @@ typedef enum { DCN4_F32 = 0, DCN4_BF16 = 1, DCN4_F16 = 2 } dcn4_dtype;
  * (16-byte vector loads, several threads per (pixel, group)) when a group's
  * channels are whole 16-byte vectors (backward: a power-of-two count of them,
  * at most 16) and the tensors are 16-byte aligned, else the scalar one.
- * GENERIC forces the scalar global-memory kernel and HALO the staged one (a
- * forced variant the call does not qualify for returns DCN4_ERR_UNSUPPORTED). */
-typedef enum { DCN4_ALGO_AUTO = 0, DCN4_ALGO_GENERIC = 1, DCN4_ALGO_HALO = 2 } dcn4_algo;
+ * GENERIC forces the scalar global-memory kernel, VECTOR the vectorised one
+ * and HALO the staged one (a forced variant the call does not qualify for
+ * returns DCN4_ERR_UNSUPPORTED). */
+typedef enum {
+    DCN4_ALGO_AUTO = 0,
+    DCN4_ALGO_GENERIC = 1,
+    DCN4_ALGO_HALO = 2,
+    DCN4_ALGO_VECTOR = 3
+} dcn4_algo;
 
 /* Multiply precision of the bilinear weights in the bf16/fp16 halo kernels
  * (fp32 calls and the generic kernels always use fp32).

@@ -529,8 +529,30 @@ FWD_VEC = {
 
 
 @pytest.mark.parametrize("name", sorted(FWD_VEC))
-@pytest.mark.parametrize("algo", ["auto", "generic"])
+@pytest.mark.parametrize("algo", ["auto", "vector", "generic"])
 def test_forward_global_kernels(orc, name, algo):
     wl = FWD_VEC[name]
     err = forward_case(orc, wl, algo)
     assert err <= TOL[wl.dtype], f"{name}/{algo}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", ["internimage_bf16", "highres_bf16", "flowdcn_msdcn_bf16",
+                                  "internimage_f32"])
+def test_vector_kernels_on_staged_shapes(orc, name):
+    """DCN4_ALGO_VECTOR forces the vectorised global-memory kernels on shapes
+    AUTO would stage: same oracle, same gates."""
+    wl = REDUCED[name]
+    assert forward_case(orc, wl, "vector") <= TOL[wl.dtype]
+    if wl.kind == "msdcn":
+        errs = msdcn_backward_case(orc, wl.replace(N=1), algo="vector")
+        assert all(e <= TOL[wl.dtype] for e in errs), errs
+    else:
+        e_in, e_ow = backward_case(orc, wl, "vector")
+        assert e_in <= TOL[wl.dtype] and e_ow <= TOL[wl.dtype], (e_in, e_ow)
+
+
+def test_vector_request_on_unaligned_groups_is_unsupported():
+    wl = GENERIC_ONLY["d12_bf16"]
+    with pytest.raises(B.Dcn4Error) as e:
+        forward_case(None, wl, "vector")
+    assert e.value.code == 2
