@@ -140,9 +140,9 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, bool rec_tma, HaloPlan *ou
 }
 
 // Tiling and shared-memory layout of the backward halo kernel: one
-// (pixel, group) pair per thread (512 threads), 128-byte staged pixels,
-// R = 4, and the sorted sample records (14 bytes each) must fit in the
-// window buffer they reuse.
+// (pixel, group) pair per thread (256 or 512 threads), 128-byte staged
+// pixels, R = 4; the sorted sample records (8 or 16 bytes each) reuse the
+// window and record slots, so they must fit there.
 bool plan_bwd(const Geometry &g, int eb, bool rec_tma, HaloPlan *out, BwdLayout *lay) {
     if (128 % (g.D * eb) != 0) return false;
     const int Gc = 128 / (g.D * eb);

@@ -11,20 +11,22 @@
 // lane-operations per corner, so the kernel transposes instead: it sorts the
 // CTA's samples by destination cell (one integer atomic per sample), and each
 // (staged pixel, group) then gathers the contributions of the four cells it
-// is a corner of, accumulating in registers, and adds the sum to the fp32
-// workspace with 16-byte vector reductions (neighbouring tiles' windows
-// overlap, so the workspace is shared).
+// is a corner of, accumulating in registers, and adds the sum to grad_input
+// with 16-byte vector reductions (neighbouring tiles' windows overlap): packed
+// 16-bit reductions into the 16-bit grad_input itself (DIRECT), else fp32
+// reductions into the workspace.
 //
 // One CTA per (image, output tile, group slice); NW warps; phases:
-//   stage  TMA: input window + grad_out tile; bulk copies: records
+//   stage  TMA: input window + grad_out tile (+ records when the pixel stride
+//          allows a TMA tile copy); else bulk copies of the records
 //   A      per (pixel, group): corner gathers, the three gradients per tap,
 //          count each staged sample into its cell (rank = atomic result)
 //   B      exclusive scan of the cell counts
-//   C      per (pixel, group): write (lx, ly, m, pair) of each staged sample
-//          at offset[cell] + rank, into the window buffer (no longer needed)
-//   D      per (staged pixel, group): gather from its four cells, flush
+//   C      per (pixel, group): write each staged sample's record at
+//          offset[cell] + rank, over the window buffer (no longer needed)
 //   E      copy the staged grad_offset_weight out with coalesced stores
-// Samples outside the staged window take a global path with fp32 atomics.
+//   D      per (staged pixel, group): gather from its four cells, flush
+// Samples outside the staged window take a global path with atomics.
 #pragma once
 
 #include "dcn4_fwd.cuh"

@@ -79,7 +79,7 @@ struct HaloPlan {
     int tiles_h, tiles_w, slices;
     int slot_bytes;      // bytes per output pixel of staged offset/weight triples
     int halo_bytes;      // HR*HC*Gc*D*elem, rounded up to 128
-    int stages;          // 2: double-buffered (512 threads), 1: single (256 threads)
+    int stages;          // 2: double-buffered pipeline, 1: single buffer
     int smem_bytes;      // dynamic shared memory of one CTA
     int rec_tma;         // 1: records arrive by one TMA tile copy per tile (forward)
     int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)

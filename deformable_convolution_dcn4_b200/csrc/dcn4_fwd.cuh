@@ -7,14 +7,15 @@
 // p_k + dp_k)[g*D + d], with the D channels of a group sharing the offsets and
 // weights, and for MSDCN dp_k = s_g(p0) * dir_k.
 //
-// Two kernels:
+// Two kernels here (the vectorised global-memory one is in dcn4_bwd_vec.cuh):
 //  * fwd_generic_kernel: one thread per (pixel, group, run of <= 8 channels),
 //    scalar loads straight from global memory. Any shape, any alignment.
 //  * fwd_halo_kernel: one thread per (pixel, group) covering all D channels.
 //    A CTA owns an output tile x a slice of Gc groups. One TMA tile load
 //    brings the input window the tile can reach (tile +- R pixels, zeros
 //    outside the image by the TMA out-of-bounds fill) into shared memory, and
-//    bulk copies bring the tile's offset/weight records. Every corner gather
+//    a second TMA tile copy (or, when the pixel stride rules that out,
+//    per-pixel bulk copies) brings the tile's offset/weight records. Every corner gather
 //    is then a 16-byte shared-memory load; samples that leave the window use
 //    16-byte global loads instead. Lanes rotate the order of their 16-byte
 //    chunks so that the 8 lanes of each shared-memory phase hit 8 different
@@ -468,11 +469,12 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
 }
 
 // Persistent halo kernel. CTA b handles tiles b, b + gridDim.x, ...; thread
-// t of the NW warps owns (pixel, group) pairs t, t + 32NW, ... of every tile,
-// so each warp consumes the records of its own tile pixels: it bulk-copies
-// those itself and waits on its own barrier (rec[w][s]). The
-// input window is shared: warp 0 loads it (win[s]) once every warp has
-// released the buffer (empty[s], NW arrivals). With STAGES == 2 the copies of
+// t of the NW warps owns (pixel, group) pairs t, t + 32NW, ... of every tile.
+// The input window (and, with pl.rec_tma, the tile's records) is shared:
+// warp 0 loads it (win[s]) once every warp has released the buffer
+// (empty[s], NW arrivals). Without pl.rec_tma each warp consumes the records
+// of its own tile pixels: it bulk-copies those itself and waits on its own
+// barrier (rec[w][s]). With STAGES == 2 the copies of
 // the next tile are in flight while the current one is computed. Every wait
 // is bounded; on expiry the warp sets the error word, lets its own copies in
 // flight land and returns.
