@@ -126,6 +126,30 @@ template <> struct DotF<__half> {
     }
 };
 
+// <a, b> with both chunks packed 16-bit: the sm_100 mixed-precision fma
+// (exact 16x16-bit products, fp32 sums); fp32 falls back to DotF.
+template <typename T> struct PackedDotM {
+    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {
+        float bf[4] = {__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z),
+                       __uint_as_float(b.w)};
+        return DotF<float>::dot(a, bf);
+    }
+};
+#define DCN4_PDOT(TY)                                                                          \
+    static __device__ __forceinline__ float dot(const uint4 &a, const uint4 &b) {              \
+        const unsigned wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};             \
+        float s0 = 0.f, s1 = 0.f;                                                              \
+        _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                        \
+            asm("{ .reg .b16 al, ah, bl, bh; mov.b32 {al, ah}, %2; mov.b32 {bl, bh}, %3;"      \
+                " fma.rn.f32." TY " %0, al, bl, %0; fma.rn.f32." TY " %1, ah, bh, %1; }"       \
+                : "+f"(s0), "+f"(s1) : "r"(wa[e]), "r"(wb[e]));                              \
+        }                                                                                      \
+        return s0 + s1;                                                                        \
+    }
+template <> struct PackedDotM<__nv_bfloat16> { DCN4_PDOT("bf16") };
+template <> struct PackedDotM<__half> { DCN4_PDOT("f16") };
+#undef DCN4_PDOT
+
 // Block-wide exclusive scan of counts[0..n) in place; counts[n] = total.
 template <int NW>
 __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *warp_sums) {
@@ -318,16 +342,17 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         }
         float dotw = 0.0f;
         const unsigned char *row0[U], *row1[U];
-        // gof[c]: this pair's grad_out chunk (c + r) mod U, unpacked to fp32
+        // gof[c]: this pair's grad_out chunk (c + r) mod U, unpacked to fp32;
+        // gop[c] the same chunk packed
         float gof[U][VE];
+        uint4 gop[U];
 #pragma unroll
         for (int c = 0; c < U; ++c) {
             const int cc = (c + r) & (U - 1);
             row0[c] = halo + (size_t)gl * D * EB + cc * 16;
             row1[c] = row0[c] + RS;
-            ChunkUnpack<T>::get(
-                *reinterpret_cast<const uint4 *>(gotile + (size_t)pix * PS + gl * D * EB + cc * 16),
-                gof[c]);
+            gop[c] = *reinterpret_cast<const uint4 *>(gotile + (size_t)pix * PS + gl * D * EB + cc * 16);
+            ChunkUnpack<T>::get(gop[c], gof[c]);
         }
         const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
         const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
@@ -356,10 +381,10 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 for (int c = 0; c < U; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
-                    d00 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a0), gof[c]);
-                    d01 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a0 + PS), gof[c]);
-                    d10 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a1), gof[c]);
-                    d11 += DotF<T>::dot(*reinterpret_cast<const uint4 *>(a1 + PS), gof[c]);
+                    d00 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a0), gop[c]);
+                    d01 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a0 + PS), gop[c]);
+                    d10 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a1), gop[c]);
+                    d11 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a1 + PS), gop[c]);
                 }
                 gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
                 gx = g.os * m * (hy * (d01 - d00) + ly * (d11 - d10));
