@@ -43,6 +43,8 @@ class Oracle:
         lib.orc_msdcn_backward.argtypes = [P, _F32P, _F32P, _F32P, _F32P, ctypes.c_float, _F32P,
                                            _F64P, _F64P, _F64P]
         lib.orc_msdcn_backward.restype = ctypes.c_int
+        lib.orc_offset_producer.argtypes = [P, _F32P, _F32P, _F32P, _F32P, _F32P, _F64P]
+        lib.orc_offset_producer.restype = ctypes.c_int
         lib.orc_msdcn_scale.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
         lib.orc_msdcn_scale.restype = ctypes.c_float
         for name in ("orc_flops",):
@@ -111,6 +113,18 @@ class Oracle:
         if rc:
             raise ValueError("orc_msdcn_backward failed")
         return gin, gdw, graw
+
+    def offset_producer(self, prob, x, dw_weight, dw_bias, lin_weight, lin_bias):
+        """offset_weight [N][H][W][G][kh*kw][3] from the depthwise 3x3 + linear
+        sub-network (dw_weight [3][3][C], lin_weight [G*kh*kw*3][C])."""
+        J = prob.G * prob.kh * prob.kw * 3
+        out = np.empty((prob.N, prob.H, prob.W, J), np.float64)
+        rc = self.lib.orc_offset_producer(ctypes.byref(prob), self._f32(x), self._f32(dw_weight),
+                                          self._f32(dw_bias), self._f32(lin_weight),
+                                          self._f32(lin_bias), out)
+        if rc:
+            raise ValueError("orc_offset_producer failed")
+        return out.reshape(prob.N, prob.H, prob.W, prob.G, prob.kh * prob.kw, 3)
 
     def msdcn_scale(self, raw, s0, smax):
         return self.lib.orc_msdcn_scale(float(raw), float(s0), float(smax))

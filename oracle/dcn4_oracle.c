@@ -463,6 +463,56 @@ int orc_msdcn_backward(const orc_problem *p, const float *input,
 
 /* FLOPs: 4 (bilinear terms) per tap per output element, i.e. 36 HWC for a
  * 3x3 kernel with H, W the output size. */
+/* Offset/weight producer of the DCNv4 module ([DIGEST] "方法3. DCN模块的微设计优化":
+ * once softmax is gone, one linear layer emits both the offsets and the
+ * aggregation weights, and the sub-network in front of it is a plain
+ * separable convolution, a depthwise 3x3 then that linear layer, without the
+ * DCNv3 LayerNorm and GELU).  For every pixel (n, y, x) of the H x W map:
+ *   h[c]  = dw_b[c] + sum_{i,j in 0..2} dw_w[i][j][c] * x[n][y+i-1][x+j-1][c]
+ *           (stride 1, zero outside the image),
+ *   out[j] = lin_b[j] + sum_c lin_w[j][c] * h[c],   j in [0, G*kh*kw*3),
+ * so out[n][y][x] is laid out exactly like offset_weight [G][kh*kw][3].
+ * dw_w is [3][3][C] (tap-major), dw_b [C], lin_w [G*kh*kw*3][C] (output
+ * row-major), lin_b [G*kh*kw*3]; all accumulation in fp64.  Returns 0, or
+ * -1 for a malformed problem. */
+int orc_offset_producer(const orc_problem *p, const float *x, const float *dw_w,
+                        const float *dw_b, const float *lin_w, const float *lin_b,
+                        double *out)
+{
+    if (orc_out_hw(p, NULL, NULL) != 0)
+        return -1;
+    const int H = p->H, W = p->W, C = p->C;
+    const int J = p->G * p->kh * p->kw * 3;
+    double *h = (double *)malloc(sizeof(double) * (size_t)C);
+    if (!h)
+        return -1;
+    for (int n = 0; n < p->N; ++n)
+        for (int y = 0; y < H; ++y)
+            for (int xx = 0; xx < W; ++xx) {
+                for (int c = 0; c < C; ++c) {
+                    double acc = dw_b[c];
+                    for (int i = 0; i < 3; ++i)
+                        for (int j = 0; j < 3; ++j) {
+                            const int yy = y + i - 1, xs = xx + j - 1;
+                            if (yy < 0 || yy >= H || xs < 0 || xs >= W)
+                                continue;
+                            acc += (double)dw_w[(i * 3 + j) * C + c] *
+                                   (double)x[(((size_t)n * H + yy) * W + xs) * C + c];
+                        }
+                    h[c] = acc;
+                }
+                double *o = out + (((size_t)n * H + y) * W + xx) * (size_t)J;
+                for (int j = 0; j < J; ++j) {
+                    double acc = lin_b[j];
+                    for (int c = 0; c < C; ++c)
+                        acc += (double)lin_w[(size_t)j * C + c] * h[c];
+                    o[j] = acc;
+                }
+            }
+    free(h);
+    return 0;
+}
+
 double orc_flops(const orc_problem *p)
 {
     int Ho, Wo;

@@ -43,6 +43,12 @@ What pins what (pages cited by title and section):
                     DCNv4 bit for bit; s = 2, dir = 0 == DCNv4 at twice the
                     dilation (pad + dilation) bit for bit; backward by central
                     differences (dir exact at s = 2; raw smooth)
+  pin_producer      offset/weight producer (DCNv4 digest "方法3. DCN模块的微设计优化":
+                    depthwise 3x3 + one merged linear): the depthwise part ==
+                    torch conv2d(groups=C) in float64, the linear part == a
+                    float64 matmul, the composition == conv2d + F.linear, and
+                    a constant map through all-ones taps counts the in-image
+                    taps exactly (4 at corners, 6 on edges, 9 inside)
 """
 import json
 import math
@@ -657,8 +663,64 @@ def pin_msdcn_dilation(o):
         assert abs(fd - graw[idx]) <= 2e-3 * max(1.0, abs(graw[idx])), f"dilation d/d raw {idx}"
 
 
+def _producer_ref(x, dw_w, dw_b, lin_w, lin_b):
+    """torch float64: conv2d(groups=C, padding 1) then F.linear."""
+    C = x.shape[-1]
+    xt = torch.from_numpy(x.astype(np.float64)).permute(0, 3, 1, 2)
+    wt = torch.from_numpy(dw_w.astype(np.float64).transpose(2, 0, 1)[:, None].copy())
+    h = F.conv2d(xt, wt, torch.from_numpy(dw_b.astype(np.float64)), padding=1, groups=C)
+    h = h.permute(0, 2, 3, 1)
+    out = F.linear(h, torch.from_numpy(lin_w.astype(np.float64)),
+                   torch.from_numpy(lin_b.astype(np.float64)))
+    return h.numpy(), out.numpy()
+
+
+def pin_producer(o):
+    for ci, (N, H, W, C, G, kh, kw) in enumerate([(2, 5, 7, 6, 3, 3, 3), (1, 4, 3, 8, 2, 1, 3),
+                                                   (1, 1, 6, 4, 1, 3, 3)]):
+        rng = _rng(900 + ci)
+        prob = o.problem(N, H, W, C, G, kh, kw, pad=((kh - 1) // 2, (kw - 1) // 2))
+        J = G * kh * kw * 3
+        x = rng.standard_normal((N, H, W, C)).astype(np.float32)
+        dw_w = rng.standard_normal((3, 3, C)).astype(np.float32)
+        dw_b = rng.standard_normal(C).astype(np.float32)
+        lin_w = rng.standard_normal((J, C)).astype(np.float32)
+        lin_b = rng.standard_normal(J).astype(np.float32)
+        h_ref, ref = _producer_ref(x, dw_w, dw_b, lin_w, lin_b)
+        got = o.offset_producer(prob, x, dw_w, dw_b, lin_w, lin_b).reshape(N, H, W, J)
+        _close(got, ref, 1e-12, f"producer case {ci} vs conv2d + linear")
+        # selection rows: out[j] = h[j % C] isolates the depthwise part
+        sel = np.zeros((J, C), np.float32)
+        sel[np.arange(J), np.arange(J) % C] = 1.0
+        got = o.offset_producer(prob, x, dw_w, dw_b, sel, np.zeros(J, np.float32))
+        _close(got.reshape(N, H, W, J), h_ref[..., np.arange(J) % C], 1e-12,
+               f"producer case {ci} depthwise part")
+        # identity depthwise (centre tap 1): out = x @ lin_w^T + lin_b
+        ident = np.zeros((3, 3, C), np.float32)
+        ident[1, 1] = 1.0
+        got = o.offset_producer(prob, x, ident, np.zeros(C, np.float32), lin_w, lin_b)
+        lin = x.astype(np.float64) @ lin_w.astype(np.float64).T + lin_b
+        _close(got.reshape(N, H, W, J), lin, 1e-12, f"producer case {ci} linear part")
+        # all-ones taps on a constant map count the in-image taps
+        got = o.offset_producer(prob, np.ones_like(x), np.ones((3, 3, C), np.float32),
+                                np.zeros(C, np.float32), sel, np.zeros(J, np.float32))
+        cnt = np.zeros((H, W))
+        for y in range(H):
+            for xx in range(W):
+                cnt[y, xx] = (min(y + 1, H - 1) - max(y - 1, 0) + 1) * \
+                             (min(xx + 1, W - 1) - max(xx - 1, 0) + 1)
+        assert np.array_equal(got.reshape(N, H, W, J), np.broadcast_to(
+            cnt[None, :, :, None], (N, H, W, J))), f"producer case {ci} tap counts"
+    # the counts themselves, written out on a 3 x 3 map
+    prob = o.problem(1, 3, 3, 1, 1, 1, 1, pad=(0, 0))
+    got = o.offset_producer(prob, np.ones((1, 3, 3, 1), np.float32),
+                            np.ones((3, 3, 1), np.float32), np.zeros(1, np.float32),
+                            np.ones((3, 1), np.float32), np.zeros(3, np.float32))
+    assert np.array_equal(got[0, :, :, 0, 0, 0], [[4, 6, 4], [6, 9, 6], [4, 6, 4]])
+
+
 ALL_PINS = [pin_conv, pin_grid_sample, pin_gather, pin_fractions, pin_out_of_bounds,
             pin_linearity, pin_equivariance, pin_msdcn, pin_cost_model, pin_adjoint,
             pin_unit_columns, pin_finite_diff, pin_msdcn_bwd_unit, pin_msdcn_bwd_adjoint,
             pin_msdcn_bwd_dir, pin_msdcn_bwd_raw, pin_softmax_box, pin_softmax_shift,
-            pin_softmax_bwd, pin_msdcn_dilation]
+            pin_softmax_bwd, pin_msdcn_dilation, pin_producer]

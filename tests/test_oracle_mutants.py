@@ -75,6 +75,12 @@ MUTANTS = [
      "float cx = (float)(wo * p->sw - p->pw);", 1),
     ("dilation_grid_unscaled", "*x = cx + sx;", "*x = cx + kx + s * ox;", 1),
     ("dilation_ds_missing_grid", "*tx = (double)ux;", "*tx = (double)ox;", 1),
+    ("producer_dw_bias_dropped", "double acc = dw_b[c];", "double acc = 0.0;", 1),
+    ("producer_lin_bias_dropped", "double acc = lin_b[j];", "double acc = 0.0;", 1),
+    ("producer_lin_transposed", "(double)lin_w[(size_t)j * C + c]", "(double)lin_w[(size_t)c * J + j]", 1),
+    ("producer_taps_transposed", "dw_w[(i * 3 + j) * C + c]", "dw_w[(j * 3 + i) * C + c]", 1),
+    ("producer_pad_shift", "const int yy = y + i - 1, xs = xx + j - 1;",
+     "const int yy = y + i - 1, xs = xx + j;", 1),
     ("flops_factor", "return 4.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;",
      "return 2.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->C;", 1),
     ("ideal_offsets_per_channel", "double ow = 3.0 * p->kh * p->kw * (double)p->N * Ho * Wo * p->G;",
