@@ -25,7 +25,7 @@ MSDCN_MODE_CODE = {"offset": 0, "dilation": 1}
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
            "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches",
-           "msdcn_backward")
+           "msdcn_backward", "dcn4_offset_producer")
 
 
 class Dcn4Error(RuntimeError):
@@ -70,6 +70,7 @@ def load(path=LIBRARY):
     lib.dcn4_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.dcn4_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
     lib.dcn4_kernel_launches.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.dcn4_offset_producer.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -147,6 +148,29 @@ def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, di
     _require(out, "out", input.dtype, (N, ho, wo, C))
     _check("dcn4_forward", load().dcn4_forward(ctypes.byref(desc), _ptr(input), _ptr(offset_weight),
                                                _ptr(out), _stream(input)))
+    return out
+
+
+def dcn4_offset_producer(x, dw_weight, dw_bias, lin_weight, lin_bias, group, kernel_size=3,
+                         stride=1, pad=1, dilation=1, algo="auto", out=None):
+    """offset_weight [N,H,W,G,kh*kw,3] from the depthwise 3x3 + merged linear
+    sub-network: x [N,H,W,C], dw_weight [3,3,C], dw_bias [C],
+    lin_weight [G*kh*kw*3, C], lin_bias [G*kh*kw*3], all of x's dtype."""
+    desc = _desc_for(x, group, kernel_size, stride, pad, dilation, 1.0, algo)
+    N, H, W, C = x.shape
+    J = group * desc.kh * desc.kw * 3
+    _require(x, "x", x.dtype)
+    _require(dw_weight, "dw_weight", x.dtype, (3, 3, C))
+    _require(dw_bias, "dw_bias", x.dtype, (C,))
+    _require(lin_weight, "lin_weight", x.dtype, (J, C))
+    _require(lin_bias, "lin_bias", x.dtype, (J,))
+    shape = (N, H, W, group, desc.kh * desc.kw, 3)
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    _require(out, "out", x.dtype, shape)
+    _check("dcn4_offset_producer",
+           load().dcn4_offset_producer(ctypes.byref(desc), _ptr(x), _ptr(dw_weight), _ptr(dw_bias),
+                                       _ptr(lin_weight), _ptr(lin_bias), _ptr(out), _stream(x)))
     return out
 
 

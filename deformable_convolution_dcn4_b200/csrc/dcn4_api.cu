@@ -347,6 +347,46 @@ dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input, const void *o
     return run_forward(desc, input, offset_weight, output, stream, nullptr);
 }
 
+dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const void *dw_weight,
+                                 const void *dw_bias, const void *lin_weight,
+                                 const void *lin_bias, void *offset_weight, void *stream) {
+    Geometry g;
+    if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
+    if (!x || !dw_weight || !dw_bias || !lin_weight || !lin_bias || !offset_weight)
+        return DCN4_ERR_INVALID_ARG;
+    if (g.Ho != g.H || g.Wo != g.W) return DCN4_ERR_UNSUPPORTED;
+    ProducerLaunch L;
+    memset(&L, 0, sizeof(L));
+    L.dtype = static_cast<Dtype>(desc->dtype);
+    L.pg.N = g.N;
+    L.pg.H = g.H;
+    L.pg.W = g.W;
+    L.pg.C = g.C;
+    L.pg.J = g.G * g.K * 3;
+    L.pg.NP = (L.pg.J + 15) / 16 * 16;
+    L.pg.npix = (long long)g.N * g.H * g.W;
+    const long long ntiles = (L.pg.npix + 127) / 128;
+    if (ntiles > std::numeric_limits<int>::max()) return DCN4_ERR_UNSUPPORTED;
+    L.pg.ntiles = (int)ntiles;
+    L.x = x;
+    L.dw_w = dw_weight;
+    L.dw_b = dw_bias;
+    L.lin_w = lin_weight;
+    L.lin_b = lin_bias;
+    L.out = offset_weight;
+    L.stream = static_cast<cudaStream_t>(stream);
+    const int eb = elem_bytes(L.dtype);
+    // tensor-core kernel: 16-bit data, K = C in steps of 16, N = J padded to
+    // 16 <= 256, whole 16-byte output rows, lin_w resident in shared memory
+    const ProducerTcLayout lay = ProducerTcLayout::make(g.C, L.pg.J, L.pg.NP);
+    L.tc = desc->algo != DCN4_ALGO_GENERIC && eb == 2 && g.C % 16 == 0 && L.pg.NP <= 256 &&
+           (L.pg.J * eb) % 16 == 0 && aligned16(x) && aligned16(lin_weight) &&
+           aligned16(offset_weight) && lay.bytes <= max_smem_optin();
+    if (!L.tc && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+    if (!L.tc && kProducerPixels * g.C * 4 > max_smem_optin()) return DCN4_ERR_UNSUPPORTED;
+    return cuda_status(launch_producer(L));
+}
+
 dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes) {
     Geometry g;
     if (!make_geometry(desc, &g) || !bytes) return DCN4_ERR_INVALID_ARG;

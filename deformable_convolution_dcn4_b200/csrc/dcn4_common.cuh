@@ -29,6 +29,38 @@ struct Geometry {
     int msd_dil;  // MSDCN scale-as-dilation reading
 };
 
+// Pixels per CTA of the generic producer kernel.
+constexpr int kProducerPixels = 16;
+
+// Shape of one producer launch.
+struct ProducerGeo {
+    int N, H, W, C;
+    int J;   // outputs per pixel, G * kh * kw * 3
+    int NP;  // J rounded up to a multiple of 16 (tensor-core N)
+    long long npix;
+    int ntiles;  // 128-pixel tiles (tensor-core kernel)
+};
+
+// Shared-memory carve-up of the tensor-core producer kernel (byte offsets).
+struct ProducerTcLayout {
+    int b_off, a_off, s_off, dwf_off, linb_off, bar_off, bytes, tmem_cols;
+
+    static ProducerTcLayout make(int C, int J, int NP) {
+        ProducerTcLayout L;
+        L.b_off = 0;                                    // lin_w, NP rows x C
+        L.a_off = L.b_off + NP * C * 2;                 // h, 128 rows x C
+        L.s_off = L.a_off + 128 * C * 2;                // output rows, 128 x J
+        L.dwf_off = L.s_off + ((128 * J * 2 + 127) / 128) * 128;  // fp32 dw_w [9][C], dw_b [C]
+        L.linb_off = L.dwf_off + 10 * C * 4;            // fp32 lin_b [NP]
+        L.bar_off = (L.linb_off + NP * 4 + 15) / 16 * 16;  // mbarrier, tmem address
+        L.bytes = L.bar_off + 16;
+        int cols = 32;
+        while (cols < NP) cols <<= 1;
+        L.tmem_cols = cols;
+        return L;
+    }
+};
+
 // MSDCN extras: per-group scale priors travel inside the launch parameters.
 // s = min(s0 * softplus(raw), smax), softplus(r) = max(r, 0) + log1p(exp(-|r|)).
 __device__ __forceinline__ float msdcn_scale(float raw, float s0, float smax) {

@@ -17,6 +17,7 @@ __device__ unsigned int g_error_word = 0;
 #include "dcn4_fwd.cuh"
 #include "dcn4_bwd_halo.cuh"
 #include "dcn4_bwd_vec.cuh"
+#include "dcn4_producer.cuh"
 #include "dcn4_launch.h"
 
 namespace dcn4 {
@@ -321,6 +322,54 @@ cudaError_t launch_backward(const BwdLaunch &L) {
         case Dtype::F32: return launch_bwd_t<float>(L);
         case Dtype::BF16: return launch_bwd_t<__nv_bfloat16>(L);
         case Dtype::F16: return launch_bwd_t<__half>(L);
+    }
+    return cudaErrorInvalidValue;
+}
+
+namespace {
+
+template <typename T>
+cudaError_t launch_producer_t(const ProducerLaunch &L) {
+    const T *x = static_cast<const T *>(L.x), *dw_w = static_cast<const T *>(L.dw_w);
+    const T *dw_b = static_cast<const T *>(L.dw_b), *lin_w = static_cast<const T *>(L.lin_w);
+    const T *lin_b = static_cast<const T *>(L.lin_b);
+    T *out = static_cast<T *>(L.out);
+    if (L.tc) {
+        if constexpr (sizeof(T) == 2) {
+            const ProducerTcLayout lay = ProducerTcLayout::make(L.pg.C, L.pg.J, L.pg.NP);
+            cudaError_t e = cudaFuncSetAttribute(producer_tc_kernel<T>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 lay.bytes);
+            if (e != cudaSuccess) return e;
+            const int grid = L.pg.ntiles < sm_count() ? L.pg.ntiles : sm_count();
+            producer_tc_kernel<T><<<grid, 256, lay.bytes, L.stream>>>(L.pg, lay, x, dw_w, dw_b,
+                                                                    lin_w, lin_b, out);
+            count_launch();
+            return cudaGetLastError();
+        }
+        return cudaErrorInvalidValue;
+    }
+    const int smem = kProducerPixels * L.pg.C * 4;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(producer_generic_kernel<T>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    const long long blocks = (L.pg.npix + kProducerPixels - 1) / kProducerPixels;
+    producer_generic_kernel<T><<<(unsigned)blocks, 256, smem, L.stream>>>(L.pg, x, dw_w, dw_b,
+                                                                          lin_w, lin_b, out);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_producer(const ProducerLaunch &L) {
+    (void)cudaGetLastError();  // a pending error of an earlier call is not ours
+    switch (L.dtype) {
+        case Dtype::F32: return launch_producer_t<float>(L);
+        case Dtype::BF16: return launch_producer_t<__nv_bfloat16>(L);
+        case Dtype::F16: return launch_producer_t<__half>(L);
     }
     return cudaErrorInvalidValue;
 }

@@ -52,7 +52,17 @@ struct BwdLaunch {
     void *graw;             // MSDCN only: grad of scale_raw [N][Ho][Wo][G], element type
 };
 
+// Offset/weight producer (depthwise 3x3 + merged linear) of one call.
+struct ProducerLaunch {
+    ProducerGeo pg;
+    Dtype dtype;
+    const void *x, *dw_w, *dw_b, *lin_w, *lin_b;
+    void *out;
+    bool tc;  // tensor-core kernel (16-bit data), else the generic kernel
+    cudaStream_t stream;
+};
 cudaError_t launch_forward(const FwdLaunch &L);
+cudaError_t launch_producer(const ProducerLaunch &L);
 cudaError_t launch_backward(const BwdLaunch &L);
 
 // Launches the bounded-wait self-test kernel (see dcn4_selftest_bounded_wait).

@@ -79,6 +79,33 @@ def msdcn_s0(G):
     return torch.tensor([1.0 + (g // 2) for g in range(G)], dtype=torch.float32)
 
 
+def make_producer_inputs(N: int, H: int, W: int, C: int, G: int, K: int = 9,
+                         dtype: str = "bf16", seed: int = 0, offset_sigma: float = 2.0,
+                         device: Optional[str] = None):
+    """Feature map and weights of the offset/weight sub-network (depthwise
+    3x3 then one linear layer emitting G*K*3 values per pixel).
+
+    Draw order: x [N,H,W,C] ~ N(0,1); dw_weight [3,3,C] ~ N(0, 1/9);
+    dw_bias [C] ~ N(0, 0.1^2); lin_weight [G*K*3, C] ~ N(0, offset_sigma^2/C)
+    (outputs of about offset_sigma for unit-size features); lin_bias
+    [G*K*3] ~ N(0, 0.1^2). All in the storage dtype.
+    """
+    g = torch.Generator().manual_seed(seed)
+    dt = DTYPES[dtype]
+    J = G * K * 3
+    out = {
+        "x": torch.randn((N, H, W, C), generator=g),
+        "dw_weight": torch.randn((3, 3, C), generator=g) / 3.0,
+        "dw_bias": torch.randn((C,), generator=g) * 0.1,
+        "lin_weight": torch.randn((J, C), generator=g) * (offset_sigma / C ** 0.5),
+        "lin_bias": torch.randn((J,), generator=g) * 0.1,
+    }
+    out = {k: v.to(dt) for k, v in out.items()}
+    if device is not None:
+        out = {k: v.to(device) for k, v in out.items()}
+    return out
+
+
 def make_inputs(wl: Workload, out_hw: Tuple[int, int], with_grad: bool = False,
                 device: Optional[str] = None):
     """Returns a dict of tensors in the workload's storage dtype.

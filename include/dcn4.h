@@ -224,6 +224,37 @@ DCN4_API dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input,
                           void *grad_input, void *grad_dir_weight, void *grad_scale_raw,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Offset/weight producer of the DCNv4 module ("(论文速读）DCNv4：高效可变形卷积算子",
+ * "方法3. DCN模块的微设计优化": once softmax is removed the offset and weight
+ * projections merge into one linear layer, and the sub-network in front of it
+ * is a plain separable convolution: a depthwise 3x3 convolution, then that
+ * linear layer, without DCNv3's LayerNorm and GELU). For every pixel p of the
+ * H x W map x [N][H][W][C]:
+ *   h[p][c]   = dw_bias[c] + sum_{i,j in 0..2} dw_weight[i][j][c] * x[p + (i-1, j-1)][c]
+ *               (stride 1, zero outside the image)
+ *   offset_weight[p][j] = lin_bias[j] + sum_c lin_weight[j][c] * h[p][c],
+ *               j in [0, G*kh*kw*3),
+ * i.e. offset_weight comes out as [N][H][W][G][kh*kw][3] (dx, dy, m per tap),
+ * ready for dcn4_forward with the same desc. dw_weight is [3][3][C]
+ * (tap-major), dw_bias [C], lin_weight [G*kh*kw*3][C] (one row per output),
+ * lin_bias [G*kh*kw*3]; all are device pointers of desc->dtype. The layer
+ * serves the sampling grid of `desc`, so the output grid must be the input
+ * grid (Ho == H, Wo == W; else DCN4_ERR_UNSUPPORTED); stride, pad and dilation
+ * matter only through that check.
+ * Precision: fp32 accumulation throughout. bf16/fp16 calls round h to the data
+ * type before the linear layer (the tensor cores take 16-bit operands); the
+ * result is rounded once to the data type.
+ * Kernels: bf16/fp16 with C % 16 == 0, G*kh*kw*3 <= 256, whole 16-byte output
+ * rows ((G*kh*kw*3*2) % 16 == 0) and 16-byte aligned x, lin_weight and
+ * offset_weight use the tensor-core (tcgen05) kernel; every other call, and
+ * desc->algo == DCN4_ALGO_GENERIC, the CUDA-core kernel (h kept in fp32).
+ * DCN4_ALGO_HALO demands the tensor-core kernel (DCN4_ERR_UNSUPPORTED where it
+ * does not apply). */
+DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
+                                          const void *dw_weight, const void *dw_bias,
+                                          const void *lin_weight, const void *lin_bias,
+                                          void *offset_weight, void *stream);
+
 /* dcn4_backward for callers that cannot allocate device memory. The paper
  * has no counterpart; this is a deployment convenience. dcn4_backward needs
  * an fp32 scratch buffer for bf16/fp16 that the caller must allocate; callers

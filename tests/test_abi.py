@@ -146,3 +146,16 @@ def test_launch_counter_without_gpu(lib):
     pointer is rejected."""
     assert B.dcn4_kernel_launches() == 0
     assert lib.dcn4_kernel_launches(None) == 1
+
+
+def test_producer_argument_errors(lib):
+    """dcn4_offset_producer rejects null pointers and a strided output grid
+    before any launch (no GPU needed)."""
+    d = _desc()
+    fake = [ctypes.c_void_p(4096)] * 6
+    assert lib.dcn4_offset_producer(ctypes.byref(d), None, *fake[:5], None) == 1
+    assert lib.dcn4_offset_producer(ctypes.byref(d), *fake[:5], None, None) == 1
+    d2 = _desc(stride=2)
+    assert lib.dcn4_offset_producer(ctypes.byref(d2), *fake, None) == 2
+    bad = _desc(C=10, G=4)
+    assert lib.dcn4_offset_producer(ctypes.byref(bad), *fake, None) == 1
