@@ -366,7 +366,7 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
     L.pg.NP = (L.pg.J + 15) / 16 * 16;
     L.pg.npix = (long long)g.N * g.H * g.W;
     const long long ntiles = (L.pg.npix + 127) / 128;
-    if (ntiles > std::numeric_limits<int>::max()) return DCN4_ERR_UNSUPPORTED;
+    if (L.pg.npix + 128 > std::numeric_limits<int>::max()) return DCN4_ERR_UNSUPPORTED;
     L.pg.ntiles = (int)ntiles;
     L.x = x;
     L.dw_w = dw_weight;
@@ -378,10 +378,12 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
     const int eb = elem_bytes(L.dtype);
     // tensor-core kernel: 16-bit data, K = C in steps of 16, N = J padded to
     // 16 <= 256, whole 16-byte output rows, lin_w resident in shared memory
-    const ProducerTcLayout lay = ProducerTcLayout::make(g.C, L.pg.J, L.pg.NP);
+    ProducerTcLayout lay = ProducerTcLayout::make(g.C, L.pg.J, L.pg.NP, g.W, 2);
+    if (lay.bytes > max_smem_optin()) lay = ProducerTcLayout::make(g.C, L.pg.J, L.pg.NP, g.W, 1);
     L.tc = desc->algo != DCN4_ALGO_GENERIC && eb == 2 && g.C % 16 == 0 && L.pg.NP <= 256 &&
            (L.pg.J * eb) % 16 == 0 && aligned16(x) && aligned16(lin_weight) &&
            aligned16(offset_weight) && lay.bytes <= max_smem_optin();
+    L.lay = lay;
     if (!L.tc && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     if (!L.tc && kProducerPixels * g.C * 4 > max_smem_optin()) return DCN4_ERR_UNSUPPORTED;
     return cuda_status(launch_producer(L));

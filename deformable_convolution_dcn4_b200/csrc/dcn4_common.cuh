@@ -43,17 +43,25 @@ struct ProducerGeo {
 
 // Shared-memory carve-up of the tensor-core producer kernel (byte offsets).
 struct ProducerTcLayout {
-    int b_off, a_off, s_off, dwf_off, linb_off, bar_off, bytes, tmem_cols;
+    int b_off, a_off, x_off, x_bytes, x_nbuf, dwf_off, dwt_off, linb_off, row_off, bar_off,
+        bytes, tmem_cols;
 
-    static ProducerTcLayout make(int C, int J, int NP) {
+    // x_nbuf staged pixel ranges: 2 (the next tile's copy overlaps this
+    // tile's work) or 1 (it overlaps only the MMA and the epilogue)
+    static ProducerTcLayout make(int C, int J, int NP, int W, int x_nbuf) {
+        (void)J;
         ProducerTcLayout L;
-        L.b_off = 0;                                    // lin_w, NP rows x C
-        L.a_off = L.b_off + NP * C * 2;                 // h, 128 rows x C
-        L.s_off = L.a_off + 128 * C * 2;                // output rows, 128 x J
-        L.dwf_off = L.s_off + ((128 * J * 2 + 127) / 128) * 128;  // fp32 dw_w [9][C], dw_b [C]
-        L.linb_off = L.dwf_off + 10 * C * 4;            // fp32 lin_b [NP]
-        L.bar_off = (L.linb_off + NP * 4 + 15) / 16 * 16;  // mbarrier, tmem address
-        L.bytes = L.bar_off + 16;
+        L.b_off = 0;                     // lin_w, NP rows x C (core matrices)
+        L.a_off = L.b_off + NP * C * 2;  // h, 128 rows x C (core matrices)
+        L.x_off = L.a_off + 128 * C * 2;  // staged pixel ranges
+        L.x_bytes = ((128 + 2 * W + 2) * C * 2 + 127) / 128 * 128;
+        L.x_nbuf = x_nbuf;
+        L.dwf_off = L.x_off + x_nbuf * L.x_bytes;  // fp32 dw_w [9][C], dw_b [C]
+        L.dwt_off = L.dwf_off + 10 * C * 4;   // dw_w [9][C] in the data type
+        L.linb_off = L.dwt_off + (9 * C * 2 + 15) / 16 * 16;  // fp32 lin_b [NP]
+        L.row_off = (L.linb_off + NP * 4 + 15) / 16 * 16;  // int2 (y, x) per tile row
+        L.bar_off = L.row_off + 128 * 8;                     // 3 mbarriers, tmem address
+        L.bytes = L.bar_off + 32;
         int cols = 32;
         while (cols < NP) cols <<= 1;
         L.tmem_cols = cols;

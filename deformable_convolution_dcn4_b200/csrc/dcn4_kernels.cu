@@ -336,14 +336,15 @@ cudaError_t launch_producer_t(const ProducerLaunch &L) {
     T *out = static_cast<T *>(L.out);
     if (L.tc) {
         if constexpr (sizeof(T) == 2) {
-            const ProducerTcLayout lay = ProducerTcLayout::make(L.pg.C, L.pg.J, L.pg.NP);
-            cudaError_t e = cudaFuncSetAttribute(producer_tc_kernel<T>,
+            const ProducerTcLayout &lay = L.lay;
+            constexpr int NW = 8;
+            cudaError_t e = cudaFuncSetAttribute(producer_tc_kernel<T, NW>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  lay.bytes);
             if (e != cudaSuccess) return e;
             const int grid = L.pg.ntiles < sm_count() ? L.pg.ntiles : sm_count();
-            producer_tc_kernel<T><<<grid, 256, lay.bytes, L.stream>>>(L.pg, lay, x, dw_w, dw_b,
-                                                                    lin_w, lin_b, out);
+            producer_tc_kernel<T, NW><<<grid, NW * 32, lay.bytes, L.stream>>>(
+                L.pg, lay, x, dw_w, dw_b, lin_w, lin_b, out);
             count_launch();
             return cudaGetLastError();
         }

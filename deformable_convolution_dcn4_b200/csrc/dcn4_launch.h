@@ -59,6 +59,7 @@ struct ProducerLaunch {
     const void *x, *dw_w, *dw_b, *lin_w, *lin_b;
     void *out;
     bool tc;  // tensor-core kernel (16-bit data), else the generic kernel
+    ProducerTcLayout lay;  // tensor-core kernel only
     cudaStream_t stream;
 };
 cudaError_t launch_forward(const FwdLaunch &L);

@@ -10,15 +10,18 @@
 //   out[p][j] = lin_b[j] + sum_c lin_w[j][c] * h[p][c]
 //
 // Two kernels:
-//  * producer_tc_kernel (16-bit data): one CTA per SM walks 128-pixel tiles.
-//    Its warps compute h for the tile on the CUDA cores (fp32, rounded to the
-//    data type, which is the operand type of the tensor cores) straight into
-//    shared memory in the tcgen05 K-major core-matrix layout; one thread
-//    issues the K/16 tcgen05.mma (M = 128 pixels, N = the outputs padded to
-//    16, fp32 accumulators in tensor memory); all eight warps read the
-//    accumulators back with tcgen05.ld, add the bias, round, and stage the
-//    tile's rows, which leave in one bulk copy (the tile's outputs are
-//    contiguous in global memory). lin_w stays resident in shared memory.
+//  * producer_tc_kernel (16-bit data): one CTA per SM walks 128-pixel tiles
+//    (128 consecutive pixels of the flattened N*H*W grid). The pixel range a
+//    tile's 3x3 neighbourhoods touch (its pixels plus one image row and one
+//    pixel on each side) arrives in one bulk copy, double-buffered so the
+//    next tile's copy overlaps this tile's work. The warps compute h from
+//    shared memory on the CUDA cores (fp32, rounded to the data type, the
+//    operand type of the tensor cores) straight into the tcgen05 K-major
+//    core-matrix layout; one thread issues the K/16 tcgen05.mma (M = 128
+//    pixels, N = the outputs padded to 16, fp32 accumulators in tensor
+//    memory); all eight warps read the accumulators back with tcgen05.ld, add
+//    the bias, round, and store 16-byte pieces of the output rows. lin_w
+//    stays resident in shared memory.
 //  * producer_generic_kernel (any type and shape): 16 pixels per CTA, h in
 //    shared memory (fp32, not rounded), the linear layer on the CUDA cores.
 #pragma once
@@ -118,6 +121,27 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
     return v;
 }
 
+// acc[k] += w[k] * v[k] for eight 16-bit pairs: the sm_100 mixed-precision
+// fma (16-bit multiplicands, exact product, one fp32 rounding), i.e. exactly
+// fmaf on the widened values.
+template <typename T> struct MixedFma8;
+#define DCN4_MIXED_FMA8(TY, CT)                                                           \
+    template <> struct MixedFma8<CT> {                                                    \
+        static __device__ __forceinline__ void run(float *acc, const uint4 &v, const uint4 &w) { \
+            const unsigned vv[4] = {v.x, v.y, v.z, v.w}, ww[4] = {w.x, w.y, w.z, w.w};    \
+            _Pragma("unroll") for (int k = 0; k < 4; ++k) {                               \
+                asm("{\n\t.reg .b16 vl, vh, wl, wh;\n\tmov.b32 {vl, vh}, %2;\n\t"          \
+                    "mov.b32 {wl, wh}, %3;\n\tfma.rn.f32." TY " %0, vl, wl, %0;\n\t"          \
+                    "fma.rn.f32." TY " %1, vh, wh, %1;\n\t}"                              \
+                    : "+f"(acc[2 * k]), "+f"(acc[2 * k + 1])                              \
+                    : "r"(vv[k]), "r"(ww[k]));                                            \
+            }                                                                             \
+        }                                                                                 \
+    };
+DCN4_MIXED_FMA8("bf16", __nv_bfloat16)
+DCN4_MIXED_FMA8("f16", __half)
+#undef DCN4_MIXED_FMA8
+
 // ---------------------------------------------------------------------------
 // Tensor-core producer (bf16 / fp16)
 // ---------------------------------------------------------------------------
@@ -128,34 +152,59 @@ __device__ __forceinline__ uint32_t core_off(int r, int q, int C) {
     return (uint32_t)((r >> 3) * (C * 16) + q * 128 + (r & 7) * 16);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256, 1)
+template <typename T, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
     producer_tc_kernel(ProducerGeo pg, ProducerTcLayout L, const T *__restrict__ x,
                        const T *__restrict__ dw_w, const T *__restrict__ dw_b,
                        const T *__restrict__ lin_w, const T *__restrict__ lin_b,
                        T *__restrict__ out) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int C = pg.C, J = pg.J, NP = pg.NP, Q = C / 8;
+    const int C = pg.C, J = pg.J, NP = pg.NP, Q = C / 8, W = pg.W;
     float *dwf = reinterpret_cast<float *>(smem + L.dwf_off);
     float *linb = reinterpret_cast<float *>(smem + L.linb_off);
-    const uint32_t bar = smem_u32(smem + L.bar_off);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.bar_off + 8);
+    const uint32_t mma_bar = smem_u32(smem + L.bar_off);
+    const uint32_t x_bar0 = mma_bar + 8;  // x_bar[b] at +8b
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.bar_off + 24);
 
     // resident operands: lin_w in core-matrix layout (rows >= J zero), the
     // depthwise taps and both biases in fp32
-    for (int i = tid; i < NP * Q; i += 256) {
+    constexpr int NT = NW * 32;
+    for (int i = tid; i < NP * Q; i += NT) {
         const int n = i / Q, q = i - n * Q;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (n < J) v = *reinterpret_cast<const uint4 *>(lin_w + (size_t)n * C + q * 8);
         *reinterpret_cast<uint4 *>(smem + L.b_off + core_off(n, q, C)) = v;
     }
-    for (int i = tid; i < 9 * C; i += 256) dwf[i] = Elem<T>::to_f(dw_w[i]);
-    for (int i = tid; i < C; i += 256) dwf[9 * C + i] = Elem<T>::to_f(dw_b[i]);
-    for (int i = tid; i < NP; i += 256) linb[i] = i < J ? Elem<T>::to_f(lin_b[i]) : 0.f;
+    for (int i = tid; i < 9 * C; i += NT) dwf[i] = Elem<T>::to_f(dw_w[i]);
+    T *dwt = reinterpret_cast<T *>(smem + L.dwt_off);  // dw_w [9][C] as stored
+    for (int i = tid; i < 9 * C; i += NT) dwt[i] = dw_w[i];
+    for (int i = tid; i < C; i += NT) dwf[9 * C + i] = Elem<T>::to_f(dw_b[i]);
+    for (int i = tid; i < NP; i += NT) linb[i] = i < J ? Elem<T>::to_f(lin_b[i]) : 0.f;
+    int2 *rowyx = reinterpret_cast<int2 *>(smem + L.row_off);  // (y, x) of each tile row
+
+    // pixel rows a tile reads: its 128 pixels and one image row plus one
+    // pixel on either side (clipped to the tensor), one contiguous range
+    auto x_range = [&](int tile, long long &lo, long long &hi) {
+        const long long p0 = (long long)tile * 128;
+        lo = p0 - W - 1 > 0 ? p0 - W - 1 : 0;
+        hi = p0 + 128 + W + 1 < pg.npix ? p0 + 128 + W + 1 : pg.npix;
+    };
+    int inflight = -1;  // (thread 0) buffer of a copy not yet waited for
+    auto issue_x = [&](int tile, int b) {
+        inflight = b;
+        long long lo, hi;
+        x_range(tile, lo, hi);
+        const uint32_t bytes = (uint32_t)((hi - lo) * C * 2);
+        mbar_arrive_expect_tx(x_bar0 + 8 * b, bytes);
+        bulk_load(smem_u32(smem + L.x_off + b * L.x_bytes), x + lo * C, bytes, x_bar0 + 8 * b);
+    };
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(mma_bar, 1);
+        mbar_init(x_bar0, 1);
+        mbar_init(x_bar0 + 8, 1);
         fence_barrier_init();
+        if ((int)blockIdx.x < pg.ntiles) issue_x(blockIdx.x, 0);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -171,97 +220,187 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t idesc = umma_idesc_f16(std::is_same<T, __nv_bfloat16>::value, 128, NP);
     const uint32_t a_base = smem_u32(smem + L.a_off), b_base = smem_u32(smem + L.b_off);
-    const uint32_t s_base = smem_u32(smem + L.s_off);
-    const int rlo = lane & 7, qlo = lane >> 3;
-    const int qgroups = (Q + 3) / 4;
+    // lane -> (row, chunk) of the depthwise pass. With whole 8-chunk blocks
+    // the 8 lanes of each shared-memory phase take 8 different rows and 8
+    // different chunks (a diagonal), so both the staged-pixel reads (pixel
+    // stride a multiple of 128 bytes) and the core-matrix stores are free of
+    // bank conflicts.
+    const bool diag = Q % 8 == 0;
+    const int e = lane & 7, f = lane >> 3;
     bool ok = true;
 
     int iter = 0;
     for (int tile = blockIdx.x; tile < pg.ntiles; tile += gridDim.x, ++iter) {
+        const bool two = L.x_nbuf == 2;
+        const int b = two ? iter & 1 : 0;
+        const uint32_t x_par = two ? (iter >> 1) & 1 : iter & 1;
+        const bool more = tile + (int)gridDim.x < pg.ntiles;
         const long long p0 = (long long)tile * 128;
         const int rows = (int)min(128ll, pg.npix - p0);
+        long long lo, hi;
+        x_range(tile, lo, hi);
+        // two buffers: the other one was last read before the previous
+        // tile's MMA
+        if (two && tid == 0 && more) {
+            bulk_wait_read();  // the previous tile's rows, staged in that buffer, have left
+            issue_x(tile + gridDim.x, b ^ 1);
+        }
+        if (tid < 128) {
+            const int p = (int)p0 + tid;  // the pixel count fits an int
+            const int t = p / W;
+            rowyx[tid] = make_int2(t % pg.H, p - t * W);
+        }
+        if (!mbar_wait_bounded(x_bar0 + 8 * b, x_par, kWaitLimitNs)) ok = false;
+        if (inflight == b) inflight = -1;
+        const unsigned char *xs = smem + L.x_off + b * L.x_bytes;
+        const int rel0 = (int)(p0 - lo);  // staged index of the tile's first pixel
+        __syncthreads();
 
-        // depthwise 3x3 of the tile's pixels -> A (16-byte chunks; each
-        // warp item covers 8 pixels x 4 chunks, conflict-free stores)
-        for (int item = warp; item < 16 * qgroups; item += 8) {
-            const int rg = item / qgroups, q = (item - rg * qgroups) * 4 + qlo;
-            if (q >= Q) continue;
-            const int r = rg * 8 + rlo;
+        // depthwise 3x3 of the tile's pixels -> A (fp32, rounded to T)
+        auto dw_one = [&](int r, int q) {
             float acc[8];
             if (r < rows) {
-                const long long p = p0 + r;
-                const int xx = (int)(p % pg.W);
-                const long long t = p / pg.W;
-                const int y = (int)(t % pg.H);
-                const int n = (int)(t / pg.H);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = dwf[9 * C + q * 8 + e];
+                const int2 yx = rowyx[r];
+                const int y = yx.x, xx = yx.y;
+                const float4 *bb = reinterpret_cast<const float4 *>(dwf + 9 * C + q * 8);
+                const float4 b0 = bb[0], b1 = bb[1];
+                acc[0] = b0.x, acc[1] = b0.y, acc[2] = b0.z, acc[3] = b0.w;
+                acc[4] = b1.x, acc[5] = b1.y, acc[6] = b1.z, acc[7] = b1.w;
 #pragma unroll
                 for (int i = 0; i < 3; ++i) {
                     const int yy = y + i - 1;
-                    if (yy < 0 || yy >= pg.H) continue;
 #pragma unroll
                     for (int j = 0; j < 3; ++j) {
-                        const int xs = xx + j - 1;
-                        if (xs < 0 || xs >= pg.W) continue;
-                        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                            x + (((size_t)n * pg.H + yy) * pg.W + xs) * C + q * 8));
-                        float f[8];
-                        unpack8<T>(v, f);
-                        const float *w = dwf + (i * 3 + j) * C + q * 8;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[e], f[e], acc[e]);
+                        const int xj = xx + j - 1;
+                        if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
+                        const int idx = rel0 + r + (i - 1) * W + (j - 1);
+                        const uint4 v = *reinterpret_cast<const uint4 *>(xs + idx * (C * 2) + q * 16);
+                        float fv[8];
+                        unpack8<T>(v, fv);
+                        const float4 *ww =
+                            reinterpret_cast<const float4 *>(dwf + (i * 3 + j) * C + q * 8);
+                        const float4 w0 = ww[0], w1 = ww[1];
+                        acc[0] = fmaf(w0.x, fv[0], acc[0]);
+                        acc[1] = fmaf(w0.y, fv[1], acc[1]);
+                        acc[2] = fmaf(w0.z, fv[2], acc[2]);
+                        acc[3] = fmaf(w0.w, fv[3], acc[3]);
+                        acc[4] = fmaf(w1.x, fv[4], acc[4]);
+                        acc[5] = fmaf(w1.y, fv[5], acc[5]);
+                        acc[6] = fmaf(w1.z, fv[6], acc[6]);
+                        acc[7] = fmaf(w1.w, fv[7], acc[7]);
                     }
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                for (int k = 0; k < 8; ++k) acc[k] = 0.f;
             }
             *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(r, q, C)) = pack8<T>(acc);
+        };
+        if (ok) {
+            if (diag) {
+                // blocks of 8 rows x 8 chunks; lane (e, f) keeps chunk
+                // qb*8 + e and its 16-bit taps in registers and takes rows
+                // (e + f + 4 s) & 7 of the block (mixed-precision fma: the
+                // 16-bit products are exact, sums in fp32 as above)
+                const int qblocks = Q / 8;
+                for (int blk = warp; blk < 16 * qblocks; blk += NW) {
+                    const int rb = blk / qblocks, q = (blk - rb * qblocks) * 8 + e;
+                    uint4 wv[9];
+#pragma unroll
+                    for (int k = 0; k < 9; ++k)
+                        wv[k] = *reinterpret_cast<const uint4 *>(dwt + k * C + q * 8);
+                    const float4 *bb = reinterpret_cast<const float4 *>(dwf + 9 * C + q * 8);
+                    const float4 b0 = bb[0], b1 = bb[1];
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int r = rb * 8 + ((e + f + 4 * s2) & 7);
+                        float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        if (r < rows) {
+                            const int2 yx = rowyx[r];
+#pragma unroll
+                            for (int i = 0; i < 3; ++i) {
+                                const int yy = yx.x + i - 1;
+#pragma unroll
+                                for (int j = 0; j < 3; ++j) {
+                                    const int xj = yx.y + j - 1;
+                                    if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
+                                    const int idx = rel0 + r + (i - 1) * W + (j - 1);
+                                    const uint4 v = *reinterpret_cast<const uint4 *>(
+                                        xs + idx * (C * 2) + q * 16);
+                                    MixedFma8<T>::run(acc, v, wv[i * 3 + j]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+                        }
+                        *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(r, q, C)) =
+                            pack8<T>(acc);
+                    }
+                }
+            } else {
+                for (int it = tid; it < 128 * Q; it += NT) {
+                    const int r = it / Q;
+                    dw_one(r, it - r * Q);
+                }
+            }
         }
         fence_async_smem();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) break;
 
-        // one thread issues the K/16 MMAs; the staging rows of the previous
-        // tile must have left before the epilogue below rewrites them
+        // one thread issues the K/16 MMAs (M = 128 pixels, N = NP outputs);
+        // with one buffer the next tile's pixels start arriving now
         if (tid == 0) {
-            bulk_wait_read();
+            if (!two && more) issue_x(tile + gridDim.x, 0);
             tc_fence_after();
             for (int kk = 0; kk < C / 16; ++kk)
                 tc_mma_f16(tmem, umma_desc_kmajor(a_base + kk * 256, 128, C * 16),
                            umma_desc_kmajor(b_base + kk * 256, 128, C * 16), idesc, kk > 0);
-            tc_commit(bar);
+            tc_commit(mma_bar);
         }
-        if (!mbar_wait_bounded(bar, iter & 1, kWaitLimitNs)) ok = false;
+        if (!mbar_wait_bounded(mma_bar, iter & 1, kWaitLimitNs)) ok = false;
         if (__syncthreads_or(!ok)) break;
         tc_fence_after();
 
         // epilogue: warp w reads TMEM lanes 32 (w & 3) .. +31 (= tile rows),
-        // 16-column chunks of parity w >> 2
+        // every (NW / 4)-th 16-column chunk from w >> 2; bias, rounding.
+        // With two input buffers the rows are staged in this tile's (now
+        // consumed) buffer and leave in one bulk copy (the tile's outputs are
+        // contiguous); else each thread stores its 16-byte pieces.
+        const bool staged = two && L.x_bytes >= 128 * J * 2;
+        unsigned char *srows = smem + L.x_off + b * L.x_bytes;
         const int r = 32 * (warp & 3) + lane;
-        for (int c16 = warp >> 2; c16 < NP / 16; c16 += 2) {
+        T *orow = out + (p0 + r) * J;
+        for (int c16 = warp >> 2; c16 < NP / 16; c16 += NW / 4) {
             float v[16];
             tc_ld_16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c16 * 16, v);
             const int c0 = c16 * 16;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 if (c0 + 8 * h >= J || r >= rows) continue;
-                float f[8];
+                float fo[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = v[8 * h + e] + linb[c0 + 8 * h + e];
-                *reinterpret_cast<uint4 *>(smem + L.s_off + ((size_t)r * J + c0 + 8 * h) * 2) =
-                    pack8<T>(f);
+                for (int k = 0; k < 8; ++k) fo[k] = v[8 * h + k] + linb[c0 + 8 * h + k];
+                if (staged)
+                    *reinterpret_cast<uint4 *>(srows + ((size_t)r * J + c0 + 8 * h) * 2) =
+                        pack8<T>(fo);
+                else
+                    *reinterpret_cast<uint4 *>(orow + c0 + 8 * h) = pack8<T>(fo);
             }
         }
         tc_fence_before();
-        fence_async_smem();
+        if (staged) fence_async_smem();
         __syncthreads();
-        if (tid == 0) bulk_store(out + p0 * J, s_base, (uint32_t)rows * J * 2);
+        if (staged && tid == 0) bulk_store(out + p0 * J, smem_u32(srows), (uint32_t)rows * J * 2);
     }
+    if (tid == 0) bulk_wait_all();
 
-    if (tid == 0) {
-        bulk_wait_all();
-        if (!ok) atomicOr(&g_error_word, kErrTimeout);
+    if (tid == 0 && !ok) {
+        atomicOr(&g_error_word, kErrTimeout);
+        // a prefetch issued before the failure lands before the CTA exits
+        if (inflight >= 0)
+            mbar_wait_bounded(x_bar0 + 8 * inflight,
+                              L.x_nbuf == 2 ? ((iter + 1) >> 1) & 1 : (iter + 1) & 1, kWaitLimitNs);
     }
     tc_fence_before();
     __syncthreads();

@@ -3,6 +3,9 @@ command profilers (ncu) wrap to capture single kernels.
 
     python -m deformable_convolution_dcn4_b200.run_op --op forward \
         --workload internimage_bf16 --iters 3 [--N 64] [--algo auto]
+
+--op producer runs the offset/weight producer (depthwise 3x3 + merged linear)
+on the workload's N, H, W, C, G with seeded sub-network weights.
 """
 import argparse
 import sys
@@ -10,12 +13,12 @@ import sys
 import torch
 
 from . import _binding as B
-from .workloads import WORKLOADS, make_inputs
+from .workloads import WORKLOADS, make_inputs, make_producer_inputs
 
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["forward", "backward", "msdcn"], default="forward")
+    p.add_argument("--op", choices=["forward", "backward", "msdcn", "producer"], default="forward")
     p.add_argument("--workload", default="internimage_bf16")
     p.add_argument("--iters", type=int, default=3)
     p.add_argument("--N", type=int, default=None)
@@ -29,12 +32,21 @@ def main(argv=None):
     desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, 0, (wl.kh, wl.kw), wl.stride, wl.pad,
                        wl.dilation, wl.offset_scale)
     ho, wo = B.dcn4_out_shape(desc)
-    d = make_inputs(wl, (ho, wo), with_grad=a.op == "backward", device="cuda")
+    if a.op == "producer":
+        d = make_producer_inputs(wl.N, wl.H, wl.W, wl.C, wl.G, wl.kh * wl.kw, wl.dtype,
+                                 seed=wl.seed, device="cuda")
+    else:
+        d = make_inputs(wl, (ho, wo), with_grad=a.op == "backward", device="cuda")
     kw = dict(group=wl.G, kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad,
               dilation=wl.dilation, offset_scale=wl.offset_scale, algo=a.algo)
     for _ in range(a.iters):
         if a.op == "forward":
             B.dcn4_forward(d["input"], d["offset_weight"], **kw)
+        elif a.op == "producer":
+            B.dcn4_offset_producer(d["x"], d["dw_weight"], d["dw_bias"], d["lin_weight"],
+                                   d["lin_bias"], group=wl.G, kernel_size=(wl.kh, wl.kw),
+                                   stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
+                                   algo=a.algo)
         elif a.op == "backward":
             B.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"], **kw)
         else:
