@@ -380,6 +380,10 @@ def run_ours(args):
                 "peak_source": f"{peak_kind} copy bandwidth",
                 "bytes_per_launch": ib[dom]}
 
+    # next rows beyond the step (MSDCN backward; the offset/weight producer),
+    # timed the same way outside the timed region, reported on their own
+    extra = next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind)
+
     # end to end: pinned host buffers, H2D copies + the three calls + D2H reads
     e2e = run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream,
                   step_bytes, world)
@@ -391,7 +395,7 @@ def run_ours(args):
                                        "InternImage stage)",
             "config": describe(wl, Ho, Wo), "roofline": roofline, "ops": breakdown,
             "gpu_launches": args.steps * sum(launches.values()),
-            "launches_per_step": launches, "e2e": e2e,
+            "launches_per_step": launches, "e2e": e2e, "next_rows": extra,
             "clocks": clocks.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -404,6 +408,67 @@ def run_ours(args):
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
+
+
+def graph_median_ms(fn, flush, stream, reps=10):
+    """Median device time of one graph replay of fn, L2 flushed before each."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    ts = []
+    for _ in range(reps + 3):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    del g
+    return statistics.median(ts[3:])
+
+
+def next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind):
+    """MSDCN backward and the offset/weight producer (depthwise 3x3 + merged
+    linear) on the step's shape: median ms, ideal bytes, GB/s."""
+    import torch
+    from deformable_convolution_dcn4_b200.workloads import make_producer_inputs
+    eb = 4 if wl.dtype == "f32" else 2
+    nin = wl.N * wl.H * wl.W * wl.C
+    nout = wl.N * Ho * Wo * wl.C
+    now = wl.N * Ho * Wo * wl.G * wl.K * 3
+    graw = wl.N * Ho * Wo * wl.G
+    gin = torch.empty_like(m["input"])
+    gdw = torch.empty_like(m["dir_weight"])
+    gsr = torch.empty_like(m["scale_raw"])
+    go = d["grad_out"]
+    res = {}
+    ms = graph_median_ms(lambda: dcn.msdcn_backward(
+        m["input"], m["dir_weight"], m["scale_raw"], m["s0"], wl.smax, go, workspace=ws,
+        grad_input=gin, grad_dir_weight=gdw, grad_scale_raw=gsr, **kw), flush, stream)
+    ib = (nin + now + graw + nout + nin + now + graw) * eb
+    res["msdcn_backward"] = {"median_ms": round(ms, 5), "ideal_bytes": ib,
+                             "GB/s": round(ib / (ms * 1e-3) / 1e9, 1),
+                             f"frac_of_{peak_kind}_hbm": round(ib / (ms * 1e-3) / 1e9 / peak, 4)}
+    if wl.H * wl.W == Ho * Wo:
+        p = make_producer_inputs(wl.N, wl.H, wl.W, wl.C, wl.G, wl.K, wl.dtype, seed=wl.seed,
+                                 device=d["input"].device)
+        pout = torch.empty_like(d["offset_weight"])
+        J = wl.G * wl.K * 3
+        ms = graph_median_ms(lambda: dcn.dcn4_offset_producer(
+            p["x"], p["dw_weight"], p["dw_bias"], p["lin_weight"], p["lin_bias"], out=pout,
+            **kw), flush, stream)
+        ib = (nin + now + 10 * wl.C + J * wl.C + J) * eb
+        flops = 2.0 * nin * J + 18.0 * nin
+        res["dcn4_offset_producer"] = {
+            "median_ms": round(ms, 5), "ideal_bytes": ib, "GB/s": round(ib / (ms * 1e-3) / 1e9, 1),
+            f"frac_of_{peak_kind}_hbm": round(ib / (ms * 1e-3) / 1e9 / peak, 4),
+            "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)}
+    return res
 
 
 def run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream, step_bytes,

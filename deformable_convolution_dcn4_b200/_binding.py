@@ -152,11 +152,11 @@ def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, di
 
 
 def dcn4_offset_producer(x, dw_weight, dw_bias, lin_weight, lin_bias, group, kernel_size=3,
-                         stride=1, pad=1, dilation=1, algo="auto", out=None):
+                         stride=1, pad=1, dilation=1, offset_scale=1.0, algo="auto", out=None):
     """offset_weight [N,H,W,G,kh*kw,3] from the depthwise 3x3 + merged linear
     sub-network: x [N,H,W,C], dw_weight [3,3,C], dw_bias [C],
     lin_weight [G*kh*kw*3, C], lin_bias [G*kh*kw*3], all of x's dtype."""
-    desc = _desc_for(x, group, kernel_size, stride, pad, dilation, 1.0, algo)
+    desc = _desc_for(x, group, kernel_size, stride, pad, dilation, offset_scale, algo)
     N, H, W, C = x.shape
     J = group * desc.kh * desc.kw * 3
     _require(x, "x", x.dtype)

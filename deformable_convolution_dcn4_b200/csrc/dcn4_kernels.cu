@@ -337,7 +337,7 @@ cudaError_t launch_producer_t(const ProducerLaunch &L) {
     if (L.tc) {
         if constexpr (sizeof(T) == 2) {
             const ProducerTcLayout &lay = L.lay;
-            constexpr int NW = 8;
+            constexpr int NW = 16;  // measured: 16 warps 90 us, 8 warps 108 us (InternImage bf16)
             cudaError_t e = cudaFuncSetAttribute(producer_tc_kernel<T, NW>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  lay.bytes);

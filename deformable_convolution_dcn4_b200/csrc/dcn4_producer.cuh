@@ -311,31 +311,41 @@ __global__ void __launch_bounds__(NW * 32, 1)
                         wv[k] = *reinterpret_cast<const uint4 *>(dwt + k * C + q * 8);
                     const float4 *bb = reinterpret_cast<const float4 *>(dwf + 9 * C + q * 8);
                     const float4 b0 = bb[0], b1 = bb[1];
+                    // the lane's two rows together: independent loads and
+                    // fma chains in flight side by side
+                    int rr[2];
+                    int2 yx[2];
+                    float acc[2][8];
 #pragma unroll
                     for (int s2 = 0; s2 < 2; ++s2) {
-                        const int r = rb * 8 + ((e + f + 4 * s2) & 7);
-                        float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                        if (r < rows) {
-                            const int2 yx = rowyx[r];
+                        rr[s2] = rb * 8 + ((e + f + 4 * s2) & 7);
+                        yx[s2] = rr[s2] < rows ? rowyx[rr[s2]] : make_int2(-1000000, 0);
+                        acc[s2][0] = b0.x, acc[s2][1] = b0.y, acc[s2][2] = b0.z, acc[s2][3] = b0.w;
+                        acc[s2][4] = b1.x, acc[s2][5] = b1.y, acc[s2][6] = b1.z, acc[s2][7] = b1.w;
+                    }
 #pragma unroll
-                            for (int i = 0; i < 3; ++i) {
-                                const int yy = yx.x + i - 1;
+                    for (int i = 0; i < 3; ++i) {
 #pragma unroll
-                                for (int j = 0; j < 3; ++j) {
-                                    const int xj = yx.y + j - 1;
-                                    if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
-                                    const int idx = rel0 + r + (i - 1) * W + (j - 1);
-                                    const uint4 v = *reinterpret_cast<const uint4 *>(
-                                        xs + idx * (C * 2) + q * 16);
-                                    MixedFma8<T>::run(acc, v, wv[i * 3 + j]);
-                                }
+                        for (int j = 0; j < 3; ++j) {
+#pragma unroll
+                            for (int s2 = 0; s2 < 2; ++s2) {
+                                const int yy = yx[s2].x + i - 1, xj = yx[s2].y + j - 1;
+                                if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
+                                const int idx = rel0 + rr[s2] + (i - 1) * W + (j - 1);
+                                const uint4 v = *reinterpret_cast<const uint4 *>(
+                                    xs + idx * (C * 2) + q * 16);
+                                MixedFma8<T>::run(acc[s2], v, wv[i * 3 + j]);
                             }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
                         }
-                        *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(r, q, C)) =
-                            pack8<T>(acc);
+                    }
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        if (rr[s2] >= rows) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) acc[s2][k] = 0.f;
+                        }
+                        *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(rr[s2], q, C)) =
+                            pack8<T>(acc[s2]);
                     }
                 }
             } else {
