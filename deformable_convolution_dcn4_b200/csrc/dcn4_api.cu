@@ -385,7 +385,8 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
            aligned16(offset_weight) && lay.bytes <= max_smem_optin();
     L.lay = lay;
     if (!L.tc && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
-    if (!L.tc && kProducerPixels * g.C * 4 > max_smem_optin()) return DCN4_ERR_UNSUPPORTED;
+    if (!L.tc && (L.pg.npix + kProducerPixels - 1) / kProducerPixels > 0x7fffffffLL)
+        return DCN4_ERR_UNSUPPORTED;
     return cuda_status(launch_producer(L));
 }
 

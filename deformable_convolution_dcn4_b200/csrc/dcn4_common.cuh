@@ -29,8 +29,11 @@ struct Geometry {
     int msd_dil;  // MSDCN scale-as-dilation reading
 };
 
-// Pixels per CTA of the generic producer kernel.
-constexpr int kProducerPixels = 16;
+// Tile of the generic producer kernel: pixels x outputs per CTA, channels
+// per shared-memory chunk.
+constexpr int kProducerPixels = 64;
+constexpr int kProducerOuts = 64;
+constexpr int kProducerK = 32;
 
 // Shape of one producer launch.
 struct ProducerGeo {

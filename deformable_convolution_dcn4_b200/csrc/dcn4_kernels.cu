@@ -350,15 +350,9 @@ cudaError_t launch_producer_t(const ProducerLaunch &L) {
         }
         return cudaErrorInvalidValue;
     }
-    const int smem = kProducerPixels * L.pg.C * 4;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(producer_generic_kernel<T>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-    }
-    const long long blocks = (L.pg.npix + kProducerPixels - 1) / kProducerPixels;
-    producer_generic_kernel<T><<<(unsigned)blocks, 256, smem, L.stream>>>(L.pg, x, dw_w, dw_b,
-                                                                          lin_w, lin_b, out);
+    const dim3 grid((unsigned)((L.pg.npix + kProducerPixels - 1) / kProducerPixels),
+                    (unsigned)((L.pg.J + kProducerOuts - 1) / kProducerOuts));
+    producer_generic_kernel<T><<<grid, 256, 0, L.stream>>>(L.pg, x, dw_w, dw_b, lin_w, lin_b, out);
     count_launch();
     return cudaGetLastError();
 }

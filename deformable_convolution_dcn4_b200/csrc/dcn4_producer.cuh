@@ -22,8 +22,9 @@
 //    memory); all eight warps read the accumulators back with tcgen05.ld, add
 //    the bias, round, and store 16-byte pieces of the output rows. lin_w
 //    stays resident in shared memory.
-//  * producer_generic_kernel (any type and shape): 16 pixels per CTA, h in
-//    shared memory (fp32, not rounded), the linear layer on the CUDA cores.
+//  * producer_generic_kernel (any type and shape): 64 pixels x 64 outputs
+//    per CTA, h (fp32, not rounded) and lin_w in channel chunks through
+//    shared memory, 4 x 4 register blocks of outputs on the CUDA cores.
 #pragma once
 
 #include <type_traits>
@@ -426,44 +427,84 @@ __global__ void __launch_bounds__(NW * 32, 1)
 // Generic producer (any type, any C and J)
 // ---------------------------------------------------------------------------
 
+// Tile of kProducerPixels pixels x kProducerOuts outputs per 256-thread
+// CTA; K (= C) in chunks of kProducerK channels: the chunk's depthwise
+// outputs h (fp32) and the chunk of lin_w go to shared memory, k-major, and
+// each thread accumulates a 4 x 4 block of outputs in registers.
 template <typename T>
 __global__ void __launch_bounds__(256)
     producer_generic_kernel(ProducerGeo pg, const T *__restrict__ x, const T *__restrict__ dw_w,
                             const T *__restrict__ dw_b, const T *__restrict__ lin_w,
                             const T *__restrict__ lin_b, T *__restrict__ out) {
-    extern __shared__ __align__(1024) unsigned char smem[];
-    float *h = reinterpret_cast<float *>(smem);  // [kProducerPixels][C]
-    const int C = pg.C, J = pg.J;
-    const long long p0 = (long long)blockIdx.x * kProducerPixels;
-    const int rows = (int)min((long long)kProducerPixels, pg.npix - p0);
-    for (int i = threadIdx.x; i < rows * C; i += blockDim.x) {
-        const int r = i / C, c = i - r * C;
-        const long long p = p0 + r;
-        const int xx = (int)(p % pg.W);
-        const long long t = p / pg.W;
-        const int y = (int)(t % pg.H);
-        const int n = (int)(t / pg.H);
-        float acc = Elem<T>::to_f(dw_b[c]);
-        for (int a = 0; a < 3; ++a) {
-            const int yy = y + a - 1;
-            if (yy < 0 || yy >= pg.H) continue;
-            for (int b = 0; b < 3; ++b) {
-                const int xs = xx + b - 1;
-                if (xs < 0 || xs >= pg.W) continue;
-                acc = fmaf(Elem<T>::to_f(dw_w[(a * 3 + b) * C + c]),
-                           Elem<T>::to_f(x[(((size_t)n * pg.H + yy) * pg.W + xs) * C + c]), acc);
-            }
-        }
-        h[i] = acc;
+    constexpr int PM = kProducerPixels, PN = kProducerOuts, KC = kProducerK, LD = PM + 4;
+    __shared__ __align__(16) float hs[KC][LD];  // h chunk, [k][pixel]
+    __shared__ __align__(16) float ws[KC][LD];  // lin_w chunk, [k][output]
+    __shared__ int2 rowyx[PM];                  // (image row index n*H + y, x) per pixel
+    const int C = pg.C, J = pg.J, tid = threadIdx.x;
+    const long long p0 = (long long)blockIdx.x * PM;
+    const int j0 = blockIdx.y * PN;
+    const int rows = (int)min((long long)PM, pg.npix - p0);
+    if (tid < PM) {
+        const long long p = p0 + tid;
+        rowyx[tid] = make_int2((int)(p / pg.W), (int)(p % pg.W));
     }
+    const int tx = tid & 15, ty = tid >> 4;  // outputs 4tx.., pixels 4ty..
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
     __syncthreads();
-    for (int i = threadIdx.x; i < rows * J; i += blockDim.x) {
-        const int r = i / J, j = i - r * J;
-        const T *wr = lin_w + (size_t)j * C;
-        const float *hr = h + (size_t)r * C;
-        float acc = Elem<T>::to_f(lin_b[j]);
-        for (int c = 0; c < C; ++c) acc = fmaf(Elem<T>::to_f(wr[c]), hr[c], acc);
-        out[(p0 + r) * J + j] = Elem<T>::from_f(acc);
+    for (int c0 = 0; c0 < C; c0 += KC) {
+        // depthwise outputs of the chunk: lanes over channels (coalesced)
+        for (int i = tid; i < PM * KC; i += 256) {
+            const int r = i / KC, k = i - r * KC, c = c0 + k;
+            float v = 0.f;
+            if (r < rows && c < C) {
+                const int ny = rowyx[r].x, xx = rowyx[r].y, y = ny % pg.H;
+                v = Elem<T>::to_f(dw_b[c]);
+#pragma unroll
+                for (int a = 0; a < 3; ++a) {
+                    const int yy = y + a - 1;
+                    if (yy < 0 || yy >= pg.H) continue;
+#pragma unroll
+                    for (int b = 0; b < 3; ++b) {
+                        const int xs = xx + b - 1;
+                        if (xs < 0 || xs >= pg.W) continue;
+                        v = fmaf(Elem<T>::to_f(dw_w[(a * 3 + b) * C + c]),
+                                 Elem<T>::to_f(x[((size_t)(ny + a - 1) * pg.W + xs) * C + c]), v);
+                    }
+                }
+            }
+            hs[k][r] = v;
+        }
+        // the chunk of lin_w: lanes over channels (coalesced)
+        for (int i = tid; i < PN * KC; i += 256) {
+            const int jj = i / KC, k = i - jj * KC, j = j0 + jj, c = c0 + k;
+            ws[k][jj] = (j < J && c < C) ? Elem<T>::to_f(lin_w[(size_t)j * C + c]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < KC; ++k) {
+            const float4 hv = *reinterpret_cast<const float4 *>(&hs[k][4 * ty]);
+            const float4 wv = *reinterpret_cast<const float4 *>(&ws[k][4 * tx]);
+            const float h4[4] = {hv.x, hv.y, hv.z, hv.w}, w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(h4[a], w4[b], acc[a][b]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = 4 * ty + a;
+        if (r >= rows) continue;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int j = j0 + 4 * tx + b;
+            if (j < J) out[(p0 + r) * J + j] = Elem<T>::from_f(acc[a][b] + Elem<T>::to_f(lin_b[j]));
+        }
     }
 }
 
