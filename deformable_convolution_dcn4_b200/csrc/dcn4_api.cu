@@ -437,7 +437,7 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
     memset(&map_go, 0, sizeof(map_go));
     memset(&map_ow, 0, sizeof(map_ow));
     if (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) {
-        const bool base = !L.msdcn && g.kh == 3 && g.kw == 3 && aligned16(input) &&
+        const bool base = g.kh == 3 && g.kw == 3 && aligned16(input) &&
                           aligned16(offset_weight) && aligned16(grad_out) && aligned16(L.acc);
         auto maps = [&]() {
             return encode_input_map(g, L.dtype, input, L.plan, &map_in) &&

@@ -192,14 +192,19 @@ __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *wa
 // DIRECT: grad_input (16-bit T) accumulates in place: each CTA's fp32 sums
 // are rounded once to T and added with packed 16-bit reductions (no fp32
 // workspace). Otherwise sums go to the fp32 workspace `gacc`.
-template <typename T, int U, int NW, bool MIXED, bool DIRECT>
+// MS: the FlowDCN multi-scale variant ("3.1"): ow holds (dir_x, dir_y, m),
+// the offset is s * dir with s from scale_raw (ms.raw); grad_offset_weight
+// receives d/d dir and graw the gradient of scale_raw, as in
+// bwd_generic_kernel.
+template <typename T, int U, int NW, bool MIXED, bool DIRECT, bool MS>
 __global__ void __launch_bounds__(NW * 32, 512 / (NW * 32))
 bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const __grid_constant__ CUtensorMap tmap_go,
                 const __grid_constant__ CUtensorMap tmap_ow, Geometry g, HaloPlan pl,
                 BwdLayout L, const T *__restrict__ in, const T *__restrict__ ow,
                 T *__restrict__ gow, float *__restrict__ gacc, T *__restrict__ gin,
-                unsigned long long ow_bytes) {
+                unsigned long long ow_bytes, const __grid_constant__ MsdcnParams ms,
+                T *__restrict__ graw) {
     constexpr int EB = Elem<T>::kBytes;
     constexpr int VE = Elem<T>::kPerVec;
     constexpr int REC = 27 * EB;
@@ -318,9 +323,13 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
 #pragma unroll
     for (int k = 0; k < 9; ++k) kr[k] = 0xffffffffu;
     const int r = (U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1));
+    float s = 1.0f, gs = 0.0f;  // MSDCN scale of this (pixel, group), d/ds
     if (valid) {
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
         RecordReader<T>::read(rec, v);
+        if (MS)
+            s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]),
+                            ms.s0[tc.g0 + gl], ms.smax);
         // DCNv3 weights: softmax of the logits over the taps; the logit
         // gradient w_k (gw_k - sum_j w_j gw_j) is formed after the taps from
         // the staged gw_k
@@ -361,8 +370,15 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         unsigned esc = 0;
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
-            const float x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
-            const float y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            float x, y, dsx = 0.f, dsy = 0.f;  // ds*: d position / d s (MSDCN)
+            if (MS) {
+                x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, k % 3, 3, g.dw, s, v[3 * k], g.os, &dsx);
+                y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, k / 3, 3, g.dh, s, v[3 * k + 1], g.os,
+                                &dsy);
+            } else {
+                x = __fadd_rn(bxs[k % 3], __fmul_rn(v[3 * k], g.os));
+                y = __fadd_rn(bys[k / 3], __fmul_rn(v[3 * k + 1], g.os));
+            }
             const float m = v[3 * k + 2];
             float gx = 0.f, gy = 0.f, gm = 0.f;
             // a sample outside (-1, W) x (-1, H) has no gradient and no
@@ -387,16 +403,19 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                     d11 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a1 + PS), gop[c]);
                 }
                 gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
-                gx = g.os * m * (hy * (d01 - d00) + ly * (d11 - d10));
-                gy = g.os * m * (hx * (d10 - d00) + lx * (d11 - d01));
+                const float px = hy * (d01 - d00) + ly * (d11 - d10);  // d/d position
+                const float py = hx * (d10 - d00) + lx * (d11 - d01);
+                gx = g.os * m * px;
+                gy = g.os * m * py;
+                if (MS) gs = fmaf(m * px, dsx, fmaf(m * py, dsy, gs));
                 const int cell = gl * ncpg + ((int)(y0f - hy_lo)) * cells_w + (int)(x0f - hx_lo);
                 const int rank = atomicAdd(&counts[cell], 1);
                 kr[k] = ((unsigned)cell << 16) | (unsigned)rank;
             } else {
                 esc |= 1u << k;
             }
-            gout_rec[3 * k] = Elem<T>::from_f(gx);
-            gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
+            gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
+            gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
             gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
             dotw = fmaf(m, gm, dotw);
         }
@@ -410,8 +429,14 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             float dx, dy, m;
             record_tap<T>(rec, k, dx, dy, m);
             if (g.softmax) m = sn.weight(m);
-            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
-            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            float x, y, dsx = 0.f, dsy = 0.f;
+            if (MS) {
+                x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, j, 3, g.dw, s, dx, g.os, &dsx);
+                y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, i, 3, g.dh, s, dy, g.os, &dsy);
+            } else {
+                x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+                y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+            }
             float gx = 0.f, gy = 0.f, gm = 0.f;
             if (x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H) {
                 const float x0f = floorf(x), y0f = floorf(y);
@@ -448,13 +473,19 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                         }
                     }
                 }
+                if (MS) gs = fmaf(m * gx, dsx, fmaf(m * gy, dsy, gs));
                 gx *= g.os * m;
                 gy *= g.os * m;
             }
-            gout_rec[3 * k] = Elem<T>::from_f(gx);
-            gout_rec[3 * k + 1] = Elem<T>::from_f(gy);
+            gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
+            gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
             gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
             dotw = fmaf(m, gm, dotw);
+        }
+        if (MS) {
+            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]);
+            graw[gp * g.G + tc.g0 + gl] = Elem<T>::from_f(
+                gs == 0.0f ? 0.0f : gs * msdcn_scale_grad(raw, ms.s0[tc.g0 + gl], ms.smax));
         }
         if (g.softmax) {
 #pragma unroll
@@ -475,8 +506,15 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             if (kr[k] == 0xffffffffu) continue;
             const int cell = (int)(kr[k] >> 16), rank = (int)(kr[k] & 0xffffu);
             const int i = k / 3, j = k - 3 * (k / 3);
-            const float x = sample_coord(wo * g.sw - g.pw + j * g.dw, v[3 * k], g.os);
-            const float y = sample_coord(ho * g.sh - g.ph + i * g.dh, v[3 * k + 1], g.os);
+            float x, y;
+            if (MS) {
+                float dsx, dsy;
+                x = msdcn_coord(g.msd_dil, wo * g.sw - g.pw, j, 3, g.dw, s, v[3 * k], g.os, &dsx);
+                y = msdcn_coord(g.msd_dil, ho * g.sh - g.ph, i, 3, g.dh, s, v[3 * k + 1], g.os, &dsy);
+            } else {
+                x = sample_coord(wo * g.sw - g.pw + j * g.dw, v[3 * k], g.os);
+                y = sample_coord(ho * g.sh - g.ph + i * g.dh, v[3 * k + 1], g.os);
+            }
             const int pos = counts[cell] + rank;
             const float lx = x - floorf(x), ly = y - floorf(y), m = v[3 * k + 2];
             const unsigned goff = (unsigned)(pix * PS + gl * D * EB);

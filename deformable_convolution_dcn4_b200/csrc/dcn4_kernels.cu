@@ -155,8 +155,8 @@ cudaError_t launch_fwd_t(const FwdLaunch &L) {
     return L.msdcn ? launch_generic_t<T, true>(L) : launch_generic_t<T, false>(L);
 }
 
-template <typename T>
-cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
+template <typename T, bool MS>
+cudaError_t launch_bwd_halo_m(const BwdLaunch &L, bool direct) {
     const int U = L.geo.D * (int)sizeof(T) / 16;
     const long long grid = (long long)L.geo.N * L.plan.slices * L.plan.tiles_h * L.plan.tiles_w;
     const int nt = L.layout.threads;
@@ -166,25 +166,30 @@ cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
         kernel<<<(unsigned)grid, nt, L.layout.smem_bytes, L.stream>>>(
             *L.tmap_in, *L.tmap_go, *L.tmap_ow, L.geo, L.plan, L.layout, static_cast<const T *>(L.in),
             static_cast<const T *>(L.ow), static_cast<T *>(L.gow), L.acc, static_cast<T *>(L.gin),
-            L.ow_bytes);
+            L.ow_bytes, L.ms ? *L.ms : kNoMs, static_cast<T *>(L.graw));
         count_launch();
         return cudaGetLastError();
     };
     if constexpr (sizeof(T) == 2) {
         if (U == 2 && nt == 256) {
-            if (direct) return run(bwd_halo_kernel<T, 2, 8, true, true>);
-            return L.mixed ? run(bwd_halo_kernel<T, 2, 8, true, false>)
-                           : run(bwd_halo_kernel<T, 2, 8, false, false>);
+            if (direct) return run(bwd_halo_kernel<T, 2, 8, true, true, MS>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 8, true, false, MS>)
+                           : run(bwd_halo_kernel<T, 2, 8, false, false, MS>);
         }
         if (U == 2) {
-            if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true>);
-            return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false>)
-                           : run(bwd_halo_kernel<T, 2, 16, false, false>);
+            if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true, MS>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false, MS>)
+                           : run(bwd_halo_kernel<T, 2, 16, false, false, MS>);
         }
     }
-    if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false>);
-    if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false>);
+    if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false, MS>);
+    if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false, MS>);
     return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_bwd_halo(const BwdLaunch &L, bool direct) {
+    return L.msdcn ? launch_bwd_halo_m<T, true>(L, direct) : launch_bwd_halo_m<T, false>(L, direct);
 }
 
 template <typename T, bool MS, int LPP>

@@ -211,13 +211,18 @@ DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
  *       once the clamp is active (or raw is NaN).
  * Arguments as in msdcn_forward and dcn4_backward (grad outputs in
  * desc->dtype, device; the same workspace size, dcn4_backward_workspace_size).
- * grad_input accumulates with fp32 atomics in the workspace (fp32 data: in
- * grad_input): AUTO runs D*sizeof(T)/16 lanes per (pixel, group) with 16-byte
- * vector loads and atomics when the group is a power-of-two count of 16-byte
- * vectors (up to 16) and the tensors are 16-byte aligned, else (and under
- * DCN4_ALGO_GENERIC) one thread per (pixel, group) with scalar atomics;
- * DCN4_ALGO_HALO returns DCN4_ERR_UNSUPPORTED. desc->weights must be
- * DCN4_WEIGHTS_PLAIN. */
+ * Kernels: AUTO runs the staged shared-memory kernel of dcn4_backward (with
+ * the multi-scale positions; its window is the same, so more samples take its
+ * global path) when the call qualifies for it as a dcn4_backward call would
+ * (3x3 taps, a group of 2 or 4 16-byte vectors, 16-byte aligned tensors), and
+ * grad_input then accumulates as in dcn4_backward; otherwise grad_input
+ * accumulates with fp32 atomics in the workspace (fp32 data: in grad_input)
+ * from D*sizeof(T)/16 lanes per (pixel, group) with 16-byte vector loads when
+ * the group is a power-of-two count of 16-byte vectors (up to 16) and the
+ * tensors are 16-byte aligned, else (and under DCN4_ALGO_GENERIC) from one
+ * thread per (pixel, group) with scalar atomics. DCN4_ALGO_HALO and
+ * DCN4_ALGO_VECTOR demand their kernel (DCN4_ERR_UNSUPPORTED where it does not
+ * apply). desc->weights must be DCN4_WEIGHTS_PLAIN. */
 DCN4_API dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input,
                           const void *dir_weight, const void *scale_raw,
                           const float *s0_host, float smax, const void *grad_out,

@@ -345,7 +345,8 @@ def test_msdcn_backward_full_size_sampled(orc):
 
 
 def test_msdcn_backward_halo_request_is_unsupported():
-    wl = MSDCN_BWD["msdcn_d16_bf16"]
+    """D64 bf16 (8 vectors per group) is beyond the staged backward kernel."""
+    wl = MSDCN_BWD["flowdcn_msdcn_bf16"]
     data = make_inputs(wl, out_hw(wl), with_grad=True)
     with pytest.raises(B.Dcn4Error) as e:
         B.msdcn_backward(data["input"].cuda(), data["dir_weight"].cuda(), data["scale_raw"].cuda(),
@@ -442,6 +443,38 @@ def test_backward_global_kernels(orc, name, algo):
     e_in, e_ow = backward_case(orc, wl, algo)
     tol = TOL[wl.dtype]
     assert e_in <= tol and e_ow <= tol, f"{name}/{algo}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
+
+
+# the staged kernel (AUTO picks it for these) and the vectorised one, forced,
+# on the same D16 MSDCN shapes (stride, dilation and offset_scale included),
+# both readings, both math modes
+MSDCN_BWD_HALO = {
+    "msdcn_d16_bf16": MSDCN_BWD["msdcn_d16_bf16"],
+    "msdcn_d16_f32": MSDCN_BWD["msdcn_d16_f32"],
+    "msdcn_stride_bf16": MSDCN_BWD["msdcn_stride_f16"].replace(name="msdsb", dtype="bf16", C=64),
+    "dil_bf16": DILATION["dil_bf16"],
+    "dil_f32": DILATION["dil_f32"],
+    "msdcn_d16_bf16_smax8_far": MSDCN_BWD["msdcn_d16_bf16"].replace(
+        name="msdfar", N=2, H=29, W=23, offset_dist=("normal", 2.5)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MSDCN_BWD_HALO))
+@pytest.mark.parametrize("algo", ["halo", "vector"])
+@pytest.mark.parametrize("math", ["default", "f32"])
+def test_msdcn_backward_staged_and_vector(orc, name, algo, math):
+    wl = MSDCN_BWD_HALO[name]
+    errs = msdcn_backward_case(orc, wl, algo=algo, math=math)
+    tol = TOL[wl.dtype]
+    assert all(e <= tol for e in errs), f"{name}/{algo}/{math}: grad_input/dir/raw {errs}"
+
+
+def test_msdcn_backward_staged_full_size_sampled(orc):
+    """The bench's MSDCN shape (N64 56x56 C128 G8 bf16) on the staged kernel;
+    images 0 and 63 against the oracle."""
+    wl = W["internimage_bf16"].replace(kind="msdcn", offset_dist=("normal", 1.0))
+    errs = msdcn_backward_case(orc, wl, algo="halo", images=[0, 63])
+    assert all(e <= TOL["bf16"] for e in errs), errs
 
 
 @pytest.mark.parametrize("name", ["msdcn_d16_bf16", "msdcn_stride_f16"])
