@@ -19,9 +19,10 @@
 //    operand type of the tensor cores) straight into the tcgen05 K-major
 //    core-matrix layout; one thread issues the K/16 tcgen05.mma (M = 128
 //    pixels, N = the outputs padded to 16, fp32 accumulators in tensor
-//    memory); all eight warps read the accumulators back with tcgen05.ld, add
-//    the bias, round, and store 16-byte pieces of the output rows. lin_w
-//    stays resident in shared memory.
+//    memory); all warps read the accumulators back with tcgen05.ld, add the
+//    bias and round; the tile's output rows are staged in its consumed input
+//    buffer and leave in one bulk copy (else each thread stores 16-byte
+//    pieces). lin_w stays resident in shared memory.
 //  * producer_generic_kernel (any type and shape): 64 pixels x 64 outputs
 //    per CTA, h (fp32, not rounded) and lin_w in channel chunks through
 //    shared memory, 4 x 4 register blocks of outputs on the CUDA cores.
