@@ -31,9 +31,9 @@ struct Geometry {
 
 // Tile of the generic producer kernel: pixels x outputs per CTA, channels
 // per shared-memory chunk.
-constexpr int kProducerPixels = 64;
-constexpr int kProducerOuts = 64;
-constexpr int kProducerK = 32;
+constexpr int kProducerPixels = 128;
+constexpr int kProducerOuts = 128;
+constexpr int kProducerK = 16;
 
 // Shape of one producer launch.
 struct ProducerGeo {

@@ -23,9 +23,9 @@
 //    bias and round; the tile's output rows are staged in its consumed input
 //    buffer and leave in one bulk copy (else each thread stores 16-byte
 //    pieces). lin_w stays resident in shared memory.
-//  * producer_generic_kernel (any type and shape): 64 pixels x 64 outputs
+//  * producer_generic_kernel (any type and shape): 128 pixels x 128 outputs
 //    per CTA, h (fp32, not rounded) and lin_w in channel chunks through
-//    shared memory, 4 x 4 register blocks of outputs on the CUDA cores.
+//    shared memory, 8 x 8 register blocks of outputs on the CUDA cores.
 #pragma once
 
 #include <type_traits>
@@ -431,13 +431,14 @@ __global__ void __launch_bounds__(NW * 32, 1)
 // Tile of kProducerPixels pixels x kProducerOuts outputs per 256-thread
 // CTA; K (= C) in chunks of kProducerK channels: the chunk's depthwise
 // outputs h (fp32) and the chunk of lin_w go to shared memory, k-major, and
-// each thread accumulates a 4 x 4 block of outputs in registers.
+// each thread accumulates an 8 x 8 block of outputs in registers.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     producer_generic_kernel(ProducerGeo pg, const T *__restrict__ x, const T *__restrict__ dw_w,
                             const T *__restrict__ dw_b, const T *__restrict__ lin_w,
                             const T *__restrict__ lin_b, T *__restrict__ out) {
     constexpr int PM = kProducerPixels, PN = kProducerOuts, KC = kProducerK, LD = PM + 4;
+    static_assert(PM == 128 && PN == 128, "16 x 16 threads of 8 x 8 outputs");
     __shared__ __align__(16) float hs[KC][LD];  // h chunk, [k][pixel]
     __shared__ __align__(16) float ws[KC][LD];  // lin_w chunk, [k][output]
     __shared__ int2 rowyx[PM];                  // (image row index n*H + y, x) per pixel
@@ -449,12 +450,12 @@ __global__ void __launch_bounds__(256)
         const long long p = p0 + tid;
         rowyx[tid] = make_int2((int)(p / pg.W), (int)(p % pg.W));
     }
-    const int tx = tid & 15, ty = tid >> 4;  // outputs 4tx.., pixels 4ty..
-    float acc[4][4];
+    const int tx = tid & 15, ty = tid >> 4;  // outputs 8tx.., pixels 8ty..
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
     __syncthreads();
     for (int c0 = 0; c0 < C; c0 += KC) {
         // depthwise outputs of the chunk: lanes over channels (coalesced)
@@ -485,25 +486,28 @@ __global__ void __launch_bounds__(256)
             ws[k][jj] = (j < J && c < C) ? Elem<T>::to_f(lin_w[(size_t)j * C + c]) : 0.f;
         }
         __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
         for (int k = 0; k < KC; ++k) {
-            const float4 hv = *reinterpret_cast<const float4 *>(&hs[k][4 * ty]);
-            const float4 wv = *reinterpret_cast<const float4 *>(&ws[k][4 * tx]);
-            const float h4[4] = {hv.x, hv.y, hv.z, hv.w}, w4[4] = {wv.x, wv.y, wv.z, wv.w};
+            const float4 h0 = *reinterpret_cast<const float4 *>(&hs[k][8 * ty]);
+            const float4 h1 = *reinterpret_cast<const float4 *>(&hs[k][8 * ty + 4]);
+            const float4 w0 = *reinterpret_cast<const float4 *>(&ws[k][8 * tx]);
+            const float4 w1 = *reinterpret_cast<const float4 *>(&ws[k][8 * tx + 4]);
+            const float h8[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 8; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(h4[a], w4[b], acc[a][b]);
+                for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(h8[a], w8[b], acc[a][b]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int r = 4 * ty + a;
+    for (int a = 0; a < 8; ++a) {
+        const int r = 8 * ty + a;
         if (r >= rows) continue;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int j = j0 + 4 * tx + b;
+        for (int b = 0; b < 8; ++b) {
+            const int j = j0 + 8 * tx + b;
             if (j < J) out[(p0 + r) * J + j] = Elem<T>::from_f(acc[a][b] + Elem<T>::to_f(lin_b[j]));
         }
     }
