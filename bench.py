@@ -9,6 +9,9 @@ events on the launching stream time each op. The reported value is effective
 bandwidth: the operator's ideal bytes (input and output once, 27 offset/weight
 values per pixel and group; DCNv4 digest "GPU效率的理论分析") per second of device
 time, summed over all ranks (weak scaling: every rank runs a full batch).
+Outside the timed step, `next_rows` times MSDCN backward and the offset/weight
+producer (depthwise 3x3 + merged linear) on the same shape, graph-replayed
+with the same L2 flush; they are reported, not counted in the value.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
