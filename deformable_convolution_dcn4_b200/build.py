@@ -14,11 +14,13 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libdcn4.so")
-SOURCES = ["dcn4_api.cu", "dcn4_kernels.cu", "dcn4_noalloc.cu"]
+SOURCES = ["dcn4_api.cu", "dcn4_kernels.cu", "dcn4_kernels_fwd.cu", "dcn4_kernels_bwd.cu",
+           "dcn4_noalloc.cu"]
+OBJDIR = os.path.join(PKG, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-         "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden",
+         "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-DDCN4_BUILDING_LIBRARY", "-I", INCLUDE, "-I", CSRC]
 
 
@@ -36,13 +38,24 @@ def up_to_date():
 
 
 def build(force=False, verbose=False):
+    """Compiles each translation unit to an object (in parallel), then links
+    the shared library."""
     if not force and up_to_date():
         return LIBRARY
-    cmd = [NVCC, *FLAGS]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", LIBRARY]
-    subprocess.run(cmd, check=True)
+    os.makedirs(OBJDIR, exist_ok=True)
+    procs, objs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJDIR, src[:-3] + ".o")
+        cmd = [NVCC, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(failed)})")
+    subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs,
+                    "-o", LIBRARY], check=True)
     return LIBRARY
 
 

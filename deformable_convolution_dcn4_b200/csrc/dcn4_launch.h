@@ -1,5 +1,5 @@
 // dcn4_launch.h -- host-side launch interface between the C ABI (dcn4_api.cu)
-// and the kernel translation unit (dcn4_kernels.cu).
+// and the kernel translation units (dcn4_kernels*.cu).
 #pragma once
 
 #include "dcn4_common.cuh"
@@ -69,8 +69,18 @@ cudaError_t launch_backward(const BwdLaunch &L);
 // Launches the bounded-wait self-test kernel (see dcn4_selftest_bounded_wait).
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 
-// Reads and clears the device error word of the current device.
+// Reads and clears the device error words of the current device (one per
+// kernel translation unit, ORed).
 cudaError_t read_clear_device_error(unsigned *bits);
+cudaError_t read_clear_error_fwd(unsigned *bits);
+cudaError_t read_clear_error_bwd(unsigned *bits);
+
+// Shared launch helpers (dcn4_kernels.cu): count one issued kernel; raise a
+// kernel's dynamic shared-memory limit once per (kernel, device); a grid of
+// ceil(work / block) blocks capped at 16 per SM.
+void count_launch();
+cudaError_t allow_smem(const void *kernel, int bytes);
+int grid_for(long long work, int block);
 
 // Kernels issued by this library so far (launched, or captured into a graph).
 unsigned long long launches_issued();

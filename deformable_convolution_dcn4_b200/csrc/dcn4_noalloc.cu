@@ -13,7 +13,13 @@
 // GPU that loads the library holds it until the process exits. Host code may
 // not pass the array's name to a kernel (on the host it is only a stand-in
 // symbol), so the first call on each device looks up its device address with
-// cudaGetSymbolAddress while that device is current and caches it.
+// cudaGetSymbolAddress while that device is current and caches it. The
+// address belongs to the CUDA context it was looked up in, so the cache is
+// keyed by the context's unique id as well: after cudaDeviceReset, or when a
+// caller makes another context current on the same device, the next call
+// looks the address up again instead of using a stale one.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "dcn4.h"
@@ -26,18 +32,51 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_backward_scratch[kScratchBytes];
 
-// Device address of g_backward_scratch on the current device (looked up once
-// per device); nullptr when the lookup fails.
+// Unique id of the current driver context (cuCtxGetId, found through the
+// runtime's driver entry-point query, so libcuda need not be linked); 0 when
+// there is no current context or the query is unavailable.
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_backward_scratch in the current device's current
+// context, looked up once per (device, context); nullptr when the lookup
+// fails.
 float *scratch_on_current_device() {
     static std::mutex mu;
     static void *addr[kMaxDevices] = {nullptr};
+    static unsigned long long ctx_of[kMaxDevices] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_backward_scratch) != cudaSuccess) return nullptr;
+        // also creates the device's primary context if none was current
+        if (cudaGetSymbolAddress(&p, g_backward_scratch) != cudaSuccess || !p) return nullptr;
         addr[dev] = p;
+        ctx_of[dev] = current_context_id();
     }
     return static_cast<float *>(addr[dev]);
 }

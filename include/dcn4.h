@@ -31,8 +31,10 @@
  *
  * Conventions for every entry point:
  *   - Device pointers are owned by the caller; the library allocates no memory
- *     and keeps no per-call state (the one exception is a device error word,
- *     see dcn4_last_device_error).
+ *     and keeps no per-call state. Exceptions: a device error word (see
+ *     dcn4_last_device_error), a launch counter (dcn4_kernel_launches), and
+ *     the fixed 32 MiB scratch array of dcn4_backward_noalloc together with
+ *     its per-(device, context) address cache (see that entry point).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Calls only enqueue work; they never synchronise the device.
  *   - Outputs are overwritten, never accumulated into.
@@ -271,10 +273,14 @@ DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
  * and allocates nothing.
  *   - Limit: dcn4_backward_workspace_size(desc) must be <= 32 MiB
  *     (N*H*W*C <= 8,388,608 for bf16/fp16); larger calls return
- *     DCN4_ERR_WORKSPACE without launching. fp32 calls need no scratch.
+ *     DCN4_ERR_WORKSPACE without launching. The limit applies to every
+ *     bf16/fp16 call, also to those whose kernels end up not touching the
+ *     scratch. fp32 calls need no scratch and have no limit.
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress); make that first call before any stream
- *     capture.
+ *     capture. The address is cached per (device, CUDA context): a call made
+ *     under another context (after cudaDeviceReset, or a context the caller
+ *     made current through the driver API) looks it up again.
  *   - All calls on a device share the one array; each call zeroes the part it
  *     uses first, but calls that overlap on the GPU (different streams, or
  *     several host threads) race on it and give wrong results.

@@ -515,6 +515,40 @@ def pin_msdcn_bwd_raw(o):
         assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), f"d/d raw at {idx}: {fd} vs {an}"
 
 
+def pin_msdcn_bwd_nan(o):
+    """A (pixel, group) whose scale is NaN, and a tap pushed far outside the
+    image, contribute nothing (the zero-outside reading applied to the
+    FlowDCN "3.1" chain rule): their direction, weight and raw-scale
+    gradients are exactly 0, grad_input equals that of the same problem with
+    their weights m set to 0, every other gradient is bit-identical to the
+    problem without the NaN, and the adjoint identity holds."""
+    prob, x, dw, raw, s0, go = _msdcn_case(o, 86)
+    smax = 3.0
+    nan_at = (1, 2, 3, 1)   # (n, ho, wo, g) with raw = NaN
+    far_at = (0, 4, 5, 2)   # (n, ho, wo, g) whose tap 4 leaves the image
+    raw[nan_at] = np.nan
+    dw[far_at + (4, 0)] = -1000.0
+    gin, gdw, graw = o.msdcn_backward(prob, x, dw, raw, s0, smax, go)
+    assert np.all(gdw[nan_at] == 0.0), "NaN scale: direction/weight gradients"
+    assert graw[nan_at] == 0.0, "NaN scale: raw gradient"
+    assert np.all(gdw[far_at + (4,)] == 0.0), "tap outside the image: its gradients"
+    assert np.all(np.isfinite(gin)) and np.all(np.isfinite(gdw)) and np.all(np.isfinite(graw))
+    # the same problem with the two contributions removed through m = 0
+    raw2, dw2 = raw.copy(), dw.copy()
+    raw2[nan_at] = 0.25
+    dw2[nan_at + (slice(None), 2)] = 0.0
+    dw2[far_at + (4, 2)] = 0.0
+    rgin, rgdw, rgraw = o.msdcn_backward(prob, x, dw2, raw2, s0, smax, go)
+    assert np.array_equal(gin, rgin), "grad_input without the two contributions"
+    keep = np.ones(raw.shape, bool)
+    keep[nan_at] = False
+    assert np.array_equal(graw[keep], rgraw[keep]), "raw gradients of the other pairs"
+    assert np.array_equal(gdw[keep], rgdw[keep]), "dir/weight gradients of the other pairs"
+    lhs = float(np.sum(o.msdcn_forward(prob, x, dw, raw, s0, smax) * go))
+    rhs = float(np.sum(x.astype(np.float64) * gin))
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs)), "adjoint with a NaN scale"
+
+
 def _box(x, K, stride, pad, dil, kh=3, kw=3):
     """Depthwise conv with every weight 1/K (float64, torch)."""
     C = x.shape[-1]
@@ -722,5 +756,5 @@ def pin_producer(o):
 ALL_PINS = [pin_conv, pin_grid_sample, pin_gather, pin_fractions, pin_out_of_bounds,
             pin_linearity, pin_equivariance, pin_msdcn, pin_cost_model, pin_adjoint,
             pin_unit_columns, pin_finite_diff, pin_msdcn_bwd_unit, pin_msdcn_bwd_adjoint,
-            pin_msdcn_bwd_dir, pin_msdcn_bwd_raw, pin_softmax_box, pin_softmax_shift,
+            pin_msdcn_bwd_dir, pin_msdcn_bwd_raw, pin_msdcn_bwd_nan, pin_softmax_box, pin_softmax_shift,
             pin_softmax_bwd, pin_msdcn_dilation, pin_producer]

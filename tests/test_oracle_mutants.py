@@ -55,6 +55,8 @@ MUTANTS = [
      "float s = orc_msdcn_scale(scale_raw[pix * p->G + g], s0[0], smax);", 1),
     ("msdcn_grad_dir_missing_s", "gt[3 * k] = gdx == 0.0 ? 0.0 : (double)s * gdx;",
      "gt[3 * k] = gdx;", 1),
+    ("msdcn_nan_scale_dir_grad_unguarded", "gt[3 * k] = gdx == 0.0 ? 0.0 : (double)s * gdx;",
+     "gt[3 * k] = (double)s * gdx;", 1),
     ("msdcn_sigmoid_sign", "return (double)s0 / (1.0 + exp(-(double)raw));",
      "return (double)s0 / (1.0 + exp((double)raw));", 1),
     ("msdcn_clamp_gradient_kept", "if (!(u <= smax))\n        return 0.0;",
