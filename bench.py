@@ -12,6 +12,14 @@ time, summed over all ranks (weak scaling: every rank runs a full batch).
 Outside the timed step, `next_rows` times MSDCN backward and the offset/weight
 producer (depthwise 3x3 + merged linear) on the same shape, graph-replayed
 with the same L2 flush; they are reported, not counted in the value.
+`configs` times every workload of the table below the same way (median of
+graph replays, L2 flushed before each): forward, backward (fp32 accumulation
+of grad_input across CTAs, the default, and the 16-bit cross-CTA variant
+acc16), MSDCN forward and backward, each with ideal bytes, GB/s, the
+fraction of the HBM peak and the fraction of samples outside the image.
+The CPU-baseline leg, which runs the oracle, also checks one image of every
+(config, op) against it (scaled max error and an elementwise error with an
+rms floor).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
@@ -32,6 +40,19 @@ if ROOT not in sys.path:
 METRIC = "DCNv4 fwd/bwd GB/s and Gsample·ch/s at 1 B200; % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
+
+# (label, workload, ops) timed outside the step; "bwd" is the default
+# backward (fp32 accumulation across CTAs), "bwd_acc16" the 16-bit cross-CTA
+# accumulation, "msbwd" the MSDCN backward (default math)
+CONFIG_TABLE = [
+    ("c1", "tiny_f32", ["fwd", "bwd"]),
+    ("c2", "internimage_bf16", ["fwd", "bwd", "bwd_acc16", "msfwd", "msbwd"]),
+    ("c2", "internimage_f32", ["fwd", "bwd"]),
+    ("c3a", "ldm64_f16", ["fwd", "bwd", "bwd_acc16"]),
+    ("c3b", "ldm32_f16", ["fwd", "bwd", "bwd_acc16"]),
+    ("c4", "flowdcn_msdcn_bf16", ["msfwd", "msbwd"]),
+    ("c5", "highres_bf16", ["fwd", "bwd", "bwd_acc16"]),
+]
 
 
 def parse_args(argv=None):
@@ -387,6 +408,9 @@ def run_ours(args):
     # timed the same way outside the timed region, reported on their own
     extra = next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind)
 
+    # every workload of the table, each op timed on its own (outside the step)
+    configs, samples = time_configs(dcn, flush, stream, peak, peak_kind)
+
     # end to end: pinned host buffers, H2D copies + the three calls + D2H reads
     e2e = run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream,
                   step_bytes, world)
@@ -399,9 +423,12 @@ def run_ours(args):
             "config": describe(wl, Ho, Wo), "roofline": roofline, "ops": breakdown,
             "gpu_launches": args.steps * sum(launches.values()),
             "launches_per_step": launches, "e2e": e2e, "next_rows": extra,
-            "clocks": clocks.summary()}
+            "configs": configs, "clocks": clocks.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+        for key, per_op in oracle_config_checks(samples).items():
+            for op, errs in per_op.items():
+                configs[key]["ops"][op].update(errs)
     barrier(dev)
     for g in graphs.values():
         del g
@@ -471,6 +498,157 @@ def next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind):
             "median_ms": round(ms, 5), "ideal_bytes": ib, "GB/s": round(ib / (ms * 1e-3) / 1e9, 1),
             f"frac_of_{peak_kind}_hbm": round(ib / (ms * 1e-3) / 1e9 / peak, 4),
             "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)}
+    return res
+
+
+def op_ideal_bytes(wl, Ho, Wo, op):
+    """Ideal bytes of one op: every tensor it reads or writes once (DCNv4
+    digest "GPU效率的理论分析" for the forward; the backward reads input,
+    grad_out and offset_weight and writes grad_input and grad_offset_weight;
+    MSDCN adds the raw scales, read and, in the backward, their gradient)."""
+    eb = 4 if wl.dtype == "f32" else 2
+    nin = wl.N * wl.H * wl.W * wl.C
+    nout = wl.N * Ho * Wo * wl.C
+    now = wl.N * Ho * Wo * wl.G * wl.K * 3
+    nraw = wl.N * Ho * Wo * wl.G
+    elems = {"fwd": nin + nout + now, "bwd": 2 * nin + nout + 2 * now,
+             "bwd_acc16": 2 * nin + nout + 2 * now, "msfwd": nin + nout + now + nraw,
+             "msbwd": 2 * nin + nout + 2 * now + 2 * nraw}[op]
+    return elems * eb
+
+
+def oob_fraction(wl, d, Ho, Wo, msdcn):
+    """Fraction of bilinear samples whose position lies outside (-1, W) x
+    (-1, H), i.e. that contribute nothing (a statistic of the synthetic
+    inputs, printed next to the timings)."""
+    import torch
+    ow = (d["dir_weight"] if msdcn else d["offset_weight"]).float()
+    dx, dy = ow[..., 0], ow[..., 1]
+    if msdcn:
+        raw = d["scale_raw"].float()
+        s0 = d["s0"].to(raw.device).view(1, 1, 1, -1)
+        s = torch.clamp(s0 * torch.nn.functional.softplus(raw), max=wl.smax).unsqueeze(-1)
+        dx, dy = s * dx, s * dy
+    dev = ow.device
+    i = torch.arange(wl.kh, device=dev).repeat_interleave(wl.kw).view(1, 1, 1, 1, -1)
+    j = torch.arange(wl.kw, device=dev).repeat(wl.kh).view(1, 1, 1, 1, -1)
+    ho = torch.arange(Ho, device=dev).view(1, -1, 1, 1, 1)
+    wo = torch.arange(Wo, device=dev).view(1, 1, -1, 1, 1)
+    x = (wo * wl.stride[1] - wl.pad[1] + j * wl.dilation[1]).float() + dx * wl.offset_scale
+    y = (ho * wl.stride[0] - wl.pad[0] + i * wl.dilation[0]).float() + dy * wl.offset_scale
+    inside = (x > -1) & (x < wl.W) & (y > -1) & (y < wl.H)
+    return round(1.0 - inside.float().mean().item(), 4)
+
+
+def time_configs(dcn, flush, stream, peak, peak_kind):
+    """Times every (config, op) of CONFIG_TABLE; returns (table, samples) where
+    samples keep one image's inputs and GPU outputs (host, fp32) per op for the
+    oracle check of the CPU-baseline leg."""
+    import torch
+    from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
+    table, samples = {}, []
+    dev = flush.device
+    for label, wname, ops in CONFIG_TABLE:
+        wl = WORKLOADS[wname]
+        desc = dcn.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, 0, (wl.kh, wl.kw), wl.stride, wl.pad,
+                             wl.dilation, wl.offset_scale)
+        Ho, Wo = dcn.dcn4_out_shape(desc)
+        kw = dict(group=wl.G, kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad,
+                  dilation=wl.dilation, offset_scale=wl.offset_scale)
+        entry = {"label": label, "shape": f"N{wl.N} {wl.H}x{wl.W} C{wl.C} G{wl.G} (D{wl.D}) "
+                                          f"{wl.dtype}", "ops": {}}
+        needs_dcn = any(not o.startswith("ms") for o in ops)
+        needs_ms = any(o.startswith("ms") for o in ops)
+        dh = make_inputs(wl, (Ho, Wo), with_grad=True) if needs_dcn and wl.kind != "msdcn" else None
+        mwl = wl if wl.kind == "msdcn" else msdcn_variant(wl)
+        mh = make_inputs(mwl, (Ho, Wo), with_grad=True) if needs_ms else None
+        d = {k: v.to(dev) for k, v in dh.items()} if dh else None
+        m = {k: (v if k == "s0" else v.to(dev)) for k, v in mh.items()} if mh else None
+        ws = torch.empty(max(wl.N * wl.H * wl.W * wl.C * 4, 16), dtype=torch.uint8, device=dev)
+        n_s = wl.N - 1  # the image the oracle checks
+        for op in ops:
+            src = m if op.startswith("ms") else d
+            x = src["input"]
+            if op == "fwd":
+                outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
+                fn = lambda: dcn.dcn4_forward(d["input"], d["offset_weight"], out=outs[0], **kw)
+            elif op in ("bwd", "bwd_acc16"):
+                outs = [torch.empty_like(x), torch.empty_like(d["offset_weight"])]
+                math = "acc16" if op == "bwd_acc16" else "default"
+                fn = lambda: dcn.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"],
+                                               workspace=ws, grad_input=outs[0],
+                                               grad_offset_weight=outs[1], math=math, **kw)
+            elif op == "msfwd":
+                outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
+                fn = lambda: dcn.msdcn_forward(m["input"], m["dir_weight"], m["scale_raw"],
+                                               m["s0"], mwl.smax, out=outs[0], **kw)
+            else:  # msbwd
+                outs = [torch.empty_like(x), torch.empty_like(m["dir_weight"]),
+                        torch.empty_like(m["scale_raw"])]
+                fn = lambda: dcn.msdcn_backward(m["input"], m["dir_weight"], m["scale_raw"],
+                                                m["s0"], mwl.smax, m["grad_out"], workspace=ws,
+                                                grad_input=outs[0], grad_dir_weight=outs[1],
+                                                grad_scale_raw=outs[2], **kw)
+            n0 = dcn.dcn4_kernel_launches()
+            fn()
+            launches = dcn.dcn4_kernel_launches() - n0
+            ms = graph_median_ms(fn, flush, stream)
+            ib = op_ideal_bytes(wl, Ho, Wo, op)
+            gbs = ib / (ms * 1e-3) / 1e9
+            rec = {"median_ms": round(ms, 5), "ideal_bytes": ib, "GB/s": round(gbs, 1),
+                   f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4), "launches": launches,
+                   "oob_fraction": oob_fraction(mwl if op.startswith("ms") else wl, src, Ho, Wo,
+                                                op.startswith("ms"))}
+            if op in ("fwd", "msfwd"):
+                rec["Gsample_ch_per_s"] = round(samples_ch(wl, Ho, Wo) / (ms * 1e-3) / 1e9, 1)
+            entry["ops"][op] = rec
+            torch.cuda.synchronize()
+            samples.append({"key": f"{label}_{wname}", "op": op,
+                            "wl": (mwl if op.startswith("ms") else wl).replace(N=1),
+                            "inputs": {k: (v if k == "s0" else v[n_s:n_s + 1].float().cpu())
+                                       for k, v in src.items()},
+                            "outputs": [t[n_s:n_s + 1].float().cpu() for t in outs]})
+        table[f"{label}_{wname}"] = entry
+        del d, m, ws, dh, mh
+        torch.cuda.empty_cache()
+    return table, samples
+
+
+def oracle_config_checks(samples):
+    """Part of the CPU-baseline leg: the oracle on the one sampled image of
+    every (config, op), compared with the GPU result. Returns
+    {key: {op: {max_scaled_err, max_rel_err_rms_floor}}} over all outputs."""
+    import numpy as np
+
+    import oracle
+    orc = oracle.default()
+    res = {}
+    for smp in samples:
+        wl, op, a = smp["wl"], smp["op"], {k: (v if k == "s0" else v.numpy())
+                                            for k, v in smp["inputs"].items()}
+        prob = orc.problem(1, wl.H, wl.W, wl.C, wl.G, wl.kh, wl.kw, wl.stride, wl.pad,
+                           wl.dilation, wl.offset_scale)
+        if op == "fwd":
+            refs = [orc.forward(prob, a["input"], a["offset_weight"])]
+        elif op in ("bwd", "bwd_acc16"):
+            refs = list(orc.backward(prob, a["input"], a["offset_weight"], a["grad_out"]))
+        elif op == "msfwd":
+            refs = [orc.msdcn_forward(prob, a["input"], a["dir_weight"], a["scale_raw"],
+                                      a["s0"].numpy(), wl.smax)]
+        else:
+            refs = list(orc.msdcn_backward(prob, a["input"], a["dir_weight"], a["scale_raw"],
+                                           a["s0"].numpy(), wl.smax, a["grad_out"]))
+        scaled, elem = 0.0, 0.0
+        for got, ref in zip(smp["outputs"], refs):
+            got = got.numpy().astype(np.float64)
+            ref = np.asarray(ref, np.float64)
+            diff = np.abs(got - ref)
+            scale = np.abs(ref).max()
+            rms = float(np.sqrt(np.mean(ref * ref)))
+            scaled = max(scaled, float(diff.max() / scale) if scale > 0 else float(diff.max()))
+            elem = max(elem, float((diff / (np.abs(ref) + rms)).max()) if rms > 0 else 0.0)
+        res.setdefault(smp["key"], {})[op] = {"max_scaled_err": float(f"{scaled:.3e}"),
+                                              "max_rel_err_rms_floor": float(f"{elem:.3e}")}
     return res
 
 

@@ -12,13 +12,14 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(_PKG, "libdcn4.so")
+CHECKED_LIBRARY = os.path.join(_PKG, "libdcn4_checked.so")
 
 STATUS = {0: "DCN4_OK", 1: "DCN4_ERR_INVALID_ARG", 2: "DCN4_ERR_UNSUPPORTED",
           3: "DCN4_ERR_WORKSPACE", 4: "DCN4_ERR_CUDA", 5: "DCN4_ERR_TIMEOUT",
           6: "DCN4_ERR_INTERNAL"}
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "generic": 1, "halo": 2, "vector": 3}
-MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2, "packed16": 3}
+MATH_CODE = {"default": 0, "f32": 1, "mixed16": 2, "packed16": 3, "acc16": 4}
 MSDCN_MODE_CODE = {"offset": 0, "dilation": 1}
 
 # Every symbol include/dcn4.h declares.
@@ -50,8 +51,28 @@ def load(path=LIBRARY):
     global _lib
     if _lib is not None:
         return _lib
+    _lib = _open(path)
+    return _lib
+
+
+def use_library(path):
+    """Makes every call of this module go to the library at `path` (e.g. the
+    bounds-checked build, libdcn4_checked.so); returns the library used
+    before, for restore_library."""
+    global _lib
+    prev = _lib
+    _lib = _open(path)
+    return prev
+
+
+def restore_library(prev):
+    global _lib
+    _lib = prev
+
+
+def _open(path):
     if not os.path.exists(path):
-        raise RuntimeError(f"libdcn4.so not built ({path}); run "
+        raise RuntimeError(f"{os.path.basename(path)} not built ({path}); run "
                            "`python -m deformable_convolution_dcn4_b200.build`")
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER(Desc)
@@ -74,7 +95,6 @@ def load(path=LIBRARY):
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
-    _lib = lib
     return lib
 
 

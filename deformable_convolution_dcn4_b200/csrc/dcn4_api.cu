@@ -38,7 +38,7 @@ bool make_geometry(const dcn4_desc *d, Geometry *g) {
         d->algo != DCN4_ALGO_VECTOR)
         return false;
     if (d->math != DCN4_MATH_DEFAULT && d->math != DCN4_MATH_F32 && d->math != DCN4_MATH_MIXED16 &&
-        d->math != DCN4_MATH_PACKED16)
+        d->math != DCN4_MATH_PACKED16 && d->math != DCN4_MATH_ACC16)
         return false;
     if (d->weights != DCN4_WEIGHTS_PLAIN && d->weights != DCN4_WEIGHTS_SOFTMAX) return false;
     if (d->msdcn_mode != DCN4_MSDCN_SCALE_OFFSET && d->msdcn_mode != DCN4_MSDCN_SCALE_DILATION)
@@ -140,44 +140,52 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, bool rec_tma, HaloPlan *ou
 }
 
 // Tiling and shared-memory layout of the backward halo kernel: one
-// (pixel, group) pair per thread (256 or 512 threads), 128-byte staged
-// pixels, R = 4; the sorted sample records (8 or 16 bytes each) reuse the
-// window and record slots, so they must fit there.
-bool plan_bwd(const Geometry &g, int eb, bool rec_tma, HaloPlan *out, BwdLayout *lay) {
+// (pixel, group) pair per thread, or per two lanes when a group is 8 chunks
+// (128 bytes: each lane owns 4); 256 or 512 threads; 128-byte staged pixels.
+// The window reaches R = 4 pixels beyond the tile; for the multi-scale
+// variant, whose scaled offsets reach far, the whole image (plus its zero
+// border) is tried first. The sorted sample records (16 bytes each) and the
+// owner list reuse the window and record slots, so they must fit there.
+bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out,
+              BwdLayout *lay) {
     if (128 % (g.D * eb) != 0) return false;
     const int Gc = 128 / (g.D * eb);
     if (g.G % Gc != 0) return false;
     const int U = g.D * eb / 16;
-    if (!(U == 4 || (U == 2 && eb == 2))) return false;
+    if (!(U == 4 || (U == 2 && eb == 2) || U == 8)) return false;
+    const int lpp = U == 8 ? 2 : 1;
     const int R = 4;
     const int smem_max = max_smem_optin() - 1024;  // static shared memory of the kernel
     // record slots as in plan_halo: per-pixel bulk copies, or one TMA tile copy
     const int al = 16 / eb;
     const int rec_box = ceil_to(Gc * 27 + al - 1, al);
     const int slot = rec_tma ? rec_box * eb : ceil_to(Gc * 27 * eb + 16, 128) + 16;
-    // first choice: a 256-pair tile small enough for two CTAs per SM (the
-    // phases of one CTA then overlap the other's); else the largest tile
-    static const int cands[][2] = {{8, 8}, {16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
-                                   {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
     const int per_sm = max_smem_per_sm();
-    for (int ci = 0; ci < (int)(sizeof(cands) / sizeof(cands[0])); ++ci) {
-        const int *c = cands[ci];
-        const int TH = c[0] < g.Ho ? c[0] : g.Ho;
-        const int TW = c[1] < pow2_ceil(g.Wo) ? c[1] : pow2_ceil(g.Wo);
-        if (TH * TW * Gc > 512) continue;
+    // tile (TH, TW), whole-image window or not; `first` demands a 256-pair
+    // tile that runs two CTAs per SM (the phases of one CTA then overlap the
+    // other's)
+    auto try_plan = [&](int TH, int TW, bool force_full, bool first) -> bool {
+        TH = TH < g.Ho ? TH : g.Ho;
+        TW = TW < pow2_ceil(g.Wo) ? TW : pow2_ceil(g.Wo);
+        const int pairs = TH * TW * Gc;
+        if (pairs * lpp > (lpp == 1 ? 512 : 256)) return false;
         int HR = (TH - 1) * g.sh + (g.kh - 1) * g.dh + 2 * R + 2;
         int HC = (TW - 1) * g.sw + (g.kw - 1) * g.dw + 2 * R + 2;
-        const int full_h = HR >= g.H + 2, full_w = HC >= g.W + 2;
+        const int full_h = force_full || HR >= g.H + 2, full_w = force_full || HC >= g.W + 2;
         if (full_h) HR = g.H + 2;
         if (full_w) HC = g.W + 2;
-        if (HR > 256 || HC > 256 || TH > 256 || TW > 256) continue;
+        if (HR > 256 || HC > 256 || TH > 256 || TW > 256) return false;
         const int halo = HR * HC * 128;
-        const int max_samples = TH * TW * Gc * 9;
+        const int max_samples = pairs * 9;
         const int ncells = (HR - 1) * (HC - 1) * Gc;
-        if (16 * max_samples > halo + TH * TW * slot || ncells > 65535) continue;
+        const int nown = HR * HC * Gc;
+        // sorted records (16 bytes each) and then the owner list (2 bytes
+        // per staged (pixel, group)) reuse the window and record slots
+        const int olist_off = ceil_to(16 * max_samples, 16);
+        if (olist_off + 2 * nown > halo + TH * TW * slot || ncells > 65535 || nown > 65535)
+            return false;
         BwdLayout L;
-        // window and record slots first: both are free after phase A and
-        // together hold the sorted 16-byte sample records
+        // window and record slots first: both are free after phase A
         L.slots_off = halo;
         L.go_off = ceil_to(L.slots_off + TH * TW * slot, 128);  // TMA destination
         L.gows_off = L.go_off + TH * TW * 128;
@@ -185,18 +193,29 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, HaloPlan *out, BwdLayout 
         L.bar_off = ceil_to(L.counts_off + (ncells + 1) * 4, 16);
         L.ncells = ncells;
         L.max_samples = max_samples;
+        L.olist_off = olist_off;
         L.hc_magic = (unsigned)(((1ull << 32) + HC - 1) / HC);
         L.smem_bytes = L.bar_off + 16;
-        if (L.smem_bytes > smem_max) continue;
-        const bool two = TH * TW * Gc <= 256 && 2 * (L.smem_bytes + 1024 + 1024) <= per_sm;
-        if (ci == 0 && !(two && TH * TW * Gc == 256)) continue;
-        L.threads = two ? 256 : 512;
+        if (L.smem_bytes > smem_max) return false;
+        const bool two = pairs * lpp <= 256 && 2 * (L.smem_bytes + 1024 + 1024) <= per_sm;
+        if (first && !(two && pairs * lpp == 256)) return false;
+        L.threads = (lpp == 1 && !two) ? 512 : 256;
+        L.lpp = lpp;
         *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                         (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
                         L.smem_bytes, rec_tma ? 1 : 0, rec_box};
         *lay = L;
         return true;
+    };
+    static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
+                                   {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    if (msdcn && lpp == 2) {  // wide groups: the whole image when it fits
+        for (auto &c : cands)
+            if (try_plan(c[0], c[1], true, false)) return true;
     }
+    if (try_plan(8, 8, false, true)) return true;
+    for (auto &c : cands)
+        if (try_plan(c[0], c[1], false, false)) return true;
     return false;
 }
 
@@ -284,7 +303,7 @@ dcn4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DCN4_OK : DCN
 bool use_mixed(const dcn4_desc *d) {
     if (d->dtype == DCN4_F32) return false;
     return d->math == DCN4_MATH_MIXED16 || d->math == DCN4_MATH_DEFAULT ||
-           d->math == DCN4_MATH_PACKED16;
+           d->math == DCN4_MATH_PACKED16 || d->math == DCN4_MATH_ACC16;
 }
 
 // forward multiply variant: 0 fp32 weights, 1 mixed-precision fma, 2 packed
@@ -426,6 +445,7 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
     L.gow = grad_offset_weight;
     L.acc = need > 0 ? static_cast<float *>(workspace) : static_cast<float *>(grad_input);
     L.mixed = use_mixed(desc);
+    L.acc16 = desc->math == DCN4_MATH_ACC16;
     L.stream = static_cast<cudaStream_t>(stream);
     L.msdcn = ms != nullptr;
     L.ms = ms;
@@ -446,12 +466,12 @@ dcn4_status run_backward(const dcn4_desc *desc, const void *input, const void *o
         };
         // records by one TMA tile copy when a pixel's G*27 values span a
         // multiple of 16 bytes, else by per-pixel bulk copies
-        L.halo = base && (g.G * 27 * eb) % 16 == 0 && plan_bwd(g, eb, true, &L.plan, &L.layout) &&
+        L.halo = base && (g.G * 27 * eb) % 16 == 0 && plan_bwd(g, eb, true, L.msdcn, &L.plan, &L.layout) &&
                  maps() &&
                  encode_map(L.dtype, offset_weight, g.N, g.Ho, g.Wo, g.G * 27, L.plan.rec_box,
                             L.plan.TW, L.plan.TH, &map_ow);
         if (!L.halo)
-            L.halo = base && plan_bwd(g, eb, false, &L.plan, &L.layout) && maps();
+            L.halo = base && plan_bwd(g, eb, false, L.msdcn, &L.plan, &L.layout) && maps();
         if (!L.halo && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     }
     // vectorised global-memory kernel: whole 16-byte vectors per group, a

@@ -40,6 +40,14 @@ bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
         const T *go = gout + (size_t)pix * g.C + (size_t)grp * g.D;
         const T *src = in + (size_t)n * img + (size_t)grp * g.D;
         float *dst = gin + (size_t)n * img + (size_t)grp * g.D;
+        const unsigned long long owb = ow_bytes_of(g, sizeof(T));
+        if (!DCN4_GMEM_OK(rec, g.K * 3 * sizeof(T), ow, owb) ||
+            !DCN4_GMEM_OK(grec, g.K * 3 * sizeof(T), gow, owb) ||
+            !DCN4_GMEM_OK(go, g.D * sizeof(T), gout, output_bytes(g, sizeof(T))) ||
+            (MS && !DCN4_GMEM_OK(static_cast<const T *>(ms.raw) + t, sizeof(T), ms.raw,
+                                 raw_bytes(g, sizeof(T)))) ||
+            (MS && !DCN4_GMEM_OK(graw + t, sizeof(T), graw, raw_bytes(g, sizeof(T)))))
+            continue;
         float s = 1.0f, gs = 0.0f;
         if (MS) s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[t]), ms.s0[grp], ms.smax);
         // DCNv3 weights: softmax over the taps; the gradients with respect to
@@ -84,6 +92,9 @@ bwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
                             const float wx = b ? lx : 1.0f - lx;
                             const float w = wy * wx;
                             const size_t at = ((size_t)yy * g.W + xx) * g.C;
+                            if (!DCN4_GMEM_OK(src + at, g.D * sizeof(T), in, input_bytes(g, sizeof(T))) ||
+                                !DCN4_GMEM_OK(dst + at, g.D * 4, gin, input_bytes(g, 4)))
+                                continue;
                             float dot = 0.0f;
                             for (int d = 0; d < g.D; ++d) {
                                 const float god = Elem<T>::to_f(go[d]);
@@ -124,7 +135,7 @@ __global__ void __launch_bounds__(256) zero_f32_kernel(float *__restrict__ p, lo
     const long long stride = (long long)gridDim.x * blockDim.x;
     const long long nv = ((reinterpret_cast<uintptr_t>(p) & 15) == 0) ? n / 4 : 0;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride)
-        reinterpret_cast<float4 *>(p)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (DCN4_CHECK(4 * i + 4 <= n)) reinterpret_cast<float4 *>(p)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (long long i = nv * 4 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
         p[i] = 0.0f;
 }
@@ -134,7 +145,7 @@ __global__ void __launch_bounds__(256) zero_bytes_kernel(unsigned char *__restri
     const long long stride = (long long)gridDim.x * blockDim.x;
     const long long nv = ((reinterpret_cast<uintptr_t>(p) & 15) == 0) ? bytes / 16 : 0;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride)
-        reinterpret_cast<uint4 *>(p)[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (DCN4_CHECK(16 * i + 16 <= bytes)) reinterpret_cast<uint4 *>(p)[i] = make_uint4(0u, 0u, 0u, 0u);
     for (long long i = nv * 16 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < bytes; i += stride)
         p[i] = 0;
 }
@@ -149,6 +160,7 @@ convert_f32_kernel(const float *__restrict__ src, T *__restrict__ dst, long long
     const long long nv = vec ? n / 4 : 0;
     if constexpr (sizeof(T) == 2) {
         for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride) {
+            if (!DCN4_CHECK(4 * i + 4 <= n)) continue;
             const float4 f = reinterpret_cast<const float4 *>(src)[i];
             uint2 o;
             o.x = VecMath<T>::pk(f.x, f.y);

@@ -24,8 +24,11 @@
 //   B      exclusive scan of the cell counts
 //   C      per (pixel, group): write each staged sample's record at
 //          offset[cell] + rank, over the window buffer (no longer needed)
+//   O      list the (staged pixel, group) owners that receive samples, sorted
+//          by their sample count (largest first), so the lanes of a warp
+//          take owners of about equal work in phase D
 //   E      copy the staged grad_offset_weight out with coalesced stores
-//   D      per (staged pixel, group): gather from its four cells, flush
+//   D      per listed owner: gather from its four cells, flush
 // Samples outside the staged window take a global path with atomics.
 #pragma once
 
@@ -196,7 +199,7 @@ __device__ __forceinline__ void block_exclusive_scan(int *counts, int n, int *wa
 // the offset is s * dir with s from scale_raw (ms.raw); grad_offset_weight
 // receives d/d dir and graw the gradient of scale_raw, as in
 // bwd_generic_kernel.
-template <typename T, int U, int NW, bool MIXED, bool DIRECT, bool MS>
+template <typename T, int U, int NW, bool MIXED, bool DIRECT, bool MS, int LPP>
 __global__ void __launch_bounds__(NW * 32, 512 / (NW * 32))
 bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const __grid_constant__ CUtensorMap tmap_go,
@@ -210,35 +213,45 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     constexpr int REC = 27 * EB;
     constexpr int PS = 128;
     constexpr int NT = NW * 32;
+    constexpr int NB = 64;  // owner-count buckets (counts >= NB - 1 share bucket 0)
+    constexpr int UL = U / LPP;  // 16-byte chunks of a group each of its LPP lanes owns
+    static_assert(UL * LPP == U && (LPP & (LPP - 1)) == 0, "LPP lanes split the U chunks");
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ int warp_sums[NW + 1];
+    __shared__ int obkt[NB + 1];
     unsigned char *halo = smem;
     unsigned char *gotile = smem + L.go_off;
     unsigned char *slots = smem + L.slots_off;
     T *gows = reinterpret_cast<T *>(smem + L.gows_off);
     int *counts = reinterpret_cast<int *>(smem + L.counts_off);
     const uint32_t bar = smem_u32(smem + L.bar_off);
-    // sorted sample records (lx, ly, m, byte offset of the source grad_out
-    // vector), written over the window and record slots after phase A
+    // sorted sample records, 16 bytes, written over the window and record
+    // slots after phase A: fp32 weights (lx, ly, byte offset of the source
+    // grad_out vector, m); with 16-bit weights (MIXED) the four corner
+    // weights m*w_c already rounded to T ({w00 | w01, w10 | w11}, then the
+    // offset), so the owner gather takes its corner's weight as it is
+    constexpr bool CR = MIXED && sizeof(T) == 2;
     float4 *srec = reinterpret_cast<float4 *>(smem);
-    // DIRECT (16-bit weights, 16-bit grad_input): 8-byte records instead,
-    // {bf16 (1-ly)*m | bf16 ly*m, fp16 lx | grad_out offset / 16}: the owner
-    // gather reads them at random addresses, where bytes are the cost
-    constexpr bool CR = DIRECT && sizeof(T) == 2;
-    uint2 *srec8 = reinterpret_cast<uint2 *>(smem);
+    uint4 *srecw = reinterpret_cast<uint4 *>(smem);
 
     const TileCoord tc = tile_coord(blockIdx.x, g, pl);
     const int D = g.D;
     const int RS = pl.HC * PS;
     const int lane = threadIdx.x & 31;
     const size_t img = (size_t)g.H * g.W * g.C;
+    // tensor extents (bounds of the checked build; unused otherwise)
+    const unsigned long long in_b = input_bytes(g, EB), raw_b = raw_bytes(g, EB);
+    const unsigned long long acc_b = input_bytes(g, 4);
+    (void)in_b, (void)raw_b, (void)acc_b;
 
     // ---------------- stage ----------------
     if (threadIdx.x == 0) {
         mbar_init(bar, NT);
         fence_barrier_init();
     }
-    for (int i = threadIdx.x; i <= L.ncells; i += NT) counts[i] = 0;
+    for (int i = threadIdx.x; i <= L.ncells; i += NT)
+        if (DCN4_SMEM_OK(counts + i, 4, smem)) counts[i] = 0;
+    for (int i = threadIdx.x; i <= NB; i += NT) obkt[i] = 0;
     __syncthreads();
     {
         uint32_t tx = 0;
@@ -258,6 +271,8 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             unsigned char *slot = slots + (size_t)p * pl.slot_bytes;
             for (unsigned long long q = e; q < end; q += EB) {
                 const unsigned char *sp = reinterpret_cast<const unsigned char *>(ow) + q;
+                if (!DCN4_GMEM_OK(sp, EB, ow, ow_bytes) || !DCN4_SMEM_OK(slot + (q - a), EB, smem))
+                    continue;
                 if (EB == 4)
                     *reinterpret_cast<unsigned *>(slot + (q - a)) = *reinterpret_cast<const unsigned *>(sp);
                 else
@@ -267,9 +282,11 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         }
         mbar_arrive_expect_tx(bar, tx);
         if (threadIdx.x == 0) {
-            tma_load_4d(smem_u32(halo), &tmap_in, tc.g0 * D, tc.hx0, tc.hy0, tc.n, bar);
-            tma_load_4d(smem_u32(gotile), &tmap_go, tc.g0 * D, tc.wo0, tc.ho0, tc.n, bar);
-            if (pl.rec_tma)
+            if (DCN4_SMEM_OK(halo, (unsigned)pl.HR * pl.HC * PS, smem))
+                tma_load_4d(smem_u32(halo), &tmap_in, tc.g0 * D, tc.hx0, tc.hy0, tc.n, bar);
+            if (DCN4_SMEM_OK(gotile, (unsigned)pl.TH * pl.TW * PS, smem))
+                tma_load_4d(smem_u32(gotile), &tmap_go, tc.g0 * D, tc.wo0, tc.ho0, tc.n, bar);
+            if (pl.rec_tma && DCN4_SMEM_OK(slots, (unsigned)pl.TH * pl.TW * pl.rec_box * EB, smem))
                 tma_load_4d(smem_u32(slots), &tmap_ow, (tc.g0 * 27) & ~(16 / EB - 1), tc.wo0, tc.ho0,
                             tc.n, bar);
         }
@@ -281,7 +298,9 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const unsigned long long end = start + (unsigned long long)pl.Gc * REC;
             const unsigned long long a = start & ~15ull;
             const unsigned long long e = min((end + 15ull) & ~15ull, ow_bytes & ~15ull);
-            if (e > a)
+            if (e > a && DCN4_SMEM_OK(slots + (size_t)p * pl.slot_bytes, (unsigned)(e - a), smem) &&
+                DCN4_GMEM_OK(reinterpret_cast<const unsigned char *>(ow) + a, (unsigned)(e - a), ow,
+                             ow_bytes))
                 bulk_load(smem_u32(slots + (size_t)p * pl.slot_bytes),
                           reinterpret_cast<const unsigned char *>(ow) + a, (uint32_t)(e - a), bar);
         }
@@ -303,7 +322,15 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     const int ncpg = (pl.HR - 1) * cells_w;  // cells per group; cell = gl * ncpg + y * cells_w + x
     unsigned kr[9];          // (cell << 16) | rank of each staged tap; 0xffffffff otherwise
     float v[27];
-    int f = threadIdx.x;
+    // LPP consecutive lanes share one (pixel, group) pair: lane `sub` owns
+    // its chunks sub*UL .. sub*UL + UL-1; their partial dot products are
+    // summed across the pair (pmask), and lane 0 of the pair alone counts,
+    // records and writes the pair's gradients
+    const int f = threadIdx.x / LPP;
+    const int sub = threadIdx.x & (LPP - 1);
+    const unsigned pmask = (LPP == 1) ? (1u << lane)
+                                      : (((1u << LPP) - 1u) << (lane & ~(LPP - 1)));
+    (void)pmask;
     const bool has_pair = f < npairs;
     int pix = 0, gl = 0, ho = 0, wo = 0;
     bool valid = false;
@@ -322,14 +349,27 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     }
 #pragma unroll
     for (int k = 0; k < 9; ++k) kr[k] = 0xffffffffu;
-    const int r = (U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1));
+    // chunk rotation: the 8 lanes of a shared-memory phase start at different
+    // 16-byte chunks of the 128-byte staged pixel (different bank quads)
+    const int r = (LPP == 1) ? ((U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1)))
+                             : ((lane / LPP) & (UL - 1));
+    auto chunk = [&](int c) -> int { return sub * UL + ((c + r) & (UL - 1)); };
     float s = 1.0f, gs = 0.0f;  // MSDCN scale of this (pixel, group), d/ds
+    const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
+    T *gout_rec = gows + ((size_t)pix * pl.Gc + gl) * 27;
+    // the reader takes whole words from the record's 4-byte boundary
+    if (valid && (!DCN4_SMEM_OK(reinterpret_cast<const unsigned char *>(
+                                    reinterpret_cast<uintptr_t>(rec) & ~uintptr_t(3)),
+                                EB == 4 ? 108u : 60u, smem) ||
+                  !DCN4_SMEM_OK(gout_rec, 27 * EB, smem)))
+        valid = false;
     if (valid) {
-        const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + start + gl * REC;
         RecordReader<T>::read(rec, v);
-        if (MS)
-            s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]),
+        if (MS) {
+            const T *rp = static_cast<const T *>(ms.raw) + gp * g.G + tc.g0 + gl;
+            s = msdcn_scale(DCN4_GMEM_OK(rp, EB, ms.raw, raw_b) ? Elem<T>::to_f(*rp) : 0.0f,
                             ms.s0[tc.g0 + gl], ms.smax);
+        }
         // DCNv3 weights: softmax of the logits over the taps; the logit
         // gradient w_k (gw_k - sum_j w_j gw_j) is formed after the taps from
         // the staged gw_k
@@ -350,23 +390,19 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             sn = SoftmaxNorm{mx, inv};
         }
         float dotw = 0.0f;
-        const unsigned char *row0[U], *row1[U];
-        // gof[c]: this pair's grad_out chunk (c + r) mod U, unpacked to fp32;
-        // gop[c] the same chunk packed
-        float gof[U][VE];
-        uint4 gop[U];
+        const unsigned char *row0[UL], *row1[UL];
+        // gop[c]: this lane's grad_out chunk chunk(c), packed
+        uint4 gop[UL];
 #pragma unroll
-        for (int c = 0; c < U; ++c) {
-            const int cc = (c + r) & (U - 1);
+        for (int c = 0; c < UL; ++c) {
+            const int cc = chunk(c);
             row0[c] = halo + (size_t)gl * D * EB + cc * 16;
             row1[c] = row0[c] + RS;
-            gop[c] = *reinterpret_cast<const uint4 *>(gotile + (size_t)pix * PS + gl * D * EB + cc * 16);
-            ChunkUnpack<T>::get(gop[c], gof[c]);
+            gop[c] = DCN4_LDS16(gotile + (size_t)pix * PS + gl * D * EB + cc * 16, smem);
         }
         const float fbx = (float)(wo * g.sw - g.pw), fby = (float)(ho * g.sh - g.ph);
         const float bxs[3] = {fbx, fbx + dwf, fbx + 2.0f * dwf};
         const float bys[3] = {fby, fby + dhf, fby + 2.0f * dhf};
-        T *gout_rec = gows + ((size_t)pix * pl.Gc + gl) * 27;
         unsigned esc = 0;
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
@@ -394,13 +430,20 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const int off = __float2int_rz(fmaf(y0f - hy_lo, RSf, (x0f - hx_lo) * PSf));
                 float d00 = 0.f, d01 = 0.f, d10 = 0.f, d11 = 0.f;
 #pragma unroll
-                for (int c = 0; c < U; ++c) {
+                for (int c = 0; c < UL; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
-                    d00 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a0), gop[c]);
-                    d01 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a0 + PS), gop[c]);
-                    d10 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a1), gop[c]);
-                    d11 += PackedDotM<T>::dot(*reinterpret_cast<const uint4 *>(a1 + PS), gop[c]);
+                    d00 += PackedDotM<T>::dot(DCN4_LDS16(a0, smem), gop[c]);
+                    d01 += PackedDotM<T>::dot(DCN4_LDS16(a0 + PS, smem), gop[c]);
+                    d10 += PackedDotM<T>::dot(DCN4_LDS16(a1, smem), gop[c]);
+                    d11 += PackedDotM<T>::dot(DCN4_LDS16(a1 + PS, smem), gop[c]);
+                }
+#pragma unroll
+                for (int o = 1; o < LPP; o <<= 1) {  // both lanes take this branch
+                    d00 += __shfl_xor_sync(pmask, d00, o);
+                    d01 += __shfl_xor_sync(pmask, d01, o);
+                    d10 += __shfl_xor_sync(pmask, d10, o);
+                    d11 += __shfl_xor_sync(pmask, d11, o);
                 }
                 gm = hy * (hx * d00 + lx * d01) + ly * (hx * d10 + lx * d11);
                 const float px = hy * (d01 - d00) + ly * (d11 - d10);  // d/d position
@@ -409,14 +452,18 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 gy = g.os * m * py;
                 if (MS) gs = fmaf(m * px, dsx, fmaf(m * py, dsy, gs));
                 const int cell = gl * ncpg + ((int)(y0f - hy_lo)) * cells_w + (int)(x0f - hx_lo);
-                const int rank = atomicAdd(&counts[cell], 1);
-                kr[k] = ((unsigned)cell << 16) | (unsigned)rank;
+                if (sub == 0 && DCN4_CHECK(cell >= 0 && cell < L.ncells)) {
+                    const int rank = atomicAdd(&counts[cell], 1);
+                    kr[k] = ((unsigned)cell << 16) | (unsigned)rank;
+                }
             } else {
                 esc |= 1u << k;
             }
-            gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
-            gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
-            gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            if (sub == 0) {
+                gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
+                gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
+                gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            }
             dotw = fmaf(m, gm, dotw);
         }
         // samples outside the staged window: global gathers, fp32 atomics
@@ -442,6 +489,23 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 const float x0f = floorf(x), y0f = floorf(y);
                 const float lx = x - x0f, ly = y - y0f;
                 const int x0 = (int)x0f, y0 = (int)y0f;
+                // the four dot products <grad_out, V_c> (this lane's chunks,
+                // then summed across the pair)
+                float dq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int yy = y0 + (q >> 1), xx = x0 + (q & 1);
+                    if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
+                    const uint4 *p =
+                        reinterpret_cast<const uint4 *>(gsrc + ((size_t)yy * g.W + xx) * g.C);
+#pragma unroll
+                    for (int c = 0; c < UL; ++c)
+                        dq[q] += PackedDotM<T>::dot(DCN4_LDG16(p + chunk(c), in, in_b), gop[c]);
+                }
+#pragma unroll
+                for (int o = 1; o < LPP; o <<= 1)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) dq[q] += __shfl_xor_sync(pmask, dq[q], o);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int a = q >> 1, b = q & 1;
@@ -449,27 +513,27 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                     if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
                     const float wy = a ? ly : 1.0f - ly, wx = b ? lx : 1.0f - lx;
                     const size_t at = ((size_t)yy * g.W + xx) * g.C;
-                    const uint4 *p = reinterpret_cast<const uint4 *>(gsrc + at);
-                    float dot = 0.f;
-#pragma unroll
-                    for (int c = 0; c < U; ++c) dot += DotF<T>::dot(__ldg(p + ((c + r) & (U - 1))), gof[c]);
+                    const float dot = dq[q];
                     gm = fmaf(wy * wx, dot, gm);
                     gx = fmaf(b ? wy : -wy, dot, gx);
                     gy = fmaf(a ? wx : -wx, dot, gy);
                     const float cw = m * wy * wx;
 #pragma unroll
-                    for (int c = 0; c < U; ++c) {
-                        const int cc = (c + r) & (U - 1);
-                        float go[VE];
+                    for (int c = 0; c < UL; ++c) {
+                        const int cc = chunk(c);
+                        float gf[VE], go[VE];
+                        ChunkUnpack<T>::get(gop[c], gf);
 #pragma unroll
-                        for (int d = 0; d < VE; ++d) go[d] = cw * gof[c][d];
+                        for (int d = 0; d < VE; ++d) go[d] = cw * gf[d];
                         if (DIRECT) {
-                            Red16<T>::add(gin + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D + at +
-                                              cc * VE,
-                                          VecMath<T>::pack(go));
-                        } else {
+                            T *gp16 = gin + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D + at + cc * VE;
+                            if (DCN4_GMEM_OK(gp16, 16, gin, in_b))
+                                Red16<T>::add(gp16, VecMath<T>::pack(go));
+                        } else if (DCN4_GMEM_OK(gdst + at + cc * VE, VE * 4, gacc, acc_b)) {
 #pragma unroll
-                            for (int d = 0; d < VE; ++d) atomicAdd(gdst + at + cc * VE + d, go[d]);
+                            for (int d = 0; d < VE; d += 4)
+                                red_add_v4(gdst + at + cc * VE + d, go[d], go[d + 1], go[d + 2],
+                                           go[d + 3]);
                         }
                     }
                 }
@@ -477,17 +541,22 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
                 gx *= g.os * m;
                 gy *= g.os * m;
             }
-            gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
-            gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
-            gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            if (sub == 0) {
+                gout_rec[3 * k] = Elem<T>::from_f(MS && gx != 0.f ? s * gx : gx);
+                gout_rec[3 * k + 1] = Elem<T>::from_f(MS && gy != 0.f ? s * gy : gy);
+                gout_rec[3 * k + 2] = Elem<T>::from_f(gm);
+            }
             dotw = fmaf(m, gm, dotw);
         }
-        if (MS) {
-            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]);
-            graw[gp * g.G + tc.g0 + gl] = Elem<T>::from_f(
-                gs == 0.0f ? 0.0f : gs * msdcn_scale_grad(raw, ms.s0[tc.g0 + gl], ms.smax));
+        if (MS && sub == 0) {
+            const T *rp = static_cast<const T *>(ms.raw) + gp * g.G + tc.g0 + gl;
+            const float raw = DCN4_GMEM_OK(rp, EB, ms.raw, raw_b) ? Elem<T>::to_f(*rp) : 0.0f;
+            T *gr = graw + gp * g.G + tc.g0 + gl;
+            if (DCN4_GMEM_OK(gr, EB, graw, raw_b))
+                *gr = Elem<T>::from_f(
+                    gs == 0.0f ? 0.0f : gs * msdcn_scale_grad(raw, ms.s0[tc.g0 + gl], ms.smax));
         }
-        if (g.softmax) {
+        if (g.softmax && sub == 0) {
 #pragma unroll
             for (int k = 0; k < 9; ++k)
                 gout_rec[3 * k + 2] =
@@ -500,7 +569,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     block_exclusive_scan<NW>(counts, L.ncells, warp_sums);
 
     // ---------------- C: sorted sample records (over the window) ----------------
-    if (valid) {
+    if (valid && sub == 0) {
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
             if (kr[k] == 0xffffffffu) continue;
@@ -518,17 +587,81 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const int pos = counts[cell] + rank;
             const float lx = x - floorf(x), ly = y - floorf(y), m = v[3 * k + 2];
             const unsigned goff = (unsigned)(pix * PS + gl * D * EB);
-            if (CR) {
-                const __nv_bfloat162 wy2 = __floats2bfloat162_rn(m - ly * m, ly * m);
-                srec8[pos] = make_uint2(*reinterpret_cast<const unsigned *>(&wy2),
-                                        (unsigned)__half_as_ushort(__float2half_rn(lx)) |
-                                            ((goff >> 4) << 16));
+            if (!DCN4_SMEM_OK(srec + pos, 16, smem)) continue;
+            if (CR) {  // the corner weights as in the forward, rounded once to T
+                const float mly = m * ly, mhy = m - mly;
+                const float w01 = mhy * lx, w11 = mly * lx;
+                srecw[pos] = make_uint4(pack2_bits<T>(mhy - w01, w01), pack2_bits<T>(mly - w11, w11),
+                                        goff, 0u);
             } else {
-                srec[pos] = make_float4(lx, ly, m, __uint_as_float(goff));
+                srec[pos] = make_float4(lx, ly, __uint_as_float(goff), m);
             }
         }
     }
     __syncthreads();
+
+    // ---------------- O: owners sorted by sample count ----------------
+    // Owner o = (staged pixel q, group ogl) receives the samples of the four
+    // cells it is a corner of: for corner row a (cell row qy - a) the cells
+    // (cy, qx - 1) (corner b = 1) and (cy, qx) (b = 0), one contiguous range
+    // of the sorted records split at es. Owners outside the image or without
+    // samples are left out; the rest are bucketed by count, largest first.
+    const int nown = pl.HR * pl.HC * pl.Gc;
+    unsigned short *olist = reinterpret_cast<unsigned short *>(smem + L.olist_off);
+    struct Ranges {
+        int e0[2], es[2], n[2];  // per corner row a: first entry, split, entry count
+    };
+    auto owner_ranges = [&](int o, Ranges &rg) -> bool {
+        const int ogl = o & (pl.Gc - 1);
+        const int q = o >> pl.lgGc;
+        const int qy = (int)__umulhi((unsigned)q, L.hc_magic), qx = q - qy * pl.HC;
+        const int iy = tc.hy0 + qy, ix = tc.hx0 + qx;
+        rg.n[0] = rg.n[1] = 0;
+        rg.e0[0] = rg.e0[1] = rg.es[0] = rg.es[1] = 0;
+        if (iy < 0 || iy >= g.H || ix < 0 || ix >= g.W) return false;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            const int cy = qy - a;
+            if (cy < 0 || cy >= pl.HR - 1) continue;
+            const int row = ogl * ncpg + cy * cells_w;
+            const int c0 = row + max(qx - 1, 0), c1 = row + min(qx, cells_w - 1) + 1;
+            if (!DCN4_CHECK(c0 >= 0 && c1 <= L.ncells)) continue;
+            rg.e0[a] = counts[c0];
+            rg.es[a] = counts[row + min(qx, cells_w)];
+            rg.n[a] = counts[c1] - rg.e0[a];
+        }
+        return true;
+    };
+    for (int o = threadIdx.x; o < nown; o += NT) {
+        Ranges rg;
+        if (!owner_ranges(o, rg)) continue;
+        const int n = rg.n[0] + rg.n[1];
+        if (n > 0) atomicAdd(&obkt[NB - 1 - min(n, NB - 1)], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {  // exclusive scan of the NB bucket sizes, 2 per lane
+        const int v0 = obkt[2 * lane], v1 = obkt[2 * lane + 1];
+        int incl = v0 + v1;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        const int excl = incl - v0 - v1;
+        obkt[2 * lane] = excl;
+        obkt[2 * lane + 1] = excl + v0;
+        if (lane == 31) obkt[NB] = incl;
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < nown; o += NT) {
+        Ranges rg;
+        if (!owner_ranges(o, rg)) continue;
+        const int n = rg.n[0] + rg.n[1];
+        if (n > 0) {
+            const int pos = atomicAdd(&obkt[NB - 1 - min(n, NB - 1)], 1);
+            if (DCN4_SMEM_OK(olist + pos, 2, smem)) olist[pos] = (unsigned short)o;
+        }
+    }
 
     // ---------------- E: grad_offset_weight out (one warp per pixel) ----------------
     {
@@ -540,6 +673,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const unsigned long long q = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
             unsigned char *dst = reinterpret_cast<unsigned char *>(gow + (q * g.G + tc.g0) * 27);
             const unsigned char *src = reinterpret_cast<const unsigned char *>(gows) + (size_t)p * span;
+            if (!DCN4_SMEM_OK(src, span, smem) || !DCN4_GMEM_OK(dst, span, gow, ow_bytes)) continue;
             // widest word that divides both addresses and the span
             const unsigned al = (unsigned)(reinterpret_cast<uintptr_t>(dst) |
                                            reinterpret_cast<uintptr_t>(src) | (uintptr_t)span);
@@ -556,74 +690,80 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         }
     }
 
-    // ---------------- D: gather per (staged pixel, group) and flush ----------------
-    const int nown = pl.HR * pl.HC * pl.Gc;
-    for (int o = threadIdx.x; o < nown; o += NT) {
+    // ---------------- D: gather per listed owner and flush ----------------
+    __syncthreads();  // owner list complete
+    const int nlist = obkt[NB];
+    // LPP consecutive lanes share an owner, each with its UL chunks (NT is a
+    // multiple of LPP, so a thread keeps its `sub`)
+    for (int t = threadIdx.x; t < nlist * LPP; t += NT) {
+        const int li = t / LPP;
+        if (!DCN4_SMEM_OK(olist + li, 2, smem)) continue;
+        const int o = olist[li];
         const int ogl = o & (pl.Gc - 1);
         const int q = o >> pl.lgGc;
         const int qy = (int)__umulhi((unsigned)q, L.hc_magic), qx = q - qy * pl.HC;
         const int iy = tc.hy0 + qy, ix = tc.hx0 + qx;
-        if (iy < 0 || iy >= g.H || ix < 0 || ix >= g.W) continue;
-        const int rr = (U <= 8) ? (((lane & 7) * U) >> 3) : (o & (U - 1));
-        float acc[U][VE];
+        Ranges rg;
+        owner_ranges(o, rg);
+        const int rr = (LPP == 1) ? ((U <= 8) ? (((lane & 7) * U) >> 3) : (o & (U - 1)))
+                                  : ((lane / LPP) & (UL - 1));
+        float acc[UL][VE];
 #pragma unroll
-        for (int c = 0; c < U; ++c)
+        for (int c = 0; c < UL; ++c)
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
-        // cells are numbered group-major, so for each corner row a the two
-        // cells (cy, qx - 1) (corner b = 1) and (cy, qx) (b = 0) are adjacent
-        // and their entries form one contiguous range split at es
-        bool any = false;
+        // one loop over the entries of both corner rows: the lanes of a warp
+        // then run for their total counts, not for the longer row of each
+        const int ntot = rg.n[0] + rg.n[1];
+        // entry j of the owner's list; the next record is loaded while the
+        // current one is used
+        auto entry = [&](int j) -> int {
+            return j >= rg.n[0] ? rg.e0[1] + (j - rg.n[0]) : rg.e0[0] + j;
+        };
+        uint4 nxt = make_uint4(0u, 0u, 0u, 0u);
+        if (ntot > 0 && DCN4_SMEM_OK(srecw + entry(0), 16, smem)) nxt = srecw[entry(0)];
+        for (int j = 0; j < ntot; ++j) {
+            const bool a = j >= rg.n[0];
+            const int e = entry(j);
+            const bool b1 = e < (a ? rg.es[1] : rg.es[0]);  // owner is the cell's x0 + 1 corner
+            const uint4 r = nxt;
+            if (j + 1 < ntot && DCN4_SMEM_OK(srecw + entry(j + 1), 16, smem)) nxt = srecw[entry(j + 1)];
+            const unsigned char *gsrc = gotile + r.z;
+            if (CR) {
+                const unsigned wd = a ? r.y : r.x;
+                const unsigned short cw = (unsigned short)(b1 ? (wd >> 16) : (wd & 0xffffu));
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-            const int cy = qy - a;
-            if (cy < 0 || cy >= pl.HR - 1) continue;
-            const int row = ogl * ncpg + cy * cells_w;
-            const int e0 = counts[row + max(qx - 1, 0)];
-            const int es = counts[row + min(qx, cells_w)];
-            const int e1 = counts[row + min(qx, cells_w - 1) + 1];
-            any |= e1 > e0;
-            for (int e = e0; e < e1; ++e) {
-                float w;
-                const unsigned char *gsrc;
-                if (CR) {
-                    const uint2 r = srec8[e];
-                    const float wy = __uint_as_float(a ? (r.x & 0xffff0000u) : (r.x << 16));
-                    const float lx = __half2float(__ushort_as_half((unsigned short)(r.y & 0xffffu)));
-                    w = wy * (e < es ? lx : 1.0f - lx);
-                    gsrc = gotile + ((r.y >> 16) << 4);
-                } else {
-                    const float4 rec4 = srec[e];
-                    const float wy = a ? rec4.y : 1.0f - rec4.y;
-                    const float wx = e < es ? rec4.x : 1.0f - rec4.x;
-                    w = wy * wx * rec4.z;
-                    gsrc = gotile + __float_as_uint(rec4.w);
+                for (int c = 0; c < UL; ++c) {
+                    const int cc = sub * UL + ((c + rr) & (UL - 1));
+                    VecMathMixed<T>::fma_bits(acc[c], DCN4_LDS16(gsrc + cc * 16, smem), cw);
                 }
+            } else {
+                const float lx = __uint_as_float(r.x), ly = __uint_as_float(r.y);
+                const float w = (a ? ly : 1.0f - ly) * (b1 ? lx : 1.0f - lx) * __uint_as_float(r.w);
 #pragma unroll
-                for (int c = 0; c < U; ++c) {
-                    const int cc = (c + rr) & (U - 1);
-                    const uint4 q = *reinterpret_cast<const uint4 *>(gsrc + cc * 16);
+                for (int c = 0; c < UL; ++c) {
+                    const int cc = sub * UL + ((c + rr) & (UL - 1));
+                    const uint4 qv = DCN4_LDS16(gsrc + cc * 16, smem);
                     if (MIXED)
-                        VecMathMixed<T>::fma(acc[c], q, w);
+                        VecMathMixed<T>::fma(acc[c], qv, w);
                     else
-                        VecMath<T>::fma(acc[c], q, w);
+                        VecMath<T>::fma(acc[c], qv, w);
                 }
             }
         }
-        if (any) {
-            const size_t at = (size_t)tc.n * img + ((size_t)iy * g.W + ix) * g.C +
-                              (size_t)(tc.g0 + ogl) * D;
+        const size_t at = (size_t)tc.n * img + ((size_t)iy * g.W + ix) * g.C +
+                          (size_t)(tc.g0 + ogl) * D;
 #pragma unroll
-            for (int c = 0; c < U; ++c) {
-                const int cc = (c + rr) & (U - 1);
-                if (DIRECT) {
+        for (int c = 0; c < UL; ++c) {
+            const int cc = sub * UL + ((c + rr) & (UL - 1));
+            if (DIRECT) {
+                if (DCN4_GMEM_OK(gin + at + cc * VE, 16, gin, in_b))
                     Red16<T>::add(gin + at + cc * VE, VecMath<T>::pack(acc[c]));
-                } else {
+            } else if (DCN4_GMEM_OK(gacc + at + cc * VE, VE * 4, gacc, acc_b)) {
 #pragma unroll
-                    for (int e = 0; e < VE; e += 4)
-                        red_add_v4(gacc + at + cc * VE + e, acc[c][e], acc[c][e + 1],
-                                   acc[c][e + 2], acc[c][e + 3]);
-                }
+                for (int e = 0; e < VE; e += 4)
+                    red_add_v4(gacc + at + cc * VE + e, acc[c][e], acc[c][e + 1],
+                               acc[c][e + 2], acc[c][e + 3]);
             }
         }
     }

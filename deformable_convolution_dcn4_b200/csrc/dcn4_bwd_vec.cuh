@@ -44,6 +44,11 @@ fwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
         const T *rec = ow + (size_t)pr * g.K * 3;
         const int c0 = grp * g.D + sub * VE;
         const T *src = in + (size_t)n * img + c0;
+        if (!DCN4_GMEM_OK(rec, g.K * 3 * sizeof(T), ow, ow_bytes_of(g, sizeof(T))) ||
+            !DCN4_GMEM_OK(out + (size_t)pix * g.C + c0, 16, out, output_bytes(g, sizeof(T))) ||
+            (MS && !DCN4_GMEM_OK(static_cast<const T *>(ms.raw) + pr, sizeof(T), ms.raw,
+                                 raw_bytes(g, sizeof(T)))))
+            continue;
         float s = 1.0f;
         if (MS) s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[pr]), ms.s0[grp], ms.smax);
         SoftmaxNorm sn{0.0f, 1.0f};
@@ -80,7 +85,8 @@ fwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                 for (int c = 0; c < 4; ++c) {
                     const int yy = y0 + (c >> 1), xx = x0 + (c & 1);
                     q[c] = (yy >= 0 && yy < g.H && xx >= 0 && xx < g.W)
-                               ? __ldg(reinterpret_cast<const uint4 *>(src + ((size_t)yy * g.W + xx) * g.C))
+                               ? DCN4_LDG16(src + ((size_t)yy * g.W + xx) * g.C, in,
+                                            input_bytes(g, sizeof(T)))
                                : make_uint4(0u, 0u, 0u, 0u);
                 }
                 const float mly = m * ly, mhy = m - mly;
@@ -121,17 +127,28 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
         const T *rec = ow + (size_t)pr * g.K * 3;
         T *grec = gow + (size_t)pr * g.K * 3;
         const int c0 = grp * g.D + sub * VE;  // this lane's first channel
+        const unsigned long long owb = ow_bytes_of(g, sizeof(T)), rawb = raw_bytes(g, sizeof(T));
+        const bool in_range =
+            !active || (DCN4_GMEM_OK(rec, g.K * 3 * sizeof(T), ow, owb) &&
+                        DCN4_GMEM_OK(grec, g.K * 3 * sizeof(T), gow, owb) &&
+                        (!MS || (DCN4_GMEM_OK(static_cast<const T *>(ms.raw) + pr, sizeof(T), ms.raw,
+                                              rawb) &&
+                                 DCN4_GMEM_OK(graw + pr, sizeof(T), graw, rawb))));
+        // a lane whose tensors fail the checked build's bounds takes no part
+        // (it still runs the shuffles, as an inactive lane)
+        const bool act = active && in_range;
         float gof[VE];
-        ChunkUnpack<T>::get(active ? __ldg(reinterpret_cast<const uint4 *>(gout + (size_t)pix * g.C + c0))
-                                   : make_uint4(0u, 0u, 0u, 0u),
+        ChunkUnpack<T>::get(act ? DCN4_LDG16(gout + (size_t)pix * g.C + c0, gout,
+                                             output_bytes(g, sizeof(T)))
+                                : make_uint4(0u, 0u, 0u, 0u),
                             gof);
         const T *src = in + (size_t)n * img + c0;
         float *dst = gin + (size_t)n * img + c0;
         float s = 1.0f, gs = 0.0f;
-        if (MS && active)
+        if (MS && act)
             s = msdcn_scale(Elem<T>::to_f(static_cast<const T *>(ms.raw)[pr]), ms.s0[grp], ms.smax);
         SoftmaxNorm sn{0.0f, 1.0f};
-        if (!MS && g.softmax && active) {
+        if (!MS && g.softmax && act) {
             float mx = -INFINITY, sum = 0.0f;
             for (int k = 0; k < g.K; ++k) mx = fmaxf(mx, Elem<T>::to_f(rec[3 * k + 2]));
             for (int k = 0; k < g.K; ++k) sum += expf(Elem<T>::to_f(rec[3 * k + 2]) - mx);
@@ -142,7 +159,7 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
             for (int j = 0; j < g.kw; ++j) {
                 const int k = i * g.kw + j;
                 float dx = 0.0f, dy = 0.0f, m = 0.0f;
-                if (active) {
+                if (act) {
                     dx = Elem<T>::to_f(rec[3 * k]);
                     dy = Elem<T>::to_f(rec[3 * k + 1]);
                     m = Elem<T>::to_f(rec[3 * k + 2]);
@@ -157,7 +174,7 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                     y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
                 }
                 const bool inside =
-                    active && x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H;
+                    act && x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H;
                 float lx = 0.0f, ly = 0.0f;
                 int x0 = 0, y0 = 0;
                 float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -171,9 +188,9 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                     for (int q = 0; q < 4; ++q) {
                         const int yy = y0 + (q >> 1), xx = x0 + (q & 1);
                         if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
-                        d[q] = DotF<T>::dot(
-                            __ldg(reinterpret_cast<const uint4 *>(src + ((size_t)yy * g.W + xx) * g.C)),
-                            gof);
+                        d[q] = DotF<T>::dot(DCN4_LDG16(src + ((size_t)yy * g.W + xx) * g.C, in,
+                                                       input_bytes(g, sizeof(T))),
+                                            gof);
                     }
                 }
 #pragma unroll
@@ -192,6 +209,7 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                         if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
                         const float w = m * ((q >> 1) ? ly : hy) * ((q & 1) ? lx : hx);
                         float *p = dst + ((size_t)yy * g.W + xx) * g.C;
+                        if (!DCN4_GMEM_OK(p, VE * 4, gin, input_bytes(g, 4))) continue;
 #pragma unroll
                         for (int e = 0; e < VE; e += 4)
                             red_add_v4(p + e, w * gof[e], w * gof[e + 1], w * gof[e + 2],
@@ -199,7 +217,7 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                     }
                 }
                 const float tx = g.os * m * gx, ty = g.os * m * gy;  // d/d offset
-                if (active && sub == 0) {
+                if (act && sub == 0) {
                     grec[3 * k] = Elem<T>::from_f(MS && tx != 0.0f ? s * tx : tx);
                     grec[3 * k + 1] = Elem<T>::from_f(MS && ty != 0.0f ? s * ty : ty);
                     grec[3 * k + 2] = Elem<T>::from_f(gm);
@@ -208,7 +226,7 @@ bwd_vec_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ ow,
                 if (MS) gs = fmaf(m * gx, dsx, fmaf(m * gy, dsy, gs));
             }
         }
-        if (active && sub == 0) {
+        if (act && sub == 0) {
             if (!MS && g.softmax) {
                 // logit gradient w_k (d/dw_k - sum_j w_j d/dw_j); d/dw_k was
                 // staged in grec (rounded to T)

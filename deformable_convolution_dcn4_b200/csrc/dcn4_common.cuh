@@ -106,9 +106,11 @@ struct BwdLayout {
     int bar_off;      // one mbarrier
     int ncells;       // (HR-1)*(HC-1)*Gc destination cells
     int max_samples;  // TH*TW*Gc*9; sorted sample records reuse the window
+    int olist_off;    // owner list (u16 per owner, sorted by sample count), after the records
     unsigned hc_magic;  // ceil(2^32 / HC): q / HC == __umulhi(q, hc_magic) for q < 2^16
     int smem_bytes;
     int threads;      // 256 (two CTAs per SM) or 512
+    int lpp;          // lanes per (pixel, group): 1, or 2 for 8 chunks (128-byte groups)
 };
 
 // Tiling of the shared-memory halo kernels (chosen on the host).
@@ -127,6 +129,20 @@ struct HaloPlan {
     int rec_tma;         // 1: records arrive by one TMA tile copy per tile (forward)
     int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)
 };
+
+// Byte sizes of the tensors of one call (bounds of the checked build).
+__host__ __device__ __forceinline__ unsigned long long input_bytes(const Geometry &g, int eb) {
+    return (unsigned long long)g.N * g.H * g.W * g.C * eb;
+}
+__host__ __device__ __forceinline__ unsigned long long output_bytes(const Geometry &g, int eb) {
+    return (unsigned long long)g.N * g.Ho * g.Wo * g.C * eb;
+}
+__host__ __device__ __forceinline__ unsigned long long ow_bytes_of(const Geometry &g, int eb) {
+    return (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * eb;
+}
+__host__ __device__ __forceinline__ unsigned long long raw_bytes(const Geometry &g, int eb) {
+    return (unsigned long long)g.N * g.Ho * g.Wo * g.G * eb;
+}
 
 // ---- element types -------------------------------------------------------
 template <typename T> struct Elem;
@@ -248,6 +264,7 @@ template <> struct VecMathMixed<float> {
     static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {
         VecMath<float>::fma(acc, v, w);
     }
+    static __device__ __forceinline__ void fma_bits(float *, const uint4 &, unsigned short) {}
 };
 __device__ __forceinline__ unsigned short bf16_bits(float w) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(w));
@@ -255,9 +272,24 @@ __device__ __forceinline__ unsigned short bf16_bits(float w) {
 __device__ __forceinline__ unsigned short f16_bits(float w) {
     return __half_as_ushort(__float2half_rn(w));
 }
+// Two fp32 values rounded to the 16-bit type T, packed (lo in bits 0-15).
+template <typename T> __device__ __forceinline__ unsigned pack2_bits(float lo, float hi);
+template <> __device__ __forceinline__ unsigned pack2_bits<__nv_bfloat16>(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const unsigned *>(&h);
+}
+template <> __device__ __forceinline__ unsigned pack2_bits<__half>(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const unsigned *>(&h);
+}
+template <> __device__ __forceinline__ unsigned pack2_bits<float>(float, float) { return 0u; }
 #define DCN4_MIXED_FMA(TY, CONV)                                                              \
     static __device__ __forceinline__ void fma(float *acc, const uint4 &v, float w) {        \
-        const unsigned short cw = CONV(w);                                                    \
+        fma_bits(acc, v, CONV(w));                                                            \
+    }                                                                                         \
+    /* the weight already rounded to the 16-bit type (its bits) */                            \
+    static __device__ __forceinline__ void fma_bits(float *acc, const uint4 &v,               \
+                                                    unsigned short cw) {                      \
         const unsigned wd[4] = {v.x, v.y, v.z, v.w};                                          \
         _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                       \
             const unsigned short lo = (unsigned short)(wd[e] & 0xffffu);                      \
@@ -313,6 +345,61 @@ template <> struct VecMathPacked<__half> { DCN4_PACKED_BLEND(__half2, __float2ha
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// ---- bounds-checked build (compiled with -DDCN4_CHECKED) -------------------
+// Every shared- and global-memory access of the kernels is guarded by
+// DCN4_SMEM_OK(p, n, base) (n bytes at p inside the CTA's dynamic shared
+// memory, which starts at base) or DCN4_GMEM_OK(p, n, base, bytes) (n bytes
+// at p inside the `bytes`-byte global tensor at base), or by DCN4_CHECK(cond)
+// for an index bound. In a checked build a
+// failing guard sets kErrInternal in the translation unit's device error word
+// (g_error_word, defined before the kernels are included) and the access is
+// skipped: a load yields zero, a store or atomic does nothing, a bulk copy is
+// not issued (the barrier it would complete then times out, which is also
+// reported). In a normal build both guards are the constant true and vanish.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+    uint32_t r;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ bool smem_in(const void *p, unsigned n, const void *base) {
+    const uint32_t a = smem_u32(p), b = smem_u32(base);
+    return a >= b && (unsigned long long)(a - b) + n <= dynamic_smem_bytes();
+}
+__device__ __forceinline__ bool smem_in_u32(uint32_t a, unsigned n, const void *base) {
+    const uint32_t b = smem_u32(base);
+    return a >= b && (unsigned long long)(a - b) + n <= dynamic_smem_bytes();
+}
+__device__ __forceinline__ bool gmem_in(const void *p, unsigned n, const void *base,
+                                        unsigned long long bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+    return a >= b && (unsigned long long)(a - b) + n <= bytes;
+}
+__device__ __forceinline__ bool flag_internal(unsigned int *word) {
+    atomicOr(word, kErrInternal);
+    return false;
+}
+#ifdef DCN4_CHECKED
+#define DCN4_CHECK(cond) ((cond) || ::dcn4::flag_internal(&g_error_word))
+#define DCN4_SMEM_OK(p, n, base) \
+    (::dcn4::smem_in((p), (n), (base)) || ::dcn4::flag_internal(&g_error_word))
+#define DCN4_SMEM_OK_U32(a, n, base) \
+    (::dcn4::smem_in_u32((a), (n), (base)) || ::dcn4::flag_internal(&g_error_word))
+#define DCN4_GMEM_OK(p, n, base, bytes) \
+    (::dcn4::gmem_in((p), (n), (base), (bytes)) || ::dcn4::flag_internal(&g_error_word))
+#else
+#define DCN4_CHECK(cond) true
+#define DCN4_SMEM_OK(p, n, base) true
+#define DCN4_SMEM_OK_U32(a, n, base) true
+#define DCN4_GMEM_OK(p, n, base, bytes) true
+#endif
+
+// Guarded 16-byte loads (zero when the guard fails).
+#define DCN4_LDS16(p, base) \
+    (DCN4_SMEM_OK((p), 16, (base)) ? *reinterpret_cast<const uint4 *>(p) : make_uint4(0u, 0u, 0u, 0u))
+#define DCN4_LDG16(p, base, bytes)                                                   \
+    (DCN4_GMEM_OK((p), 16, (base), (bytes)) ? __ldg(reinterpret_cast<const uint4 *>(p)) \
+                                            : make_uint4(0u, 0u, 0u, 0u))
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;

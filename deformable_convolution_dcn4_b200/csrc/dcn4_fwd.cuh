@@ -54,9 +54,12 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
         const int d0 = ch * CH;
         const int cnt = min(CH, g.D - d0);
         const T *rec = ow + (size_t)(pix * g.G + grp) * g.K * 3;
+        if (!DCN4_GMEM_OK(rec, g.K * 3 * sizeof(T), ow, ow_bytes_of(g, sizeof(T)))) continue;
         float s = 1.0f;
         if (MS) {
-            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[pix * g.G + grp]);
+            const T *rp = static_cast<const T *>(ms.raw) + pix * g.G + grp;
+            const float raw = DCN4_GMEM_OK(rp, sizeof(T), ms.raw, raw_bytes(g, sizeof(T)))
+                                  ? Elem<T>::to_f(*rp) : 0.0f;
             s = msdcn_scale(raw, ms.s0[grp], ms.smax);
         }
         SoftmaxNorm sn{0.0f, 1.0f};
@@ -97,6 +100,8 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
                         if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
                         const float w = (a ? ly : 1.0f - ly) * (b ? lx : 1.0f - lx) * m;
                         const T *p = src + ((size_t)yy * g.W + xx) * g.C;
+                        if (!DCN4_GMEM_OK(p, cnt * sizeof(T), in, input_bytes(g, sizeof(T))))
+                            continue;
 #pragma unroll
                         for (int d = 0; d < CH; ++d)
                             if (d < cnt) acc[d] = fmaf(w, Elem<T>::to_f(p[d]), acc[d]);
@@ -105,6 +110,7 @@ fwd_generic_kernel(Geometry g, const T *__restrict__ in, const T *__restrict__ o
             }
         }
         T *dst = out + (size_t)pix * g.C + (size_t)grp * g.D + d0;
+        if (!DCN4_GMEM_OK(dst, cnt * sizeof(T), out, output_bytes(g, sizeof(T)))) continue;
 #pragma unroll
         for (int d = 0; d < CH; ++d)
             if (d < cnt) dst[d] = Elem<T>::from_f(acc[d]);
@@ -218,7 +224,8 @@ template <typename T>
 __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometry &g,
                                               const HaloPlan &pl, const T *__restrict__ ow,
                                               unsigned long long ow_bytes, unsigned char *slots,
-                                              int nt, uint32_t bar) {
+                                              int nt, uint32_t bar, const unsigned char *sbase) {
+    (void)sbase;
     constexpr int EB = Elem<T>::kBytes;
     constexpr unsigned long long REC = 27ull * EB;
     const int lane = threadIdx.x & 31;
@@ -245,6 +252,8 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
         unsigned char *slot = slots + (size_t)p * pl.slot_bytes;
         for (unsigned long long q = e; q < end; q += EB) {
             const unsigned char *sp = reinterpret_cast<const unsigned char *>(ow) + q;
+            if (!DCN4_GMEM_OK(sp, EB, ow, ow_bytes) || !DCN4_SMEM_OK(slot + (q - a), EB, sbase))
+                continue;
             if (EB == 4)
                 *reinterpret_cast<unsigned *>(slot + (q - a)) = *reinterpret_cast<const unsigned *>(sp);
             else
@@ -265,6 +274,10 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
         const int p = base + lane;
         unsigned long long a, e, end;
         if (!mine || !span(p, a, e, end) || e <= a) continue;
+        if (!DCN4_SMEM_OK(slots + (size_t)p * pl.slot_bytes, (unsigned)(e - a), sbase) ||
+            !DCN4_GMEM_OK(reinterpret_cast<const unsigned char *>(ow) + a, (unsigned)(e - a), ow,
+                          ow_bytes))
+            continue;
         bulk_load(smem_u32(slots + (size_t)p * pl.slot_bytes),
                   reinterpret_cast<const unsigned char *>(ow) + a, (uint32_t)(e - a), bar);
     }
@@ -274,10 +287,14 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
 // (arrival count 1); called by one thread.
 __device__ __forceinline__ void stage_window(const TileCoord &tc, const CUtensorMap *tmap,
                                              const Geometry &g, const HaloPlan &pl, int eb,
-                                             unsigned char *halo, uint32_t bar) {
+                                             unsigned char *halo, uint32_t bar,
+                                             const unsigned char *sbase) {
+    (void)sbase;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(bar, (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb);
-    tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
+    const uint32_t wbytes = (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb;
+    mbar_arrive_expect_tx(bar, wbytes);
+    if (DCN4_SMEM_OK(halo, wbytes, sbase))
+        tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
 }
 
 // With pl.rec_tma: the tile's input window and its records ([TH][TW]
@@ -287,13 +304,17 @@ __device__ __forceinline__ void stage_window_records(const TileCoord &tc, const 
                                                      const CUtensorMap *tmap_ow, const Geometry &g,
                                                      const HaloPlan &pl, int eb,
                                                      unsigned char *halo, unsigned char *slots,
-                                                     uint32_t bar) {
+                                                     uint32_t bar, const unsigned char *sbase) {
+    (void)sbase;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(bar, (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb +
-                                   (uint32_t)pl.TH * pl.TW * pl.rec_box * eb);
-    tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
+    const uint32_t wbytes = (uint32_t)pl.HR * pl.HC * pl.Gc * g.D * eb;
+    const uint32_t rbytes = (uint32_t)pl.TH * pl.TW * pl.rec_box * eb;
+    mbar_arrive_expect_tx(bar, wbytes + rbytes);
+    if (DCN4_SMEM_OK(halo, wbytes, sbase))
+        tma_load_4d(smem_u32(halo), tmap, tc.g0 * g.D, tc.hx0, tc.hy0, tc.n, bar);
     const int x0 = (tc.g0 * 27) & ~(16 / eb - 1);
-    tma_load_4d(smem_u32(slots), tmap_ow, x0, tc.wo0, tc.ho0, tc.n, bar);
+    if (DCN4_SMEM_OK(slots, rbytes, sbase))
+        tma_load_4d(smem_u32(slots), tmap_ow, x0, tc.wo0, tc.ho0, tc.n, bar);
 }
 
 // The gathers of one staged tile: one thread per (pixel, group).
@@ -302,7 +323,9 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                                              const HaloPlan &pl, const T *__restrict__ in,
                                              T *__restrict__ out, const MsdcnParams &ms,
                                              const unsigned char *halo,
-                                             const unsigned char *slots, int ct, int nct) {
+                                             const unsigned char *slots, int ct, int nct,
+                                             const unsigned char *sbase) {
+    (void)sbase;
     constexpr int EB = Elem<T>::kBytes;
     constexpr int VE = Elem<T>::kPerVec;  // elements per 16-byte chunk
     constexpr int REC = 27 * EB;          // bytes of one (pixel, group) record
@@ -330,12 +353,19 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                                  ? ((unsigned)(tc.g0 * 27) & (unsigned)(16 / EB - 1)) * (unsigned)EB
                                  : ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + mis + gl * REC;
+        // the reader takes whole words from the record's 4-byte boundary
+        if (!DCN4_SMEM_OK(reinterpret_cast<const unsigned char *>(
+                              reinterpret_cast<uintptr_t>(rec) & ~uintptr_t(3)),
+                          EB == 4 ? 108u : 60u, sbase))
+            continue;
         float v[27];
         RecordReader<T>::read(rec, v);
         float s = 1.0f;
         const bool dil = MS && g.msd_dil;
         if (MS) {
-            const float raw = Elem<T>::to_f(static_cast<const T *>(ms.raw)[gp * g.G + tc.g0 + gl]);
+            const T *rp = static_cast<const T *>(ms.raw) + gp * g.G + tc.g0 + gl;
+            const float raw = DCN4_GMEM_OK(rp, EB, ms.raw, raw_bytes(g, EB)) ? Elem<T>::to_f(*rp)
+                                                                              : 0.0f;
             s = msdcn_scale(raw, ms.s0[tc.g0 + gl], ms.smax);
             if (!dil) {
 #pragma unroll
@@ -405,10 +435,10 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                 for (int c = 0; c < U; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
-                    const uint4 q00 = *reinterpret_cast<const uint4 *>(a0);
-                    const uint4 q01 = *reinterpret_cast<const uint4 *>(a0 + PS);
-                    const uint4 q10 = *reinterpret_cast<const uint4 *>(a1);
-                    const uint4 q11 = *reinterpret_cast<const uint4 *>(a1 + PS);
+                    const uint4 q00 = DCN4_LDS16(a0, sbase);
+                    const uint4 q01 = DCN4_LDS16(a0 + PS, sbase);
+                    const uint4 q10 = DCN4_LDS16(a1, sbase);
+                    const uint4 q11 = DCN4_LDS16(a1 + PS, sbase);
                     if (MV == 2) {
                         VecMathPacked<T>::blend4(acc[c], q00, q01, q10, q11, w00, w01, w10, w11);
                     } else if (MV == 1) {
@@ -434,7 +464,7 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
             const int k = __ffs(esc) - 1;
             esc &= esc - 1;
             float dx, dy, m;
-            record_tap<T>(rec, k, dx, dy, m);
+            record_tap<T>(rec, k, dx, dy, m);  // inside the record checked above
             if (!MS && g.softmax) m = sn.weight(m);
             const int i = k / 3, j = k - 3 * (k / 3);
             float x, y, dsx, dsy;
@@ -459,12 +489,15 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                 const uint4 *p = reinterpret_cast<const uint4 *>(gbase + ((size_t)yy * g.W + xx) * g.C);
 #pragma unroll
                 for (int c = 0; c < U; ++c)
-                    VecMath<T>::fma(acc[c], __ldg(p + ((c + r) & (U - 1))), wc[q]);
+                    VecMath<T>::fma(acc[c], DCN4_LDG16(p + ((c + r) & (U - 1)), in, input_bytes(g, EB)),
+                                    wc[q]);
             }
         }
         uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)(tc.g0 + gl) * D);
 #pragma unroll
-        for (int c = 0; c < U; ++c) dst[(c + r) & (U - 1)] = VecMath<T>::pack(acc[c]);
+        for (int c = 0; c < U; ++c)
+            if (DCN4_GMEM_OK(dst + ((c + r) & (U - 1)), 16, out, output_bytes(g, EB)))
+                dst[(c + r) & (U - 1)] = VecMath<T>::pack(acc[c]);
     }
 }
 
@@ -513,9 +546,9 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
             unsigned char *buf = smem + s * stage_bytes;
             if (pl.rec_tma)
                 stage_window_records(tc, &tmap, &tmap_ow, g, pl, Elem<T>::kBytes, buf,
-                                     buf + pl.halo_bytes, win0 + 8 * s);
+                                     buf + pl.halo_bytes, win0 + 8 * s, smem);
             else
-                stage_window(tc, &tmap, g, pl, Elem<T>::kBytes, buf, win0 + 8 * s);
+                stage_window(tc, &tmap, g, pl, Elem<T>::kBytes, buf, win0 + 8 * s, smem);
         }
         return true;
     };
@@ -525,7 +558,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
         if (pl.rec_tma) return;
         const int s = k % STAGES;
         stage_records<T>(tc, g, pl, ow, ow_bytes, smem + s * stage_bytes + pl.halo_bytes, NW * 32,
-                         myrec + 8 * s);
+                         myrec + 8 * s, smem);
     };
     auto records_ready = [&](int k) -> bool {
         return pl.rec_tma ||
@@ -572,7 +605,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
         }
         const unsigned char *buf = smem + s * stage_bytes;
         compute_tile<T, U, MS, MV>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
-                                      threadIdx.x, NW * 32);
+                                   threadIdx.x, NW * 32, smem);
         __syncwarp();
         if (leader) mbar_arrive(empty0 + 8 * s);
         if (STAGES == 1 && tn < ntiles) {

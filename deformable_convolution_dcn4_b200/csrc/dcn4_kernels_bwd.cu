@@ -39,18 +39,28 @@ cudaError_t launch_bwd_halo_m(const BwdLaunch &L, bool direct) {
     };
     if constexpr (sizeof(T) == 2) {
         if (U == 2 && nt == 256) {
-            if (direct) return run(bwd_halo_kernel<T, 2, 8, true, true, MS>);
-            return L.mixed ? run(bwd_halo_kernel<T, 2, 8, true, false, MS>)
-                           : run(bwd_halo_kernel<T, 2, 8, false, false, MS>);
+            if (direct) return run(bwd_halo_kernel<T, 2, 8, true, true, MS, 1>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 8, true, false, MS, 1>)
+                           : run(bwd_halo_kernel<T, 2, 8, false, false, MS, 1>);
         }
         if (U == 2) {
-            if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true, MS>);
-            return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false, MS>)
-                           : run(bwd_halo_kernel<T, 2, 16, false, false, MS>);
+            if (direct) return run(bwd_halo_kernel<T, 2, 16, true, true, MS, 1>);
+            return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false, MS, 1>)
+                           : run(bwd_halo_kernel<T, 2, 16, false, false, MS, 1>);
         }
+        // 64 channels: two lanes per (pixel, group), 256 threads
+        if (U == 8 && nt == 256 && L.layout.lpp == 2) {
+            if (direct) return run(bwd_halo_kernel<T, 8, 8, true, true, MS, 2>);
+            return L.mixed ? run(bwd_halo_kernel<T, 8, 8, true, false, MS, 2>)
+                           : run(bwd_halo_kernel<T, 8, 8, false, false, MS, 2>);
+        }
+    } else {
+        // fp32, 32 channels: two lanes per (pixel, group), 256 threads
+        if (U == 8 && nt == 256 && L.layout.lpp == 2)
+            return run(bwd_halo_kernel<T, 8, 8, false, false, MS, 2>);
     }
-    if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false, MS>);
-    if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false, MS>);
+    if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false, MS, 1>);
+    if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false, MS, 1>);
     return cudaErrorInvalidValue;
 }
 
@@ -92,9 +102,10 @@ template <typename T>
 cudaError_t launch_bwd_t(const BwdLaunch &L) {
     const Geometry &g = L.geo;
     const long long nin = (long long)g.N * g.H * g.W * g.C;
-    // 16-bit grad_input accumulates in place when the halo kernel runs in
-    // the 16-bit weight mode; otherwise through the fp32 workspace
-    const bool direct = L.halo && L.mixed && sizeof(T) == 2;
+    // 16-bit grad_input accumulates in place when the caller asked for
+    // 16-bit cross-CTA accumulation and the halo kernel runs; otherwise
+    // through the fp32 workspace (zeroed, then converted once)
+    const bool direct = L.halo && L.mixed && L.acc16 && sizeof(T) == 2;
     cudaError_t e;
     if (direct) {
         zero_bytes_kernel<<<grid_for(nin * (long long)sizeof(T) / 16 + 1, 256), 256, 0, L.stream>>>(

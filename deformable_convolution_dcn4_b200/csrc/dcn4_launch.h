@@ -40,6 +40,7 @@ struct BwdLaunch {
     bool halo;     // use the shared-memory halo kernel
     bool vec;      // otherwise the vectorised global-memory kernel (else scalar)
     bool mixed;    // 16-bit weights with mixed-precision fma (bf16/fp16 grad_input)
+    bool acc16;    // staged 16-bit kernel adds CTA partials into grad_input (no workspace)
     HaloPlan plan;
     BwdLayout layout;
     const CUtensorMap *tmap_in;

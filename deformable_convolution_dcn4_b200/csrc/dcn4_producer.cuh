@@ -172,17 +172,26 @@ __global__ void __launch_bounds__(NW * 32, 1)
     // resident operands: lin_w in core-matrix layout (rows >= J zero), the
     // depthwise taps and both biases in fp32
     constexpr int NT = NW * 32;
+    // tensor extents (bounds of the checked build; unused otherwise)
+    const unsigned long long x_b = (unsigned long long)pg.npix * C * 2;
+    const unsigned long long out_b = (unsigned long long)pg.npix * J * 2;
+    const unsigned long long lw_b = (unsigned long long)J * C * 2;
+    (void)x_b, (void)out_b, (void)lw_b;
     for (int i = tid; i < NP * Q; i += NT) {
         const int n = i / Q, q = i - n * Q;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < J) v = *reinterpret_cast<const uint4 *>(lin_w + (size_t)n * C + q * 8);
-        *reinterpret_cast<uint4 *>(smem + L.b_off + core_off(n, q, C)) = v;
+        if (n < J) v = DCN4_LDG16(lin_w + (size_t)n * C + q * 8, lin_w, lw_b);
+        if (DCN4_SMEM_OK(smem + L.b_off + core_off(n, q, C), 16, smem))
+            *reinterpret_cast<uint4 *>(smem + L.b_off + core_off(n, q, C)) = v;
     }
-    for (int i = tid; i < 9 * C; i += NT) dwf[i] = Elem<T>::to_f(dw_w[i]);
     T *dwt = reinterpret_cast<T *>(smem + L.dwt_off);  // dw_w [9][C] as stored
-    for (int i = tid; i < 9 * C; i += NT) dwt[i] = dw_w[i];
-    for (int i = tid; i < C; i += NT) dwf[9 * C + i] = Elem<T>::to_f(dw_b[i]);
-    for (int i = tid; i < NP; i += NT) linb[i] = i < J ? Elem<T>::to_f(lin_b[i]) : 0.f;
+    if (DCN4_SMEM_OK(dwf, 10 * C * 4, smem) && DCN4_SMEM_OK(dwt, 9 * C * 2, smem) &&
+        DCN4_SMEM_OK(linb, NP * 4, smem)) {
+        for (int i = tid; i < 9 * C; i += NT) dwf[i] = Elem<T>::to_f(dw_w[i]);
+        for (int i = tid; i < 9 * C; i += NT) dwt[i] = dw_w[i];
+        for (int i = tid; i < C; i += NT) dwf[9 * C + i] = Elem<T>::to_f(dw_b[i]);
+        for (int i = tid; i < NP; i += NT) linb[i] = i < J ? Elem<T>::to_f(lin_b[i]) : 0.f;
+    }
     int2 *rowyx = reinterpret_cast<int2 *>(smem + L.row_off);  // (y, x) of each tile row
 
     // pixel rows a tile reads: its 128 pixels and one image row plus one
@@ -199,7 +208,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
         x_range(tile, lo, hi);
         const uint32_t bytes = (uint32_t)((hi - lo) * C * 2);
         mbar_arrive_expect_tx(x_bar0 + 8 * b, bytes);
-        bulk_load(smem_u32(smem + L.x_off + b * L.x_bytes), x + lo * C, bytes, x_bar0 + 8 * b);
+        if (DCN4_CHECK(bytes <= (uint32_t)L.x_bytes) &&
+            DCN4_SMEM_OK(smem + L.x_off + b * L.x_bytes, bytes, smem) &&
+            DCN4_GMEM_OK(x + lo * C, bytes, x, x_b))
+            bulk_load(smem_u32(smem + L.x_off + b * L.x_bytes), x + lo * C, bytes, x_bar0 + 8 * b);
     };
     if (tid == 0) {
         mbar_init(mma_bar, 1);
@@ -247,7 +259,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
             bulk_wait_read();  // the previous tile's rows, staged in that buffer, have left
             issue_x(tile + gridDim.x, b ^ 1);
         }
-        if (tid < 128) {
+        if (tid < 128 && DCN4_SMEM_OK(rowyx + tid, 8, smem)) {
             const int p = (int)p0 + tid;  // the pixel count fits an int
             const int t = p / W;
             rowyx[tid] = make_int2(t % pg.H, p - t * W);
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
                         const int xj = xx + j - 1;
                         if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
                         const int idx = rel0 + r + (i - 1) * W + (j - 1);
-                        const uint4 v = *reinterpret_cast<const uint4 *>(xs + idx * (C * 2) + q * 16);
+                        const uint4 v = DCN4_LDS16(xs + idx * (C * 2) + q * 16, smem);
                         float fv[8];
                         unpack8<T>(v, fv);
                         const float4 *ww =
@@ -296,7 +308,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) acc[k] = 0.f;
             }
-            *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(r, q, C)) = pack8<T>(acc);
+            if (DCN4_SMEM_OK(smem + L.a_off + core_off(r, q, C), 16, smem))
+                *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(r, q, C)) = pack8<T>(acc);
         };
         if (ok) {
             if (diag) {
@@ -334,8 +347,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
                                 const int yy = yx[s2].x + i - 1, xj = yx[s2].y + j - 1;
                                 if (yy < 0 || yy >= pg.H || xj < 0 || xj >= W) continue;
                                 const int idx = rel0 + rr[s2] + (i - 1) * W + (j - 1);
-                                const uint4 v = *reinterpret_cast<const uint4 *>(
-                                    xs + idx * (C * 2) + q * 16);
+                                const uint4 v = DCN4_LDS16(xs + idx * (C * 2) + q * 16, smem);
                                 MixedFma8<T>::run(acc[s2], v, wv[i * 3 + j]);
                             }
                         }
@@ -346,8 +358,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
 #pragma unroll
                             for (int k = 0; k < 8; ++k) acc[s2][k] = 0.f;
                         }
-                        *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(rr[s2], q, C)) =
-                            pack8<T>(acc[s2]);
+                        if (DCN4_SMEM_OK(smem + L.a_off + core_off(rr[s2], q, C), 16, smem))
+                            *reinterpret_cast<uint4 *>(smem + L.a_off + core_off(rr[s2], q, C)) =
+                                pack8<T>(acc[s2]);
                     }
                 }
             } else {
@@ -393,17 +406,21 @@ __global__ void __launch_bounds__(NW * 32, 1)
                 float fo[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) fo[k] = v[8 * h + k] + linb[c0 + 8 * h + k];
-                if (staged)
-                    *reinterpret_cast<uint4 *>(srows + ((size_t)r * J + c0 + 8 * h) * 2) =
-                        pack8<T>(fo);
-                else
+                if (staged) {
+                    if (DCN4_SMEM_OK(srows + ((size_t)r * J + c0 + 8 * h) * 2, 16, smem))
+                        *reinterpret_cast<uint4 *>(srows + ((size_t)r * J + c0 + 8 * h) * 2) =
+                            pack8<T>(fo);
+                } else if (DCN4_GMEM_OK(orow + c0 + 8 * h, 16, out, out_b)) {
                     *reinterpret_cast<uint4 *>(orow + c0 + 8 * h) = pack8<T>(fo);
+                }
             }
         }
         tc_fence_before();
         if (staged) fence_async_smem();
         __syncthreads();
-        if (staged && tid == 0) bulk_store(out + p0 * J, smem_u32(srows), (uint32_t)rows * J * 2);
+        if (staged && tid == 0 && DCN4_SMEM_OK(srows, (unsigned)rows * J * 2, smem) &&
+            DCN4_GMEM_OK(out + p0 * J, (unsigned)rows * J * 2, out, out_b))
+            bulk_store(out + p0 * J, smem_u32(srows), (uint32_t)rows * J * 2);
     }
     if (tid == 0) bulk_wait_all();
 
@@ -473,8 +490,11 @@ __global__ void __launch_bounds__(256, 2)
                     for (int b = 0; b < 3; ++b) {
                         const int xs = xx + b - 1;
                         if (xs < 0 || xs >= pg.W) continue;
-                        v = fmaf(Elem<T>::to_f(dw_w[(a * 3 + b) * C + c]),
-                                 Elem<T>::to_f(x[((size_t)(ny + a - 1) * pg.W + xs) * C + c]), v);
+                        const T *xp = x + ((size_t)(ny + a - 1) * pg.W + xs) * C + c;
+                        if (!DCN4_GMEM_OK(xp, sizeof(T), x,
+                                          (unsigned long long)pg.npix * C * sizeof(T)))
+                            continue;
+                        v = fmaf(Elem<T>::to_f(dw_w[(a * 3 + b) * C + c]), Elem<T>::to_f(*xp), v);
                     }
                 }
             }
@@ -508,7 +528,9 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
             const int j = j0 + 8 * tx + b;
-            if (j < J) out[(p0 + r) * J + j] = Elem<T>::from_f(acc[a][b] + Elem<T>::to_f(lin_b[j]));
+            if (j < J && DCN4_GMEM_OK(out + (p0 + r) * J + j, sizeof(T), out,
+                                      (unsigned long long)pg.npix * J * sizeof(T)))
+                out[(p0 + r) * J + j] = Elem<T>::from_f(acc[a][b] + Elem<T>::to_f(lin_b[j]));
         }
     }
 }

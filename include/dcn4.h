@@ -103,14 +103,24 @@ typedef enum {
  *            twice the error of MIXED16 (rms relative ~3e-3 for bf16,
  *            ~4e-4 for fp16, against ~1.7e-3 / ~2e-4 for the rounding of
  *            the output itself), for fewer instructions per tap.
+ *   ACC16    bf16/fp16 backward only (the forward runs as MIXED16): as
+ *            MIXED16, but the staged kernel adds each CTA's fp32 partial sum
+ *            of grad_input straight into the 16-bit grad_input with packed
+ *            16-bit atomic adds (one rounding per contributing CTA, up to
+ *            ~6 per element, plus one per sample that leaves the staged
+ *            window), skipping the fp32 workspace and its zero and convert
+ *            passes. Faster, not fp32-accumulated across CTAs.
  *   DEFAULT  MIXED16 for bf16/fp16 data, F32 for fp32 data.
+ * In every mode except ACC16, grad_input is accumulated in fp32 across the
+ * whole call (the workspace for bf16/fp16) and rounded once at the end.
  * Dot products of two stored tensors (the backward's <grad_out, input>) are
  * exact products of the stored values summed in fp32 in every mode. */
 typedef enum {
     DCN4_MATH_DEFAULT = 0,
     DCN4_MATH_F32 = 1,
     DCN4_MATH_MIXED16 = 2,
-    DCN4_MATH_PACKED16 = 3
+    DCN4_MATH_PACKED16 = 3,
+    DCN4_MATH_ACC16 = 4
 } dcn4_math;
 
 /* Aggregation weights ("(论文速读）DCNv4：高效可变形卷积算子", "移除Softmax归一化"):
@@ -161,9 +171,10 @@ DCN4_API dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input,
                          const void *offset_weight, void *output, void *stream);
 
 /* Bytes of device workspace dcn4_backward needs for `desc`: an fp32 copy of
- * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. (In the default
- * math mode the staged bf16/fp16 kernel accumulates in grad_input itself and
- * leaves the workspace unused; the generic kernel and DCN4_MATH_F32 use it.) */
+ * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. (Under
+ * DCN4_MATH_ACC16 the staged bf16/fp16 kernel accumulates in grad_input
+ * itself and leaves the workspace unused; every other bf16/fp16 call uses
+ * it.) */
 DCN4_API dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes);
 
 /* DCNv4 backward: the derivative of the forward (the pages only say that
@@ -175,10 +186,11 @@ DCN4_API dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t 
  * At an integer sample position the derivative is that of the cell floor()
  * selects. `workspace` (>= dcn4_backward_workspace_size bytes, 16-byte
  * aligned, device memory owned by the caller) may be NULL when that size is 0.
- * grad_input sums partial results with atomic adds, so its last bits may vary
- * from run to run: in fp32 (the workspace) for fp32 data and DCN4_MATH_F32;
- * in the default mode the staged bf16/fp16 kernel sums each CTA's
- * contribution in fp32 and adds it to grad_input with one 16-bit rounding. */
+ * grad_input sums partial results with fp32 atomic adds (in the workspace for
+ * bf16/fp16, rounded once to the element type at the end), so its last bits
+ * may vary from run to run; under DCN4_MATH_ACC16 the staged bf16/fp16
+ * kernel adds each CTA's fp32 partial sum to grad_input with one 16-bit
+ * rounding instead. */
 DCN4_API dcn4_status dcn4_backward(const dcn4_desc *desc, const void *input,
                           const void *offset_weight, const void *grad_out,
                           void *grad_input, void *grad_offset_weight,

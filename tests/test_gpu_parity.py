@@ -246,10 +246,13 @@ BWD = {
 }
 
 
+@pytest.mark.parametrize("math", ["default", "acc16"])
 @pytest.mark.parametrize("name", sorted(BWD))
-def test_backward(orc, name):
+def test_backward(orc, name, math):
+    """Default: fp32 accumulation of grad_input across CTAs; acc16: each CTA's
+    fp32 partial sum added to the 16-bit grad_input directly."""
     wl = BWD[name]
-    e_in, e_ow = backward_case(orc, wl)
+    e_in, e_ow = backward_case(orc, wl, math=math)
     tol = TOL[wl.dtype]
     assert e_in <= tol and e_ow <= tol, f"{name}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
 
@@ -299,21 +302,24 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(orc):
 
 
 def test_launch_counter_counts_each_kernel():
-    """Forward on the halo path is one kernel; the 16-bit backward in the
-    default math mode is two (zero grad_input, halo kernel); with fp32
-    accumulation it is three (zero workspace, halo kernel, convert)."""
+    """Forward on the halo path is one kernel; the 16-bit backward with 16-bit
+    cross-CTA accumulation (acc16) is two (zero grad_input, halo kernel);
+    with fp32 accumulation (the default, and f32) it is three (zero
+    workspace, halo kernel, convert)."""
     wl = REDUCED["internimage_bf16"]
     data = make_inputs(wl, out_hw(wl), with_grad=True)
     x, ow, go = (data[k].cuda() for k in ("input", "offset_weight", "grad_out"))
     n0 = B.dcn4_kernel_launches()
     B.dcn4_forward(x, ow, group=wl.G, algo="halo")
     n1 = B.dcn4_kernel_launches()
-    B.dcn4_backward(x, ow, go, group=wl.G, algo="halo")
+    B.dcn4_backward(x, ow, go, group=wl.G, algo="halo", math="acc16")
     n2 = B.dcn4_kernel_launches()
     B.dcn4_backward(x, ow, go, group=wl.G, algo="halo", math="f32")
     n3 = B.dcn4_kernel_launches()
+    B.dcn4_backward(x, ow, go, group=wl.G, algo="halo")
+    n4 = B.dcn4_kernel_launches()
     torch.cuda.synchronize()
-    assert (n1 - n0, n2 - n1, n3 - n2) == (1, 2, 3)
+    assert (n1 - n0, n2 - n1, n3 - n2, n4 - n3) == (1, 2, 3, 3)
 
 
 MSDCN_BWD = {
@@ -330,7 +336,7 @@ MSDCN_BWD = {
 
 
 @pytest.mark.parametrize("name", sorted(MSDCN_BWD))
-@pytest.mark.parametrize("math", ["default", "f32"])
+@pytest.mark.parametrize("math", ["default", "f32", "acc16"])
 def test_msdcn_backward(orc, name, math):
     wl = MSDCN_BWD[name]
     errs = msdcn_backward_case(orc, wl, math=math)
@@ -344,14 +350,42 @@ def test_msdcn_backward_full_size_sampled(orc):
     assert all(e <= TOL["bf16"] for e in errs), errs
 
 
-def test_msdcn_backward_halo_request_is_unsupported():
-    """D64 bf16 (8 vectors per group) is beyond the staged backward kernel."""
-    wl = MSDCN_BWD["flowdcn_msdcn_bf16"]
-    data = make_inputs(wl, out_hw(wl), with_grad=True)
-    with pytest.raises(B.Dcn4Error) as e:
-        B.msdcn_backward(data["input"].cuda(), data["dir_weight"].cuda(), data["scale_raw"].cuda(),
-                         data["s0"], wl.smax, data["grad_out"].cuda(), group=wl.G, algo="halo")
-    assert e.value.code == 2
+# 64-channel groups (8 16-byte vectors): the staged backward with two lanes
+# per (pixel, group), the whole image as its window for MSDCN (FlowDCN token
+# grid) and a 4-pixel margin for DCNv4; forced, against the oracle, in all
+# three accumulation modes, plus the vectorised kernel on the same shapes
+D64_STAGED = {
+    "flowdcn_msdcn_bf16": MSDCN_BWD["flowdcn_msdcn_bf16"],
+    "flowdcn_msdcn_f16_ragged": W["flowdcn_msdcn_bf16"].replace(name="fd16", N=2, H=21, W=19,
+                                                                C=256, G=4, dtype="f16"),
+    "msdcn_d32_f32": W["internimage_f32"].replace(name="msd32f", N=1, H=18, W=14, C=64, G=2,
+                                                  kind="msdcn", offset_dist=("normal", 1.0),
+                                                  smax=4.0),
+    "dcn4_d64_bf16": W["internimage_bf16"].replace(name="d64s", N=2, H=23, W=29, C=128, G=2),
+}
+
+
+@pytest.mark.parametrize("math", ["default", "f32", "acc16"])
+@pytest.mark.parametrize("name", sorted(D64_STAGED))
+def test_backward_staged_wide_groups(orc, name, math):
+    wl = D64_STAGED[name]
+    if wl.dtype == "f32" and math == "acc16":
+        pytest.skip("16-bit accumulation applies to bf16/fp16 only")
+    tol = TOL[wl.dtype]
+    if wl.kind == "msdcn":
+        errs = msdcn_backward_case(orc, wl, algo="halo", math=math)
+        assert max(errs) <= tol, f"{name}/{math}: {errs}"
+    else:
+        e_in, e_ow = backward_case(orc, wl, algo="halo", math=math)
+        assert e_in <= tol and e_ow <= tol, f"{name}/{math}: {e_in:.3e} {e_ow:.3e}"
+
+
+def test_backward_staged_wide_groups_full_size_sampled(orc):
+    """The FlowDCN shape (N32 32x32 C1152 G18 bf16) on the staged kernel:
+    images 0 and 31 against the oracle."""
+    wl = W["flowdcn_msdcn_bf16"]
+    errs = msdcn_backward_case(orc, wl, algo="halo", images=[0, 31])
+    assert all(e <= TOL["bf16"] for e in errs), errs
 
 
 # DCNv3 compatibility (softmax over the taps) and the MSDCN scale-as-dilation
@@ -418,9 +452,11 @@ def test_msdcn_rejects_softmax():
     assert rc == 2
 
 
-# Shapes the shared-memory backward does not take: AUTO runs the vectorised
-# global-memory kernel (whole 16-byte vectors per group) or, for group widths
-# that are not, the scalar one; "generic" forces the scalar kernel.
+# Shapes on the global-memory backward kernels: AUTO runs the staged kernel
+# where it applies (d64_bf16, softmax_d64_bf16: 64-channel groups), else the
+# vectorised global-memory kernel (whole 16-byte vectors per group) or, for
+# group widths that are not, the scalar one; "generic" forces the scalar
+# kernel, "vector" the vectorised one.
 BWD_VEC = {
     "d64_bf16": W["flowdcn_msdcn_bf16"].replace(name="d64", kind="dcn4", N=1, H=12, W=14,
                                                 C=256, G=4, offset_dist=("normal", 2.0)),
@@ -437,9 +473,12 @@ BWD_VEC = {
 
 
 @pytest.mark.parametrize("name", sorted(BWD_VEC))
-@pytest.mark.parametrize("algo", ["auto", "generic"])
+@pytest.mark.parametrize("algo", ["auto", "generic", "vector"])
 def test_backward_global_kernels(orc, name, algo):
     wl = BWD_VEC[name]
+    vb = wl.D * (4 if wl.dtype == "f32" else 2)
+    if algo == "vector" and (vb % 16 or vb > 256 or (vb // 16) & (vb // 16 - 1)):
+        pytest.skip("group channels are not whole 16-byte vectors")
     e_in, e_ow = backward_case(orc, wl, algo)
     tol = TOL[wl.dtype]
     assert e_in <= tol and e_ow <= tol, f"{name}/{algo}: grad_input {e_in:.3e} grad_ow {e_ow:.3e}"
