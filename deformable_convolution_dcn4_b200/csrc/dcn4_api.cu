@@ -179,10 +179,11 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
         const int max_samples = pairs * 9;
         const int ncells = (HR - 1) * (HC - 1) * Gc;
         const int nown = HR * HC * Gc;
-        // sorted records (16 bytes each) and then the owner list (2 bytes
-        // per staged (pixel, group)) reuse the window and record slots
+        // sorted samples (16 bytes each), then the owner list and the owners'
+        // ranks (2 bytes each per staged (pixel, group)) and their counts
+        // (1 byte each) reuse the window and record slots
         const int olist_off = ceil_to(16 * max_samples, 16);
-        if (olist_off + 2 * nown > halo + TH * TW * slot || ncells > 65535 || nown > 65535)
+        if (olist_off + 5 * nown > halo + TH * TW * slot || ncells > 65535 || nown > 65535)
             return false;
         BwdLayout L;
         // window and record slots first: both are free after phase A

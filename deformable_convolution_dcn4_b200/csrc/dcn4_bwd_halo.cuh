@@ -218,21 +218,19 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     static_assert(UL * LPP == U && (LPP & (LPP - 1)) == 0, "LPP lanes split the U chunks");
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ int warp_sums[NW + 1];
-    __shared__ int obkt[NB + 1];
+    __shared__ int obkt[4][NB];  // per group: owners per count bucket, then bucket offsets
+    __shared__ int onon[4];      // per group: owners with samples
     unsigned char *halo = smem;
     unsigned char *gotile = smem + L.go_off;
     unsigned char *slots = smem + L.slots_off;
     T *gows = reinterpret_cast<T *>(smem + L.gows_off);
     int *counts = reinterpret_cast<int *>(smem + L.counts_off);
     const uint32_t bar = smem_u32(smem + L.bar_off);
-    // sorted sample records, 16 bytes, written over the window and record
-    // slots after phase A: fp32 weights (lx, ly, byte offset of the source
-    // grad_out vector, m); with 16-bit weights (MIXED) the four corner
-    // weights m*w_c already rounded to T ({w00 | w01, w10 | w11}, then the
-    // offset), so the owner gather takes its corner's weight as it is
+    // sorted samples, written over the window and record slots after phase
+    // A (16 bytes per sample either way; see phase C): per-corner entry
+    // lists with 16-bit weights (CR), else fp32 records
     constexpr bool CR = MIXED && sizeof(T) == 2;
     float4 *srec = reinterpret_cast<float4 *>(smem);
-    uint4 *srecw = reinterpret_cast<uint4 *>(smem);
 
     const TileCoord tc = tile_coord(blockIdx.x, g, pl);
     const int D = g.D;
@@ -251,7 +249,7 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     }
     for (int i = threadIdx.x; i <= L.ncells; i += NT)
         if (DCN4_SMEM_OK(counts + i, 4, smem)) counts[i] = 0;
-    for (int i = threadIdx.x; i <= NB; i += NT) obkt[i] = 0;
+    for (int i = threadIdx.x; i < 4 * NB; i += NT) obkt[i / NB][i % NB] = 0;
     __syncthreads();
     {
         uint32_t tx = 0;
@@ -568,7 +566,14 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     // ---------------- B: cell offsets ----------------
     block_exclusive_scan<NW>(counts, L.ncells, warp_sums);
 
-    // ---------------- C: sorted sample records (over the window) ----------------
+    // ---------------- C: sorted sample entries (over the window) ----------------
+    // CR (16-bit weights): four lists, one per corner (a, b) of the cells,
+    // each in cell order; entry = weight m*w_ab rounded to T (bits 0-15) |
+    // byte offset / 16 of the sample's grad_out vector (bits 16-31). An owner
+    // then reads its own corner's entries straight. Otherwise one 16-byte
+    // record per sample: (lx, ly, grad_out offset, m), fp32.
+    const int ML = L.max_samples;  // entries per corner list
+    unsigned *lists = reinterpret_cast<unsigned *>(smem);
     if (valid && sub == 0) {
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
@@ -587,13 +592,18 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             const int pos = counts[cell] + rank;
             const float lx = x - floorf(x), ly = y - floorf(y), m = v[3 * k + 2];
             const unsigned goff = (unsigned)(pix * PS + gl * D * EB);
-            if (!DCN4_SMEM_OK(srec + pos, 16, smem)) continue;
             if (CR) {  // the corner weights as in the forward, rounded once to T
+                if (!DCN4_CHECK(pos >= 0 && pos < ML)) continue;
                 const float mly = m * ly, mhy = m - mly;
                 const float w01 = mhy * lx, w11 = mly * lx;
-                srecw[pos] = make_uint4(pack2_bits<T>(mhy - w01, w01), pack2_bits<T>(mly - w11, w11),
-                                        goff, 0u);
+                const unsigned top = pack2_bits<T>(mhy - w01, w01), bot = pack2_bits<T>(mly - w11, w11);
+                const unsigned hi = (goff >> 4) << 16;
+                lists[pos] = (top & 0xffffu) | hi;
+                lists[ML + pos] = (top >> 16) | hi;
+                lists[2 * ML + pos] = (bot & 0xffffu) | hi;
+                lists[3 * ML + pos] = (bot >> 16) | hi;
             } else {
+                if (!DCN4_SMEM_OK(srec + pos, 16, smem)) continue;
                 srec[pos] = make_float4(lx, ly, __uint_as_float(goff), m);
             }
         }
@@ -601,46 +611,59 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
     __syncthreads();
 
     // ---------------- O: owners sorted by sample count ----------------
-    // Owner o = (staged pixel q, group ogl) receives the samples of the four
-    // cells it is a corner of: for corner row a (cell row qy - a) the cells
-    // (cy, qx - 1) (corner b = 1) and (cy, qx) (b = 0), one contiguous range
-    // of the sorted records split at es. Owners outside the image or without
-    // samples are left out; the rest are bucketed by count, largest first.
+    // Owner o = (staged pixel q = (qy, qx), group ogl) receives the samples
+    // of the four cells it is a corner of: corner (a, b) of cell
+    // (qy - a, qx - b). Within each group the owners are ordered by their
+    // sample count, largest first (counting sort over NB buckets; owners
+    // outside the image count 0), and the groups are interleaved: list slot
+    // Gc * k + g holds group g's k-th owner. The lanes of a warp then take
+    // owners of about equal work, and consecutive lanes keep consecutive
+    // groups, so the 16-byte grad_out reads of phase D stay free of bank
+    // conflicts (the lanes of a phase hit different 16-byte bank quads).
     const int nown = pl.HR * pl.HC * pl.Gc;
+    const int nq = pl.HR * pl.HC;  // owners per group
     unsigned short *olist = reinterpret_cast<unsigned short *>(smem + L.olist_off);
-    struct Ranges {
-        int e0[2], es[2], n[2];  // per corner row a: first entry, split, entry count
+    unsigned short *orank = olist + nown;  // owner's rank in its (group, bucket)
+    unsigned char *ocnt = smem + L.olist_off + 4 * nown;  // count per owner (<= 255 kept)
+    struct Corners {
+        int beg[4], n[4];  // corner ab: first entry (cell offset), entry count
     };
-    auto owner_ranges = [&](int o, Ranges &rg) -> bool {
+    auto owner_corners = [&](int o, Corners &cr) -> bool {
         const int ogl = o & (pl.Gc - 1);
         const int q = o >> pl.lgGc;
         const int qy = (int)__umulhi((unsigned)q, L.hc_magic), qx = q - qy * pl.HC;
         const int iy = tc.hy0 + qy, ix = tc.hx0 + qx;
-        rg.n[0] = rg.n[1] = 0;
-        rg.e0[0] = rg.e0[1] = rg.es[0] = rg.es[1] = 0;
+#pragma unroll
+        for (int ab = 0; ab < 4; ++ab) cr.beg[ab] = cr.n[ab] = 0;
         if (iy < 0 || iy >= g.H || ix < 0 || ix >= g.W) return false;
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-            const int cy = qy - a;
-            if (cy < 0 || cy >= pl.HR - 1) continue;
-            const int row = ogl * ncpg + cy * cells_w;
-            const int c0 = row + max(qx - 1, 0), c1 = row + min(qx, cells_w - 1) + 1;
-            if (!DCN4_CHECK(c0 >= 0 && c1 <= L.ncells)) continue;
-            rg.e0[a] = counts[c0];
-            rg.es[a] = counts[row + min(qx, cells_w)];
-            rg.n[a] = counts[c1] - rg.e0[a];
+        for (int ab = 0; ab < 4; ++ab) {
+            const int cy = qy - (ab >> 1), cx = qx - (ab & 1);
+            if (cy < 0 || cy >= pl.HR - 1 || cx < 0 || cx >= cells_w) continue;
+            const int cell = ogl * ncpg + cy * cells_w + cx;
+            if (!DCN4_CHECK(cell >= 0 && cell < L.ncells)) continue;
+            cr.beg[ab] = counts[cell];
+            cr.n[ab] = counts[cell + 1] - cr.beg[ab];
         }
         return true;
     };
+    auto bucket_of = [&](int n) -> int { return n > 0 ? NB - 2 - min(n - 1, NB - 2) : NB - 1; };
+    // pass 1: count, bucket histogram per group; the atomic's result is the
+    // owner's rank in its bucket
     for (int o = threadIdx.x; o < nown; o += NT) {
-        Ranges rg;
-        if (!owner_ranges(o, rg)) continue;
-        const int n = rg.n[0] + rg.n[1];
-        if (n > 0) atomicAdd(&obkt[NB - 1 - min(n, NB - 1)], 1);
+        Corners cr;
+        int n = 0;
+        if (owner_corners(o, cr)) n = cr.n[0] + cr.n[1] + cr.n[2] + cr.n[3];
+        const int rank = atomicAdd(&obkt[o & (pl.Gc - 1)][bucket_of(n)], 1);
+        if (DCN4_SMEM_OK(ocnt + o, 1, smem) && DCN4_SMEM_OK(orank + o, 2, smem)) {
+            ocnt[o] = (unsigned char)min(n, 255);
+            orank[o] = (unsigned short)rank;
+        }
     }
     __syncthreads();
-    if (threadIdx.x < 32) {  // exclusive scan of the NB bucket sizes, 2 per lane
-        const int v0 = obkt[2 * lane], v1 = obkt[2 * lane + 1];
+    if ((threadIdx.x >> 5) < pl.Gc) {  // warp g: exclusive scan of group g's buckets
+        const int gg = threadIdx.x >> 5;
+        const int v0 = obkt[gg][2 * lane], v1 = obkt[gg][2 * lane + 1];
         int incl = v0 + v1;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -648,21 +671,18 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             if (lane >= d) incl += y;
         }
         const int excl = incl - v0 - v1;
-        obkt[2 * lane] = excl;
-        obkt[2 * lane + 1] = excl + v0;
-        if (lane == 31) obkt[NB] = incl;
+        if (lane == 31) onon[gg] = nq - v1;  // all but the empty (last) bucket
+        obkt[gg][2 * lane] = excl;
+        obkt[gg][2 * lane + 1] = excl + v0;
     }
     __syncthreads();
+    // pass 2: place every owner at its slot
     for (int o = threadIdx.x; o < nown; o += NT) {
-        Ranges rg;
-        if (!owner_ranges(o, rg)) continue;
-        const int n = rg.n[0] + rg.n[1];
-        if (n > 0) {
-            const int pos = atomicAdd(&obkt[NB - 1 - min(n, NB - 1)], 1);
-            if (DCN4_SMEM_OK(olist + pos, 2, smem)) olist[pos] = (unsigned short)o;
-        }
+        if (!DCN4_SMEM_OK(ocnt + o, 1, smem) || !DCN4_SMEM_OK(orank + o, 2, smem)) continue;
+        const int gg = o & (pl.Gc - 1);
+        const int slot = (obkt[gg][bucket_of(ocnt[o])] + orank[o]) * pl.Gc + gg;
+        if (DCN4_CHECK(slot < nown)) olist[slot] = (unsigned short)o;
     }
-
     // ---------------- E: grad_offset_weight out (one warp per pixel) ----------------
     {
         const int npix = pl.TH * pl.TW;
@@ -692,19 +712,22 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
 
     // ---------------- D: gather per listed owner and flush ----------------
     __syncthreads();  // owner list complete
-    const int nlist = obkt[NB];
+    int nmax = 0;  // slots past Gc * (largest per-group count of owners with samples) are empty
+    for (int gg = 0; gg < pl.Gc; ++gg) nmax = max(nmax, onon[gg]);
+    const int nlist = nmax * pl.Gc;
     // LPP consecutive lanes share an owner, each with its UL chunks (NT is a
     // multiple of LPP, so a thread keeps its `sub`)
     for (int t = threadIdx.x; t < nlist * LPP; t += NT) {
         const int li = t / LPP;
         if (!DCN4_SMEM_OK(olist + li, 2, smem)) continue;
         const int o = olist[li];
+        if (!DCN4_CHECK(o < nown) || ocnt[o] == 0) continue;  // an empty slot of a shorter group
         const int ogl = o & (pl.Gc - 1);
         const int q = o >> pl.lgGc;
         const int qy = (int)__umulhi((unsigned)q, L.hc_magic), qx = q - qy * pl.HC;
         const int iy = tc.hy0 + qy, ix = tc.hx0 + qx;
-        Ranges rg;
-        owner_ranges(o, rg);
+        Corners cr;
+        owner_corners(o, cr);
         const int rr = (LPP == 1) ? ((U <= 8) ? (((lane & 7) * U) >> 3) : (o & (U - 1)))
                                   : ((lane / LPP) & (UL - 1));
         float acc[UL][VE];
@@ -712,34 +735,39 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
         for (int c = 0; c < UL; ++c)
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
-        // one loop over the entries of both corner rows: the lanes of a warp
-        // then run for their total counts, not for the longer row of each
-        const int ntot = rg.n[0] + rg.n[1];
-        // entry j of the owner's list; the next record is loaded while the
-        // current one is used
-        auto entry = [&](int j) -> int {
-            return j >= rg.n[0] ? rg.e0[1] + (j - rg.n[0]) : rg.e0[0] + j;
-        };
-        uint4 nxt = make_uint4(0u, 0u, 0u, 0u);
-        if (ntot > 0 && DCN4_SMEM_OK(srecw + entry(0), 16, smem)) nxt = srecw[entry(0)];
-        for (int j = 0; j < ntot; ++j) {
-            const bool a = j >= rg.n[0];
-            const int e = entry(j);
-            const bool b1 = e < (a ? rg.es[1] : rg.es[0]);  // owner is the cell's x0 + 1 corner
-            const uint4 r = nxt;
-            if (j + 1 < ntot && DCN4_SMEM_OK(srecw + entry(j + 1), 16, smem)) nxt = srecw[entry(j + 1)];
-            const unsigned char *gsrc = gotile + r.z;
-            if (CR) {
-                const unsigned wd = a ? r.y : r.x;
-                const unsigned short cw = (unsigned short)(b1 ? (wd >> 16) : (wd & 0xffffu));
+        // one loop over the entries of the four corners: the lanes of a warp
+        // then run for their total counts. Entry j belongs to corner ab where
+        // the running total c_ab passes j; its index is j + d_ab.
+        const int c1 = cr.n[0], c2 = c1 + cr.n[1], c3 = c2 + cr.n[2], ntot = c3 + cr.n[3];
+        if (CR) {
+            const int d0 = cr.beg[0], d1 = ML + cr.beg[1] - c1, d2 = 2 * ML + cr.beg[2] - c2,
+                      d3 = 3 * ML + cr.beg[3] - c3;
+            auto at_j = [&](int j) -> int {
+                return j + (j < c1 ? d0 : j < c2 ? d1 : j < c3 ? d2 : d3);
+            };
+            // the next entry is loaded while the current one is used
+            unsigned nxt = 0u;
+            if (ntot > 0 && DCN4_SMEM_OK(lists + at_j(0), 4, smem)) nxt = lists[at_j(0)];
+            for (int j = 0; j < ntot; ++j) {
+                const unsigned en = nxt;
+                if (j + 1 < ntot && DCN4_SMEM_OK(lists + at_j(j + 1), 4, smem)) nxt = lists[at_j(j + 1)];
+                const unsigned char *gsrc = gotile + ((en >> 16) << 4);
+                const unsigned short cw = (unsigned short)(en & 0xffffu);
 #pragma unroll
                 for (int c = 0; c < UL; ++c) {
                     const int cc = sub * UL + ((c + rr) & (UL - 1));
                     VecMathMixed<T>::fma_bits(acc[c], DCN4_LDS16(gsrc + cc * 16, smem), cw);
                 }
-            } else {
-                const float lx = __uint_as_float(r.x), ly = __uint_as_float(r.y);
-                const float w = (a ? ly : 1.0f - ly) * (b1 ? lx : 1.0f - lx) * __uint_as_float(r.w);
+            }
+        } else {
+            for (int j = 0; j < ntot; ++j) {
+                const int ab = j < c1 ? 0 : j < c2 ? 1 : j < c3 ? 2 : 3;
+                const int e = j + (ab == 0 ? cr.beg[0] : ab == 1 ? cr.beg[1] - c1
+                                   : ab == 2 ? cr.beg[2] - c2 : cr.beg[3] - c3);
+                if (!DCN4_SMEM_OK(srec + e, 16, smem)) continue;
+                const float4 r = srec[e];
+                const float w = ((ab & 2) ? r.y : 1.0f - r.y) * ((ab & 1) ? r.x : 1.0f - r.x) * r.w;
+                const unsigned char *gsrc = gotile + __float_as_uint(r.z);
 #pragma unroll
                 for (int c = 0; c < UL; ++c) {
                     const int cc = sub * UL + ((c + rr) & (UL - 1));

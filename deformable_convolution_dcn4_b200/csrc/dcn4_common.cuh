@@ -106,7 +106,8 @@ struct BwdLayout {
     int bar_off;      // one mbarrier
     int ncells;       // (HR-1)*(HC-1)*Gc destination cells
     int max_samples;  // TH*TW*Gc*9; sorted sample records reuse the window
-    int olist_off;    // owner list (u16 per owner, sorted by sample count), after the records
+    int olist_off;    // owner list (u16 per owner, sorted by sample count), a u16 rank and
+                      // a u8 count per owner, after the sorted samples
     unsigned hc_magic;  // ceil(2^32 / HC): q / HC == __umulhi(q, hc_magic) for q < 2^16
     int smem_bytes;
     int threads;      // 256 (two CTAs per SM) or 512
