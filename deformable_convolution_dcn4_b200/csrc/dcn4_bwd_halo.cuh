@@ -745,12 +745,31 @@ bwd_halo_kernel(const __grid_constant__ CUtensorMap tmap_in,
             auto at_j = [&](int j) -> int {
                 return j + (j < c1 ? d0 : j < c2 ? d1 : j < c3 ? d2 : d3);
             };
-            // the next entry is loaded while the current one is used
-            unsigned nxt = 0u;
-            if (ntot > 0 && DCN4_SMEM_OK(lists + at_j(0), 4, smem)) nxt = lists[at_j(0)];
-            for (int j = 0; j < ntot; ++j) {
-                const unsigned en = nxt;
-                if (j + 1 < ntot && DCN4_SMEM_OK(lists + at_j(j + 1), 4, smem)) nxt = lists[at_j(j + 1)];
+            // BJ entries at a time: their entry and grad_out loads are all
+            // issued before the multiply-adds, so the loads' latency overlaps
+            constexpr int BJ = UL <= 2 ? 4 : 2;
+            int j = 0;
+            for (; j + BJ <= ntot; j += BJ) {
+                unsigned en[BJ];
+#pragma unroll
+                for (int u = 0; u < BJ; ++u)
+                    en[u] = DCN4_SMEM_OK(lists + at_j(j + u), 4, smem) ? lists[at_j(j + u)] : 0u;
+                uint4 qv[BJ][UL];
+#pragma unroll
+                for (int u = 0; u < BJ; ++u) {
+                    const unsigned char *gsrc = gotile + ((en[u] >> 16) << 4);
+#pragma unroll
+                    for (int c = 0; c < UL; ++c)
+                        qv[u][c] = DCN4_LDS16(gsrc + (sub * UL + ((c + rr) & (UL - 1))) * 16, smem);
+                }
+#pragma unroll
+                for (int u = 0; u < BJ; ++u)
+#pragma unroll
+                    for (int c = 0; c < UL; ++c)
+                        VecMathMixed<T>::fma_bits(acc[c], qv[u][c], (unsigned short)(en[u] & 0xffffu));
+            }
+            for (; j < ntot; ++j) {
+                const unsigned en = DCN4_SMEM_OK(lists + at_j(j), 4, smem) ? lists[at_j(j)] : 0u;
                 const unsigned char *gsrc = gotile + ((en >> 16) << 4);
                 const unsigned short cw = (unsigned short)(en & 0xffffu);
 #pragma unroll
