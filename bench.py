@@ -63,6 +63,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="internimage_bf16")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    # time the step alone: skip the next_rows and configs diagnostics and the
+    # end-to-end leg (used by the profiler's launch list)
+    p.add_argument("--step-only", action="store_true")
     return p.parse_args(argv)
 
 
@@ -406,14 +409,16 @@ def run_ours(args):
 
     # next rows beyond the step (MSDCN backward; the offset/weight producer),
     # timed the same way outside the timed region, reported on their own
-    extra = next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind)
+    extra, configs, samples, e2e = None, None, [], None
+    if not args.step_only:
+        extra = next_rows(dcn, wl, Ho, Wo, d, m, kw, ws, flush, stream, peak, peak_kind)
 
-    # every workload of the table, each op timed on its own (outside the step)
-    configs, samples = time_configs(dcn, flush, stream, peak, peak_kind)
+        # every workload of the table, each op timed on its own (outside the step)
+        configs, samples = time_configs(dcn, flush, stream, peak, peak_kind)
 
-    # end to end: pinned host buffers, H2D copies + the three calls + D2H reads
-    e2e = run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream,
-                  step_bytes, world)
+        # end to end: pinned host buffers, H2D copies + the three calls + D2H reads
+        e2e = run_e2e(args, dcn, host, mhost, ops, d, m, out, ms_out, gin, gow, dev, stream,
+                      step_bytes, world)
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
@@ -424,7 +429,7 @@ def run_ours(args):
             "gpu_launches": args.steps * sum(launches.values()),
             "launches_per_step": launches, "e2e": e2e, "next_rows": extra,
             "configs": configs, "clocks": clocks.summary()}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.step_only:
         line["cpu_baseline"] = cpu_baseline(wl)
         for key, per_op in oracle_config_checks(samples).items():
             for op, errs in per_op.items():
