@@ -140,8 +140,8 @@ bool plan_halo(const Geometry &g, int eb, bool msdcn, bool rec_tma, HaloPlan *ou
 }
 
 // Tiling and shared-memory layout of the backward halo kernel: one
-// (pixel, group) pair per thread, or per two lanes when a group is 8 chunks
-// (128 bytes: each lane owns 4); 256 or 512 threads; 128-byte staged pixels.
+// (pixel, group) pair per thread, or per four lanes when a group is 8 chunks
+// (128 bytes: each lane owns 2); 256 or 512 threads; 128-byte staged pixels.
 // The window reaches R = 4 pixels beyond the tile; for the multi-scale
 // variant, whose scaled offsets reach far, the whole image (plus its zero
 // border) is tried first. The sorted sample records (16 bytes each) and the
@@ -153,7 +153,7 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
     if (g.G % Gc != 0) return false;
     const int U = g.D * eb / 16;
     if (!(U == 4 || (U == 2 && eb == 2) || U == 8)) return false;
-    const int lpp = U == 8 ? 2 : 1;
+    const int lpp = U == 8 ? 4 : 1;
     const int R = 4;
     const int smem_max = max_smem_optin() - 1024;  // static shared memory of the kernel
     // record slots as in plan_halo: per-pixel bulk copies, or one TMA tile copy
@@ -168,7 +168,7 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
         TH = TH < g.Ho ? TH : g.Ho;
         TW = TW < pow2_ceil(g.Wo) ? TW : pow2_ceil(g.Wo);
         const int pairs = TH * TW * Gc;
-        if (pairs * lpp > (lpp == 1 ? 512 : 256)) return false;
+        if (pairs * lpp > 512) return false;
         int HR = (TH - 1) * g.sh + (g.kh - 1) * g.dh + 2 * R + 2;
         int HC = (TW - 1) * g.sw + (g.kw - 1) * g.dw + 2 * R + 2;
         const int full_h = force_full || HR >= g.H + 2, full_w = force_full || HC >= g.W + 2;
@@ -200,7 +200,7 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
         if (L.smem_bytes > smem_max) return false;
         const bool two = pairs * lpp <= 256 && 2 * (L.smem_bytes + 1024 + 1024) <= per_sm;
         if (first && !(two && pairs * lpp == 256)) return false;
-        L.threads = (lpp == 1 && !two) ? 512 : 256;
+        L.threads = two ? 256 : 512;
         L.lpp = lpp;
         *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
                         (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
@@ -210,7 +210,7 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
     };
     static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8},
                                    {4, 4}, {4, 2}, {2, 4}, {2, 2}, {2, 1}, {1, 2}, {1, 1}};
-    if (msdcn && lpp == 2) {  // wide groups: the whole image when it fits
+    if (msdcn && lpp > 1) {  // wide groups: the whole image when it fits
         for (auto &c : cands)
             if (try_plan(c[0], c[1], true, false)) return true;
     }

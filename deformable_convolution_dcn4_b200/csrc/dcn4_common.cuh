@@ -111,7 +111,7 @@ struct BwdLayout {
     unsigned hc_magic;  // ceil(2^32 / HC): q / HC == __umulhi(q, hc_magic) for q < 2^16
     int smem_bytes;
     int threads;      // 256 (two CTAs per SM) or 512
-    int lpp;          // lanes per (pixel, group): 1, or 2 for 8 chunks (128-byte groups)
+    int lpp;          // lanes per (pixel, group): 1, or 4 for 8 chunks (128-byte groups)
 };
 
 // Tiling of the shared-memory halo kernels (chosen on the host).

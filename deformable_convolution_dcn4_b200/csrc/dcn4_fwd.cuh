@@ -216,11 +216,12 @@ __device__ __forceinline__ TileCoord tile_coord(int t, const Geometry &g, const 
 }
 
 // Bulk-copies into their slots the records of the tile pixels whose pairs
-// this warp computes: with NT threads, thread t handles pairs t, t + NT, ...,
-// so warp w owns pixel blocks [(32w + k*NT)/Gc, +32/Gc) for k = 0, 1, ...
+// this warp computes: with NT threads and LPP lanes per pair, thread t
+// handles pairs t/LPP, (t + NT)/LPP, ..., so warp w owns pixel blocks
+// [(32w + k*NT)/(LPP*Gc), +32/(LPP*Gc)) for k = 0, 1, ...
 // Completes on `bar` (arrival count 1); all 32 lanes call it, lane l copies
 // pixel l of each block it has, lane 0 arrives with the warp's byte count.
-template <typename T>
+template <typename T, int LPP = 1>
 __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometry &g,
                                               const HaloPlan &pl, const T *__restrict__ ow,
                                               unsigned long long ow_bytes, unsigned char *slots,
@@ -230,7 +231,7 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
     constexpr unsigned long long REC = 27ull * EB;
     const int lane = threadIdx.x & 31;
     const int npix = pl.TH * pl.TW;
-    const bool mine = lane < (32 >> pl.lgGc);
+    const bool mine = lane < ((32 / LPP) >> pl.lgGc);
     auto span = [&](int p, unsigned long long &a, unsigned long long &e,
                     unsigned long long &end) -> bool {
         const int ty = p >> pl.lgTW, tx_ = p & (pl.TW - 1);
@@ -243,7 +244,8 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
         return true;
     };
     uint32_t tx = 0;
-    for (int base = (threadIdx.x & ~31) >> pl.lgGc; base < npix; base += nt >> pl.lgGc) {
+    for (int base = ((threadIdx.x & ~31) / LPP) >> pl.lgGc; base < npix;
+         base += (nt / LPP) >> pl.lgGc) {
         const int p = base + lane;
         unsigned long long a, e, end;
         if (!mine || !span(p, a, e, end)) continue;
@@ -270,7 +272,8 @@ __device__ __forceinline__ void stage_records(const TileCoord &tc, const Geometr
     __syncwarp();
     if (lane == 0) mbar_arrive_expect_tx(bar, total);
     __syncwarp();
-    for (int base = (threadIdx.x & ~31) >> pl.lgGc; base < npix; base += nt >> pl.lgGc) {
+    for (int base = ((threadIdx.x & ~31) / LPP) >> pl.lgGc; base < npix;
+         base += (nt / LPP) >> pl.lgGc) {
         const int p = base + lane;
         unsigned long long a, e, end;
         if (!mine || !span(p, a, e, end) || e <= a) continue;
@@ -317,8 +320,9 @@ __device__ __forceinline__ void stage_window_records(const TileCoord &tc, const 
         tma_load_4d(smem_u32(slots), tmap_ow, x0, tc.wo0, tc.ho0, tc.n, bar);
 }
 
-// The gathers of one staged tile: one thread per (pixel, group).
-template <typename T, int U, bool MS, int MV>
+// The gathers of one staged tile: LPP lanes per (pixel, group), each with
+// U/LPP of its 16-byte chunks (one lane with all of them when LPP = 1).
+template <typename T, int U, bool MS, int MV, int LPP>
 __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry &g,
                                              const HaloPlan &pl, const T *__restrict__ in,
                                              T *__restrict__ out, const MsdcnParams &ms,
@@ -341,7 +345,10 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
     const float hy_lo = (float)tc.hy0, hy_hi = (float)(tc.hy0 + pl.HR - 1);
     const float PSf = (float)PS, RSf = (float)RS;
     const float dwf = (float)g.dw, dhf = (float)g.dh;
-    for (int f = ct; f < npairs; f += nct) {
+    constexpr int UL = U / LPP;  // chunks of this lane
+    // nct is a multiple of LPP, so a thread keeps its lane-in-pair `sub`
+    for (int t = ct; t < npairs * LPP; t += nct) {
+        const int f = t / LPP, sub = t & (LPP - 1);
         const int pix = f >> pl.lgGc;
         const int gl = f & (pl.Gc - 1);
         const int ty = pix >> pl.lgTW, tx = pix & (pl.TW - 1);
@@ -393,16 +400,19 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
         }
         // chunk rotation: the 8 lanes of a shared-memory phase start at
         // different 16-byte chunks, so their loads hit 8 different bank quads
-        const int r = (U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1));
-        const unsigned char *row0[U], *row1[U];
+        const int r = (LPP == 1) ? ((U <= 8) ? (((lane & 7) * U) >> 3) : (f & (U - 1)))
+                                 : ((lane / LPP) & (UL - 1));
+        // this lane's c-th chunk
+        auto chunk = [&](int c) -> int { return sub * UL + ((c + r) & (UL - 1)); };
+        const unsigned char *row0[UL], *row1[UL];
 #pragma unroll
-        for (int c = 0; c < U; ++c) {
-            row0[c] = halo + (size_t)gl * D * EB + ((c + r) & (U - 1)) * 16;
+        for (int c = 0; c < UL; ++c) {
+            row0[c] = halo + (size_t)gl * D * EB + chunk(c) * 16;
             row1[c] = row0[c] + RS;
         }
-        float acc[U][VE];
+        float acc[UL][VE];
 #pragma unroll
-        for (int c = 0; c < U; ++c)
+        for (int c = 0; c < UL; ++c)
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[c][e] = 0.0f;
 
@@ -432,7 +442,7 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                 // integer-valued floats below 2^24: the byte offset is exact
                 const int off = __float2int_rz(fmaf(y0f - hy_lo, RSf, (x0f - hx_lo) * PSf));
 #pragma unroll
-                for (int c = 0; c < U; ++c) {
+                for (int c = 0; c < UL; ++c) {
                     const unsigned char *a0 = row0[c] + off;
                     const unsigned char *a1 = row1[c] + off;
                     const uint4 q00 = DCN4_LDS16(a0, sbase);
@@ -488,16 +498,15 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                 if (yy < 0 || yy >= g.H || xx < 0 || xx >= g.W) continue;
                 const uint4 *p = reinterpret_cast<const uint4 *>(gbase + ((size_t)yy * g.W + xx) * g.C);
 #pragma unroll
-                for (int c = 0; c < U; ++c)
-                    VecMath<T>::fma(acc[c], DCN4_LDG16(p + ((c + r) & (U - 1)), in, input_bytes(g, EB)),
-                                    wc[q]);
+                for (int c = 0; c < UL; ++c)
+                    VecMath<T>::fma(acc[c], DCN4_LDG16(p + chunk(c), in, input_bytes(g, EB)), wc[q]);
             }
         }
         uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)(tc.g0 + gl) * D);
 #pragma unroll
-        for (int c = 0; c < U; ++c)
-            if (DCN4_GMEM_OK(dst + ((c + r) & (U - 1)), 16, out, output_bytes(g, EB)))
-                dst[(c + r) & (U - 1)] = VecMath<T>::pack(acc[c]);
+        for (int c = 0; c < UL; ++c)
+            if (DCN4_GMEM_OK(dst + chunk(c), 16, out, output_bytes(g, EB)))
+                dst[chunk(c)] = VecMath<T>::pack(acc[c]);
     }
 }
 
@@ -511,7 +520,7 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
 // the next tile are in flight while the current one is computed. Every wait
 // is bounded; on expiry the warp sets the error word, lets its own copies in
 // flight land and returns.
-template <typename T, int U, bool MS, int MV, int STAGES, int NW>
+template <typename T, int U, bool MS, int MV, int STAGES, int NW, int LPP>
 __global__ void __launch_bounds__(NW * 32, 1)
 fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_ow,
                 Geometry g, HaloPlan pl, const T *__restrict__ in, const T *__restrict__ ow,
@@ -557,7 +566,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
     auto records = [&](const TileCoord &tc, int k) {
         if (pl.rec_tma) return;
         const int s = k % STAGES;
-        stage_records<T>(tc, g, pl, ow, ow_bytes, smem + s * stage_bytes + pl.halo_bytes, NW * 32,
+        stage_records<T, LPP>(tc, g, pl, ow, ow_bytes, smem + s * stage_bytes + pl.halo_bytes, NW * 32,
                          myrec + 8 * s, smem);
     };
     auto records_ready = [&](int k) -> bool {
@@ -604,7 +613,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
             return;
         }
         const unsigned char *buf = smem + s * stage_bytes;
-        compute_tile<T, U, MS, MV>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
+        compute_tile<T, U, MS, MV, LPP>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
                                    threadIdx.x, NW * 32, smem);
         __syncwarp();
         if (leader) mbar_arrive(empty0 + 8 * s);

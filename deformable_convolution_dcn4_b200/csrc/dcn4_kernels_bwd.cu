@@ -48,16 +48,22 @@ cudaError_t launch_bwd_halo_m(const BwdLaunch &L, bool direct) {
             return L.mixed ? run(bwd_halo_kernel<T, 2, 16, true, false, MS, 1>)
                            : run(bwd_halo_kernel<T, 2, 16, false, false, MS, 1>);
         }
-        // 64 channels: two lanes per (pixel, group), 256 threads
-        if (U == 8 && nt == 256 && L.layout.lpp == 2) {
-            if (direct) return run(bwd_halo_kernel<T, 8, 8, true, true, MS, 2>);
-            return L.mixed ? run(bwd_halo_kernel<T, 8, 8, true, false, MS, 2>)
-                           : run(bwd_halo_kernel<T, 8, 8, false, false, MS, 2>);
+        // 64 channels: four lanes per (pixel, group), 256 or 512 threads
+        if (U == 8 && L.layout.lpp == 4 && nt == 256) {
+            if (direct) return run(bwd_halo_kernel<T, 8, 8, true, true, MS, 4>);
+            return L.mixed ? run(bwd_halo_kernel<T, 8, 8, true, false, MS, 4>)
+                           : run(bwd_halo_kernel<T, 8, 8, false, false, MS, 4>);
+        }
+        if (U == 8 && L.layout.lpp == 4) {
+            if (direct) return run(bwd_halo_kernel<T, 8, 16, true, true, MS, 4>);
+            return L.mixed ? run(bwd_halo_kernel<T, 8, 16, true, false, MS, 4>)
+                           : run(bwd_halo_kernel<T, 8, 16, false, false, MS, 4>);
         }
     } else {
-        // fp32, 32 channels: two lanes per (pixel, group), 256 threads
-        if (U == 8 && nt == 256 && L.layout.lpp == 2)
-            return run(bwd_halo_kernel<T, 8, 8, false, false, MS, 2>);
+        // fp32, 32 channels: four lanes per (pixel, group), 256 or 512 threads
+        if (U == 8 && L.layout.lpp == 4 && nt == 256)
+            return run(bwd_halo_kernel<T, 8, 8, false, false, MS, 4>);
+        if (U == 8 && L.layout.lpp == 4) return run(bwd_halo_kernel<T, 8, 16, false, false, MS, 4>);
     }
     if (U == 4 && nt == 256) return run(bwd_halo_kernel<T, 4, 8, false, false, MS, 1>);
     if (U == 4) return run(bwd_halo_kernel<T, 4, 16, false, false, MS, 1>);

@@ -19,9 +19,9 @@ namespace {
 // Kernel argument for launches without the multi-scale variant.
 const MsdcnParams kNoMs = {};
 
-template <typename T, int U, bool MS, int MV, int STAGES, int NW>
+template <typename T, int U, bool MS, int MV, int STAGES, int NW, int LPP = 1>
 cudaError_t launch_halo_t(const FwdLaunch &L) {
-    auto k = fwd_halo_kernel<T, U, MS, MV, STAGES, NW>;
+    auto k = fwd_halo_kernel<T, U, MS, MV, STAGES, NW, LPP>;
     constexpr int NT = NW * 32;
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.plan.smem_bytes);
     if (e != cudaSuccess) return e;
@@ -41,7 +41,8 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
 
 // Stage count and warps: two stages with 16 warps when a tile has 512
 // (pixel, group) pairs, 8 warps when it has fewer; the large single-stage
-// plans (MSDCN whole-image windows, 64-channel groups) use 8.
+// plans (MSDCN whole-image windows) use 8, and groups of 8 chunks (64 bf16 /
+// 32 fp32 channels) run two lanes per pair on 16 warps.
 template <typename T, int U, bool MS, int MV>
 cudaError_t launch_halo_s(const FwdLaunch &L) {
     if constexpr (U <= 4) {
@@ -50,8 +51,10 @@ cudaError_t launch_halo_s(const FwdLaunch &L) {
                 return launch_halo_t<T, U, MS, MV, 2, 16>(L);
             return launch_halo_t<T, U, MS, MV, 2, 8>(L);
         }
+        return launch_halo_t<T, U, MS, MV, 1, 8>(L);
+    } else {
+        return launch_halo_t<T, U, MS, MV, 1, 16, 2>(L);
     }
-    return launch_halo_t<T, U, MS, MV, 1, 8>(L);
 }
 
 template <typename T, int U, bool MS>
