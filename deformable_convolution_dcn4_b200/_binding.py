@@ -26,7 +26,8 @@ MSDCN_MODE_CODE = {"offset": 0, "dilation": 1}
 EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dcn4_backward",
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
            "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches",
-           "msdcn_backward", "dcn4_offset_producer")
+           "msdcn_backward", "dcn4_offset_producer", "dcn4_fused_forward_workspace_size",
+           "dcn4_fused_forward")
 
 
 class Dcn4Error(RuntimeError):
@@ -92,6 +93,9 @@ def _open(path):
     lib.dcn4_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
     lib.dcn4_kernel_launches.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     lib.dcn4_offset_producer.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.dcn4_fused_forward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.dcn4_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                       vp]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -191,6 +195,54 @@ def dcn4_offset_producer(x, dw_weight, dw_bias, lin_weight, lin_bias, group, ker
     _check("dcn4_offset_producer",
            load().dcn4_offset_producer(ctypes.byref(desc), _ptr(x), _ptr(dw_weight), _ptr(dw_bias),
                                        _ptr(lin_weight), _ptr(lin_bias), _ptr(out), _stream(x)))
+    return out
+
+
+def dcn4_fused_forward_workspace_size(desc):
+    n = ctypes.c_size_t()
+    _check("dcn4_fused_forward_workspace_size",
+           load().dcn4_fused_forward_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def dcn4_fused_forward(input, x, dw_weight, dw_bias, lin_weight, lin_bias, group, kernel_size=3,
+                       stride=1, pad=1, dilation=1, offset_scale=1.0, algo="auto", out=None,
+                       math="default", softmax=False, workspace=None, offset_weight_out=None):
+    """DCNv4 forward with the offset/weight sub-network in front:
+    dcn4_forward(input, dcn4_offset_producer(x, ...)) in one call. input and x
+    [N,H,W,C]; dw_weight [3,3,C], dw_bias [C], lin_weight [G*kh*kw*3, C],
+    lin_bias [G*kh*kw*3]. offset_weight_out [N,Ho,Wo,G,kh*kw,3], when given,
+    receives the records the aggregation used. A scratch tensor is allocated
+    when the call takes the two-kernel chain and neither it nor
+    offset_weight_out is given."""
+    desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
+                     softmax)
+    ho, wo = dcn4_out_shape(desc)
+    N, H, W, C = input.shape
+    J = group * desc.kh * desc.kw * 3
+    _require(input, "input", input.dtype)
+    _require(x, "x", input.dtype, (N, H, W, C))
+    _require(dw_weight, "dw_weight", input.dtype, (3, 3, C))
+    _require(dw_bias, "dw_bias", input.dtype, (C,))
+    _require(lin_weight, "lin_weight", input.dtype, (J, C))
+    _require(lin_bias, "lin_bias", input.dtype, (J,))
+    if out is None:
+        out = torch.empty((N, ho, wo, C), dtype=input.dtype, device=input.device)
+    _require(out, "out", input.dtype, (N, ho, wo, C))
+    if offset_weight_out is not None:
+        _require(offset_weight_out, "offset_weight_out", input.dtype,
+                 (N, ho, wo, group, desc.kh * desc.kw, 3))
+    if workspace is None and offset_weight_out is None:
+        need = dcn4_fused_forward_workspace_size(desc)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=input.device)
+    ws, nws = (_ptr(workspace), workspace.numel() * workspace.element_size()) \
+        if workspace is not None else (None, 0)
+    _check("dcn4_fused_forward",
+           load().dcn4_fused_forward(ctypes.byref(desc), _ptr(input), _ptr(x), _ptr(dw_weight),
+                                     _ptr(dw_bias), _ptr(lin_weight), _ptr(lin_bias), _ptr(out),
+                                     None if offset_weight_out is None else _ptr(offset_weight_out),
+                                     ws, nws, _stream(input)))
     return out
 
 

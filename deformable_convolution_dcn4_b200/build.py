@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libdcn4.so")
 CHECKED_LIBRARY = os.path.join(PKG, "libdcn4_checked.so")
 SOURCES = ["dcn4_api.cu", "dcn4_kernels.cu", "dcn4_kernels_fwd.cu", "dcn4_kernels_bwd.cu",
-           "dcn4_noalloc.cu"]
+           "dcn4_kernels_fused.cu", "dcn4_noalloc.cu"]
 OBJDIR = os.path.join(PKG, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -220,6 +220,68 @@ bool plan_bwd(const Geometry &g, int eb, bool rec_tma, bool msdcn, HaloPlan *out
     return false;
 }
 
+// Tiling and shared-memory carve-up of the fused producer + forward kernel:
+// 16-bit data, 3x3 taps, 128-byte staged pixels of Gc groups with 2 or 4
+// chunks each (so C is a multiple of 64: whole MMA K steps and whole blocks
+// of 8 depthwise chunks), C <= 256 (one TMA box row), the offset grid equal
+// to the input grid. One stage: the input window (reach R,
+// 5 where the tile fits, else 4 or 3), the record slots, x's neighbourhood
+// of the tile, A (128 rows), the slice's lin_w rows, taps and biases; a tile
+// of at most 128 pixels (the MMA's M).
+bool plan_fused(const Geometry &g, int eb, HaloPlan *out, FusedLayout *lay) {
+    if (eb != 2 || g.kh != 3 || g.kw != 3) return false;
+    if (g.Ho != g.H || g.Wo != g.W) return false;
+    if ((g.D * eb) % 16 != 0) return false;
+    const int U = g.D * eb / 16;
+    if (U != 2 && U != 4) return false;
+    if (g.C % 64 != 0 || g.C > 256) return false;
+    const int Gc = 128 / (g.D * eb);
+    if (g.G % Gc != 0) return false;
+    const int JS = Gc * 27, NP = ceil_to(JS, 16);
+    const int slot = NP * eb + 16;  // an odd multiple of 16 bytes
+    const int smem_max = max_smem_optin();
+    auto try_tile = [&](int TH, int TW, int R) -> bool {
+        TH = TH < g.Ho ? TH : g.Ho;
+        TW = TW < pow2_ceil(g.Wo) ? TW : pow2_ceil(g.Wo);
+        if (TH * TW > 128) return false;
+        int HR = (TH - 1) * g.sh + (g.kh - 1) * g.dh + 2 * R + 2;
+        int HC = (TW - 1) * g.sw + (g.kw - 1) * g.dw + 2 * R + 2;
+        const int full_h = HR >= g.H + 2, full_w = HC >= g.W + 2;
+        if (full_h) HR = g.H + 2;
+        if (full_w) HC = g.W + 2;
+        if (HR > 256 || HC > 256) return false;
+        const int halo = HR * HC * 128;
+        FusedLayout L;
+        L.win_off = 0;
+        L.slots_off = ceil_to(halo, 128);
+        L.x_off = ceil_to(L.slots_off + TH * TW * slot, 128);
+        L.x_bytes = (TH + 2) * (TW + 2) * g.C * eb;
+        L.a_off = ceil_to(L.x_off + L.x_bytes, 1024);
+        L.b_off = L.a_off + 128 * g.C * eb;
+        L.dwt_off = L.b_off + NP * g.C * eb;
+        L.dwb_off = ceil_to(L.dwt_off + 9 * g.C * eb, 16);
+        L.linb_off = L.dwb_off + g.C * 4;
+        L.bar_off = ceil_to(L.linb_off + NP * 4, 16);
+        L.bytes = L.bar_off + 32;
+        L.JS = JS;
+        L.NP = NP;
+        L.tmem_cols = 32;
+        while (L.tmem_cols < NP) L.tmem_cols <<= 1;
+        if (L.bytes > smem_max) return false;
+        *out = HaloPlan{TH, TW, Gc, log2_exact(TW), log2_exact(Gc), R, HR, HC, full_h, full_w,
+                        (g.Ho + TH - 1) / TH, (g.Wo + TW - 1) / TW, g.G / Gc, slot, halo, 1,
+                        L.bytes, 2, 0};
+        *lay = L;
+        return true;
+    };
+    static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8}, {4, 4},
+                                   {4, 2},  {2, 4},  {2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    for (auto &c : cands)
+        for (int R : {5, 4, 3})
+            if (try_tile(c[0], c[1], R)) return true;
+    return false;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -408,6 +470,78 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
     if (!L.tc && (L.pg.npix + kProducerPixels - 1) / kProducerPixels > 0x7fffffffLL)
         return DCN4_ERR_UNSUPPORTED;
     return cuda_status(launch_producer(L));
+}
+
+dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *bytes) {
+    Geometry g;
+    if (!make_geometry(desc, &g) || !bytes) return DCN4_ERR_INVALID_ARG;
+    HaloPlan plan;
+    FusedLayout lay;
+    const int eb = elem_bytes(static_cast<Dtype>(desc->dtype));
+    const bool fused = (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) &&
+                       plan_fused(g, eb, &plan, &lay);
+    *bytes = fused ? 0 : (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
+    return DCN4_OK;
+}
+
+dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const void *x,
+                               const void *dw_weight, const void *dw_bias,
+                               const void *lin_weight, const void *lin_bias, void *output,
+                               void *offset_weight_out, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    Geometry g;
+    if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
+    if (!input || !x || !dw_weight || !dw_bias || !lin_weight || !lin_bias || !output)
+        return DCN4_ERR_INVALID_ARG;
+    if (g.Ho != g.H || g.Wo != g.W) return DCN4_ERR_UNSUPPORTED;
+    const Dtype dt = static_cast<Dtype>(desc->dtype);
+    const int eb = elem_bytes(dt);
+    if (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) {
+        FusedLaunch L;
+        memset(&L, 0, sizeof(L));
+        CUtensorMap map_in, map_x;
+        memset(&map_in, 0, sizeof(map_in));
+        memset(&map_x, 0, sizeof(map_x));
+        const bool fused =
+            plan_fused(g, eb, &L.plan, &L.lay) && aligned16(input) && aligned16(x) &&
+            aligned16(lin_weight) && aligned16(output) &&
+            (reinterpret_cast<uintptr_t>(offset_weight_out) & 3) == 0 &&
+            encode_input_map(g, dt, input, L.plan, &map_in) &&
+            encode_map(dt, x, g.N, g.H, g.W, g.C, g.C, L.plan.TW + 2, L.plan.TH + 2, &map_x);
+        if (fused) {
+            L.geo = g;
+            L.dtype = dt;
+            L.in = input;
+            L.x = x;
+            L.dw_w = dw_weight;
+            L.dw_b = dw_bias;
+            L.lin_w = lin_weight;
+            L.lin_b = lin_bias;
+            L.out = output;
+            L.rec_out = offset_weight_out;
+            L.mathv = forward_math(desc);
+            L.tmap_in = &map_in;
+            L.tmap_x = &map_x;
+            L.stream = static_cast<cudaStream_t>(stream);
+            return cuda_status(launch_fused(L));
+        }
+        if (desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+    }
+    // the two-kernel chain, through offset_weight_out when given, else
+    // through the caller's scratch
+    void *records = offset_weight_out;
+    if (!records) {
+        const size_t need = (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
+        if (!workspace || workspace_bytes < need) return DCN4_ERR_WORKSPACE;
+        records = workspace;
+    }
+    dcn4_desc d = *desc;
+    d.algo = desc->algo == DCN4_ALGO_GENERIC ? DCN4_ALGO_GENERIC : DCN4_ALGO_AUTO;
+    const dcn4_status st =
+        dcn4_offset_producer(&d, x, dw_weight, dw_bias, lin_weight, lin_bias, records, stream);
+    if (st != DCN4_OK) return st;
+    d.algo = desc->algo;
+    return dcn4_forward(&d, input, records, output, stream);
 }
 
 dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes) {

@@ -127,8 +127,28 @@ struct HaloPlan {
     int halo_bytes;      // HR*HC*Gc*D*elem, rounded up to 128
     int stages;          // 2: double-buffered pipeline, 1: single buffer
     int smem_bytes;      // dynamic shared memory of one CTA
-    int rec_tma;         // 1: records arrive by one TMA tile copy per tile (forward)
+    int rec_tma;         // 1: records arrive by one TMA tile copy per tile (forward);
+                         // 2: the fused kernel writes them, slot-aligned, in place
     int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)
+};
+
+// Shared-memory carve-up of the fused producer + forward kernel (byte offsets
+// from the start of dynamic shared memory; chosen on the host).
+struct FusedLayout {
+    int win_off;    // input window of the tile's group slice (HaloPlan::halo_bytes)
+    int slots_off;  // the tile's records, TH*TW slots of HaloPlan::slot_bytes
+    int x_off;      // x neighbourhood of the tile, (TH+2) x (TW+2) pixels x C
+    int x_bytes;    // bytes of that copy
+    int a_off;      // depthwise outputs: 128 rows x C, tcgen05 K-major core matrices
+    int b_off;      // the slice's rows of lin_weight: NP rows x C, core matrices
+    int dwt_off;    // dw_weight [9][C] in the data type
+    int dwb_off;    // dw_bias [C] in fp32
+    int linb_off;   // the slice's lin_bias [NP] in fp32 (zero past JS)
+    int bar_off;    // three mbarriers and the tensor-memory address
+    int bytes;      // dynamic shared memory of one CTA
+    int JS;         // outputs of one slice, Gc * 27
+    int NP;         // JS rounded up to 16 (the MMA's N)
+    int tmem_cols;  // tensor-memory columns allocated: a power of two >= NP, >= 32
 };
 
 // Byte sizes of the tensors of one call (bounds of the checked build).

@@ -355,10 +355,12 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
         if (ty >= tc.th_eff || tx >= tc.tw_eff) continue;
         const int ho = tc.ho0 + ty, wo = tc.wo0 + tx;
         const unsigned long long gp = tc.gp0 + (unsigned long long)ty * g.Wo + tx;
-        // the record's offset within its 16-byte-aligned copy (arithmetic mod 2^32)
-        const unsigned mis = pl.rec_tma
-                                 ? ((unsigned)(tc.g0 * 27) & (unsigned)(16 / EB - 1)) * (unsigned)EB
-                                 : ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
+        // the record's offset within its 16-byte-aligned copy (arithmetic mod
+        // 2^32); records written in place (rec_tma == 2) start their slot
+        const unsigned mis =
+            pl.rec_tma == 2 ? 0u
+            : pl.rec_tma    ? ((unsigned)(tc.g0 * 27) & (unsigned)(16 / EB - 1)) * (unsigned)EB
+                            : ((unsigned)gp * (unsigned)g.G + (unsigned)tc.g0) * (unsigned)REC & 15u;
         const unsigned char *rec = slots + (size_t)pix * pl.slot_bytes + mis + gl * REC;
         // the reader takes whole words from the record's 4-byte boundary
         if (!DCN4_SMEM_OK(reinterpret_cast<const unsigned char *>(

@@ -150,7 +150,7 @@ cudaError_t launch_producer(const ProducerLaunch &L) {
 }
 
 cudaError_t read_clear_device_error(unsigned *bits) {
-    unsigned v = 0, f = 0, b = 0;
+    unsigned v = 0, f = 0, b = 0, u = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v));
     if (e != cudaSuccess) return e;
     if (v != 0) {
@@ -162,7 +162,9 @@ cudaError_t read_clear_device_error(unsigned *bits) {
     if (e != cudaSuccess) return e;
     e = read_clear_error_bwd(&b);
     if (e != cudaSuccess) return e;
-    *bits = v | f | b;
+    e = read_clear_error_fused(&u);
+    if (e != cudaSuccess) return e;
+    *bits = v | f | b | u;
     return cudaSuccess;
 }
 

@@ -63,8 +63,25 @@ struct ProducerLaunch {
     ProducerTcLayout lay;  // tensor-core kernel only
     cudaStream_t stream;
 };
+
+// The fused producer + forward kernel of one call.
+struct FusedLaunch {
+    Geometry geo;
+    Dtype dtype;  // BF16 or F16
+    const void *in, *x, *dw_w, *dw_b, *lin_w, *lin_b;
+    void *out;
+    void *rec_out;  // optional copy of the records (offset_weight layout)
+    int mathv;      // as FwdLaunch::mathv
+    HaloPlan plan;
+    FusedLayout lay;
+    const CUtensorMap *tmap_in;  // input windows
+    const CUtensorMap *tmap_x;   // x neighbourhoods of the tiles
+    cudaStream_t stream;
+};
+
 cudaError_t launch_forward(const FwdLaunch &L);
 cudaError_t launch_producer(const ProducerLaunch &L);
+cudaError_t launch_fused(const FusedLaunch &L);
 cudaError_t launch_backward(const BwdLaunch &L);
 
 // Launches the bounded-wait self-test kernel (see dcn4_selftest_bounded_wait).
@@ -75,6 +92,7 @@ cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t strea
 cudaError_t read_clear_device_error(unsigned *bits);
 cudaError_t read_clear_error_fwd(unsigned *bits);
 cudaError_t read_clear_error_bwd(unsigned *bits);
+cudaError_t read_clear_error_fused(unsigned *bits);
 
 // Shared launch helpers (dcn4_kernels.cu): count one issued kernel; raise a
 // kernel's dynamic shared-memory limit once per (kernel, device); a grid of

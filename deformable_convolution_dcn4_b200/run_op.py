@@ -4,10 +4,11 @@ command profilers (ncu) wrap to capture single kernels.
     python -m deformable_convolution_dcn4_b200.run_op --op forward \
         --workload internimage_bf16 --iters 3 [--N 64] [--algo auto] [--math default]
 
---op: forward, backward, msdcn (MSDCN forward), msdcn_backward, producer.
+--op: forward, backward, msdcn (MSDCN forward), msdcn_backward, producer, fused.
 msdcn / msdcn_backward on a DCNv4 workload use MSDCN inputs of its shape.
 --op producer runs the offset/weight producer (depthwise 3x3 + merged linear)
-on the workload's N, H, W, C, G with seeded sub-network weights.
+on the workload's N, H, W, C, G with seeded sub-network weights; --op fused
+the sub-network fused into the forward (dcn4_fused_forward) on the same shape.
 """
 import argparse
 import sys
@@ -15,13 +16,13 @@ import sys
 import torch
 
 from . import _binding as B
-from .workloads import WORKLOADS, make_inputs, make_producer_inputs
+from .workloads import WORKLOADS, make_fused_inputs, make_inputs, make_producer_inputs
 
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["forward", "backward", "msdcn", "msdcn_backward", "producer"],
-                   default="forward")
+    p.add_argument("--op", choices=["forward", "backward", "msdcn", "msdcn_backward", "producer",
+                                    "fused"], default="forward")
     p.add_argument("--workload", default="internimage_bf16")
     p.add_argument("--iters", type=int, default=3)
     p.add_argument("--N", type=int, default=None)
@@ -39,6 +40,8 @@ def main(argv=None):
     if a.op == "producer":
         d = make_producer_inputs(wl.N, wl.H, wl.W, wl.C, wl.G, wl.kh * wl.kw, wl.dtype,
                                  seed=wl.seed, device="cuda")
+    elif a.op == "fused":
+        d = make_fused_inputs(wl.N, wl.H, wl.W, wl.C, wl.G, wl.dtype, seed=wl.seed, device="cuda")
     else:
         d = make_inputs(wl, (ho, wo), with_grad=a.op in ("backward", "msdcn_backward"),
                         device="cuda")
@@ -52,6 +55,9 @@ def main(argv=None):
                                    d["lin_bias"], group=wl.G, kernel_size=(wl.kh, wl.kw),
                                    stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
                                    algo=a.algo)
+        elif a.op == "fused":
+            B.dcn4_fused_forward(d["input"], d["x"], d["dw_weight"], d["dw_bias"],
+                                 d["lin_weight"], d["lin_bias"], math=a.math, **kw)
         elif a.op == "backward":
             B.dcn4_backward(d["input"], d["offset_weight"], d["grad_out"], math=a.math, **kw)
         elif a.op == "msdcn_backward":

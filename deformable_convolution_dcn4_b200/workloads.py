@@ -106,6 +106,21 @@ def make_producer_inputs(N: int, H: int, W: int, C: int, G: int, K: int = 9,
     return out
 
 
+def make_fused_inputs(N: int, H: int, W: int, C: int, G: int, dtype: str = "bf16",
+                      seed: int = 0, offset_sigma: float = 2.0, device: Optional[str] = None):
+    """Inputs of the fused call (offset/weight sub-network in front of the
+    aggregation): make_producer_inputs(..., seed) for x and the weights, then
+    the sampled map input [N,H,W,C] ~ N(0,1) from a generator seeded seed + 1.
+    """
+    out = make_producer_inputs(N, H, W, C, G, K=9, dtype=dtype, seed=seed,
+                               offset_sigma=offset_sigma)
+    g = torch.Generator().manual_seed(seed + 1)
+    out["input"] = torch.randn((N, H, W, C), generator=g).to(DTYPES[dtype])
+    if device is not None:
+        out = {k: v.to(device) for k, v in out.items()}
+    return out
+
+
 def make_inputs(wl: Workload, out_hw: Tuple[int, int], with_grad: bool = False,
                 device: Optional[str] = None):
     """Returns a dict of tensors in the workload's storage dtype.

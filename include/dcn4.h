@@ -274,6 +274,56 @@ DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
                                           const void *lin_weight, const void *lin_bias,
                                           void *offset_weight, void *stream);
 
+/* Scratch bytes dcn4_fused_forward may need for this desc: 0 when the fused
+ * kernel takes the call's shape and desc->algo (it may still need the scratch
+ * when a pointer is not aligned, see below), else the size of the
+ * offset_weight tensor the two-kernel chain passes through,
+ * N*Ho*Wo*G*kh*kw*3 elements of desc->dtype (none is needed when the call
+ * passes offset_weight_out). */
+DCN4_API dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *bytes);
+
+/* The DCNv4 module's aggregation with its offset/weight sub-network in front
+ * ("(论文速读）DCNv4：高效可变形卷积算子", "方法3. DCN模块的微设计优化": the offset
+ * and weight projections become one linear layer after a depthwise 3x3
+ * convolution): output = dcn4_forward(input, dcn4_offset_producer(x, ...))
+ * with the same desc, without the N*Ho*Wo*G*kh*kw*3 offset_weight tensor
+ * going through global memory when the fused kernel runs.
+ *   input [N][H][W][C] (the sampled map), x [N][H][W][C] (the map the
+ *   offsets and weights are computed from), dw_weight [3][3][C], dw_bias [C],
+ *   lin_weight [G*kh*kw*3][C], lin_bias [G*kh*kw*3], output [N][Ho][Wo][C]:
+ *   device pointers of desc->dtype, owned by the caller. As for the producer,
+ *   Ho == H and Wo == W (else DCN4_ERR_UNSUPPORTED).
+ *   offset_weight_out: NULL, or [N][Ho][Wo][G][kh*kw][3] of desc->dtype, which
+ *   then receives the records the aggregation used (what dcn4_backward takes
+ *   as offset_weight in a training step; one extra write of that tensor).
+ * Result: what the two calls give, records rounded to the data type in
+ * between, fp32 accumulation in both steps.
+ * Kernels: bf16/fp16 with a 3x3 kernel, D*2 in {32, 64} bytes, G a multiple
+ * of 128 / (D*2) (hence C a multiple of 64), C <= 256, 16-byte aligned
+ * input, x, lin_weight and output, a 4-byte aligned offset_weight_out,
+ * desc->weights either mode and a tile that fits shared memory run one
+ * persistent tcgen05 kernel per call: each CTA owns an output tile x a slice
+ * of groups, loads the tile's x neighbourhood by TMA, computes the depthwise
+ * outputs on the CUDA cores, the slice's rows of the linear layer on the
+ * tensor cores (accumulators in tensor memory), and writes the records
+ * straight into the shared-memory slots the gathers read. Every other call
+ * (and DCN4_ALGO_GENERIC or DCN4_ALGO_VECTOR, which select the forward kernel
+ * of the second step) runs dcn4_offset_producer into offset_weight_out, or
+ * when that is NULL into `workspace` (at least
+ * N*Ho*Wo*G*kh*kw*3*sizeof(element) bytes, else DCN4_ERR_WORKSPACE before any
+ * launch; 16-byte aligned to take the tensor-core producer and the staged
+ * forward), and then dcn4_forward on it. The chain's records are the
+ * tensor-core producer's where that applies and the CUDA-core producer's
+ * (h kept in fp32) otherwise, so on shapes the tensor-core producer does not
+ * take the chain and the fused kernel may round a record differently.
+ * DCN4_ALGO_HALO demands the fused kernel (DCN4_ERR_UNSUPPORTED where it does
+ * not apply). */
+DCN4_API dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const void *x,
+                                        const void *dw_weight, const void *dw_bias,
+                                        const void *lin_weight, const void *lin_bias,
+                                        void *output, void *offset_weight_out,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
 /* dcn4_backward for callers that cannot allocate device memory. The paper
  * has no counterpart; this is a deployment convenience. dcn4_backward needs
  * an fp32 scratch buffer for bf16/fp16 that the caller must allocate; callers

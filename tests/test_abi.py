@@ -159,3 +159,24 @@ def test_producer_argument_errors(lib):
     assert lib.dcn4_offset_producer(ctypes.byref(d2), *fake, None) == 2
     bad = _desc(C=10, G=4)
     assert lib.dcn4_offset_producer(ctypes.byref(bad), *fake, None) == 1
+
+
+def test_fused_forward_argument_errors(lib):
+    """dcn4_fused_forward rejects null pointers and a strided output grid, and
+    a call that must take the two-kernel chain (fp32 has no fused kernel)
+    without scratch is refused with DCN4_ERR_WORKSPACE before any launch."""
+    d = _desc()  # fp32, N2 9x11 C16 G4
+    fake = [ctypes.c_void_p(4096)] * 7
+    n = ctypes.c_size_t()
+    assert lib.dcn4_fused_forward_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0
+    assert n.value == 2 * 9 * 11 * 4 * 27 * 4  # the offset_weight tensor, fp32
+    assert lib.dcn4_fused_forward_workspace_size(ctypes.byref(d), None) == 1
+    assert lib.dcn4_fused_forward(ctypes.byref(d), None, *fake[:6], None, None, 0, None) == 1
+    assert lib.dcn4_fused_forward(ctypes.byref(d), *fake[:6], None, None, None, 0, None) == 1
+    assert lib.dcn4_fused_forward(ctypes.byref(_desc(stride=2)), *fake, None, None, 0,
+                                  None) == 2
+    assert lib.dcn4_fused_forward(ctypes.byref(d), *fake, None, None, 0, None) == 3
+    assert lib.dcn4_fused_forward(ctypes.byref(d), *fake, None, ctypes.c_void_p(4096),
+                                  n.value - 1, None) == 3
+    d.algo = B.ALGO_CODE["halo"]  # demands the fused kernel: none for fp32
+    assert lib.dcn4_fused_forward(ctypes.byref(d), *fake, None, None, 0, None) == 2

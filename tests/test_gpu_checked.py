@@ -14,7 +14,8 @@ import torch
 
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200 import build as libbuild
-from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_producer_inputs
+from deformable_convolution_dcn4_b200.workloads import (WORKLOADS, make_fused_inputs,
+                                                        make_producer_inputs)
 
 from parity_util import (TOL, backward_case, f32, forward_case, gpu_forward, msdcn_backward_case,
                          out_hw, scaled_err)
@@ -142,4 +143,24 @@ def test_checked_producer(orc, checked, case, algo):
     prob = orc.problem(N, H, Wd, C, G, k, k, pad=((k - 1) // 2, (k - 1) // 2))
     ref = orc.offset_producer(prob, f32(d["x"]), f32(d["dw_weight"]), f32(d["dw_bias"]),
                               f32(d["lin_weight"]), f32(d["lin_bias"]))
+    assert scaled_err(f32(out), ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("case", [(2, 24, 20, 128, 8, "bf16"), (1, 12, 10, 256, 16, "bf16"),
+                                  (3, 2, 3, 64, 4, "f16"), (1, 20, 21, 64, 2, "bf16")])
+def test_checked_fused_forward(orc, checked, case):
+    """The fused producer + forward kernel (x neighbourhoods, depthwise into
+    the MMA operand, lin_w rows, accumulators into the record slots, the
+    gathers) through the checked build, against the oracle chain."""
+    N, H, Wd, C, G, dtype = case
+    d = make_fused_inputs(N, H, Wd, C, G, dtype=dtype, seed=11, offset_sigma=0.5)
+    dev = {n: t.cuda() for n, t in d.items()}
+    out = B.dcn4_fused_forward(dev["input"], dev["x"], dev["dw_weight"], dev["dw_bias"],
+                               dev["lin_weight"], dev["lin_bias"], group=G, algo="halo")
+    _clear()
+    prob = orc.problem(N, H, Wd, C, G, 3, 3)
+    ow = orc.offset_producer(prob, f32(d["x"]), f32(d["dw_weight"]), f32(d["dw_bias"]),
+                             f32(d["lin_weight"]), f32(d["lin_bias"]))
+    ow = torch.from_numpy(ow).to(d["x"].dtype).float().numpy().reshape(N, H, Wd, G, 9, 3)
+    ref = orc.forward(prob, f32(d["input"]), ow)
     assert scaled_err(f32(out), ref) <= TOL[dtype]
