@@ -15,8 +15,10 @@ with the same L2 flush; they are reported, not counted in the value.
 `configs` times every workload of the table below the same way (median of
 graph replays, L2 flushed before each): forward, backward (fp32 accumulation
 of grad_input across CTAs, the default, and the 16-bit cross-CTA variant
-acc16), MSDCN forward and backward, each with ideal bytes, GB/s, the
-fraction of the HBM peak and the fraction of samples outside the image.
+acc16), MSDCN forward and backward, and the forward with the offset/weight
+sub-network fused in (dcn4_fused_forward, next to the producer + forward
+chain it replaces), each with ideal bytes, GB/s, the fraction of the HBM
+peak and the fraction of samples outside the image.
 The CPU-baseline leg, which runs the oracle, also checks one image of every
 (config, op) against it (scaled max error and an elementwise error with an
 rms floor).
@@ -43,15 +45,16 @@ FLUSH_BYTES = 256 << 20
 
 # (label, workload, ops) timed outside the step; "bwd" is the default
 # backward (fp32 accumulation across CTAs), "bwd_acc16" the 16-bit cross-CTA
-# accumulation, "msbwd" the MSDCN backward (default math)
+# accumulation, "msbwd" the MSDCN backward (default math), "fused" the
+# forward with the offset/weight sub-network in front (one call)
 CONFIG_TABLE = [
     ("c1", "tiny_f32", ["fwd", "bwd"]),
-    ("c2", "internimage_bf16", ["fwd", "bwd", "bwd_acc16", "msfwd", "msbwd"]),
+    ("c2", "internimage_bf16", ["fwd", "bwd", "bwd_acc16", "msfwd", "msbwd", "fused"]),
     ("c2", "internimage_f32", ["fwd", "bwd"]),
     ("c3a", "ldm64_f16", ["fwd", "bwd", "bwd_acc16"]),
     ("c3b", "ldm32_f16", ["fwd", "bwd", "bwd_acc16"]),
     ("c4", "flowdcn_msdcn_bf16", ["msfwd", "msbwd"]),
-    ("c5", "highres_bf16", ["fwd", "bwd", "bwd_acc16"]),
+    ("c5", "highres_bf16", ["fwd", "bwd", "bwd_acc16", "fused"]),
 ]
 
 
@@ -516,9 +519,13 @@ def op_ideal_bytes(wl, Ho, Wo, op):
     nout = wl.N * Ho * Wo * wl.C
     now = wl.N * Ho * Wo * wl.G * wl.K * 3
     nraw = wl.N * Ho * Wo * wl.G
+    J = wl.G * wl.K * 3
     elems = {"fwd": nin + nout + now, "bwd": 2 * nin + nout + 2 * now,
              "bwd_acc16": 2 * nin + nout + 2 * now, "msfwd": nin + nout + now + nraw,
-             "msbwd": 2 * nin + nout + 2 * now + 2 * nraw}[op]
+             "msbwd": 2 * nin + nout + 2 * now + 2 * nraw,
+             # input and x read once, output written once, the sub-network's
+             # weights; the records stay on chip
+             "fused": 2 * nin + nout + 10 * wl.C + J * wl.C + J}[op]
     return elems * eb
 
 
@@ -550,7 +557,7 @@ def time_configs(dcn, flush, stream, peak, peak_kind):
     samples keep one image's inputs and GPU outputs (host, fp32) per op for the
     oracle check of the CPU-baseline leg."""
     import torch
-    from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
+    from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_fused_inputs, make_inputs
     table, samples = {}, []
     dev = flush.device
     for label, wname, ops in CONFIG_TABLE:
@@ -562,18 +569,30 @@ def time_configs(dcn, flush, stream, peak, peak_kind):
                   dilation=wl.dilation, offset_scale=wl.offset_scale)
         entry = {"label": label, "shape": f"N{wl.N} {wl.H}x{wl.W} C{wl.C} G{wl.G} (D{wl.D}) "
                                           f"{wl.dtype}", "ops": {}}
-        needs_dcn = any(not o.startswith("ms") for o in ops)
+        needs_dcn = any(not o.startswith("ms") and o != "fused" for o in ops)
         needs_ms = any(o.startswith("ms") for o in ops)
         dh = make_inputs(wl, (Ho, Wo), with_grad=True) if needs_dcn and wl.kind != "msdcn" else None
         mwl = wl if wl.kind == "msdcn" else msdcn_variant(wl)
         mh = make_inputs(mwl, (Ho, Wo), with_grad=True) if needs_ms else None
         d = {k: v.to(dev) for k, v in dh.items()} if dh else None
         m = {k: (v if k == "s0" else v.to(dev)) for k, v in mh.items()} if mh else None
+        f = None
+        if "fused" in ops:
+            f = make_fused_inputs(wl.N, wl.H, wl.W, wl.C, wl.G, wl.dtype, seed=wl.seed,
+                                  device=dev)
+            # the records the call uses (written out once, untimed): the oob
+            # statistic and the oracle check of the aggregation read them
+            f["offset_weight"] = torch.empty((wl.N, Ho, Wo, wl.G, wl.K, 3), dtype=f["x"].dtype,
+                                             device=dev)
+            dcn.dcn4_fused_forward(f["input"], f["x"], f["dw_weight"], f["dw_bias"],
+                                   f["lin_weight"], f["lin_bias"],
+                                   offset_weight_out=f["offset_weight"], **kw)
         ws = torch.empty(max(wl.N * wl.H * wl.W * wl.C * 4, 16), dtype=torch.uint8, device=dev)
         n_s = wl.N - 1  # the image the oracle checks
         for op in ops:
-            src = m if op.startswith("ms") else d
+            src = m if op.startswith("ms") else f if op == "fused" else d
             x = src["input"]
+            chain_ms = None
             if op == "fwd":
                 outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
                 fn = lambda: dcn.dcn4_forward(d["input"], d["offset_weight"], out=outs[0], **kw)
@@ -587,6 +606,20 @@ def time_configs(dcn, flush, stream, peak, peak_kind):
                 outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
                 fn = lambda: dcn.msdcn_forward(m["input"], m["dir_weight"], m["scale_raw"],
                                                m["s0"], mwl.smax, out=outs[0], **kw)
+            elif op == "fused":
+                outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
+                fn = lambda: dcn.dcn4_fused_forward(f["input"], f["x"], f["dw_weight"],
+                                                    f["dw_bias"], f["lin_weight"],
+                                                    f["lin_bias"], out=outs[0], **kw)
+                # the two-kernel chain it replaces, same inputs, same flush
+                rec_buf = torch.empty_like(f["offset_weight"])
+                chain_out = torch.empty_like(outs[0])
+
+                def chain():
+                    dcn.dcn4_offset_producer(f["x"], f["dw_weight"], f["dw_bias"],
+                                             f["lin_weight"], f["lin_bias"], out=rec_buf, **kw)
+                    dcn.dcn4_forward(f["input"], rec_buf, out=chain_out, **kw)
+                chain_ms = graph_median_ms(chain, flush, stream)
             else:  # msbwd
                 outs = [torch.empty_like(x), torch.empty_like(m["dir_weight"]),
                         torch.empty_like(m["scale_raw"])]
@@ -604,19 +637,31 @@ def time_configs(dcn, flush, stream, peak, peak_kind):
                    f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4), "launches": launches,
                    "oob_fraction": oob_fraction(mwl if op.startswith("ms") else wl, src, Ho, Wo,
                                                 op.startswith("ms"))}
-            if op in ("fwd", "msfwd"):
+            if op in ("fwd", "msfwd", "fused"):
                 rec["Gsample_ch_per_s"] = round(samples_ch(wl, Ho, Wo) / (ms * 1e-3) / 1e9, 1)
+            if chain_ms is not None:
+                rec["producer_plus_forward_ms"] = round(chain_ms, 5)
+                rec["speedup_vs_chain"] = round(chain_ms / ms, 3)
             entry["ops"][op] = rec
             torch.cuda.synchronize()
             samples.append({"key": f"{label}_{wname}", "op": op,
                             "wl": (mwl if op.startswith("ms") else wl).replace(N=1),
-                            "inputs": {k: (v if k == "s0" else v[n_s:n_s + 1].float().cpu())
-                                       for k, v in src.items()},
+                            "inputs": {k: sample_of(op, k, v, n_s) for k, v in src.items()},
                             "outputs": [t[n_s:n_s + 1].float().cpu() for t in outs]})
         table[f"{label}_{wname}"] = entry
-        del d, m, ws, dh, mh
+        del d, m, f, ws, dh, mh
         torch.cuda.empty_cache()
     return table, samples
+
+
+def sample_of(op, k, v, n):
+    """Image n of an input tensor (host, fp32) for the oracle check; s0 and
+    the fused call's sub-network weights as they are."""
+    if k == "s0":
+        return v
+    if op == "fused" and v.dim() < 4:
+        return v.float().cpu()
+    return v[n:n + 1].float().cpu()
 
 
 def oracle_config_checks(samples):
@@ -640,6 +685,15 @@ def oracle_config_checks(samples):
         elif op == "msfwd":
             refs = [orc.msdcn_forward(prob, a["input"], a["dir_weight"], a["scale_raw"],
                                       a["s0"].numpy(), wl.smax)]
+        elif op == "fused":
+            # the aggregation on the records the call used; those records
+            # against the oracle's producer
+            refs = [orc.forward(prob, a["input"], a["offset_weight"])]
+            rec_ref = orc.offset_producer(prob, a["x"], a["dw_weight"], a["dw_bias"],
+                                          a["lin_weight"], a["lin_bias"])
+            rd = np.abs(a["offset_weight"].reshape(rec_ref.shape) - rec_ref)
+            res.setdefault(smp["key"], {}).setdefault(op, {})["records_max_scaled_err"] = \
+                float(f"{rd.max() / np.abs(rec_ref).max():.3e}")
         else:
             refs = list(orc.msdcn_backward(prob, a["input"], a["dir_weight"], a["scale_raw"],
                                            a["s0"].numpy(), wl.smax, a["grad_out"]))
@@ -652,8 +706,9 @@ def oracle_config_checks(samples):
             rms = float(np.sqrt(np.mean(ref * ref)))
             scaled = max(scaled, float(diff.max() / scale) if scale > 0 else float(diff.max()))
             elem = max(elem, float((diff / (np.abs(ref) + rms)).max()) if rms > 0 else 0.0)
-        res.setdefault(smp["key"], {})[op] = {"max_scaled_err": float(f"{scaled:.3e}"),
-                                              "max_rel_err_rms_floor": float(f"{elem:.3e}")}
+        res.setdefault(smp["key"], {}).setdefault(op, {}).update(
+            {"max_scaled_err": float(f"{scaled:.3e}"),
+             "max_rel_err_rms_floor": float(f"{elem:.3e}")})
     return res
 
 
