@@ -282,6 +282,44 @@ bool plan_fused(const Geometry &g, int eb, HaloPlan *out, FusedLayout *lay) {
     return false;
 }
 
+// Tiling and shared-memory carve-up of the 2-D tiled tensor-core producer:
+// 16-bit data, C a multiple of 64 (whole blocks of 8 depthwise chunks) and at
+// most 256 (one TMA box row), J <= 256 outputs in whole 16-byte rows (the TMA
+// store's inner box). Tiles of at most 128 pixels (the MMA's M), 16 x 8 first.
+bool plan_producer_2d(int H, int W, int C, int J, int NP, ProducerTc2dLayout *out) {
+    if (C % 64 != 0 || C > 256 || J > 256 || (J * 2) % 16 != 0) return false;
+    const int smem_max = max_smem_optin();
+    static const int cands[][2] = {{16, 8}, {8, 16}, {8, 8}, {8, 4}, {4, 8}, {4, 4},
+                                   {4, 2},  {2, 4},  {2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    for (auto &c : cands) {
+        const int TH = c[0] < H ? c[0] : H;
+        const int TW = c[1] < pow2_ceil(W) ? c[1] : pow2_ceil(W);
+        if (TH * TW > 128) continue;
+        ProducerTc2dLayout L;
+        L.TH = TH;
+        L.TW = TW;
+        L.lgTW = log2_exact(TW);
+        L.tiles_h = (H + TH - 1) / TH;
+        L.tiles_w = (W + TW - 1) / TW;
+        L.x_off = 0;
+        L.x_bytes = (TH + 2) * (TW + 2) * C * 2;
+        L.a_off = ceil_to(L.x_off + L.x_bytes, 1024);
+        L.b_off = L.a_off + 128 * C * 2;
+        L.o_off = ceil_to(L.b_off + NP * C * 2, 1024);
+        L.dwt_off = ceil_to(L.o_off + TH * TW * J * 2, 16);
+        L.dwb_off = ceil_to(L.dwt_off + 9 * C * 2, 16);
+        L.linb_off = L.dwb_off + C * 4;
+        L.bar_off = ceil_to(L.linb_off + NP * 4, 16);
+        L.bytes = L.bar_off + 32;
+        L.tmem_cols = 32;
+        while (L.tmem_cols < NP) L.tmem_cols <<= 1;
+        if (L.bytes > smem_max) continue;
+        *out = L;
+        return true;
+    }
+    return false;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -467,6 +505,19 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
            aligned16(offset_weight) && lay.bytes <= max_smem_optin();
     L.lay = lay;
     if (!L.tc && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+    // the 2-D tiled kernel where it applies (x by TMA tile, sliding-window
+    // depthwise, one TMA store per tile)
+    CUtensorMap map_x, map_out;
+    memset(&map_x, 0, sizeof(map_x));
+    memset(&map_out, 0, sizeof(map_out));
+    L.tc2d = L.tc && plan_producer_2d(g.H, g.W, g.C, L.pg.J, L.pg.NP, &L.lay2) &&
+             encode_map(L.dtype, x, g.N, g.H, g.W, g.C, g.C, L.lay2.TW + 2, L.lay2.TH + 2,
+                        &map_x) &&
+             encode_map(L.dtype, offset_weight, g.N, g.H, g.W, L.pg.J, L.pg.J, L.lay2.TW,
+                        L.lay2.TH, &map_out) &&
+             (long long)g.N * L.lay2.tiles_h * L.lay2.tiles_w <= 0x7fffffffLL;
+    L.tmap_x = &map_x;
+    L.tmap_out = &map_out;
     if (!L.tc && (L.pg.npix + kProducerPixels - 1) / kProducerPixels > 0x7fffffffLL)
         return DCN4_ERR_UNSUPPORTED;
     return cuda_status(launch_producer(L));

@@ -132,6 +132,23 @@ struct HaloPlan {
     int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)
 };
 
+// Tiling and shared-memory carve-up of the 2-D tiled tensor-core producer
+// (byte offsets from the start of dynamic shared memory; chosen on the host).
+struct ProducerTc2dLayout {
+    int TH, TW, lgTW;      // pixel tile (TW a power of two, TH * TW <= 128)
+    int tiles_h, tiles_w;  // tiles per image
+    int x_off, x_bytes;    // x neighbourhood of a tile, (TH+2) x (TW+2) pixels x C
+    int a_off;             // depthwise outputs: 128 rows x C, tcgen05 core matrices
+    int b_off;             // lin_w: NP rows x C, core matrices (rows >= J zero)
+    int o_off;             // the tile's outputs, TH*TW rows of J values (TMA store source)
+    int dwt_off;           // dw_weight [9][C] in the data type
+    int dwb_off;           // dw_bias [C] in fp32
+    int linb_off;          // lin_bias [NP] in fp32 (zero past J)
+    int bar_off;           // two mbarriers and the tensor-memory address
+    int bytes;             // dynamic shared memory of one CTA
+    int tmem_cols;         // a power of two >= NP, >= 32
+};
+
 // Shared-memory carve-up of the fused producer + forward kernel (byte offsets
 // from the start of dynamic shared memory; chosen on the host).
 struct FusedLayout {
@@ -479,6 +496,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
+}
+
+// TMA tile store shared -> global of a 4-D box (coordinates >= 0; elements
+// past the tensor's extent are not written); one bulk group per call.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
 // Plain (untiled) bulk copy global -> shared; 16-byte aligned addresses and size.

@@ -57,81 +57,12 @@ __device__ __forceinline__ TileCoord fused_coord(int u, const Geometry &g, const
     return c;
 }
 
-// Depthwise 3x3 outputs of the tile's pixels (A row r = tile pixel
-// ty*TW + tx) from the staged neighbourhood xs ((TH+2) x (TW+2) pixels of C
-// values, the tile's top-left pixel at (1, 1)): bias, then the nine taps in
-// row-major order as fp32 fma of the exact 16-bit products, rounded to T.
-// Rows past the tile are left alone (zero since the CTA started).
-// One item per thread: an 8-channel chunk q of one tile column tx over S
-// consecutive rows. The item walks the S+2 staged rows it needs once, and
-// each row's three vectors feed up to three output rows, so a staged vector
-// is read (S+2)*3/S times per output row instead of 9, and the S*8
-// accumulators give independent fma chains. C is a multiple of 64 (the
-// host's plan: 128-byte staged pixels of whole groups). Eight consecutive
-// items (one shared-memory phase) take 8 different chunks l = 0..7 of one
-// block and columns (l + kx) mod TW: their staged reads hit 8 different
-// bank quads (the pixel stride is a multiple of 128 bytes), and so do their
-// core-matrix stores when TW >= 8.
-template <typename T, int NW, int S>
-__device__ __forceinline__ void fused_depthwise(const unsigned char *xs, unsigned char *a,
-                                                const T *dwt, const float *dwb, int C, int TH,
-                                                int TW, int lgTW, const unsigned char *sbase) {
-    (void)sbase;
-    constexpr int NT = NW * 32;
-    const int XW = TW + 2;  // staged pixels per row
-    const int PX = C * 2;   // bytes per staged pixel
-    const int QB = C / 64;  // blocks of 8 chunks
-    const int items = (TH + S - 1) / S * TW * QB * 8;
-    for (int it = threadIdx.x; it < items; it += NT) {
-        const int l = it & 7;
-        int rest = it >> 3;
-        const int qb = rest % QB;
-        rest /= QB;
-        const int kx = rest & (TW - 1), seg = rest >> lgTW;
-        const int q = qb * 8 + l, tx = (l + kx) & (TW - 1), y0 = seg * S;
-        const int ns = min(S, TH - y0);
-        uint4 wv[9];
-#pragma unroll
-        for (int k = 0; k < 9; ++k) wv[k] = *reinterpret_cast<const uint4 *>(dwt + k * C + q * 8);
-        const float4 *bb = reinterpret_cast<const float4 *>(dwb + q * 8);
-        const float4 b0 = bb[0], b1 = bb[1];
-        float acc[S][8];
-#pragma unroll
-        for (int y = 0; y < S; ++y) {
-            acc[y][0] = b0.x, acc[y][1] = b0.y, acc[y][2] = b0.z, acc[y][3] = b0.w;
-            acc[y][4] = b1.x, acc[y][5] = b1.y, acc[y][6] = b1.z, acc[y][7] = b1.w;
-        }
-        // staged row y0 + r, columns tx .. tx + 2 (tile rows y0 + r - 1)
-        const unsigned char *col = xs + ((size_t)y0 * XW + tx) * PX + q * 16;
-#pragma unroll
-        for (int r = 0; r < S + 2; ++r) {
-            if (r < ns + 2) {
-                uint4 xv[3];
-#pragma unroll
-                for (int j = 0; j < 3; ++j) xv[j] = DCN4_LDS16(col + (r * XW + j) * PX, sbase);
-#pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    const int y = r - i;  // output row fed by tap row i
-                    if (y < 0 || y >= S) continue;
-#pragma unroll
-                    for (int j = 0; j < 3; ++j) MixedFma8<T>::run(acc[y], xv[j], wv[i * 3 + j]);
-                }
-            }
-        }
-#pragma unroll
-        for (int y = 0; y < S; ++y) {
-            if (y >= ns) continue;
-            unsigned char *dst = a + core_off((y0 + y) * TW + tx, q, C);
-            if (DCN4_SMEM_OK(dst, 16, sbase)) *reinterpret_cast<uint4 *>(dst) = pack8<T>(acc[y]);
-        }
-    }
-}
-
 // Accumulators -> records: warp w reads tensor-memory lanes 32 (w & 3) ..
-// +31 (tile pixels) and every (NW / 4)-th 16-column chunk from w >> 2, adds
-// the bias and rounds; pixel r's outputs land at the start of its slot, in
-// the forward's record order (group, tap, (dx, dy, m)). The slot stride is an
-// odd multiple of 16 bytes, so the 16-byte stores are free of bank conflicts.
+// +31 (tile pixels) and every (NW / 4)-th 32-column chunk from w >> 2 (a
+// 16-column tail when NP % 32 != 0), adds the bias and rounds; pixel r's
+// outputs land at the start of its slot, in the forward's record order
+// (group, tap, (dx, dy, m)). The slot stride is an odd multiple of 16 bytes,
+// so the 16-byte stores are free of bank conflicts.
 template <typename T, int NW>
 __device__ __forceinline__ void fused_epilogue(uint32_t tmem, const float *linb,
                                                unsigned char *slots, int slot_bytes, int NP,
@@ -139,18 +70,26 @@ __device__ __forceinline__ void fused_epilogue(uint32_t tmem, const float *linb,
     (void)sbase;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = 32 * (warp & 3) + lane;
-    for (int c16 = warp >> 2; c16 < NP / 16; c16 += NW / 4) {
+    const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    auto store8 = [&](const float *v, int c0) {
+        if (r >= npx) return;
+        float fo[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) fo[k] = v[k] + linb[c0 + k];
+        unsigned char *dst = slots + (size_t)r * slot_bytes + c0 * 2;
+        if (DCN4_SMEM_OK(dst, 16, sbase)) *reinterpret_cast<uint4 *>(dst) = pack8<T>(fo);
+    };
+    for (int c32 = warp >> 2; c32 < NP / 32; c32 += NW / 4) {
+        float v[32];
+        tc_ld_32(trow + c32 * 32, v);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) store8(v + 8 * h, c32 * 32 + 8 * h);
+    }
+    if ((NP & 16) && (warp >> 2) == (NP / 32) % (NW / 4)) {
         float v[16];
-        tc_ld_16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c16 * 16, v);
-        if (r >= npx) continue;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float fo[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) fo[k] = v[8 * h + k] + linb[c16 * 16 + 8 * h + k];
-            unsigned char *dst = slots + (size_t)r * slot_bytes + c16 * 32 + h * 16;
-            if (DCN4_SMEM_OK(dst, 16, sbase)) *reinterpret_cast<uint4 *>(dst) = pack8<T>(fo);
-        }
+        tc_ld_16(trow + (NP / 32) * 32, v);
+        store8(v, (NP / 32) * 32);
+        store8(v + 8, (NP / 32) * 32 + 8);
     }
 }
 
@@ -247,7 +186,7 @@ __global__ void __launch_bounds__(NW * 32, 1)
         if (!mbar_wait_bounded(x_bar, (uint32_t)k & 1u, kWaitLimitNs)) ok = false;
         else if (tid == 0) ++x_done;
         if (__syncthreads_or(!ok)) return false;
-        fused_depthwise<T, NW, 4>(xs, abuf, dwt, dwb, C, pl.TH, pl.TW, pl.lgTW, smem);
+        depthwise_tile<T, NW, 4>(xs, abuf, dwt, dwb, C, pl.TH, pl.TW, pl.lgTW, smem);
         fence_async_smem();
         __syncthreads();
         if (tid == 0) {

@@ -58,6 +58,21 @@ cudaError_t launch_producer_t(const ProducerLaunch &L) {
     const T *dw_b = static_cast<const T *>(L.dw_b), *lin_w = static_cast<const T *>(L.lin_w);
     const T *lin_b = static_cast<const T *>(L.lin_b);
     T *out = static_cast<T *>(L.out);
+    if (L.tc2d) {
+        if constexpr (sizeof(T) == 2) {
+            constexpr int NW = 16;
+            auto k = producer_tc2d_kernel<T, NW>;
+            cudaError_t e = allow_smem(reinterpret_cast<const void *>(k), L.lay2.bytes);
+            if (e != cudaSuccess) return e;
+            const int tiles = L.pg.N * L.lay2.tiles_h * L.lay2.tiles_w;
+            const int grid = tiles < sm_count() ? tiles : sm_count();
+            k<<<grid, NW * 32, L.lay2.bytes, L.stream>>>(*L.tmap_x, *L.tmap_out, L.pg, L.lay2,
+                                                        dw_w, dw_b, lin_w, lin_b);
+            count_launch();
+            return cudaGetLastError();
+        }
+        return cudaErrorInvalidValue;
+    }
     if (L.tc) {
         if constexpr (sizeof(T) == 2) {
             const ProducerTcLayout &lay = L.lay;

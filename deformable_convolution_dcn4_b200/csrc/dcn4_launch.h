@@ -59,8 +59,12 @@ struct ProducerLaunch {
     Dtype dtype;
     const void *x, *dw_w, *dw_b, *lin_w, *lin_b;
     void *out;
-    bool tc;  // tensor-core kernel (16-bit data), else the generic kernel
-    ProducerTcLayout lay;  // tensor-core kernel only
+    bool tc;    // tensor-core kernel over pixel ranges (16-bit data), else the generic kernel
+    bool tc2d;  // 2-D tiled tensor-core kernel (takes precedence over tc)
+    ProducerTcLayout lay;      // tc only
+    ProducerTc2dLayout lay2;   // tc2d only
+    const CUtensorMap *tmap_x;    // tc2d: x neighbourhoods of the tiles
+    const CUtensorMap *tmap_out;  // tc2d: the tiles' output rows
     cudaStream_t stream;
 };
 

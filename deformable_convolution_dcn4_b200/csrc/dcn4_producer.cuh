@@ -93,6 +93,24 @@ __device__ __forceinline__ void tc_ld_16(uint32_t taddr, float *v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 32 consecutive 32-bit columns: thread t gets lane (base lane + t).
+__device__ __forceinline__ void tc_ld_32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Bulk copy shared -> global (16-byte aligned addresses and size).
 __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
@@ -152,6 +170,76 @@ DCN4_MIXED_FMA8("f16", __half)
 // K-major core-matrix tile whose rows hold C channels.
 __device__ __forceinline__ uint32_t core_off(int r, int q, int C) {
     return (uint32_t)((r >> 3) * (C * 16) + q * 128 + (r & 7) * 16);
+}
+
+// Depthwise 3x3 outputs of the tile's pixels (A row r = tile pixel
+// ty*TW + tx) from the staged neighbourhood xs ((TH+2) x (TW+2) pixels of C
+// values, the tile's top-left pixel at (1, 1)): bias, then the nine taps in
+// row-major order as fp32 fma of the exact 16-bit products, rounded to T.
+// Rows past the tile are left alone (zero since the CTA started).
+// One item per thread: an 8-channel chunk q of one tile column tx over S
+// consecutive rows. The item walks the S+2 staged rows it needs once, and
+// each row's three vectors feed up to three output rows, so a staged vector
+// is read (S+2)*3/S times per output row instead of 9, and the S*8
+// accumulators give independent fma chains. C is a multiple of 64 (the
+// host's plan: 128-byte staged pixels of whole groups). Eight consecutive
+// items (one shared-memory phase) take 8 different chunks l = 0..7 of one
+// block and columns (l + kx) mod TW: their staged reads hit 8 different
+// bank quads (the pixel stride is a multiple of 128 bytes), and so do their
+// core-matrix stores when TW >= 8.
+template <typename T, int NW, int S>
+__device__ __forceinline__ void depthwise_tile(const unsigned char *xs, unsigned char *a,
+                                                const T *dwt, const float *dwb, int C, int TH,
+                                                int TW, int lgTW, const unsigned char *sbase) {
+    (void)sbase;
+    constexpr int NT = NW * 32;
+    const int XW = TW + 2;  // staged pixels per row
+    const int PX = C * 2;   // bytes per staged pixel
+    const int QB = C / 64;  // blocks of 8 chunks
+    const int items = (TH + S - 1) / S * TW * QB * 8;
+    for (int it = threadIdx.x; it < items; it += NT) {
+        const int l = it & 7;
+        int rest = it >> 3;
+        const int qb = rest % QB;
+        rest /= QB;
+        const int kx = rest & (TW - 1), seg = rest >> lgTW;
+        const int q = qb * 8 + l, tx = (l + kx) & (TW - 1), y0 = seg * S;
+        const int ns = min(S, TH - y0);
+        uint4 wv[9];
+#pragma unroll
+        for (int k = 0; k < 9; ++k) wv[k] = *reinterpret_cast<const uint4 *>(dwt + k * C + q * 8);
+        const float4 *bb = reinterpret_cast<const float4 *>(dwb + q * 8);
+        const float4 b0 = bb[0], b1 = bb[1];
+        float acc[S][8];
+#pragma unroll
+        for (int y = 0; y < S; ++y) {
+            acc[y][0] = b0.x, acc[y][1] = b0.y, acc[y][2] = b0.z, acc[y][3] = b0.w;
+            acc[y][4] = b1.x, acc[y][5] = b1.y, acc[y][6] = b1.z, acc[y][7] = b1.w;
+        }
+        // staged row y0 + r, columns tx .. tx + 2 (tile rows y0 + r - 1)
+        const unsigned char *col = xs + ((size_t)y0 * XW + tx) * PX + q * 16;
+#pragma unroll
+        for (int r = 0; r < S + 2; ++r) {
+            if (r < ns + 2) {
+                uint4 xv[3];
+#pragma unroll
+                for (int j = 0; j < 3; ++j) xv[j] = DCN4_LDS16(col + (r * XW + j) * PX, sbase);
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {
+                    const int y = r - i;  // output row fed by tap row i
+                    if (y < 0 || y >= S) continue;
+#pragma unroll
+                    for (int j = 0; j < 3; ++j) MixedFma8<T>::run(acc[y], xv[j], wv[i * 3 + j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int y = 0; y < S; ++y) {
+            if (y >= ns) continue;
+            unsigned char *dst = a + core_off((y0 + y) * TW + tx, q, C);
+            if (DCN4_SMEM_OK(dst, 16, sbase)) *reinterpret_cast<uint4 *>(dst) = pack8<T>(acc[y]);
+        }
+    }
 }
 
 template <typename T, int NW>
@@ -430,6 +518,174 @@ __global__ void __launch_bounds__(NW * 32, 1)
         if (inflight >= 0)
             mbar_wait_bounded(x_bar0 + 8 * inflight,
                               L.x_nbuf == 2 ? ((iter + 1) >> 1) & 1 : (iter + 1) & 1, kWaitLimitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(L.tmem_cols)
+                     : "memory");
+    }
+}
+
+// 2-D tiled tensor-core producer (bf16 / fp16, C a multiple of 64, J <= 256,
+// whole 16-byte output rows): one CTA per SM walks TH x TW pixel tiles. Per
+// tile, x's (TH+2) x (TW+2) neighbourhood arrives by one TMA tile load whose
+// zero fill is the depthwise padding; the warps compute h with depthwise_tile
+// (each staged vector read 4.5 times per output row instead of 9); one thread
+// issues the C/16 MMAs (M = 128, N = NP, all J outputs) and the next tile's x
+// load; the warps read the accumulators back, add the bias, round, and stage
+// the tile's TH*TW rows of J values, which leave in one TMA tile store
+// (columns and rows past the image are not written). Every wait is bounded.
+template <typename T, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
+    producer_tc2d_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                         const __grid_constant__ CUtensorMap tmap_out, ProducerGeo pg,
+                         ProducerTc2dLayout L, const T *__restrict__ dw_w,
+                         const T *__restrict__ dw_b, const T *__restrict__ lin_w,
+                         const T *__restrict__ lin_b) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    constexpr int NT = NW * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int C = pg.C, J = pg.J, NP = pg.NP, Q = C / 8;
+    const int npx = L.TH * L.TW;
+    const int ntiles = pg.N * L.tiles_h * L.tiles_w;
+    unsigned char *xs = smem + L.x_off, *abuf = smem + L.a_off, *obuf = smem + L.o_off;
+    T *dwt = reinterpret_cast<T *>(smem + L.dwt_off);
+    float *dwb = reinterpret_cast<float *>(smem + L.dwb_off);
+    float *linb = reinterpret_cast<float *>(smem + L.linb_off);
+    const uint32_t x_bar = smem_u32(smem + L.bar_off), mma_bar = x_bar + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.bar_off + 16);
+    const unsigned long long lw_b = (unsigned long long)J * C * 2;
+    (void)lw_b;
+
+    // resident operands; rows of h past the tile zero for good
+    for (int i = tid; i < NP * Q; i += NT) {
+        const int n = i / Q, q = i - n * Q;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < J) v = DCN4_LDG16(lin_w + (size_t)n * C + q * 8, lin_w, lw_b);
+        if (DCN4_SMEM_OK(smem + L.b_off + core_off(n, q, C), 16, smem))
+            *reinterpret_cast<uint4 *>(smem + L.b_off + core_off(n, q, C)) = v;
+    }
+    for (int i = npx * Q + tid; i < 128 * Q; i += NT) {
+        const int r = i / Q, q = i - r * Q;
+        if (DCN4_SMEM_OK(abuf + core_off(r, q, C), 16, smem))
+            *reinterpret_cast<uint4 *>(abuf + core_off(r, q, C)) = make_uint4(0, 0, 0, 0);
+    }
+    if (DCN4_SMEM_OK(dwt, 9 * C * 2, smem) && DCN4_SMEM_OK(dwb, C * 4, smem) &&
+        DCN4_SMEM_OK(linb, NP * 4, smem)) {
+        for (int i = tid; i < 9 * C; i += NT) dwt[i] = dw_w[i];
+        for (int i = tid; i < C; i += NT) dwb[i] = Elem<T>::to_f(dw_b[i]);
+        for (int i = tid; i < NP; i += NT) linb[i] = i < J ? Elem<T>::to_f(lin_b[i]) : 0.f;
+    }
+    if (tid == 0) {
+        mbar_init(x_bar, 1);
+        mbar_init(mma_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(L.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t idesc = umma_idesc_f16(std::is_same<T, __nv_bfloat16>::value, 128, NP);
+    const uint32_t a_base = smem_u32(abuf), b_base = smem_u32(smem + L.b_off);
+
+    // tile t: image n, output rows ho0.., columns wo0..
+    auto coord = [&](int t, int &n, int &ho0, int &wo0) {
+        const int tw = t % L.tiles_w;
+        t /= L.tiles_w;
+        ho0 = (t % L.tiles_h) * L.TH;
+        n = t / L.tiles_h;
+        wo0 = tw * L.TW;
+    };
+    // thread 0 issues every copy and MMA and counts them (for the drain on an
+    // expired wait)
+    int x_issued = 0, x_done = 0, mma_issued = 0, mma_done = 0;
+    auto issue_x = [&](int t) {
+        int n, ho0, wo0;
+        coord(t, n, ho0, wo0);
+        fence_async_smem();
+        mbar_arrive_expect_tx(x_bar, (uint32_t)L.x_bytes);
+        if (DCN4_SMEM_OK(xs, (unsigned)L.x_bytes, smem))
+            tma_load_4d(smem_u32(xs), &tmap_x, 0, wo0 - 1, ho0 - 1, n, x_bar);
+        ++x_issued;
+    };
+    if (tid == 0 && (int)blockIdx.x < ntiles) issue_x(blockIdx.x);
+
+    bool ok = true;
+    int k = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+        const uint32_t par = (uint32_t)k & 1u;
+        if (!mbar_wait_bounded(x_bar, par, kWaitLimitNs)) ok = false;
+        else if (tid == 0) ++x_done;
+        if (__syncthreads_or(!ok)) break;
+        depthwise_tile<T, NW, 4>(xs, abuf, dwt, dwb, C, L.TH, L.TW, L.lgTW, smem);
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            if (t + (int)gridDim.x < ntiles) issue_x(t + gridDim.x);
+            tc_fence_after();
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc_mma_f16(tmem, umma_desc_kmajor(a_base + kk * 256, 128, C * 16),
+                           umma_desc_kmajor(b_base + kk * 256, 128, C * 16), idesc, kk > 0);
+            tc_commit(mma_bar);
+            ++mma_issued;
+            bulk_wait_read();  // the previous tile's store has read the staged rows
+        }
+        if (!mbar_wait_bounded(mma_bar, par, kWaitLimitNs)) ok = false;
+        else if (tid == 0) ++mma_done;
+        if (__syncthreads_or(!ok)) break;
+        tc_fence_after();
+
+        // accumulators -> staged rows (row stride J*2 bytes, a multiple of 16):
+        // 32-column reads (one wait each), a 16-column tail when NP % 32 != 0
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        auto stage8 = [&](const float *v, int c0) {
+            if (r >= npx || c0 >= J) return;
+            float fo[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) fo[e] = v[e] + linb[c0 + e];
+            unsigned char *dst = obuf + (size_t)r * J * 2 + c0 * 2;
+            if (DCN4_SMEM_OK(dst, 16, smem)) *reinterpret_cast<uint4 *>(dst) = pack8<T>(fo);
+        };
+        for (int c32 = warp >> 2; c32 < NP / 32; c32 += NW / 4) {
+            float v[32];
+            tc_ld_32(trow + c32 * 32, v);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) stage8(v + 8 * h, c32 * 32 + 8 * h);
+        }
+        if ((NP & 16) && (warp >> 2) == (NP / 32) % (NW / 4)) {
+            float v[16];
+            tc_ld_16(trow + (NP / 32) * 32, v);
+            stage8(v, (NP / 32) * 32);
+            stage8(v + 8, (NP / 32) * 32 + 8);
+        }
+        tc_fence_before();
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            int n, ho0, wo0;
+            coord(t, n, ho0, wo0);
+            if (DCN4_SMEM_OK(obuf, (unsigned)npx * J * 2, smem))
+                tma_store_4d(&tmap_out, smem_u32(obuf), 0, wo0, ho0, n);
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+    if (tid == 0 && !ok) {
+        atomicOr(&g_error_word, kErrTimeout);
+        if (x_issued > x_done) mbar_wait_bounded(x_bar, (uint32_t)(x_issued - 1) & 1u, kWaitLimitNs);
+        if (mma_issued > mma_done)
+            mbar_wait_bounded(mma_bar, (uint32_t)(mma_issued - 1) & 1u, kWaitLimitNs);
     }
     tc_fence_before();
     __syncthreads();
