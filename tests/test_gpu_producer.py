@@ -31,6 +31,12 @@ CASES = {
     "ldm_f16": (1, 8, 8, 320, 20, 3, "f16", False),
     # C not a multiple of 16
     "c24_bf16": (1, 6, 9, 24, 8, 3, "bf16", False),
+    # the 2-D tiled kernel on an image smaller than one 16 x 8 tile (2 x 4
+    # tiles, columns and rows past the image not stored), three images
+    "tiny_2d_bf16": (3, 2, 3, 64, 8, 3, "bf16", True),
+    # the 2-D tiled kernel over a tall narrow image: 16 x 8 tiles whose
+    # columns 5..7 and, in the last tile row, rows 8..15 lie past the image
+    "tall_2d_f16": (1, 40, 5, 64, 8, 3, "f16", True),
 }
 
 
