@@ -9,8 +9,14 @@
 //   h[p][c]   = dw_b[c] + sum_{i,j} dw_w[i][j][c] * x[p + (i-1, j-1)][c]
 //   out[p][j] = lin_b[j] + sum_c lin_w[j][c] * h[p][c]
 //
-// Two kernels:
-//  * producer_tc_kernel (16-bit data): one CTA per SM walks 128-pixel tiles
+// Three kernels:
+//  * producer_tc2d_kernel (16-bit data, C a multiple of 64 up to 256, at most
+//    256 outputs in whole 16-byte rows): 2-D pixel tiles, x by TMA tile load,
+//    the sliding-window depthwise pass of depthwise_tile (shared with the
+//    fused forward), one MMA over all outputs, rows written by one TMA tile
+//    store (described at the kernel).
+//  * producer_tc_kernel (16-bit data, the other tensor-core shapes): one CTA
+//    per SM walks 128-pixel tiles
 //    (128 consecutive pixels of the flattened N*H*W grid). The pixel range a
 //    tile's 3x3 neighbourhoods touch (its pixels plus one image row and one
 //    pixel on each side) arrives in one bulk copy, double-buffered so the
