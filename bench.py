@@ -105,11 +105,19 @@ def hbm_peak():
 
 
 def kernel_source_hash():
+    """Hash of the kernel sources' code: comments removed and whitespace
+    collapsed, so that a documentation edit does not invalidate recorded
+    measurements while any change to the code does."""
+    import re
     csrc = os.path.join(ROOT, "deformable_convolution_dcn4_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            code = f.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        code = " ".join(code.split())
+        h.update(name.encode() + code.encode())
     return h.hexdigest()[:16]
 
 
