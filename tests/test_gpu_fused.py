@@ -253,3 +253,68 @@ def test_fused_given_workspace(orc):
     ws = torch.empty(10 * 12 * 8 * 27 * 2, dtype=torch.uint8, device="cuda")
     err = scaled_err(f32(_gpu(d, 8, "auto", workspace=ws)), _oracle(orc, d, 8))
     assert err <= TOL["bf16"]
+
+
+def test_fused_unaligned_pointers_take_the_chain(orc):
+    """An input and output that start 2 bytes past a 16-byte boundary rule
+    the fused kernel out (TMA and 16-byte stores); the call runs the
+    two-kernel chain through the scratch it is given and still matches the
+    oracle chain, while the forced fused kernel is refused."""
+    N, H, W, C, G, dtype, _ = CASES["internimage_bf16"]
+    d = _inputs("internimage_bf16", sigma=0.5)
+    dev = {k: v.cuda() for k, v in d.items()}
+    n = N * H * W * C
+    inp_buf = torch.empty(n + 1, dtype=d["input"].dtype, device="cuda")
+    inp = inp_buf[1:].view(N, H, W, C)
+    inp.copy_(dev["input"])
+    out_buf = torch.empty(n + 1, dtype=d["input"].dtype, device="cuda")
+    out = out_buf[1:].view(N, H, W, C)
+    ws = torch.empty(N * H * W * G * 27 * 2, dtype=torch.uint8, device="cuda")
+    B.dcn4_fused_forward(inp, dev["x"], dev["dw_weight"], dev["dw_bias"], dev["lin_weight"],
+                         dev["lin_bias"], group=G, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert B.dcn4_last_device_error() == (0, 0)
+    err = scaled_err(f32(out), _oracle(orc, d, G))
+    assert err <= TOL[dtype], f"scaled error {err:.2e}"
+    with pytest.raises(B.Dcn4Error) as e:
+        B.dcn4_fused_forward(inp, dev["x"], dev["dw_weight"], dev["dw_bias"],
+                             dev["lin_weight"], dev["lin_bias"], group=G, out=out, workspace=ws,
+                             algo="halo")
+    assert e.value.code == 2
+
+
+def _random_shapes(count=14, seed=2024):
+    """Seeded fused-call shapes: N 1..3, H and W 1..37, C in {64, 96, 128,
+    192, 256} with G giving D = 8, 16 or 32 (the fused kernel for D 16/32 with
+    whole group slices, the chain for D 8 and for C 96), bf16/fp16."""
+    rng = np.random.default_rng(seed)
+    shapes = []
+    while len(shapes) < count:
+        C = int(rng.choice([64, 96, 128, 192, 256]))
+        D = int(rng.choice([8, 16, 32]))
+        if C % D:
+            continue
+        shapes.append((int(rng.integers(1, 4)), int(rng.integers(1, 38)),
+                       int(rng.integers(1, 38)), C, C // D, str(rng.choice(["bf16", "f16"]))))
+    return shapes
+
+
+@pytest.mark.parametrize("shape", _random_shapes())
+def test_fused_random_shapes(orc, shape):
+    """End to end against the oracle chain on seeded random shapes (the fused
+    kernel where it takes the shape, else the chain through scratch)."""
+    N, H, W, C, G, dtype = shape
+    d = make_fused_inputs(N, H, W, C, G, dtype=dtype, seed=N * 1000 + H * 37 + W,
+                          offset_sigma=0.5)
+    err = scaled_err(f32(_gpu(d, G)), _oracle(orc, d, G))
+    assert err <= TOL[dtype], f"{shape}: scaled error {err:.2e}"
+
+
+def test_fused_random_shapes_cover_the_fused_kernel():
+    """The sweep above reaches the fused kernel (no scratch needed) and the
+    chain (scratch needed) both."""
+    kinds = set()
+    for N, H, W, C, G, dtype in _random_shapes():
+        desc = B.make_desc(N, H, W, C, G, DTYPES[dtype])
+        kinds.add(B.dcn4_fused_forward_workspace_size(desc) == 0)
+    assert kinds == {True, False}
