@@ -163,8 +163,11 @@ __global__ void __launch_bounds__(NW * 32, 1)
     const uint32_t idesc = umma_idesc_f16(std::is_same<T, __nv_bfloat16>::value, 128, L.NP);
     const uint32_t a_base = smem_u32(abuf), b_base = smem_u32(smem + L.b_off);
 
-    // thread 0 issues every copy and MMA and counts them, so that a CTA
-    // leaving on an expired wait can let the outstanding ones land first
+    // thread 32 issues the x loads, thread 0 the window loads and the MMAs
+    // (so the next x load and the MMAs go out side by side); each counts its
+    // own, so that a CTA leaving on an expired wait can let the outstanding
+    // ones land first
+    constexpr int kXThread = 32;
     int x_issued = 0, x_done = 0, win_issued = 0, win_done = 0, mma_issued = 0, mma_done = 0;
     auto issue_x = [&](const TileCoord &tc) {
         fence_async_smem();  // the generic reads of the buffer come first
@@ -184,13 +187,14 @@ __global__ void __launch_bounds__(NW * 32, 1)
     // (every thread gets the same answer)
     auto produce = [&](int k, int u) -> bool {
         if (!mbar_wait_bounded(x_bar, (uint32_t)k & 1u, kWaitLimitNs)) ok = false;
-        else if (tid == 0) ++x_done;
+        else if (tid == kXThread) ++x_done;
         if (__syncthreads_or(!ok)) return false;
         depthwise_tile<T, NW, 4>(xs, abuf, dwt, dwb, C, pl.TH, pl.TW, pl.lgTW, smem);
         fence_async_smem();
         __syncthreads();
+        if (tid == kXThread && u + (int)gridDim.x < units)
+            issue_x(fused_coord(u + gridDim.x, g, pl));
         if (tid == 0) {
-            if (u + (int)gridDim.x < units) issue_x(fused_coord(u + gridDim.x, g, pl));
             tc_fence_after();
             for (int kk = 0; kk < C / 16; ++kk)
                 tc_mma_f16(tmem, umma_desc_kmajor(a_base + kk * 256, 128, C * 16),
@@ -233,11 +237,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
     // (Issuing unit k+1's MMA before unit k's gathers, so that it runs under
     // them, measured slower on the InternImage stage: 244 against 231 us.)
     if ((int)blockIdx.x < units) {
-        if (tid == 0) {
-            const TileCoord t0 = fused_coord(blockIdx.x, g, pl);
-            issue_x(t0);
-            issue_win(t0);
-        }
+        const TileCoord t0 = fused_coord(blockIdx.x, g, pl);
+        if (tid == kXThread) issue_x(t0);
+        if (tid == 0) issue_win(t0);
         int k = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++k) {
             const TileCoord tc = fused_coord(u, g, pl);
@@ -252,10 +254,11 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
     }
 
+    // at most one copy of each kind and one MMA batch are outstanding
+    if (tid == kXThread && !ok && x_issued > x_done)
+        mbar_wait_bounded(x_bar, (uint32_t)(x_issued - 1) & 1u, kWaitLimitNs);
     if (tid == 0 && !ok) {
         atomicOr(&g_error_word, kErrTimeout);
-        // at most one copy of each kind and one MMA batch are outstanding
-        if (x_issued > x_done) mbar_wait_bounded(x_bar, (uint32_t)(x_issued - 1) & 1u, kWaitLimitNs);
         if (win_issued > win_done)
             mbar_wait_bounded(win_bar, (uint32_t)(win_issued - 1) & 1u, kWaitLimitNs);
         if (mma_issued > mma_done)

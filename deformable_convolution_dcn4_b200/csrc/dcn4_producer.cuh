@@ -613,8 +613,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
         n = t / L.tiles_h;
         wo0 = tw * L.TW;
     };
-    // thread 0 issues every copy and MMA and counts them (for the drain on an
-    // expired wait)
+    // thread 32 issues the x loads, thread 0 the MMAs and the stores (so the
+    // next x load and the MMAs go out side by side); each counts its own, for
+    // the drain on an expired wait
+    constexpr int kXThread = 32;
     int x_issued = 0, x_done = 0, mma_issued = 0, mma_done = 0;
     auto issue_x = [&](int t) {
         int n, ho0, wo0;
@@ -625,20 +627,20 @@ __global__ void __launch_bounds__(NW * 32, 1)
             tma_load_4d(smem_u32(xs), &tmap_x, 0, wo0 - 1, ho0 - 1, n, x_bar);
         ++x_issued;
     };
-    if (tid == 0 && (int)blockIdx.x < ntiles) issue_x(blockIdx.x);
+    if (tid == kXThread && (int)blockIdx.x < ntiles) issue_x(blockIdx.x);
 
     bool ok = true;
     int k = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
         const uint32_t par = (uint32_t)k & 1u;
         if (!mbar_wait_bounded(x_bar, par, kWaitLimitNs)) ok = false;
-        else if (tid == 0) ++x_done;
+        else if (tid == kXThread) ++x_done;
         if (__syncthreads_or(!ok)) break;
         depthwise_tile<T, NW, 4>(xs, abuf, dwt, dwb, C, L.TH, L.TW, L.lgTW, smem);
         fence_async_smem();
         __syncthreads();
+        if (tid == kXThread && t + (int)gridDim.x < ntiles) issue_x(t + gridDim.x);
         if (tid == 0) {
-            if (t + (int)gridDim.x < ntiles) issue_x(t + gridDim.x);
             tc_fence_after();
             for (int kk = 0; kk < C / 16; ++kk)
                 tc_mma_f16(tmem, umma_desc_kmajor(a_base + kk * 256, 128, C * 16),
@@ -687,9 +689,10 @@ __global__ void __launch_bounds__(NW * 32, 1)
         }
     }
     if (tid == 0) bulk_wait_all();
+    if (tid == kXThread && !ok && x_issued > x_done)
+        mbar_wait_bounded(x_bar, (uint32_t)(x_issued - 1) & 1u, kWaitLimitNs);
     if (tid == 0 && !ok) {
         atomicOr(&g_error_word, kErrTimeout);
-        if (x_issued > x_done) mbar_wait_bounded(x_bar, (uint32_t)(x_issued - 1) & 1u, kWaitLimitNs);
         if (mma_issued > mma_done)
             mbar_wait_bounded(mma_bar, (uint32_t)(mma_issued - 1) & 1u, kWaitLimitNs);
     }
