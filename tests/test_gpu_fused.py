@@ -318,3 +318,26 @@ def test_fused_random_shapes_cover_the_fused_kernel():
         desc = B.make_desc(N, H, W, C, G, DTYPES[dtype])
         kinds.add(B.dcn4_fused_forward_workspace_size(desc) == 0)
     assert kinds == {True, False}
+
+
+@pytest.mark.parametrize("algo", ["halo", "generic"])
+def test_fused_dilation_and_offset_scale(orc, algo):
+    """Dilation 2 with pad 2 keeps the output grid equal to the input grid, so
+    the fused call takes it; with offset_scale 0.5 the sampling grid and the
+    offsets both differ from the plain case (the depthwise 3x3 of the
+    sub-network is unchanged). Against the oracle chain of the same
+    geometry."""
+    N, H, W, C, G, dtype, _ = CASES["internimage_bf16"]
+    d = _inputs("internimage_bf16", sigma=0.5)
+    dev = {k: v.cuda() for k, v in d.items()}
+    out = B.dcn4_fused_forward(dev["input"], dev["x"], dev["dw_weight"], dev["dw_bias"],
+                               dev["lin_weight"], dev["lin_bias"], group=G, pad=2, dilation=2,
+                               offset_scale=0.5, algo=algo)
+    torch.cuda.synchronize()
+    assert B.dcn4_last_device_error() == (0, 0)
+    prob = orc.problem(N, H, W, C, G, 3, 3, pad=(2, 2), dilation=(2, 2), offset_scale=0.5)
+    rec = orc.offset_producer(prob, f32(d["x"]), f32(d["dw_weight"]), f32(d["dw_bias"]),
+                              f32(d["lin_weight"]), f32(d["lin_bias"]))
+    rec = torch.from_numpy(rec).to(d["x"].dtype).float().numpy().reshape(N, H, W, G, 9, 3)
+    err = scaled_err(f32(out), orc.forward(prob, f32(d["input"]), rec))
+    assert err <= TOL[dtype], f"{algo}: scaled error {err:.2e}"
