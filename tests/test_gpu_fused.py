@@ -341,3 +341,22 @@ def test_fused_dilation_and_offset_scale(orc, algo):
     rec = torch.from_numpy(rec).to(d["x"].dtype).float().numpy().reshape(N, H, W, G, 9, 3)
     err = scaled_err(f32(out), orc.forward(prob, f32(d["input"]), rec))
     assert err <= TOL[dtype], f"{algo}: scaled error {err:.2e}"
+
+
+def test_fused_full_size_highres(orc):
+    """N4 128x128 C256 G16 bf16 (four group slices, 8 x 8 tiles, 432 outputs
+    per pixel: the tensor-core producer of the chain does not take it), image
+    3: against the oracle forward on the records the call used, those records
+    against the oracle's producer, and end to end against the oracle chain."""
+    d = make_fused_inputs(4, 128, 128, 256, 16, dtype="bf16", seed=2)
+    got, rec = _gpu(d, 16, "halo", records=True)
+    got = f32(got)
+    assert np.isfinite(got).all()
+    images = [3]
+    err = scaled_err(got[images], _oracle_on(orc, d, 16, rec.cpu(), images=images))
+    assert err <= TOL["bf16"], f"on its records: {err:.2e}"
+    err = scaled_err(f32(rec[images]), _oracle_records(orc, d, 16, images=images))
+    assert err <= TOL["bf16"], f"records: {err:.2e}"
+    d = make_fused_inputs(4, 128, 128, 256, 16, dtype="bf16", seed=3, offset_sigma=0.5)
+    err = scaled_err(f32(_gpu(d, 16, "halo"))[images], _oracle(orc, d, 16, images=images))
+    assert err <= TOL["bf16"], f"end to end: {err:.2e}"
