@@ -34,7 +34,7 @@ import torch
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200.workloads import DTYPES, make_fused_inputs
 
-from parity_util import TOL, f32, scaled_err
+from parity_util import TOL, checked_err, f32, scaled_err
 
 pytestmark = pytest.mark.gpu
 
@@ -143,7 +143,7 @@ def test_fused_parity(orc, name, algo):
         assert e.value.code == 2
         return
     got, rec = _gpu(d, G, algo, records=True)
-    err = scaled_err(f32(got), _oracle_on(orc, d, G, rec))
+    err = checked_err(f32(got), _oracle_on(orc, d, G, rec), dtype, "aggregation")
     assert err <= TOL[dtype], f"{name} {algo}: aggregation, scaled error {err:.2e}"
     err = scaled_err(f32(rec), _oracle_records(orc, d, G))
     assert err <= TOL[dtype], f"{name} {algo}: records, scaled error {err:.2e}"
@@ -155,7 +155,7 @@ def test_fused_parity_oracle_chain(orc, name, algo):
     """End to end against the oracle's producer and forward (offsets ~0.5 px)."""
     G, dtype = CASES[name][4], CASES[name][5]
     d = _inputs(name, sigma=0.5)
-    err = scaled_err(f32(_gpu(d, G, algo)), _oracle(orc, d, G))
+    err = checked_err(f32(_gpu(d, G, algo)), _oracle(orc, d, G), dtype, "end to end")
     assert err <= TOL[dtype], f"{name} {algo}: scaled error {err:.2e}"
 
 
@@ -214,7 +214,8 @@ def test_fused_full_size_internimage(orc):
     got, rec = _gpu(d, 8, "halo", records=True)
     got = f32(got)
     assert np.isfinite(got).all()
-    err = scaled_err(got[images], _oracle_on(orc, d, 8, rec.cpu(), images=images))
+    err = checked_err(got[images], _oracle_on(orc, d, 8, rec.cpu(), images=images), "bf16",
+                      "on its records")
     assert err <= TOL["bf16"], f"on its records: {err:.2e}"
     err = scaled_err(f32(rec[images]), _oracle_records(orc, d, 8, images=images))
     assert err <= TOL["bf16"], f"records: {err:.2e}"
@@ -353,7 +354,8 @@ def test_fused_full_size_highres(orc):
     got = f32(got)
     assert np.isfinite(got).all()
     images = [3]
-    err = scaled_err(got[images], _oracle_on(orc, d, 16, rec.cpu(), images=images))
+    err = checked_err(got[images], _oracle_on(orc, d, 16, rec.cpu(), images=images), "bf16",
+                      "on its records")
     assert err <= TOL["bf16"], f"on its records: {err:.2e}"
     err = scaled_err(f32(rec[images]), _oracle_records(orc, d, 16, images=images))
     assert err <= TOL["bf16"], f"records: {err:.2e}"

@@ -9,8 +9,9 @@ import torch
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
 
-from parity_util import (TOL, backward_case, desc_kw, msdcn_backward_case, f32, forward_case,
-                         gpu_forward, oracle_forward, out_hw, problem, scaled_err)
+from parity_util import (TOL, backward_case, checked_err, desc_kw, msdcn_backward_case, f32,
+                         forward_case, gpu_forward, oracle_forward, out_hw, problem,
+                         scaled_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -93,7 +94,7 @@ def test_forward_math_modes(orc, name, math):
     else:
         got = B.dcn4_forward(data["input"].to(dev), data["offset_weight"].to(dev), group=wl.G,
                              math=math, **_kw(wl))
-    err = scaled_err(f32(got), oracle_forward(orc, wl, data))
+    err = checked_err(f32(got), oracle_forward(orc, wl, data), wl.dtype, f"{name}/{math}")
     assert err <= TOL[wl.dtype], f"{name}: {err:.3e}"
 
 

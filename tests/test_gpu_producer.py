@@ -10,7 +10,7 @@ import torch
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200.workloads import make_producer_inputs
 
-from parity_util import TOL, f32, scaled_err
+from parity_util import TOL, checked_err, f32, scaled_err
 
 pytestmark = pytest.mark.gpu
 
@@ -73,7 +73,7 @@ def test_producer_parity(orc, name, algo):
         assert e.value.code == 2
         return
     got = f32(_gpu(d, G, k, algo))
-    err = scaled_err(got, _oracle(orc, d, G, k))
+    err = checked_err(got, _oracle(orc, d, G, k), dtype, f"{name} {algo}")
     assert err <= TOL[dtype], f"{name} {algo}: scaled error {err:.2e}"
 
 
@@ -83,7 +83,7 @@ def test_producer_full_size_internimage(orc):
     d = _inputs(64, 56, 56, 128, 8, 3, "bf16", seed=0)
     got = f32(_gpu(d, 8, 3, "halo"))
     images = [0, 1, 63]
-    err = scaled_err(got[images], _oracle(orc, d, 8, 3, images))
+    err = checked_err(got[images], _oracle(orc, d, 8, 3, images), "bf16", "full size")
     assert err <= TOL["bf16"], f"scaled error {err:.2e}"
 
 
@@ -106,6 +106,9 @@ def test_producer_feeds_forward(orc):
     prob = orc.problem(N, H, W, C, G)
     ow_ref = _oracle(orc, d, G, 3)
     ref = orc.forward(prob, f32(d["x"]), ow_ref.astype(np.float32))
+    # scaled gate only: the records reach the forward rounded to bf16, which
+    # moves a sample by up to half an ulp of its offset, so single outputs
+    # near zero can differ by more than the elementwise gate allows
     err = scaled_err(got, ref)
     assert err <= TOL["bf16"], f"scaled error {err:.2e}"
 
