@@ -320,6 +320,23 @@ bool plan_producer_2d(int H, int W, int C, int J, int NP, ProducerTc2dLayout *ou
     return false;
 }
 
+// Where the fused kernel splits a tile's groups over several slices, each
+// slice's CTA computes the whole depthwise pass; when the 2-D tensor-core
+// producer takes the shape in one pass (J <= 256 outputs, lin_w resident),
+// the two-kernel chain is then the faster one (InternImage stage, N64 56x56
+// C128 G8 bf16: 174 us against 225 us), while on every shape that leaves the
+// chain's producer on the CUDA cores the fused kernel wins by 3-5x.
+bool chain_preferred(const Geometry &g, int eb, const HaloPlan &fused_plan) {
+    if (fused_plan.slices < 2 || eb != 2) return false;
+    const int J = g.G * g.K * 3, NP = (J + 15) / 16 * 16;
+    if (g.C % 16 != 0 || NP > 256 || (J * eb) % 16 != 0) return false;
+    ProducerTcLayout lay = ProducerTcLayout::make(g.C, J, NP, g.W, 2);
+    if (lay.bytes > max_smem_optin()) lay = ProducerTcLayout::make(g.C, J, NP, g.W, 1);
+    if (lay.bytes > max_smem_optin()) return false;
+    ProducerTc2dLayout l2;
+    return plan_producer_2d(g.H, g.W, g.C, J, NP, &l2);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -530,7 +547,8 @@ dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *byt
     FusedLayout lay;
     const int eb = elem_bytes(static_cast<Dtype>(desc->dtype));
     const bool fused = (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) &&
-                       plan_fused(g, eb, &plan, &lay);
+                       plan_fused(g, eb, &plan, &lay) &&
+                       !(desc->algo == DCN4_ALGO_AUTO && chain_preferred(g, eb, plan));
     *bytes = fused ? 0 : (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
     return DCN4_OK;
 }
@@ -559,7 +577,15 @@ dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const v
             (reinterpret_cast<uintptr_t>(offset_weight_out) & 3) == 0 &&
             encode_input_map(g, dt, input, L.plan, &map_in) &&
             encode_map(dt, x, g.N, g.H, g.W, g.C, g.C, L.plan.TW + 2, L.plan.TH + 2, &map_x);
-        if (fused) {
+        // AUTO takes the chain where it is faster, when there is room for
+        // the records (aligned for the producer's TMA store)
+        void *rec = offset_weight_out;
+        const size_t rec_bytes = (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
+        if (!rec && workspace && workspace_bytes >= rec_bytes) rec = workspace;
+        const bool to_chain = fused && desc->algo == DCN4_ALGO_AUTO &&
+                              chain_preferred(g, eb, L.plan) && rec != nullptr && aligned16(rec) &&
+                              aligned16(lin_weight);
+        if (fused && !to_chain) {
             L.geo = g;
             L.dtype = dt;
             L.in = input;
@@ -576,7 +602,7 @@ dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const v
             L.stream = static_cast<cudaStream_t>(stream);
             return cuda_status(launch_fused(L));
         }
-        if (desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
+        if (!fused && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     }
     // the two-kernel chain, through offset_weight_out when given, else
     // through the caller's scratch

@@ -274,12 +274,14 @@ DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
                                           const void *lin_weight, const void *lin_bias,
                                           void *offset_weight, void *stream);
 
-/* Scratch bytes dcn4_fused_forward may need for this desc: 0 when the fused
- * kernel takes the call's shape and desc->algo (it may still need the scratch
- * when a pointer is not aligned, see below), else the size of the
+/* Scratch bytes dcn4_fused_forward may need for this desc: 0 when the call
+ * runs the fused kernel (its shape and desc->algo; it may still need the
+ * scratch when a pointer is not aligned, see below), else the size of the
  * offset_weight tensor the two-kernel chain passes through,
  * N*Ho*Wo*G*kh*kw*3 elements of desc->dtype (none is needed when the call
- * passes offset_weight_out). */
+ * passes offset_weight_out). With DCN4_ALGO_AUTO that includes the shapes on
+ * which the chain is the faster path (see dcn4_fused_forward); a call given
+ * no scratch there runs the fused kernel instead. */
 DCN4_API dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *bytes);
 
 /* The DCNv4 module's aggregation with its offset/weight sub-network in front
@@ -316,6 +318,14 @@ DCN4_API dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, si
  * tensor-core producer's where that applies and the CUDA-core producer's
  * (h kept in fp32) otherwise, so on shapes the tensor-core producer does not
  * take the chain and the fused kernel may round a record differently.
+ * DCN4_ALGO_AUTO also takes the chain on a fused-kernel shape where the
+ * chain is faster, when it has 16-byte aligned room for the records
+ * (offset_weight_out, or a large enough workspace): where the groups span
+ * two or more slices (every slice's CTA then repeats the depthwise pass) and
+ * the tensor-core producer takes the shape in one 2-D tiled pass (at most 256
+ * outputs per pixel in whole 16-byte rows, C and lin_weight fitting shared
+ * memory) -- the InternImage stage, C128 G8, is one. Given no room it runs
+ * the fused kernel.
  * DCN4_ALGO_HALO demands the fused kernel (DCN4_ERR_UNSUPPORTED where it does
  * not apply). */
 DCN4_API dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const void *x,

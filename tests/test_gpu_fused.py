@@ -59,6 +59,10 @@ CASES = {
     "c24_bf16": (1, 6, 9, 24, 8, "bf16", False),
 }
 FUSED = sorted(k for k, v in CASES.items() if v[6])
+# fused-kernel shapes where AUTO takes the two-kernel chain when it has room
+# for the records: two or more group slices (each slice's CTA repeats the
+# depthwise pass) and a shape the 2-D tensor-core producer takes in one pass
+AUTO_CHAIN = {"internimage_bf16", "internimage_f16"}
 
 
 def _inputs(name, seed=7, sigma=2.0):
@@ -226,15 +230,20 @@ def test_fused_full_size_internimage(orc):
 
 
 def test_fused_workspace_size_and_refusal():
-    """The fused kernel's shapes need no scratch; the others need the
-    offset_weight tensor's bytes, and refuse a smaller scratch before any
-    launch."""
+    """Shapes on which AUTO runs the fused kernel need no scratch; the others
+    (the chain's shapes, and those where AUTO prefers the chain) ask for the
+    offset_weight tensor's bytes; the forced fused kernel never does. A chain
+    shape refuses a smaller scratch before any launch."""
     for name in sorted(CASES):
         N, H, W, C, G, dtype, fused = CASES[name]
         desc = B.make_desc(N, H, W, C, G, DTYPES[dtype])
         need = B.dcn4_fused_forward_workspace_size(desc)
         eb = 4 if dtype == "f32" else 2
-        assert need == (0 if fused else N * H * W * G * 27 * eb), name
+        auto_fused = fused and name not in AUTO_CHAIN
+        assert need == (0 if auto_fused else N * H * W * G * 27 * eb), name
+        if fused:
+            desc = B.make_desc(N, H, W, C, G, DTYPES[dtype], algo="halo")
+            assert B.dcn4_fused_forward_workspace_size(desc) == 0, name
     d = {k: v.cuda() for k, v in _inputs("d8_bf16").items()}
     desc = B.make_desc(1, 10, 12, 64, 8, torch.bfloat16)
     out = torch.empty_like(d["input"])
@@ -246,6 +255,33 @@ def test_fused_workspace_size_and_refusal():
         ctypes.c_void_p(out.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
     assert rc == 3
     assert B.dcn4_kernel_launches() == before
+
+
+@pytest.mark.parametrize("name", sorted(AUTO_CHAIN))
+def test_fused_auto_route(orc, name):
+    """AUTO on a shape where the chain is faster: with scratch (or an
+    offset_weight_out) it launches the producer and the forward, without it
+    the fused kernel; both against the oracle chain."""
+    N, H, W, C, G, dtype, _ = CASES[name]
+    d = _inputs(name, sigma=0.5)
+    ref = _oracle(orc, d, G)
+    ws = torch.empty(N * H * W * G * 27 * 2, dtype=torch.uint8, device="cuda")
+    for workspace, launches in ((ws, 2), (None, 1)):
+        dev = {k: v.cuda() for k, v in d.items()}
+        out = torch.empty_like(dev["input"])
+        desc = B.make_desc(N, H, W, C, G, DTYPES[dtype])
+        before = B.dcn4_kernel_launches()
+        rc = B.load().dcn4_fused_forward(
+            ctypes.byref(desc), *(ctypes.c_void_p(dev[k].data_ptr()) for k in (
+                "input", "x", "dw_weight", "dw_bias", "lin_weight", "lin_bias")),
+            ctypes.c_void_p(out.data_ptr()), None,
+            None if workspace is None else ctypes.c_void_p(workspace.data_ptr()),
+            0 if workspace is None else workspace.numel(), None)
+        torch.cuda.synchronize()
+        assert rc == 0 and B.dcn4_last_device_error() == (0, 0)
+        assert B.dcn4_kernel_launches() - before == launches
+        err = scaled_err(f32(out), ref)
+        assert err <= TOL[dtype], f"{name} scratch={workspace is not None}: {err:.2e}"
 
 
 def test_fused_given_workspace(orc):
