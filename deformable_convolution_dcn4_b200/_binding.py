@@ -27,7 +27,8 @@ EXPORTS = ("dcn4_out_shape", "dcn4_forward", "dcn4_backward_workspace_size", "dc
            "msdcn_forward", "dcn4_status_string", "dcn4_last_device_error",
            "dcn4_backward_noalloc", "dcn4_selftest_bounded_wait", "dcn4_kernel_launches",
            "msdcn_backward", "dcn4_offset_producer", "dcn4_fused_forward_workspace_size",
-           "dcn4_fused_forward")
+           "dcn4_fused_forward", "dcn4_forward_workspace_size", "dcn4_forward_ws",
+           "msdcn_forward_ws")
 
 
 class Dcn4Error(RuntimeError):
@@ -96,6 +97,10 @@ def _open(path):
     lib.dcn4_fused_forward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.dcn4_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                                        vp]
+    lib.dcn4_forward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.dcn4_forward_ws.argtypes = [P, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.msdcn_forward_ws.argtypes = [P, vp, vp, vp, ctypes.POINTER(ctypes.c_float),
+                                     ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
     for name in EXPORTS:
         if name != "dcn4_status_string":
             getattr(lib, name).restype = st
@@ -156,10 +161,36 @@ def _desc_for(inp, group, kernel_size, stride, pad, dilation, offset_scale, algo
                      offset_scale, algo, math, softmax, msdcn_mode)
 
 
+def dcn4_forward_workspace_size(desc):
+    n = ctypes.c_size_t()
+    _check("dcn4_forward_workspace_size",
+           load().dcn4_forward_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def _forward_scratch(desc, input, workspace, defer_escapes):
+    """(pointer, bytes, tensor) of the escape scratch: the caller's tensor,
+    else one from PyTorch's allocator of dcn4_forward_workspace_size bytes
+    (the caller keeps the tensor until the launch is issued; the allocator
+    reuses it only in stream order after that); None when escapes are to be
+    handled in place."""
+    if not defer_escapes:
+        return None
+    if workspace is None:
+        need = dcn4_forward_workspace_size(desc)
+        if need == 0:
+            return (None, 0, None)
+        workspace = torch.empty(need, dtype=torch.uint8, device=input.device)
+    return (_ptr(workspace), workspace.numel() * workspace.element_size(), workspace)
+
+
 def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, dilation=1,
-                 offset_scale=1.0, algo="auto", out=None, math="default", softmax=False):
+                 offset_scale=1.0, algo="auto", out=None, math="default", softmax=False,
+                 workspace=None, defer_escapes=True):
     """DCNv4 forward. input [N,H,W,C]; offset_weight [N,Ho,Wo,G,kh*kw,3].
-    softmax=True normalises m over the taps (DCNv3 weights)."""
+    softmax=True normalises m over the taps (DCNv3 weights). The staged
+    kernel's escaped samples go through scratch (dcn4_forward_ws; `workspace`,
+    else one allocated here) unless defer_escapes=False (dcn4_forward)."""
     desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
                      softmax)
     ho, wo = dcn4_out_shape(desc)
@@ -170,8 +201,15 @@ def dcn4_forward(input, offset_weight, group, kernel_size=3, stride=1, pad=1, di
     if out is None:
         out = torch.empty((N, ho, wo, C), dtype=input.dtype, device=input.device)
     _require(out, "out", input.dtype, (N, ho, wo, C))
-    _check("dcn4_forward", load().dcn4_forward(ctypes.byref(desc), _ptr(input), _ptr(offset_weight),
-                                               _ptr(out), _stream(input)))
+    ws = _forward_scratch(desc, input, workspace, defer_escapes)
+    if ws is None:
+        _check("dcn4_forward", load().dcn4_forward(ctypes.byref(desc), _ptr(input),
+                                                   _ptr(offset_weight), _ptr(out),
+                                                   _stream(input)))
+    else:
+        _check("dcn4_forward_ws", load().dcn4_forward_ws(ctypes.byref(desc), _ptr(input),
+                                                         _ptr(offset_weight), _ptr(out), ws[0],
+                                                         ws[1], _stream(input)))
     return out
 
 
@@ -305,9 +343,10 @@ def dcn4_backward_noalloc(input, offset_weight, grad_out, group, kernel_size=3, 
 
 def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, stride=1, pad=1,
                   dilation=1, offset_scale=1.0, algo="auto", out=None, math="default",
-                  msdcn_mode="offset"):
+                  msdcn_mode="offset", workspace=None, defer_escapes=True):
     """MSDCN forward. dir_weight [N,Ho,Wo,G,K,3]; scale_raw [N,Ho,Wo,G]; s0 host floats [G].
-    msdcn_mode "offset" (s * dir) or "dilation" (s * (p_k + dir))."""
+    msdcn_mode "offset" (s * dir) or "dilation" (s * (p_k + dir)). Escape
+    scratch as in dcn4_forward (msdcn_forward_ws)."""
     desc = _desc_for(input, group, kernel_size, stride, pad, dilation, offset_scale, algo, math,
                      False, msdcn_mode)
     ho, wo = dcn4_out_shape(desc)
@@ -322,9 +361,15 @@ def msdcn_forward(input, dir_weight, scale_raw, s0, smax, group, kernel_size=3, 
     if out is None:
         out = torch.empty((N, ho, wo, C), dtype=input.dtype, device=input.device)
     _require(out, "out", input.dtype, (N, ho, wo, C))
-    _check("msdcn_forward", load().msdcn_forward(
-        ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr,
-        float(smax), _ptr(out), _stream(input)))
+    ws = _forward_scratch(desc, input, workspace, defer_escapes)
+    if ws is None:
+        _check("msdcn_forward", load().msdcn_forward(
+            ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr,
+            float(smax), _ptr(out), _stream(input)))
+    else:
+        _check("msdcn_forward_ws", load().msdcn_forward_ws(
+            ctypes.byref(desc), _ptr(input), _ptr(dir_weight), _ptr(scale_raw), s0_arr,
+            float(smax), _ptr(out), ws[0], ws[1], _stream(input)))
     return out
 
 

@@ -431,7 +431,8 @@ int forward_math(const dcn4_desc *d) {
 }
 
 dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow, void *output,
-                        void *stream, const MsdcnParams *ms) {
+                        void *stream, const MsdcnParams *ms, void *ws = nullptr,
+                        size_t ws_bytes = 0) {
     Geometry g;
     if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
     if (!input || !ow || !output) return DCN4_ERR_INVALID_ARG;
@@ -448,6 +449,10 @@ dcn4_status run_forward(const dcn4_desc *desc, const void *input, const void *ow
     L.mathv = forward_math(desc);
     L.stream = static_cast<cudaStream_t>(stream);
     L.ow_bytes = (unsigned long long)g.N * g.Ho * g.Wo * g.G * g.K * 3 * elem_bytes(L.dtype);
+    if (ws != nullptr && aligned16(ws)) {
+        L.ws = ws;
+        L.ws_bytes = ws_bytes;
+    }
     CUtensorMap map, map_ow;
     memset(&map, 0, sizeof(map));
     memset(&map_ow, 0, sizeof(map_ow));
@@ -482,6 +487,27 @@ dcn4_status dcn4_out_shape(const dcn4_desc *desc, int *Ho, int *Wo) {
 dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input, const void *offset_weight,
                          void *output, void *stream) {
     return run_forward(desc, input, offset_weight, output, stream, nullptr);
+}
+
+dcn4_status dcn4_forward_workspace_size(const dcn4_desc *desc, size_t *bytes) {
+    Geometry g;
+    if (!make_geometry(desc, &g) || !bytes) return DCN4_ERR_INVALID_ARG;
+    const int eb = elem_bytes(static_cast<Dtype>(desc->dtype));
+    // the staged kernel with one lane per (pixel, group): 3x3 taps, groups of
+    // 2 (16-bit) or 4 16-byte chunks
+    const int U = (g.D * eb) % 16 == 0 ? g.D * eb / 16 : 0;
+    const bool staged = g.kh == 3 && g.kw == 3 && (U == 4 || (U == 2 && eb == 2)) &&
+                        (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO);
+    *bytes = staged ? forward_escape_bytes((long long)g.N * g.Ho * g.Wo * g.G, g.D, eb,
+                                           sm_count() * 8)
+                    : 0;
+    return DCN4_OK;
+}
+
+dcn4_status dcn4_forward_ws(const dcn4_desc *desc, const void *input, const void *offset_weight,
+                            void *output, void *workspace, size_t workspace_bytes, void *stream) {
+    return run_forward(desc, input, offset_weight, output, stream, nullptr, workspace,
+                       workspace_bytes);
 }
 
 dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const void *dw_weight,
@@ -739,6 +765,21 @@ dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input, const void *
     ms.smax = smax;
     for (int i = 0; i < g.G; ++i) ms.s0[i] = s0_host[i];
     return run_forward(desc, input, dir_weight, output, stream, &ms);
+}
+
+dcn4_status msdcn_forward_ws(const dcn4_desc *desc, const void *input, const void *dir_weight,
+                             const void *scale_raw, const float *s0_host, float smax,
+                             void *output, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+    Geometry g;
+    if (!make_geometry(desc, &g)) return DCN4_ERR_INVALID_ARG;
+    if (!s0_host || !scale_raw) return DCN4_ERR_INVALID_ARG;
+    if (g.softmax) return DCN4_ERR_UNSUPPORTED;
+    static thread_local MsdcnParams ms;
+    ms.raw = scale_raw;
+    ms.smax = smax;
+    for (int i = 0; i < g.G; ++i) ms.s0[i] = s0_host[i];
+    return run_forward(desc, input, dir_weight, output, stream, &ms, workspace, workspace_bytes);
 }
 
 const char *dcn4_status_string(dcn4_status s) {

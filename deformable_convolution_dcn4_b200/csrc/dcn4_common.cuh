@@ -132,6 +132,24 @@ struct HaloPlan {
     int rec_box;         // elements per pixel of that copy (Gc*27 plus alignment slack)
 };
 
+// Deferred escapes of the staged forward (chosen on the host). A (pixel,
+// group) pair with taps outside the staged window does not wait for their
+// global loads: it leaves an entry here, and the CTA adds those taps and
+// writes the pair's output after its last tile, with all its warps busy on
+// such entries. Entry layout, entry_bytes = 16 + 4*D:
+//   bytes 0-7    pair index P = ((n*Ho + ho)*Wo + wo)*G + g   (u64)
+//   bytes 8-11   mask of the escaped taps (bit k: tap k)
+//   bytes 16-    the in-window partial sums, D fp32 values in channel order
+// CTA b of the staged kernel appends to entries [b*cap, (b+1)*cap) while
+// it works through its tiles, and finishes them itself once all its warps
+// are done; once its region is full it handles further escapes in place.
+struct EscList {
+    unsigned char *entries;    // nullptr: every escape handled in place
+    int cap;                   // entries per CTA
+    int entry_bytes;
+    unsigned long long bytes;  // of the entries area (bounds of the checked build)
+};
+
 // Tiling and shared-memory carve-up of the 2-D tiled tensor-core producer
 // (byte offsets from the start of dynamic shared memory; chosen on the host).
 struct ProducerTc2dLayout {

@@ -321,14 +321,19 @@ __device__ __forceinline__ void stage_window_records(const TileCoord &tc, const 
 }
 
 // The gathers of one staged tile: LPP lanes per (pixel, group), each with
-// U/LPP of its 16-byte chunks (one lane with all of them when LPP = 1).
-template <typename T, int U, bool MS, int MV, int LPP>
+// U/LPP of its 16-byte chunks (one lane with all of them when LPP = 1). With
+// DEF (LPP = 1) and el.entries set, a pair with escaped taps appends an
+// EscList entry (slot from the CTA's counter *esc_n) instead of loading them.
+template <typename T, int U, bool MS, int MV, int LPP, bool DEF = false>
 __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry &g,
                                              const HaloPlan &pl, const T *__restrict__ in,
                                              T *__restrict__ out, const MsdcnParams &ms,
                                              const unsigned char *halo,
                                              const unsigned char *slots, int ct, int nct,
-                                             const unsigned char *sbase) {
+                                             const unsigned char *sbase,
+                                             const EscList &el = EscList{},
+                                             int *esc_n = nullptr) {
+    static_assert(!DEF || LPP == 1, "deferred escapes take one lane per pair");
     (void)sbase;
     constexpr int EB = Elem<T>::kBytes;
     constexpr int VE = Elem<T>::kPerVec;  // elements per 16-byte chunk
@@ -469,6 +474,26 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
                 esc |= 1u << k;
             }
         }
+        if (DEF && esc != 0u && el.entries != nullptr) {
+            const int slot = atomicAdd(esc_n, 1);
+            if (slot < el.cap) {
+                unsigned char *e =
+                    el.entries + ((size_t)blockIdx.x * el.cap + slot) * (size_t)el.entry_bytes;
+                const unsigned long long P = gp * g.G + tc.g0 + gl;
+                if (DCN4_GMEM_OK(e, (unsigned)el.entry_bytes, el.entries, el.bytes)) {
+                    *reinterpret_cast<uint4 *>(e) =
+                        make_uint4((unsigned)P, (unsigned)(P >> 32), esc, 0u);
+                    float4 *pf = reinterpret_cast<float4 *>(e + 16);
+#pragma unroll
+                    for (int c = 0; c < UL; ++c)
+#pragma unroll
+                        for (int q = 0; q < VE; q += 4)
+                            pf[(chunk(c) * VE + q) >> 2] =
+                                make_float4(acc[c][q], acc[c][q + 1], acc[c][q + 2], acc[c][q + 3]);
+                }
+                continue;
+            }
+        }
         // samples outside the staged window (rare): 16-byte loads from global
         // memory, each corner tested against the image
         const T *gbase = in + (size_t)tc.n * img + (size_t)(tc.g0 + gl) * D;
@@ -512,6 +537,117 @@ __device__ __forceinline__ void compute_tile(const TileCoord &tc, const Geometry
     }
 }
 
+// One deferred escape (an EscList entry of the staged forward): starts from
+// the entry's partial sums and adds the escaped taps in ascending order with
+// the staged kernel's own arithmetic (the pair's record read again from
+// global memory; position, softmax weight or MSDCN scale, corner weights,
+// fp32 multiply-adds of 16-byte global loads, out-of-image corners skipped),
+// then writes the pair's output: the in-place result, bit for bit.
+template <typename T, int U, bool MS>
+__device__ __forceinline__ void finish_escape(const unsigned char *e, const Geometry &g,
+                                              const T *__restrict__ in,
+                                              const T *__restrict__ ow, T *__restrict__ out,
+                                              const MsdcnParams &ms) {
+    constexpr int EB = Elem<T>::kBytes;
+    constexpr int VE = Elem<T>::kPerVec;
+    const size_t img = (size_t)g.H * g.W * g.C;
+    const unsigned long long npairs = (unsigned long long)g.N * g.Ho * g.Wo * g.G;
+    const unsigned long long in_b = input_bytes(g, EB), out_b = output_bytes(g, EB);
+    const unsigned long long ow_b = npairs * 27 * EB;
+    (void)in_b, (void)out_b, (void)ow_b, (void)npairs;
+    const uint4 meta = *reinterpret_cast<const uint4 *>(e);
+    const unsigned long long P = meta.x | ((unsigned long long)meta.y << 32);
+    const unsigned esc = meta.z;
+    if (!DCN4_CHECK(P < npairs)) return;
+    const T *rec = ow + P * 27;
+    if (!DCN4_GMEM_OK(rec, 27 * EB, ow, ow_b)) return;
+    float acc[U][VE];
+    const float4 *pf = reinterpret_cast<const float4 *>(e + 16);
+#pragma unroll
+    for (int c = 0; c < U; ++c)
+#pragma unroll
+        for (int q = 0; q < VE / 4; ++q) {
+            const float4 f = pf[c * (VE / 4) + q];
+            acc[c][4 * q] = f.x, acc[c][4 * q + 1] = f.y;
+            acc[c][4 * q + 2] = f.z, acc[c][4 * q + 3] = f.w;
+        }
+    const int gg = (int)(P % (unsigned)g.G);
+    const unsigned long long gp = P / (unsigned)g.G;
+    const int wo = (int)(gp % (unsigned)g.Wo);
+    const unsigned long long rr = gp / (unsigned)g.Wo;
+    const int ho = (int)(rr % (unsigned)g.Ho), n = (int)(rr / (unsigned)g.Ho);
+    float s = 1.0f;
+    const bool dil = MS && g.msd_dil;
+    if (MS) {
+        const T *rp = static_cast<const T *>(ms.raw) + P;
+        const float raw = DCN4_GMEM_OK(rp, EB, ms.raw, raw_bytes(g, EB))
+                              ? Elem<T>::to_f(*rp) : 0.0f;
+        s = msdcn_scale(raw, ms.s0[gg], ms.smax);
+    }
+    SoftmaxNorm sn{0.0f, 1.0f};
+    if (!MS && g.softmax) {
+        float mx = Elem<T>::to_f(rec[2]);
+#pragma unroll
+        for (int k = 1; k < 9; ++k) mx = fmaxf(mx, Elem<T>::to_f(rec[3 * k + 2]));
+        float sum = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 9; ++k) sum += expf(Elem<T>::to_f(rec[3 * k + 2]) - mx);
+        sn = SoftmaxNorm{mx, 1.0f / sum};
+    }
+    const T *gbase = in + (size_t)n * img + (size_t)gg * g.D;
+    // tap k: its corner weights and which corners lie in the image (none
+    // when the sample is outside), loads into qv
+    auto tap = [&](int k, float *wc, bool *ok, uint4 (*qv)[U]) {
+        const float dx = Elem<T>::to_f(rec[3 * k]), dy = Elem<T>::to_f(rec[3 * k + 1]);
+        float m = Elem<T>::to_f(rec[3 * k + 2]);
+        if (!MS && g.softmax) m = sn.weight(m);
+        const int i = k / 3, j = k - 3 * i;
+        float x, y, dsx, dsy;
+        if (MS) {
+            x = msdcn_coord(dil, wo * g.sw - g.pw, j, 3, g.dw, s, dx, g.os, &dsx);
+            y = msdcn_coord(dil, ho * g.sh - g.ph, i, 3, g.dh, s, dy, g.os, &dsy);
+        } else {
+            x = sample_coord(wo * g.sw - g.pw + j * g.dw, dx, g.os);
+            y = sample_coord(ho * g.sh - g.ph + i * g.dh, dy, g.os);
+        }
+        const bool inside = x > -1.0f && x < (float)g.W && y > -1.0f && y < (float)g.H;
+        const float x0f = floorf(x), y0f = floorf(y);
+        const float lx = x - x0f, ly = y - y0f;
+        const float mly = m * ly, mhy = m - mly;
+        const float w01 = mhy * lx, w11 = mly * lx;
+        wc[0] = mhy - w01, wc[1] = w01, wc[2] = mly - w11, wc[3] = w11;
+        const int x0 = inside ? (int)x0f : 0, y0 = inside ? (int)y0f : 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int yy = y0 + (q >> 1), xx = x0 + (q & 1);
+            ok[q] = inside && yy >= 0 && yy < g.H && xx >= 0 && xx < g.W;
+            const uint4 *p =
+                reinterpret_cast<const uint4 *>(gbase + ((size_t)yy * g.W + xx) * g.C);
+#pragma unroll
+            for (int c = 0; c < U; ++c)
+                qv[q][c] = ok[q] ? DCN4_LDG16(p + c, in, in_b) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    unsigned em = esc & 0x1ffu;
+    while (em) {
+        const int k = __ffs(em) - 1;
+        em &= em - 1;
+        float wc[4];
+        bool ok[4];
+        uint4 qv[4][U];
+        tap(k, wc, ok, qv);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (ok[q])
+#pragma unroll
+                for (int c = 0; c < U; ++c) VecMath<T>::fma(acc[c], qv[q][c], wc[q]);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(out + gp * g.C + (size_t)gg * g.D);
+#pragma unroll
+    for (int c = 0; c < U; ++c)
+        if (DCN4_GMEM_OK(dst + c, 16, out, out_b)) dst[c] = VecMath<T>::pack(acc[c]);
+}
+
 // Persistent halo kernel. CTA b handles tiles b, b + gridDim.x, ...; thread
 // t of the NW warps owns (pixel, group) pairs t, t + 32NW, ... of every tile.
 // The input window (and, with pl.rec_tma, the tile's records) is shared:
@@ -527,8 +663,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
 fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_ow,
                 Geometry g, HaloPlan pl, const T *__restrict__ in, const T *__restrict__ ow,
                 T *__restrict__ out, unsigned long long ow_bytes,
-                const __grid_constant__ MsdcnParams ms) {
+                const __grid_constant__ MsdcnParams ms, const __grid_constant__ EscList el) {
     extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ int esc_n;  // deferred escapes: entries taken
     const int stage_bytes = HaloSmem::stage_bytes(pl);
     const uint32_t win0 = smem_u32(smem + STAGES * stage_bytes);  // win[s]   at +8s
     const uint32_t empty0 = win0 + 8 * STAGES;                     // empty[s] at +8s
@@ -545,6 +682,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
         }
         for (int b = 0; b < NW * STAGES; ++b) mbar_init(rec0 + 8 * b, 1);
         fence_barrier_init();
+        esc_n = 0;
     }
     __syncthreads();
 
@@ -591,6 +729,7 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
         if (warp == 0) window(cur, 0);
     }
     int i = 0;
+    bool bail = false;  // this warp stopped on an expired wait
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
         const int s = i % STAGES;
         const int tn = t + gridDim.x;
@@ -603,7 +742,8 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
                 if (leader) atomicOr(&g_error_word, kErrTimeout);
                 drain(i, i + 1, false);
                 drain(i, i, true);
-                return;
+                bail = true;
+                break;
             }
             issued = i + 1;
         }
@@ -612,11 +752,13 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
         if (!ok) {
             if (leader) atomicOr(&g_error_word, kErrTimeout);
             drain(i, issued, warp == 0);
-            return;
+            bail = true;
+            break;
         }
         const unsigned char *buf = smem + s * stage_bytes;
-        compute_tile<T, U, MS, MV, LPP>(cur, g, pl, in, out, ms, buf, buf + pl.halo_bytes,
-                                   threadIdx.x, NW * 32, smem);
+        compute_tile<T, U, MS, MV, LPP, LPP == 1>(cur, g, pl, in, out, ms, buf,
+                                                 buf + pl.halo_bytes, threadIdx.x, NW * 32, smem,
+                                                 el, &esc_n);
         __syncwarp();
         if (leader) mbar_arrive(empty0 + 8 * s);
         if (STAGES == 1 && tn < ntiles) {
@@ -624,10 +766,23 @@ fwd_halo_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant_
             if (warp == 0 && !window(nxt, i + 1)) {
                 if (leader) atomicOr(&g_error_word, kErrTimeout);
                 drain(i + 1, i + 1, false);
-                return;
+                bail = true;
+                break;
             }
         }
         cur = nxt;
+    }
+    // the CTA's deferred escapes, once every warp is done with its tiles
+    // (every warp gets here: each wait is bounded); none after an expired wait
+    if (LPP == 1 && el.entries != nullptr) {
+        if (__syncthreads_or(bail)) return;
+        const int ne = min(esc_n, el.cap);
+        for (int ei = threadIdx.x; ei < ne; ei += NW * 32) {
+            const unsigned char *e =
+                el.entries + ((size_t)blockIdx.x * el.cap + ei) * (size_t)el.entry_bytes;
+            if (DCN4_GMEM_OK(e, (unsigned)el.entry_bytes, el.entries, el.bytes))
+                finish_escape<T, U, MS>(e, g, in, ow, out, ms);
+        }
     }
 }
 

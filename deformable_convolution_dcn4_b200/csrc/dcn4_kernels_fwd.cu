@@ -1,5 +1,7 @@
 // dcn4_kernels_fwd.cu -- forward kernels of libdcn4 (staged halo, vectorised
 // and scalar global-memory, DCNv4 and MSDCN) and their launcher.
+#include <cstring>
+
 #include "dcn4_common.cuh"
 
 namespace dcn4 {
@@ -32,11 +34,27 @@ cudaError_t launch_halo_t(const FwdLaunch &L) {
     if (occ < 1) return cudaErrorInvalidConfiguration;
     long long grid = (long long)sm_count() * occ;
     if (grid > tiles) grid = tiles;
+    // deferred escapes: each CTA's region of entries
+    EscList el;
+    memset(&el, 0, sizeof(el));
+    if constexpr (LPP == 1) {
+        const size_t entry = escape_entry_bytes(L.geo.D, (int)sizeof(T));
+        if (L.ws != nullptr && L.ws_bytes >= entry * (size_t)grid) {
+            size_t cap = L.ws_bytes / entry / (size_t)grid;
+            if (cap > (size_t)(1 << 30)) cap = (size_t)1 << 30;
+            el.entries = static_cast<unsigned char *>(L.ws);
+            el.cap = (int)cap;
+            el.entry_bytes = (int)entry;
+            el.bytes = (unsigned long long)(cap * entry * (size_t)grid);
+        }
+    }
     k<<<(unsigned)grid, NT, L.plan.smem_bytes, L.stream>>>(
         *L.tmap, *L.tmap_ow, L.geo, L.plan, static_cast<const T *>(L.in),
-        static_cast<const T *>(L.ow), static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs);
+        static_cast<const T *>(L.ow), static_cast<T *>(L.out), L.ow_bytes, L.ms ? *L.ms : kNoMs,
+        el);
     count_launch();
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    return e;
 }
 
 // Stage count and warps: two stages with 16 warps when a tile has 512
@@ -115,6 +133,15 @@ cudaError_t launch_forward(const FwdLaunch &L) {
         case Dtype::F16: return launch_fwd_t<__half>(L);
     }
     return cudaErrorInvalidValue;
+}
+
+size_t escape_entry_bytes(int D, int eb) {
+    (void)eb;
+    return 16 + 4 * (size_t)D;
+}
+
+size_t forward_escape_bytes(long long npairs, int D, int eb, int ctas) {
+    return (size_t)((npairs + 3) / 4 + ctas) * escape_entry_bytes(D, eb);
 }
 
 cudaError_t read_clear_error_fwd(unsigned *bits) {

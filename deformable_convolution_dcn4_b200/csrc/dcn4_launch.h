@@ -25,8 +25,16 @@ struct FwdLaunch {
     const CUtensorMap *tmap;
     const CUtensorMap *tmap_ow;  // records, when plan.rec_tma
     unsigned long long ow_bytes;
+    void *ws;         // scratch for deferred escapes (16-byte aligned), or nullptr
+    size_t ws_bytes;
     cudaStream_t stream;
 };
+
+// Scratch the staged forward can use for deferred escapes: entries of
+// escape_entry_bytes(D, eb) for a quarter of the (pixel, group) pairs plus
+// one per CTA, for up to `ctas` CTAs (eb: bytes per element).
+size_t escape_entry_bytes(int D, int eb);
+size_t forward_escape_bytes(long long npairs, int D, int eb, int ctas);
 
 struct BwdLaunch {
     Geometry geo;

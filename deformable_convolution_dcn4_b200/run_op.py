@@ -28,6 +28,8 @@ def main(argv=None):
     p.add_argument("--N", type=int, default=None)
     p.add_argument("--algo", default="auto")
     p.add_argument("--math", default="default")
+    p.add_argument("--in-place-escapes", action="store_true",
+                   help="forward/msdcn: no escape scratch (one kernel)")
     a = p.parse_args(argv)
     wl = WORKLOADS[a.workload]
     if a.N:
@@ -49,7 +51,8 @@ def main(argv=None):
               dilation=wl.dilation, offset_scale=wl.offset_scale, algo=a.algo)
     for _ in range(a.iters):
         if a.op == "forward":
-            B.dcn4_forward(d["input"], d["offset_weight"], **kw)
+            B.dcn4_forward(d["input"], d["offset_weight"],
+                           defer_escapes=not a.in_place_escapes, **kw)
         elif a.op == "producer":
             B.dcn4_offset_producer(d["x"], d["dw_weight"], d["dw_bias"], d["lin_weight"],
                                    d["lin_bias"], group=wl.G, kernel_size=(wl.kh, wl.kw),
@@ -64,7 +67,8 @@ def main(argv=None):
             B.msdcn_backward(d["input"], d["dir_weight"], d["scale_raw"], d["s0"], wl.smax,
                              d["grad_out"], math=a.math, **kw)
         else:
-            B.msdcn_forward(d["input"], d["dir_weight"], d["scale_raw"], d["s0"], wl.smax, **kw)
+            B.msdcn_forward(d["input"], d["dir_weight"], d["scale_raw"], d["s0"], wl.smax,
+                            defer_escapes=not a.in_place_escapes, **kw)
     torch.cuda.synchronize()
     rc, bits = B.dcn4_last_device_error()
     print(f"run_op {a.op} {wl.name} N={wl.N} iters={a.iters}: device error bits {bits}")

@@ -170,6 +170,30 @@ DCN4_API dcn4_status dcn4_out_shape(const dcn4_desc *desc, int *Ho, int *Wo);
 DCN4_API dcn4_status dcn4_forward(const dcn4_desc *desc, const void *input,
                          const void *offset_weight, void *output, void *stream);
 
+/* Bytes of device scratch with which dcn4_forward_ws and msdcn_forward_ws
+ * run fastest for `desc` (0 where the staged kernel cannot use any: taps
+ * other than 3x3, groups other than 2 (bf16/fp16) or 4 16-byte vectors, or
+ * DCN4_ALGO_GENERIC/VECTOR): 16 + 4*D bytes for a quarter of the N*Ho*Wo*G
+ * (pixel, group) pairs plus one per CTA, for up to 8 CTAs per SM. */
+DCN4_API dcn4_status dcn4_forward_workspace_size(const dcn4_desc *desc, size_t *bytes);
+
+/* dcn4_forward with scratch for the staged kernel's escapes (samples outside
+ * its shared-memory window; no counterpart on the pages). In place, a warp
+ * waits on the global loads of any one lane's escaped tap; with scratch, a
+ * (pixel, group) pair with escaped taps writes its in-window partial sums
+ * (fp32) and the taps' mask to `workspace` instead of its output, and its
+ * CTA, after its last tile, adds those taps with all its threads (global
+ * loads, the same arithmetic in the same order) and writes the output. One
+ * kernel either way; the output is bit-identical to dcn4_forward's.
+ * workspace: device memory owned by the caller, 16-byte aligned, or NULL;
+ * any size is accepted (none, a misaligned pointer or too little for one
+ * entry per CTA: escapes are handled in place; a CTA whose share of the
+ * entries fills up handles further escapes in place). Two calls must not
+ * use the same workspace at the same time. */
+DCN4_API dcn4_status dcn4_forward_ws(const dcn4_desc *desc, const void *input,
+                                     const void *offset_weight, void *output, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /* Bytes of device workspace dcn4_backward needs for `desc`: an fp32 copy of
  * grad_input for bf16/fp16 (N*H*W*C*4 bytes) and 0 for fp32. (Under
  * DCN4_MATH_ACC16 the staged bf16/fp16 kernel accumulates in grad_input
@@ -210,6 +234,14 @@ DCN4_API dcn4_status msdcn_forward(const dcn4_desc *desc, const void *input,
                           const void *dir_weight, const void *scale_raw,
                           const float *s0_host, float smax, void *output,
                           void *stream);
+
+/* msdcn_forward with scratch for the staged kernel's escapes, as
+ * dcn4_forward_ws (size from dcn4_forward_workspace_size; the output is
+ * bit-identical to msdcn_forward's). */
+DCN4_API dcn4_status msdcn_forward_ws(const dcn4_desc *desc, const void *input,
+                                      const void *dir_weight, const void *scale_raw,
+                                      const float *s0_host, float smax, void *output,
+                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /* MSDCN backward: the derivative of msdcn_forward (FlowDCN article, "3.1";
  * the page prints no gradient, these follow by the chain rule). With

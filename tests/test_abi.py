@@ -4,6 +4,7 @@ import ctypes
 import re
 
 import pytest
+import torch
 
 from deformable_convolution_dcn4_b200 import _binding as B
 from deformable_convolution_dcn4_b200 import build as libbuild
@@ -180,3 +181,21 @@ def test_fused_forward_argument_errors(lib):
                                   n.value - 1, None) == 3
     d.algo = B.ALGO_CODE["halo"]  # demands the fused kernel: none for fp32
     assert lib.dcn4_fused_forward(ctypes.byref(d), *fake, None, None, 0, None) == 2
+
+
+def test_workspace_size_where_it_applies():
+    """Scratch only for the staged kernel with one lane per pair: 3x3 taps,
+    groups of 32 or 64 bytes (16-bit) or 64 bytes (fp32); AUTO or HALO."""
+    def size(C, G, dt, k=3, algo="auto"):
+        return B.dcn4_forward_workspace_size(B.make_desc(2, 9, 9, C, G, dt, kernel_size=k,
+                                                         pad=(k - 1) // 2, algo=algo))
+    npairs = 2 * 9 * 9 * 8
+    base = size(128, 8, torch.bfloat16)
+    assert base >= (npairs + 3) // 4 * (16 + 4 * 16)
+    assert size(128, 4, torch.bfloat16) > 0           # D32 bf16: 4 chunks
+    assert size(128, 8, torch.float32) > 0            # D16 fp32: 4 chunks
+    assert size(256, 4, torch.bfloat16) == 0          # D64 bf16: two lanes per pair
+    assert size(128, 16, torch.bfloat16) == 0         # D8 bf16: 16-byte groups
+    assert size(128, 8, torch.bfloat16, k=5) == 0     # 5x5 taps
+    assert size(128, 8, torch.bfloat16, algo="generic") == 0
+    assert size(128, 8, torch.bfloat16, algo="halo") == base

@@ -1,0 +1,118 @@
+"""Deferred escapes of the staged forward (dcn4_forward_ws, msdcn_forward_ws):
+pairs with taps outside the staged window leave their partial sums in
+scratch and their CTA finishes them after its last tile. The output must be
+bit-identical to the in-place path (dcn4_forward, msdcn_forward), whatever
+the scratch size, and match the oracle."""
+import ctypes
+
+import pytest
+import torch
+
+from deformable_convolution_dcn4_b200 import _binding as B
+from deformable_convolution_dcn4_b200.workloads import WORKLOADS, make_inputs
+
+from parity_util import TOL, checked_err, f32, oracle_forward, out_hw
+
+pytestmark = pytest.mark.gpu
+
+W = WORKLOADS
+# offsets of ~8 px against a window reach of 4-5 px: most pairs escape
+CASES = {
+    "dcn4_bf16": W["internimage_bf16"].replace(N=2, H=24, W=40, offset_dist=("normal", 8.0)),
+    "dcn4_f16_softmax": W["internimage_bf16"].replace(N=1, H=20, W=33, dtype="f16",
+                                                      softmax=True, offset_dist=("normal", 8.0)),
+    "dcn4_f32": W["internimage_f32"].replace(N=1, H=17, W=30, offset_dist=("normal", 8.0)),
+    "dcn4_d32_bf16": W["internimage_bf16"].replace(N=1, H=19, W=21, C=128, G=4,
+                                                   offset_dist=("normal", 6.0)),
+    "ms_offset_bf16": W["internimage_bf16"].replace(N=2, H=24, W=24, kind="msdcn",
+                                                    offset_dist=("normal", 2.0)),
+    "ms_dilation_f16": W["internimage_bf16"].replace(N=1, H=21, W=26, dtype="f16",
+                                                     kind="msdcn", msdcn_mode="dilation",
+                                                     offset_dist=("normal", 2.0)),
+}
+
+
+def _scratch(wl):
+    """Scratch of the recommended size, filled with 0xff (an entry written
+    by the kernel shows as changed bytes)."""
+    dt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[wl.dtype]
+    n = B.dcn4_forward_workspace_size(B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, dt))
+    return torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+
+
+def _used(ws):
+    return bool((ws != 255).any())
+
+
+def _run(wl, data, defer, workspace=None, algo="auto"):
+    dev = {k: (v if k == "s0" else v.cuda()) for k, v in data.items()}
+    kw = dict(kernel_size=(wl.kh, wl.kw), stride=wl.stride, pad=wl.pad, dilation=wl.dilation,
+              offset_scale=wl.offset_scale, algo=algo, workspace=workspace, defer_escapes=defer)
+    before = B.dcn4_kernel_launches()
+    if wl.kind == "msdcn":
+        out = B.msdcn_forward(dev["input"], dev["dir_weight"], dev["scale_raw"], dev["s0"],
+                              wl.smax, group=wl.G, msdcn_mode=wl.msdcn_mode, **kw)
+    else:
+        out = B.dcn4_forward(dev["input"], dev["offset_weight"], group=wl.G,
+                             softmax=wl.softmax, **kw)
+    torch.cuda.synchronize()
+    assert B.dcn4_last_device_error() == (0, 0)
+    return out, B.dcn4_kernel_launches() - before
+
+
+def _bits(t):
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_deferred_escapes_are_bit_identical(orc, name):
+    """Entries in the scratch (one kernel either way); the same bits as in
+    place; and the oracle's result."""
+    wl = CASES[name]
+    data = make_inputs(wl, out_hw(wl))
+    inplace, n0 = _run(wl, data, defer=False)
+    ws = _scratch(wl)
+    deferred, n1 = _run(wl, data, defer=True, workspace=ws)
+    assert (n0, n1) == (1, 1) and _used(ws)
+    assert torch.equal(_bits(inplace), _bits(deferred))
+    err = checked_err(f32(deferred), oracle_forward(orc, wl, data), wl.dtype, name)
+    assert err <= TOL[wl.dtype], f"{name}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", ["dcn4_bf16", "ms_offset_bf16"])
+def test_small_scratch_fills_up_and_stays_exact(name):
+    """Scratch for one or two entries per CTA: each CTA fills its share and
+    handles the rest in place; bits unchanged. Scratch too small for one
+    entry per CTA, or misaligned, stays untouched (escapes in place)."""
+    wl = CASES[name]
+    data = make_inputs(wl, out_hw(wl))
+    ref, _ = _run(wl, data, defer=False)
+    entry = 16 + 4 * wl.D  # bytes per entry
+    for extra in (2 * 148 * entry, 148 * entry + 16):
+        ws = torch.full((extra,), 255, dtype=torch.uint8, device="cuda")
+        got, n = _run(wl, data, defer=True, workspace=ws)
+        assert n == 1 and _used(ws)
+        assert torch.equal(_bits(ref), _bits(got))
+    tiny = torch.full((16,), 255, dtype=torch.uint8, device="cuda")
+    got, n = _run(wl, data, defer=True, workspace=tiny)
+    assert n == 1 and not _used(tiny) and torch.equal(_bits(ref), _bits(got))
+    big = _scratch(wl)
+    got, n = _run(wl, data, defer=True, workspace=big[8:])
+    assert n == 1 and not _used(big) and torch.equal(_bits(ref), _bits(got))
+
+
+def test_raw_entry_points_take_null_scratch(orc):
+    """dcn4_forward_ws with a NULL workspace is dcn4_forward."""
+    wl = CASES["dcn4_bf16"]
+    data = make_inputs(wl, out_hw(wl))
+    ref, _ = _run(wl, data, defer=False)
+    dev = {k: v.cuda() for k, v in data.items()}
+    out = torch.empty_like(dev["input"])
+    desc = B.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, torch.bfloat16)
+    before = B.dcn4_kernel_launches()
+    rc = B.load().dcn4_forward_ws(ctypes.byref(desc), ctypes.c_void_p(dev["input"].data_ptr()),
+                                  ctypes.c_void_p(dev["offset_weight"].data_ptr()),
+                                  ctypes.c_void_p(out.data_ptr()), None, 0, None)
+    torch.cuda.synchronize()
+    assert rc == 0 and B.dcn4_kernel_launches() - before == 1
+    assert torch.equal(_bits(ref), _bits(out))

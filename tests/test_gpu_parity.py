@@ -303,15 +303,19 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(orc):
 
 
 def test_launch_counter_counts_each_kernel():
-    """Forward on the halo path is one kernel; the 16-bit backward with 16-bit
+    """Forward on the halo path is one kernel, with escape scratch or without;
+    the 16-bit backward with 16-bit
     cross-CTA accumulation (acc16) is two (zero grad_input, halo kernel);
     with fp32 accumulation (the default, and f32) it is three (zero
     workspace, halo kernel, convert)."""
     wl = REDUCED["internimage_bf16"]
     data = make_inputs(wl, out_hw(wl), with_grad=True)
     x, ow, go = (data[k].cuda() for k in ("input", "offset_weight", "grad_out"))
-    n0 = B.dcn4_kernel_launches()
+    nf = B.dcn4_kernel_launches()
     B.dcn4_forward(x, ow, group=wl.G, algo="halo")
+    n0 = B.dcn4_kernel_launches()
+    assert n0 - nf == 1
+    B.dcn4_forward(x, ow, group=wl.G, algo="halo", defer_escapes=False)
     n1 = B.dcn4_kernel_launches()
     B.dcn4_backward(x, ow, go, group=wl.G, algo="halo", math="acc16")
     n2 = B.dcn4_kernel_launches()
