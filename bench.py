@@ -281,10 +281,20 @@ def cpu_baseline(wl, budget_s=10.0):
             break
         if n < wl.N:
             n = min(wl.N, max(n + 1, int(n * budget_s / max(dt, 1e-3) * 0.25)))
+    # once more on one thread (one image)
+    import oracle
+    orc = oracle.default()
+    orc.set_threads(1)
+    try:
+        dt1, b1 = oracle_step_sample(wl, 1)
+    finally:
+        orc.set_threads(cpu_threads())
     return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": cpu_threads(),
             "kind": "oracle",
             "sample": f"{runs} oracle runs of fwd+bwd+MSDCN fwd, the last on {n} of {wl.N} "
-                      f"images of {wl.name}, {total_t:.1f} s of oracle time"}
+                      f"images of {wl.name}, {total_t:.1f} s of oracle time",
+            "single_thread": {"value": round(b1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"1 image of {wl.name}, {dt1:.2f} s"}}
 
 
 # ---------------------------------------------------------------- our arm

@@ -55,6 +55,11 @@ class Oracle:
             getattr(lib, name).restype = ctypes.c_double
         self.lib = lib
 
+    def set_threads(self, n):
+        """Threads of the oracle's OpenMP loops (a timing knob: the loops are
+        parallel over independent outputs, so results do not depend on it)."""
+        self.lib.omp_set_num_threads(ctypes.c_int(int(n)))
+
     # -- problem description -------------------------------------------------
     @staticmethod
     def problem(N, H, W, C, G, kh=3, kw=3, stride=(1, 1), pad=(1, 1), dilation=(1, 1),
