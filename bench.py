@@ -636,9 +636,12 @@ def time_configs(dcn, flush, stream, peak, peak_kind):
                                                m["s0"], mwl.smax, out=outs[0], **kw)
             elif op == "fused":
                 outs = [torch.empty((wl.N, Ho, Wo, wl.C), dtype=x.dtype, device=dev)]
-                # scratch for the records, used where the call takes the
-                # two-kernel chain (faster than the fused kernel there)
-                fws = torch.empty_like(f["offset_weight"])
+                # scratch for the records and the forward's escapes, used
+                # where the call takes the two-kernel chain (faster than the
+                # fused kernel there)
+                fdesc = dcn.make_desc(wl.N, wl.H, wl.W, wl.C, wl.G, f["x"].dtype)
+                fws = torch.empty(max(16, dcn.dcn4_fused_forward_workspace_size(fdesc)),
+                                  dtype=torch.uint8, device=dev)
                 fn = lambda: dcn.dcn4_fused_forward(f["input"], f["x"], f["dw_weight"],
                                                     f["dw_bias"], f["lin_weight"],
                                                     f["lin_bias"], out=outs[0], workspace=fws,

@@ -321,13 +321,19 @@ bool plan_producer_2d(int H, int W, int C, int J, int NP, ProducerTc2dLayout *ou
 }
 
 // Where the fused kernel splits a tile's groups over several slices, each
-// slice's CTA computes the whole depthwise pass; when the 2-D tensor-core
-// producer takes the shape in one pass (J <= 256 outputs, lin_w resident),
-// the two-kernel chain is then the faster one (InternImage stage, N64 56x56
-// C128 G8 bf16: 174 us against 225 us), while on every shape that leaves the
-// chain's producer on the CUDA cores the fused kernel wins by 3-5x.
+// slice's CTA repeats the depthwise pass and runs the gathers with one CTA
+// per SM after it; the two-kernel chain is then the faster one when the 2-D
+// tensor-core producer takes the shape in one pass (J <= 256 outputs,
+// lin_w resident; InternImage stage, N64 56x56 C128 G8 bf16: 166-174 us
+// against 225 us), or when there are 4 slices or more, whose producer (the
+// fused kernel's producer steps alone) and forward run apart faster (C256
+// G16: 285 against 369 us; C256 G8: 684 against 829 us). With 2 or 3
+// slices and that producer the two are within a few percent (C128 G4: 266
+// against 248 us; C192 G12: 477 against 471 us) and one slice favours the
+// fused kernel (C64 G4: 111 against 141 us).
 bool chain_preferred(const Geometry &g, int eb, const HaloPlan &fused_plan) {
     if (fused_plan.slices < 2 || eb != 2) return false;
+    if (fused_plan.slices >= 4) return true;
     const int J = g.G * g.K * 3, NP = (J + 15) / 16 * 16;
     if (g.C % 16 != 0 || NP > 256 || (J * eb) % 16 != 0) return false;
     ProducerTcLayout lay = ProducerTcLayout::make(g.C, J, NP, g.W, 2);
@@ -547,6 +553,37 @@ dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x, const voi
            (L.pg.J * eb) % 16 == 0 && aligned16(x) && aligned16(lin_weight) &&
            aligned16(offset_weight) && lay.bytes <= max_smem_optin();
     L.lay = lay;
+    if (!L.tc && desc->algo != DCN4_ALGO_GENERIC && eb == 2) {
+        // the fused kernel's producer steps alone: a slice of the groups'
+        // outputs per CTA on the tensor cores, records written out
+        FusedLaunch F;
+        memset(&F, 0, sizeof(F));
+        CUtensorMap map_in, map_xs;
+        memset(&map_in, 0, sizeof(map_in));
+        memset(&map_xs, 0, sizeof(map_xs));
+        if (plan_fused(g, eb, &F.plan, &F.lay) && aligned16(x) && aligned16(lin_weight) &&
+            (reinterpret_cast<uintptr_t>(offset_weight) & 3) == 0 &&
+            encode_input_map(g, L.dtype, x, F.plan, &map_in) &&
+            encode_map(L.dtype, x, g.N, g.H, g.W, g.C, g.C, F.plan.TW + 2, F.plan.TH + 2,
+                       &map_xs)) {
+            F.geo = g;
+            F.dtype = L.dtype;
+            F.in = x;  // no window is loaded; the map only fills the argument
+            F.x = x;
+            F.dw_w = dw_weight;
+            F.dw_b = dw_bias;
+            F.lin_w = lin_weight;
+            F.lin_b = lin_bias;
+            F.out = nullptr;
+            F.rec_out = offset_weight;
+            F.records_only = true;
+            F.mathv = 1;
+            F.tmap_in = &map_in;
+            F.tmap_x = &map_xs;
+            F.stream = L.stream;
+            return cuda_status(launch_fused(F));
+        }
+    }
     if (!L.tc && desc->algo == DCN4_ALGO_HALO) return DCN4_ERR_UNSUPPORTED;
     // the 2-D tiled kernel where it applies (x by TMA tile, sliding-window
     // depthwise, one TMA store per tile)
@@ -575,7 +612,14 @@ dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *byt
     const bool fused = (desc->algo == DCN4_ALGO_AUTO || desc->algo == DCN4_ALGO_HALO) &&
                        plan_fused(g, eb, &plan, &lay) &&
                        !(desc->algo == DCN4_ALGO_AUTO && chain_preferred(g, eb, plan));
-    *bytes = fused ? 0 : (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
+    if (fused) {
+        *bytes = 0;
+        return DCN4_OK;
+    }
+    // the chain: the records, then scratch for the forward's escapes
+    size_t esc = 0;
+    dcn4_forward_workspace_size(desc, &esc);
+    *bytes = ((size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb + 15) / 16 * 16 + esc;
     return DCN4_OK;
 }
 
@@ -633,10 +677,15 @@ dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const v
     // the two-kernel chain, through offset_weight_out when given, else
     // through the caller's scratch
     void *records = offset_weight_out;
+    void *esc = workspace;  // what the records leave of the scratch: the forward's escapes
+    size_t esc_bytes = workspace ? workspace_bytes : 0;
     if (!records) {
         const size_t need = (size_t)g.N * g.Ho * g.Wo * g.G * g.K * 3 * (size_t)eb;
         if (!workspace || workspace_bytes < need) return DCN4_ERR_WORKSPACE;
         records = workspace;
+        const size_t used = (need + 15) / 16 * 16;
+        esc = workspace_bytes > used ? static_cast<unsigned char *>(workspace) + used : nullptr;
+        esc_bytes = workspace_bytes > used ? workspace_bytes - used : 0;
     }
     dcn4_desc d = *desc;
     d.algo = desc->algo == DCN4_ALGO_GENERIC ? DCN4_ALGO_GENERIC : DCN4_ALGO_AUTO;
@@ -644,7 +693,7 @@ dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const v
         dcn4_offset_producer(&d, x, dw_weight, dw_bias, lin_weight, lin_bias, records, stream);
     if (st != DCN4_OK) return st;
     d.algo = desc->algo;
-    return dcn4_forward(&d, input, records, output, stream);
+    return dcn4_forward_ws(&d, input, records, output, esc, esc_bytes, stream);
 }
 
 dcn4_status dcn4_backward_workspace_size(const dcn4_desc *desc, size_t *bytes) {

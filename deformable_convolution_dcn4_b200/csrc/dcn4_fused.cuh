@@ -29,6 +29,9 @@
 //      unit's window load then starts and overlaps its steps 1-4.
 // Every wait is bounded; on expiry the CTA sets the error word, lets its
 // copies and MMAs in flight land, frees its tensor memory and returns.
+// With records_only the kernel is the offset/weight producer alone (steps
+// 1-4 without the window, the records written to rec_out): the tensor-core
+// producer for shapes whose whole lin_w does not fit one CTA next to x and h.
 #pragma once
 
 #include "dcn4_fwd.cuh"
@@ -100,7 +103,8 @@ __global__ void __launch_bounds__(NW * 32, 1)
                       FusedLayout L, const T *__restrict__ in, const T *__restrict__ dw_w,
                       const T *__restrict__ dw_b, const T *__restrict__ lin_w,
                       const T *__restrict__ lin_b, T *__restrict__ out,
-                      T *__restrict__ rec_out, const __grid_constant__ MsdcnParams ms) {
+                      T *__restrict__ rec_out, const __grid_constant__ MsdcnParams ms,
+                      int records_only) {
     extern __shared__ __align__(1024) unsigned char smem[];
     constexpr int NT = NW * 32;
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -239,12 +243,13 @@ __global__ void __launch_bounds__(NW * 32, 1)
     if ((int)blockIdx.x < units) {
         const TileCoord t0 = fused_coord(blockIdx.x, g, pl);
         if (tid == kXThread) issue_x(t0);
-        if (tid == 0) issue_win(t0);
+        if (tid == 0 && !records_only) issue_win(t0);
         int k = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++k) {
             const TileCoord tc = fused_coord(u, g, pl);
             const int un = u + gridDim.x;
             if (!produce(k, u) || !finish(k, tc)) break;
+            if (records_only) continue;  // the producer alone: records to rec_out
             if (!mbar_wait_bounded(win_bar, (uint32_t)k & 1u, kWaitLimitNs)) ok = false;
             else if (tid == 0) ++win_done;
             if (__syncthreads_or(!ok)) break;

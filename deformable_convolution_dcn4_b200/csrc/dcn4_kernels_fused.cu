@@ -39,7 +39,7 @@ cudaError_t launch_fused_t(const FusedLaunch &L) {
         *L.tmap_in, *L.tmap_x, L.geo, L.plan, L.lay, static_cast<const T *>(L.in),
         static_cast<const T *>(L.dw_w), static_cast<const T *>(L.dw_b),
         static_cast<const T *>(L.lin_w), static_cast<const T *>(L.lin_b), static_cast<T *>(L.out),
-        static_cast<T *>(L.rec_out), kNoMs);
+        static_cast<T *>(L.rec_out), kNoMs, L.records_only ? 1 : 0);
     count_launch();
     return cudaGetLastError();
 }

@@ -83,6 +83,7 @@ struct FusedLaunch {
     const void *in, *x, *dw_w, *dw_b, *lin_w, *lin_b;
     void *out;
     void *rec_out;  // optional copy of the records (offset_weight layout)
+    bool records_only;  // the producer alone: no window, no gathers, out unused
     int mathv;      // as FwdLaunch::mathv
     HaloPlan plan;
     FusedLayout lay;

@@ -296,11 +296,18 @@ DCN4_API dcn4_status msdcn_backward(const dcn4_desc *desc, const void *input,
  * type before the linear layer (the tensor cores take 16-bit operands); the
  * result is rounded once to the data type.
  * Kernels: bf16/fp16 with C % 16 == 0, G*kh*kw*3 <= 256, whole 16-byte output
- * rows ((G*kh*kw*3*2) % 16 == 0) and 16-byte aligned x, lin_weight and
- * offset_weight use the tensor-core (tcgen05) kernel; every other call, and
- * desc->algo == DCN4_ALGO_GENERIC, the CUDA-core kernel (h kept in fp32).
- * DCN4_ALGO_HALO demands the tensor-core kernel (DCN4_ERR_UNSUPPORTED where it
- * does not apply). */
+ * rows ((G*kh*kw*3*2) % 16 == 0), lin_weight fitting one CTA's shared memory
+ * next to x and h, and 16-byte aligned x, lin_weight and offset_weight use
+ * the tensor-core (tcgen05) kernels (2-D tiles where they fit, else pixel
+ * ranges). Other bf16/fp16 calls with 3x3 taps and the shapes
+ * dcn4_fused_forward's kernel takes (D*2 in {32, 64} bytes, C a multiple of
+ * 64, C <= 256; 16-byte aligned x and lin_weight, 4-byte aligned
+ * offset_weight) run that kernel's producer steps alone: each CTA computes
+ * the outputs of one slice of 128 bytes of groups on the tensor cores (the
+ * depthwise pass repeated per slice). Every other call, and desc->algo ==
+ * DCN4_ALGO_GENERIC, runs the CUDA-core kernel (h kept in fp32).
+ * DCN4_ALGO_HALO demands a tensor-core kernel (DCN4_ERR_UNSUPPORTED where
+ * none applies). */
 DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
                                           const void *dw_weight, const void *dw_bias,
                                           const void *lin_weight, const void *lin_bias,
@@ -310,8 +317,11 @@ DCN4_API dcn4_status dcn4_offset_producer(const dcn4_desc *desc, const void *x,
  * runs the fused kernel (its shape and desc->algo; it may still need the
  * scratch when a pointer is not aligned, see below), else the size of the
  * offset_weight tensor the two-kernel chain passes through,
- * N*Ho*Wo*G*kh*kw*3 elements of desc->dtype (none is needed when the call
- * passes offset_weight_out). With DCN4_ALGO_AUTO that includes the shapes on
+ * N*Ho*Wo*G*kh*kw*3 elements of desc->dtype rounded up to 16 bytes (none is
+ * needed when the call passes offset_weight_out), plus
+ * dcn4_forward_workspace_size bytes for the forward's escapes (optional:
+ * the chain's forward uses what the records leave over, see
+ * dcn4_forward_ws). With DCN4_ALGO_AUTO that includes the shapes on
  * which the chain is the faster path (see dcn4_fused_forward); a call given
  * no scratch there runs the fused kernel instead. */
 DCN4_API dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, size_t *bytes);
@@ -347,17 +357,18 @@ DCN4_API dcn4_status dcn4_fused_forward_workspace_size(const dcn4_desc *desc, si
  * N*Ho*Wo*G*kh*kw*3*sizeof(element) bytes, else DCN4_ERR_WORKSPACE before any
  * launch; 16-byte aligned to take the tensor-core producer and the staged
  * forward), and then dcn4_forward on it. The chain's records are the
- * tensor-core producer's where that applies and the CUDA-core producer's
- * (h kept in fp32) otherwise, so on shapes the tensor-core producer does not
- * take the chain and the fused kernel may round a record differently.
+ * tensor-core producers' where one applies and the CUDA-core producer's
+ * (h kept in fp32) otherwise, so on shapes no tensor-core producer takes the
+ * chain and the fused kernel may round a record differently.
  * DCN4_ALGO_AUTO also takes the chain on a fused-kernel shape where the
  * chain is faster, when it has 16-byte aligned room for the records
  * (offset_weight_out, or a large enough workspace): where the groups span
  * two or more slices (every slice's CTA then repeats the depthwise pass) and
  * the tensor-core producer takes the shape in one 2-D tiled pass (at most 256
  * outputs per pixel in whole 16-byte rows, C and lin_weight fitting shared
- * memory) -- the InternImage stage, C128 G8, is one. Given no room it runs
- * the fused kernel.
+ * memory) -- the InternImage stage, C128 G8, is one -- and where they span
+ * four slices or more (C256 G16, C256 G8), whose producer runs this kernel's
+ * producer steps alone. Given no room it runs the fused kernel.
  * DCN4_ALGO_HALO demands the fused kernel (DCN4_ERR_UNSUPPORTED where it does
  * not apply). */
 DCN4_API dcn4_status dcn4_fused_forward(const dcn4_desc *desc, const void *input, const void *x,

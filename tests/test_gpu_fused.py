@@ -61,8 +61,9 @@ CASES = {
 FUSED = sorted(k for k, v in CASES.items() if v[6])
 # fused-kernel shapes where AUTO takes the two-kernel chain when it has room
 # for the records: two or more group slices (each slice's CTA repeats the
-# depthwise pass) and a shape the 2-D tensor-core producer takes in one pass
-AUTO_CHAIN = {"internimage_bf16", "internimage_f16"}
+# depthwise pass) and a shape the 2-D tensor-core producer takes in one
+# pass, or four slices and more (the sliced tensor-core producer)
+AUTO_CHAIN = {"internimage_bf16", "internimage_f16", "c256_bf16"}
 
 
 def _inputs(name, seed=7, sigma=2.0):
@@ -232,15 +233,17 @@ def test_fused_full_size_internimage(orc):
 def test_fused_workspace_size_and_refusal():
     """Shapes on which AUTO runs the fused kernel need no scratch; the others
     (the chain's shapes, and those where AUTO prefers the chain) ask for the
-    offset_weight tensor's bytes; the forced fused kernel never does. A chain
-    shape refuses a smaller scratch before any launch."""
+    offset_weight tensor's bytes (rounded to 16) plus the forward's escape
+    scratch; the forced fused kernel never does. A chain shape refuses
+    scratch smaller than the records before any launch."""
     for name in sorted(CASES):
         N, H, W, C, G, dtype, fused = CASES[name]
         desc = B.make_desc(N, H, W, C, G, DTYPES[dtype])
         need = B.dcn4_fused_forward_workspace_size(desc)
         eb = 4 if dtype == "f32" else 2
         auto_fused = fused and name not in AUTO_CHAIN
-        assert need == (0 if auto_fused else N * H * W * G * 27 * eb), name
+        chain = (N * H * W * G * 27 * eb + 15) // 16 * 16 + B.dcn4_forward_workspace_size(desc)
+        assert need == (0 if auto_fused else chain), name
         if fused:
             desc = B.make_desc(N, H, W, C, G, DTYPES[dtype], algo="halo")
             assert B.dcn4_fused_forward_workspace_size(desc) == 0, name

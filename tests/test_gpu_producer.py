@@ -23,8 +23,13 @@ CASES = {
     "c16_k1_bf16": (1, 5, 130, 16, 8, 1, "bf16", True),
     # C = 256 (16 K steps), 1x1 taps, one ragged tile of 35 pixels
     "c256_k1_bf16": (1, 5, 7, 256, 8, 1, "bf16", True),
-    # C = 256 with 3x3 taps: lin_w does not fit next to the tile (generic)
-    "c256_bf16": (1, 5, 7, 256, 8, 3, "bf16", False),
+    # C = 256 with 3x3 taps: lin_w does not fit next to the tile; the fused
+    # kernel's producer steps (4 slices of 2 groups) take it
+    "c256_bf16": (1, 5, 7, 256, 8, 3, "bf16", True),
+    # the high-resolution stage's channels (C256 G16: J = 432 > 256), 4
+    # slices of 108 outputs, tiles 16 x 8 with ragged edges
+    "c256_g16_bf16": (2, 19, 13, 256, 16, 3, "bf16", True),
+    "c256_g16_f16": (1, 9, 21, 256, 16, 3, "f16", True),
     # not for the tensor cores: fp32; J = 81 (odd 16-byte rows); J = 540 > 256
     "f32_g3": (2, 9, 7, 24, 3, 3, "f32", False),
     "bf16_g3": (1, 10, 12, 48, 3, 3, "bf16", False),
@@ -84,6 +89,15 @@ def test_producer_full_size_internimage(orc):
     got = f32(_gpu(d, 8, 3, "halo"))
     images = [0, 1, 63]
     err = checked_err(got[images], _oracle(orc, d, 8, 3, images), "bf16", "full size")
+    assert err <= TOL["bf16"], f"scaled error {err:.2e}"
+
+
+def test_producer_full_size_highres(orc):
+    """N4 128x128 C256 G16 bf16 (J = 432: the sliced tensor-core path, 4096
+    units of 16 x 8 pixels x 4 groups), image 2 against the oracle."""
+    d = _inputs(4, 128, 128, 256, 16, 3, "bf16", seed=1)
+    got = f32(_gpu(d, 16, 3, "halo"))
+    err = checked_err(got[[2]], _oracle(orc, d, 16, 3, [2]), "bf16", "full size")
     assert err <= TOL["bf16"], f"scaled error {err:.2e}"
 
 
