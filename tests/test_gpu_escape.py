@@ -116,3 +116,43 @@ def test_raw_entry_points_take_null_scratch(orc):
     torch.cuda.synchronize()
     assert rc == 0 and B.dcn4_kernel_launches() - before == 1
     assert torch.equal(_bits(ref), _bits(out))
+
+
+def _random_cases(count=12, seed=77):
+    """Seeded shapes for the staged kernel with one lane per pair: N 1..3, H
+    and W 1..40, 16-bit groups of 16 or 32 channels or fp32 groups of 16,
+    DCNv4 (softmax or not) or MSDCN (either reading), offsets of 3-8 px."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < count:
+        dtype = str(rng.choice(["bf16", "f16", "f32"]))
+        D = 16 if dtype == "f32" else int(rng.choice([16, 32]))
+        G = int(rng.choice([2, 4, 8]))
+        if (128 // (D * (4 if dtype == "f32" else 2))) > G:
+            continue
+        kind = str(rng.choice(["dcn4", "msdcn"]))
+        base = W["internimage_f32"] if dtype == "f32" else W["internimage_bf16"]
+        kw = dict(N=int(rng.integers(1, 4)), H=int(rng.integers(1, 41)),
+                  W=int(rng.integers(1, 41)), C=G * D, G=G, dtype=dtype, kind=kind,
+                  offset_dist=("normal", float(rng.uniform(3.0, 8.0))),
+                  seed=int(rng.integers(0, 1000)))
+        if kind == "msdcn":
+            kw["msdcn_mode"] = str(rng.choice(["offset", "dilation"]))
+            kw["offset_dist"] = ("normal", 1.5)
+        else:
+            kw["softmax"] = bool(rng.integers(0, 2))
+        cases.append(base.replace(**kw))
+    return cases
+
+
+@pytest.mark.parametrize("i", range(12))
+def test_deferred_escapes_random_shapes(orc, i):
+    """Seeded random shapes: deferred and in-place bits equal, oracle gates."""
+    wl = _random_cases()[i]
+    data = make_inputs(wl, out_hw(wl))
+    inplace, _ = _run(wl, data, defer=False)
+    deferred, _ = _run(wl, data, defer=True, workspace=_scratch(wl))
+    assert torch.equal(_bits(inplace), _bits(deferred)), wl
+    err = checked_err(f32(deferred), oracle_forward(orc, wl, data), wl.dtype, str(wl))
+    assert err <= TOL[wl.dtype], f"{wl}: {err:.3e}"
