@@ -5,8 +5,8 @@ the access) on the small and edge parity cases of every kernel: staged,
 vectorised and scalar forward and backward, DCNv4 and MSDCN, and both
 offset/weight producers. Each case must match the oracle within the usual
 gate, give the same forward output bit for bit as the normal build, and leave
-the device error word clear. compute-sanitizer is not available on the GPU
-pool, so this build is how out-of-bounds accesses are caught."""
+the device error word clear. It stands in for compute-sanitizer: the checked
+library is how out-of-bounds accesses are caught."""
 import os
 
 import pytest
